@@ -1,0 +1,69 @@
+"""Seeded synthetic inputs for the fused MoE forward.
+
+This module is shared by the tests, the benchmark and the oracle's callers.
+It holds no part of the method's arithmetic: it only draws random tensors
+with the shapes and distributions of the atrex-bench #009 "fused_moe"
+workload (its input.py, ``_make_inputs``): hidden ``randn * 0.1`` in bf16,
+w1 ``randn * H**-0.5`` and w2 ``randn * I**-0.5`` in bf16, and fp32 ``randn``
+router logits.  Routing (softmax / top-k / renormalisation) is NOT done here;
+each side computes it from the logits with its own code.
+
+The draws use torch's CPU generator so that the CPU oracle and the GPU path
+see bit-identical inputs; callers move tensors to the GPU themselves.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+
+@dataclass(frozen=True)
+class MoEShape:
+    name: str
+    T: int
+    H: int
+    I: int
+    E: int
+    k: int
+
+    @property
+    def flops(self) -> float:
+        """Useful FLOPs of one forward: 2 GEMMs of 2*T*k*H*(2I) and 2*T*k*I*H."""
+        return 6.0 * self.T * self.k * self.H * self.I
+
+    def describe(self) -> dict:
+        return {"workload": self.name, "T": self.T, "H": self.H, "I": self.I,
+                "E": self.E, "top_k": self.k}
+
+
+# The five workloads: a tiny case, and rows 4, 8, 19 and 22 of the
+# atrex-bench #009 shapes table.
+SHAPES = {
+    "tiny": MoEShape("tiny fused MoE T=64 H=256 I=128 E=8 k=2", 64, 256, 128, 8, 2),
+    "prefill_8e": MoEShape("prefill, few large experts T=1979 H=2048 I=2048 E=8 k=2",
+                           1979, 2048, 2048, 8, 2),
+    "decode": MoEShape("decode, many small experts T=1 H=2048 I=768 E=128 k=8",
+                       1, 2048, 768, 128, 8),
+    "prefill_thin": MoEShape("prefill, many thin experts T=8192 H=4096 I=384 E=128 k=8",
+                             8192, 4096, 384, 128, 8),
+    "prefill_big": MoEShape("large prefill, big experts T=15381 H=4096 I=4096 E=8 k=2",
+                            15381, 4096, 4096, 8, 2),
+}
+
+
+def make_inputs(T: int, H: int, I: int, E: int, seed: int = 0,
+                hidden_scale: float = 0.1):
+    """Draw (hidden [T,H] bf16, w1 [E,2I,H] bf16, w2 [E,H,I] bf16,
+    logits [T,E] fp32) on the CPU, in that order, from one seeded generator."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    hidden = torch.randn(T, H, dtype=torch.bfloat16, generator=g) * hidden_scale
+    w1 = torch.randn(E, 2 * I, H, dtype=torch.bfloat16, generator=g) * (H ** -0.5)
+    w2 = torch.randn(E, H, I, dtype=torch.bfloat16, generator=g) * (I ** -0.5)
+    logits = torch.randn(T, E, dtype=torch.float32, generator=g)
+    return hidden, w1, w2, logits
+
+
+def make_shape_inputs(shape: MoEShape, seed: int = 0):
+    return make_inputs(shape.T, shape.H, shape.I, shape.E, seed=seed)

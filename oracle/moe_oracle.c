@@ -1,0 +1,298 @@
+/*
+ * moe_oracle.c -- the plain, slow, fp64 CPU oracle of the fused MoE forward.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only tests/, __graft_entry__.smoke()
+ * and bench.py's cpu_baseline / reference arm may load or run this file.  It
+ * shares no code, header, table or helper with the CUDA library and includes
+ * nothing from it.
+ *
+ * What it computes (sources: the web pages this project restates):
+ *   - "tpu_inference/kernels/fused_moe/v1/kernel.py" (tpu-inference 0.11.1),
+ *     function ref_moe: softmax over the router logits, lax.top_k, then for
+ *     every token and each chosen expert x.[W_gate | W_up] -> act(gate)*up ->
+ *     .W2, and the top-k-weighted sum over the chosen experts.
+ *   - the same file at tpu-inference 0.13.2, ref_moe: optional division of
+ *     the k chosen weights by their sum (renormalize_topk_logits).
+ *   - atrex-bench operator #009 "fused_moe", reference.py Model.forward: the
+ *     same function written as a loop over experts with a token mask, the
+ *     vLLM weight layout w1 [E, 2I, H] (rows 0..I-1 gate, I..2I-1 up) and
+ *     w2 [E, H, I] applied as F.linear, and an fp32 [T, H] output that starts
+ *     at zero.
+ *
+ * Everything is computed in double precision from the bf16 inputs (bf16 ->
+ * double is exact).  Nothing is blocked, fused or reordered beyond what the
+ * definitions state; OpenMP only splits independent tokens across threads.
+ *
+ * Readings taken where the pages are silent (each is listed in the design doc):
+ *   - top-k order: largest logit first; equal logits go to the lowest expert
+ *     index (the in-kernel argmax on the TPU page returns the lowest index).
+ *     Ranking logits is ranking the exact softmax, since exp is monotone.
+ *   - logits of -inf get probability 0 and can still fill the remaining
+ *     slots, lowest untaken index first; an expert is never chosen twice.
+ *   - expert ids outside [0, E) in the forward input are skipped (the
+ *     per-expert loop of Model.forward only visits 0..E-1).
+ *   - silu(z) = z / (1 + exp(-z)).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Planted-mistake builds: tests compile this file with -DORACLE_MUTATION=n to
+ * check that the pins catch each plausible mistake.  The normal build leaves
+ * ORACLE_MUTATION at 0 and every MUTATED(n) is false. */
+#ifndef ORACLE_MUTATION
+#define ORACLE_MUTATION 0
+#endif
+#define MUTATED(n) (ORACLE_MUTATION == (n))
+
+static double bf16_to_double(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+int oracle_mutation(void) { return ORACLE_MUTATION; }
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/*
+ * Routing: per token, p_e = exp(l_e - m) / sum_e' exp(l_e' - m) with
+ * m = max_e l_e; the k experts with the largest logits in (logit desc,
+ * index asc) order; w_j = p_{id_j}; with renorm, w_j /= sum_j w_j.
+ * Pages: ref_moe (softmax, lax.top_k), ref_moe of 0.13.2 (renormalisation),
+ * atrex-bench #009 input.py (softmax -> topk -> divide by the sum).
+ * logits [T, E] fp32 row-major -> ids [T, k] int32, weights [T, k] double.
+ * Returns 0, or -1 for bad arguments.
+ */
+int oracle_route(const float *logits, int64_t T, int E, int k, int renorm,
+                 int32_t *ids, double *weights)
+{
+    if (T < 0 || E < 1 || k < 1 || k > E) return -1;
+    char *taken = (char *)malloc((size_t)E);
+    if (!taken) return -1;
+    for (int64_t t = 0; t < T; ++t) {
+        const float *l = logits + t * E;
+        double m = -INFINITY;
+        for (int e = 0; e < E; ++e)
+            if ((double)l[e] > m) m = (double)l[e];
+        double s = 0.0;
+        for (int e = 0; e < E; ++e) s += exp((double)l[e] - m);
+
+        memset(taken, 0, (size_t)E);
+        double wsum = 0.0;
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0) { best = e; continue; }
+                if (MUTATED(4) ? (l[e] >= l[best]) : (l[e] > l[best])) best = e;
+            }
+            taken[best] = 1;
+            ids[t * k + j] = best;
+            double p = exp((double)l[best] - m) / s;
+            weights[t * k + j] = p;
+            wsum += p;
+        }
+        if (renorm && !MUTATED(3))
+            for (int j = 0; j < k; ++j) weights[t * k + j] /= wsum;
+    }
+    free(taken);
+    return 0;
+}
+
+/*
+ * Permutation of the flat (token, slot) indices i = t*k + j by expert: a
+ * stable counting sort.  counts[e] = #{i : ids[i] == e}; offsets is the
+ * exclusive prefix sum (offsets[0] = 0, offsets[E] = number of valid ids);
+ * sorted_rows[offsets[e] + r] is the r-th smallest i with ids[i] == e.
+ * This is the (token, k) visiting order in which the TPU kernel's scatter
+ * hands rows to each expert (start_a2a_scatter) and the ascending token
+ * order of Model.forward's nonzero() per expert.  Ids outside [0, E) are
+ * left out.  sorted_rows must hold n entries; entries past offsets[E] are
+ * set to -1.
+ */
+int oracle_permute(const int32_t *ids, int64_t n, int E,
+                   int32_t *sorted_rows, int32_t *offsets)
+{
+    if (n < 0 || E < 1) return -1;
+    int64_t *cursor = (int64_t *)calloc((size_t)E + 1, sizeof(int64_t));
+    if (!cursor) return -1;
+    for (int64_t i = 0; i < n; ++i) {
+        int e = ids[i];
+        if (e >= 0 && e < E) cursor[e + 1] += 1;
+    }
+    for (int e = 0; e < E; ++e) cursor[e + 1] += cursor[e];
+    for (int e = 0; e <= E; ++e) offsets[e] = (int32_t)cursor[e];
+    for (int64_t i = 0; i < n; ++i) sorted_rows[i] = -1;
+    if (MUTATED(5)) {
+        /* planted mistake: visit the indices from the back (unstable order) */
+        for (int64_t i = n - 1; i >= 0; --i) {
+            int e = ids[i];
+            if (e >= 0 && e < E) sorted_rows[cursor[e]++] = (int32_t)i;
+        }
+    } else {
+        for (int64_t i = 0; i < n; ++i) {
+            int e = ids[i];
+            if (e >= 0 && e < E) sorted_rows[cursor[e]++] = (int32_t)i;
+        }
+    }
+    free(cursor);
+    return 0;
+}
+
+/*
+ * One expert's SwiGLU FFN on one token, in double:
+ *   g_i = W1[e][i,:] . x, u_i = W1[e][I+i,:] . x, a_i = silu(g_i) * u_i,
+ *   y_h = W2[e][h,:] . a.
+ * Layout of atrex-bench #009: F.linear(x, w1_e) is x . w1_e^T with w1_e of
+ * shape [2I, H]; the first I outputs are gate, the next I are up;
+ * F.linear(act, w2_e) with w2_e of shape [H, I].
+ */
+static void expert_ffn(const uint16_t *w1, const uint16_t *w2, int e,
+                       int64_t H, int64_t I, const double *x, double *a,
+                       double *y)
+{
+    const uint16_t *W1 = w1 + (size_t)e * 2 * I * H;
+    const uint16_t *W2 = w2 + (size_t)e * H * I;
+    for (int64_t i = 0; i < I; ++i) {
+        const uint16_t *rg = W1 + (size_t)i * H;
+        const uint16_t *ru = W1 + (size_t)(I + i) * H;
+        if (MUTATED(1)) { const uint16_t *tmp = rg; rg = ru; ru = tmp; }
+        double g = 0.0, u = 0.0;
+        for (int64_t h = 0; h < H; ++h) {
+            g += bf16_to_double(rg[h]) * x[h];
+            u += bf16_to_double(ru[h]) * x[h];
+        }
+        a[i] = silu(g) * u;
+    }
+    for (int64_t h = 0; h < H; ++h) {
+        double acc = 0.0;
+        for (int64_t i = 0; i < I; ++i) {
+            /* planted mistake 2 reads W2 as if it were stored [I, H]
+             * (only meaningful when H == I, which the test uses) */
+            double wv = MUTATED(2) ? bf16_to_double(W2[(size_t)i * H + h])
+                                   : bf16_to_double(W2[(size_t)h * I + i]);
+            acc += wv * a[i];
+        }
+        y[h] = acc;
+    }
+}
+
+/*
+ * Formulation A, the per-token loop of ref_moe: for every token t (or only
+ * the tokens listed in `rows`, when nrows >= 0), out[t] = sum over j of
+ * w[t,j] * FFN_{ids[t,j]}(x_t), with j ascending.  Ids outside [0, E) are
+ * skipped.  hidden [T,H], w1 [E,2I,H], w2 [E,H,I] are bf16 bit patterns;
+ * topk_w [T,k] double; out is [nrows or T, H] double, overwritten.
+ */
+int oracle_moe_token_loop(const uint16_t *hidden, const uint16_t *w1,
+                          const uint16_t *w2, const double *topk_w,
+                          const int32_t *ids, int64_t T, int64_t H, int64_t I,
+                          int E, int k, const int64_t *rows, int64_t nrows,
+                          double *out)
+{
+    if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1) return -1;
+    int64_t n = nrows >= 0 ? nrows : T;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *x = (double *)malloc(sizeof(double) * (size_t)H);
+        double *a = (double *)malloc(sizeof(double) * (size_t)I);
+        double *y = (double *)malloc(sizeof(double) * (size_t)H);
+        if (!x || !a || !y) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < n; ++r) {
+                int64_t t = nrows >= 0 ? rows[r] : r;
+                double *o = out + (size_t)r * H;
+                for (int64_t h = 0; h < H; ++h) o[h] = 0.0;
+                if (t < 0 || t >= T) continue;
+                for (int64_t h = 0; h < H; ++h) x[h] = bf16_to_double(hidden[(size_t)t * H + h]);
+                for (int j = 0; j < k; ++j) {
+                    int e = ids[t * k + j];
+                    if (e < 0 || e >= E) continue;
+                    expert_ffn(w1, w2, e, H, I, x, a, y);
+                    double wj = topk_w[t * k + j];
+                    for (int64_t h = 0; h < H; ++h) o[h] += wj * y[h];
+                }
+            }
+        }
+        free(x); free(a); free(y);
+    }
+    return err ? -1 : 0;
+}
+
+/*
+ * Formulation B, the per-expert mask loop of Model.forward: out = 0; for
+ * e = 0..E-1: w_hat[t] = sum_j w[t,j] * [ids[t,j] == e]; for every token
+ * with w_hat[t] != 0 (ascending t): out[t] += w_hat[t] * FFN_e(x_t).
+ * A token routed twice to e thus gets the summed weight.  Same argument
+ * layout as formulation A (all T rows).
+ */
+int oracle_moe_expert_loop(const uint16_t *hidden, const uint16_t *w1,
+                           const uint16_t *w2, const double *topk_w,
+                           const int32_t *ids, int64_t T, int64_t H, int64_t I,
+                           int E, int k, double *out)
+{
+    if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1) return -1;
+    double *what = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    if (!what) return -1;
+    for (int64_t i = 0; i < T * H; ++i) out[i] = 0.0;
+    int err = 0;
+    for (int e = 0; e < E; ++e) {
+        for (int64_t t = 0; t < T; ++t) {
+            double s = 0.0;
+            for (int j = 0; j < k; ++j)
+                if (ids[t * k + j] == e) s += topk_w[t * k + j];
+            what[t] = s;
+        }
+#pragma omp parallel
+        {
+            double *x = (double *)malloc(sizeof(double) * (size_t)H);
+            double *a = (double *)malloc(sizeof(double) * (size_t)I);
+            double *y = (double *)malloc(sizeof(double) * (size_t)H);
+            if (!x || !a || !y) {
+#pragma omp atomic write
+                err = 1;
+            } else {
+#pragma omp for schedule(dynamic, 1)
+                for (int64_t t = 0; t < T; ++t) {
+                    if (what[t] == 0.0) continue;
+                    for (int64_t h = 0; h < H; ++h) x[h] = bf16_to_double(hidden[(size_t)t * H + h]);
+                    expert_ffn(w1, w2, e, H, I, x, a, y);
+                    double *o = out + (size_t)t * H;
+                    for (int64_t h = 0; h < H; ++h) o[h] += what[t] * y[h];
+                }
+            }
+            free(x); free(a); free(y);
+        }
+    }
+    free(what);
+    return err ? -1 : 0;
+}
