@@ -1,0 +1,179 @@
+/*
+ * moe.h -- C ABI of libmoe.so, a fused Mixture-of-Experts forward for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The function computed is the one defined on the pages this library
+ * restates:
+ *   - "tpu_inference/kernels/fused_moe/v1/kernel.py" (tpu-inference), ref_moe:
+ *     softmax over router logits, top-k expert choice (optionally
+ *     renormalised, 0.13.2 version of that page), a SwiGLU expert FFN per
+ *     (token, chosen expert), and the top-k-weighted sum;
+ *   - atrex-bench operator #009 "fused_moe", reference.py Model.forward and
+ *     input.py: the weight layout used here (w1 [E, 2I, H], rows 0..I-1
+ *     gate and I..2I-1 up; w2 [E, H, I]), fp32 top-k weights, int32 ids and
+ *     an fp32 [T, H] output.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *     owned by the caller, dense and row-major.  bf16 tensors are passed as
+ *     uint16_t bit patterns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  No call
+ *     synchronises the stream unless its comment says so; results are ready
+ *     when the stream's work completes.
+ *   - Return value: MOE_OK (0) or a negative MOE_ERR_* code.  Nothing is
+ *     launched when an argument check fails.  No call throws.
+ *   - The library owns a grow-only device workspace per device (routing
+ *     permutation, the bf16 SwiGLU intermediate, per-(token, slot) expert
+ *     outputs).  It grows on the first call that needs more; that call
+ *     allocates (and synchronises the device if it frees a smaller one).
+ *     Calls on two different streams of one device must not overlap in time
+ *     (they share that workspace).
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG -1 /* null pointer, negative size, k outside [1, E] */
+#define MOE_ERR_UNSUPPORTED -2 /* shape this build does not handle (see each call) */
+#define MOE_ERR_CUDA -3        /* a CUDA runtime/driver call or a launch failed */
+#define MOE_ERR_TIMEOUT -4     /* a bounded device-side wait expired */
+#define MOE_ERR_NO_DEVICE -5   /* no usable sm_100 device is current */
+#define MOE_ERR_OOM -6         /* workspace allocation failed */
+
+/* Bits of the device status word (moe_get_device_status). */
+#define MOE_STATUS_TIMEOUT 0x1u  /* a pipeline wait gave up; that launch's output is invalid */
+#define MOE_STATUS_BAD_ID 0x2u   /* moe_forward met an expert id outside [0, E) and skipped it */
+
+/*
+ * moe_route -- router softmax, top-k choice and optional renormalisation.
+ * Pages: ref_moe (softmax over the experts, lax.top_k), its 0.13.2 version
+ * (renormalize_topk_logits divides the k weights by their sum), and the
+ * in-kernel top-k of the same file (an argmax that returns the lowest index
+ * among equal values).
+ *
+ *   logits        [T, E] fp32, read only.
+ *   topk_ids      [T, k] int32, written: the k experts with the largest
+ *                 logits, largest first; equal logits go to the lower index.
+ *   topk_weights  [T, k] fp32, written: p_id = exp(l_id - max) / sum exp(l - max)
+ *                 and, when renorm != 0, divided by the sum of the k values.
+ * Errors: INVALID_ARG for null pointers, T < 0, E < 1, k < 1 or k > E;
+ *         UNSUPPORTED for E > 1024.  T == 0 launches nothing.
+ * Logits may be -inf (probability 0; such experts fill leftover slots lowest
+ * index first).  Rows that are all -inf or contain NaN are undefined.
+ */
+int moe_route(const float *logits, int64_t T, int E, int k, int renorm,
+              int32_t *topk_ids, float *topk_weights, void *stream);
+
+/*
+ * moe_forward -- the expert FFNs and the weighted combine.
+ * Pages: ref_moe (per token: x.[W_gate | W_up] -> silu(gate) * up -> .W2,
+ * then sum_j w_j y_j); atrex-bench #009 Model.forward (same result written
+ * as a loop over experts; a token routed twice to one expert gets the summed
+ * weight; ids outside [0, E) never match an expert).
+ *
+ *   hidden        [T, H] bf16
+ *   w1            [E, 2I, H] bf16; rows 0..I-1 of w1[e] are the gate
+ *                 projection, rows I..2I-1 the up projection (x . w1[e]^T)
+ *   w2            [E, H, I] bf16 (act . w2[e]^T)
+ *   topk_weights  [T, k] fp32
+ *   topk_ids      [T, k] int32; ids outside [0, E) are skipped and flagged
+ *                 with MOE_STATUS_BAD_ID in the device status word
+ *   out           [T, H] fp32, every element overwritten:
+ *                 out[t] = sum over j = 0..k-1 (in that order) of
+ *                          topk_weights[t, j] * FFN_{topk_ids[t, j]}(hidden[t]),
+ *                 accumulated in fp32; a row with no valid id is 0.
+ * Numerics: bf16 inputs, fp32 accumulation; the SwiGLU intermediate is
+ * rounded to bf16 before the second projection on the grouped-GEMM path
+ * (T > small-T limit) and kept in fp32 on the small-T path.  The combine is
+ * deterministic (fixed j order, no atomics): repeated calls give identical
+ * bits.
+ * Errors: INVALID_ARG for null pointers, T < 0, H/I/E < 1, k < 1 or k > E;
+ *         UNSUPPORTED unless H % 128 == 0 and I % 128 == 0 (the alignment
+ *         the TPU page also demands), E <= 1024 and k <= 16;
+ *         OOM if the workspace cannot grow.  T == 0 launches nothing.
+ */
+int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
+                const float *topk_weights, const int32_t *topk_ids, float *out,
+                int64_t T, int H, int I, int E, int k, void *stream);
+
+/*
+ * moe_permute -- the expert grouping that moe_forward uses internally,
+ * exported so that it can be checked bit for bit.  Pages: the TPU kernel
+ * hands each expert its rows in (token, k) order (start_a2a_scatter);
+ * Model.forward visits each expert's tokens in ascending order.
+ *
+ *   topk_ids        [T, k] int32 (flat index i = t*k + j)
+ *   sorted_rows     [T*k] int32, written for positions < expert_offsets[E]:
+ *                   the flat indices grouped by expert, ascending within an
+ *                   expert (a stable counting sort); later positions are
+ *                   left untouched
+ *   expert_offsets  [E+1] int32, written: exclusive prefix sum of the
+ *                   per-expert counts; expert_offsets[E] = number of ids in
+ *                   [0, E)
+ * Errors: INVALID_ARG for null pointers, T < 0, k < 1, E < 1;
+ *         UNSUPPORTED for E > 1024.
+ */
+int moe_permute(const int32_t *topk_ids, int64_t T, int k, int E,
+                int32_t *sorted_rows, int32_t *expert_offsets, void *stream);
+
+/* Static, NUL-terminated description of an MOE_* return code. */
+const char *moe_error_string(int code);
+
+/*
+ * moe_get_device_status -- SYNCHRONISES `stream`, then returns in *status
+ * the OR of the MOE_STATUS_* bits raised by this library's kernels on the
+ * current device since the last call, and clears them.  Debug aid.
+ */
+int moe_get_device_status(void *stream, uint32_t *status);
+
+/*
+ * Tuning and debug switches (host-side, process-wide):
+ *   moe_set_small_t_max(n)  -- moe_forward uses the GEMV path when T <= n
+ *                              (default 16, also read from MOE_SMALL_T_MAX);
+ *                              n = 0 forces the grouped-GEMM path.
+ *   moe_set_sync_each_stage(on) -- synchronise and check for errors after
+ *                              every launch (also MOE_SYNC_EACH_STAGE=1);
+ *                              a failure returns MOE_ERR_CUDA and
+ *                              moe_last_failed_stage() names the kernel.
+ *   moe_set_wait_limit_ns(ns) -- bound of every device-side pipeline wait
+ *                              (default 2e9 ns); ns <= 0 restores it.
+ * Each returns the previous value.
+ */
+int moe_set_small_t_max(int n);
+int moe_set_sync_each_stage(int on);
+int64_t moe_set_wait_limit_ns(int64_t ns);
+const char *moe_last_failed_stage(void);
+
+/*
+ * moe_debug_wait_timeout -- launches one CTA that waits on a shared-memory
+ * barrier nothing will ever signal, bounded by `limit_ns`, and SYNCHRONISES
+ * the stream.  Returns MOE_ERR_TIMEOUT when the bounded wait gave up as
+ * designed (and leaves MOE_STATUS_TIMEOUT set), MOE_OK if it somehow
+ * completed.  Exercises the failure path of the pipeline waits without
+ * faulting or hanging the GPU.  limit_ns must be in (0, 1e10].
+ */
+int moe_debug_wait_timeout(int64_t limit_ns, void *stream);
+
+/*
+ * Per-kernel timing for benchmarks.  While enabled, moe_route/moe_forward/
+ * moe_permute record a CUDA event pair around each kernel launch on the
+ * caller's stream.  moe_profile_read SYNCHRONISES the device, then for each
+ * kernel name (up to max_names) writes its launch count, total milliseconds
+ * and name, and returns how many names exist.  moe_profile_reset clears.
+ */
+int moe_profile_enable(int on);
+int moe_profile_reset(void);
+int moe_profile_read(int max_names, char (*names)[64], int64_t *launches,
+                     double *total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

@@ -1,0 +1,224 @@
+"""Python binding of libmoe.so, the B200 (sm_100a) fused MoE forward.
+
+Argument marshalling only: every function checks dtypes, shapes and devices
+of torch tensors, passes raw device pointers, sizes and the current CUDA
+stream to the C ABI of ``include/moe.h`` and raises ``MoEError`` on a
+non-zero return code.  All arithmetic runs in the library's CUDA kernels;
+there is no CPU or PyTorch fallback, and importing this package fails if
+libmoe.so has not been built (``python -m mixture_experts_expert_softmax_b200.build``).
+
+    ids, w = moe_route(logits, k=8, renorm=True)          # [T,k] int32, fp32
+    out = moe_forward(hidden, w1, w2, w, ids)              # [T,H] fp32
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED = -2
+MOE_ERR_CUDA = -3
+MOE_ERR_TIMEOUT = -4
+MOE_ERR_NO_DEVICE = -5
+MOE_ERR_OOM = -6
+MOE_STATUS_TIMEOUT = 0x1
+MOE_STATUS_BAD_ID = 0x2
+
+# every symbol declared in include/moe.h
+EXPORTED = (
+    "moe_route", "moe_forward", "moe_permute", "moe_error_string",
+    "moe_get_device_status", "moe_set_small_t_max", "moe_set_sync_each_stage",
+    "moe_set_wait_limit_ns", "moe_last_failed_stage", "moe_debug_wait_timeout",
+    "moe_profile_enable", "moe_profile_reset", "moe_profile_read",
+)
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {error_string(code)} (code {code})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m mixture_experts_expert_softmax_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    sig = {
+        "moe_route": ([P, I64, I32, I32, I32, P, P, P], I32),
+        "moe_forward": ([P, P, P, P, P, P, I64, I32, I32, I32, I32, P], I32),
+        "moe_permute": ([P, I64, I32, I32, P, P, P], I32),
+        "moe_error_string": ([I32], ctypes.c_char_p),
+        "moe_get_device_status": ([P, ctypes.POINTER(ctypes.c_uint32)], I32),
+        "moe_set_small_t_max": ([I32], I32),
+        "moe_set_sync_each_stage": ([I32], I32),
+        "moe_set_wait_limit_ns": ([I64], I64),
+        "moe_last_failed_stage": ([], ctypes.c_char_p),
+        "moe_debug_wait_timeout": ([I64, P], I32),
+        "moe_profile_enable": ([I32], I32),
+        "moe_profile_reset": ([], I32),
+        "moe_profile_read": ([I32, P, P, P], I32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def error_string(code: int) -> str:
+    return _lib.moe_error_string(int(code)).decode()
+
+
+def _check(code: int, where: str) -> None:
+    if code != MOE_OK:
+        raise MoEError(code, where)
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        if not torch.cuda.is_available():
+            return None  # legacy default stream; the library reports the missing device
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def moe_route(logits: torch.Tensor, k: int, renorm: bool = True,
+              topk_ids: torch.Tensor | None = None,
+              topk_weights: torch.Tensor | None = None, stream=None):
+    """Softmax over [T, E] fp32 logits, top-k (lowest index on ties),
+    optional renormalisation.  Returns (topk_ids int32 [T,k], topk_weights fp32 [T,k])."""
+    _need(logits, "logits", torch.float32)
+    T, E = logits.shape
+    if topk_ids is None:
+        topk_ids = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    if topk_weights is None:
+        topk_weights = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    _need(topk_ids, "topk_ids", torch.int32, (T, k))
+    _need(topk_weights, "topk_weights", torch.float32, (T, k))
+    _check(_lib.moe_route(logits.data_ptr(), T, E, int(k), int(bool(renorm)),
+                          topk_ids.data_ptr(), topk_weights.data_ptr(), _stream(stream)),
+           "moe_route")
+    return topk_ids, topk_weights
+
+
+def moe_forward(hidden: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
+                topk_weights: torch.Tensor, topk_ids: torch.Tensor,
+                out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Fused MoE forward: hidden [T,H] bf16, w1 [E,2I,H] bf16, w2 [E,H,I] bf16,
+    topk_weights [T,k] fp32, topk_ids [T,k] int32 -> out [T,H] fp32."""
+    _need(hidden, "hidden", torch.bfloat16)
+    T, H = hidden.shape
+    _need(w1, "w1", torch.bfloat16)
+    E, twoI, _ = w1.shape
+    I = twoI // 2
+    _need(w1, "w1", torch.bfloat16, (E, 2 * I, H))
+    _need(w2, "w2", torch.bfloat16, (E, H, I))
+    k = topk_ids.shape[1] if topk_ids.dim() == 2 else 0
+    _need(topk_ids, "topk_ids", torch.int32, (T, k))
+    _need(topk_weights, "topk_weights", torch.float32, (T, k))
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.float32, device=hidden.device)
+    _need(out, "out", torch.float32, (T, H))
+    _check(_lib.moe_forward(hidden.data_ptr(), w1.data_ptr(), w2.data_ptr(),
+                            topk_weights.data_ptr(), topk_ids.data_ptr(), out.data_ptr(),
+                            T, H, I, E, k, _stream(stream)), "moe_forward")
+    return out
+
+
+def moe_permute(topk_ids: torch.Tensor, E: int, sorted_rows: torch.Tensor | None = None,
+                expert_offsets: torch.Tensor | None = None, stream=None):
+    """Stable grouping of the flat (token, slot) indices by expert.
+    Returns (sorted_rows int32 [T*k], expert_offsets int32 [E+1])."""
+    _need(topk_ids, "topk_ids", torch.int32)
+    T, k = topk_ids.shape
+    if sorted_rows is None:
+        sorted_rows = torch.full((T * k,), -1, dtype=torch.int32, device=topk_ids.device)
+    if expert_offsets is None:
+        expert_offsets = torch.empty((E + 1,), dtype=torch.int32, device=topk_ids.device)
+    _need(sorted_rows, "sorted_rows", torch.int32, (T * k,))
+    _need(expert_offsets, "expert_offsets", torch.int32, (E + 1,))
+    _check(_lib.moe_permute(topk_ids.data_ptr(), T, k, int(E), sorted_rows.data_ptr(),
+                            expert_offsets.data_ptr(), _stream(stream)), "moe_permute")
+    return sorted_rows, expert_offsets
+
+
+def get_device_status(stream=None) -> int:
+    """Synchronise, return and clear the OR of MOE_STATUS_* bits."""
+    v = ctypes.c_uint32(0)
+    _check(_lib.moe_get_device_status(_stream(stream), ctypes.byref(v)), "moe_get_device_status")
+    return int(v.value)
+
+
+def set_small_t_max(n: int) -> int:
+    return int(_lib.moe_set_small_t_max(int(n)))
+
+
+def set_sync_each_stage(on: bool) -> int:
+    return int(_lib.moe_set_sync_each_stage(int(bool(on))))
+
+
+def set_wait_limit_ns(ns: int) -> int:
+    return int(_lib.moe_set_wait_limit_ns(int(ns)))
+
+
+def last_failed_stage() -> str:
+    return _lib.moe_last_failed_stage().decode()
+
+
+def debug_wait_timeout(limit_ns: int, stream=None) -> int:
+    """Run the never-signalled bounded wait; returns the raw MOE_* code."""
+    return int(_lib.moe_debug_wait_timeout(int(limit_ns), _stream(stream)))
+
+
+def profile_enable(on: bool) -> bool:
+    return bool(_lib.moe_profile_enable(int(bool(on))))
+
+
+def profile_reset() -> None:
+    _lib.moe_profile_reset()
+
+
+def profile_read() -> dict[str, tuple[int, float]]:
+    """Synchronise and return {kernel name: (launches, total ms)}."""
+    n = _lib.moe_profile_read(0, None, None, None)
+    if n <= 0:
+        return {}
+    names = (ctypes.c_char * 64 * n)()
+    launches = (ctypes.c_int64 * n)()
+    ms = (ctypes.c_double * n)()
+    n = _lib.moe_profile_read(n, names, launches, ms)
+    return {bytes(names[i]).split(b"\0", 1)[0].decode(): (int(launches[i]), float(ms[i]))
+            for i in range(n)}
+
+
+__all__ = [
+    "moe_route", "moe_forward", "moe_permute", "get_device_status", "set_small_t_max",
+    "set_sync_each_stage", "set_wait_limit_ns", "last_failed_stage", "debug_wait_timeout",
+    "profile_enable", "profile_reset", "profile_read", "error_string", "MoEError",
+    "LIB_PATH", "EXPORTED",
+]

@@ -1,0 +1,422 @@
+// moe_api.cu -- the extern "C" boundary of libmoe.so (declared in
+// include/moe.h): argument checks, the per-device workspace, dispatch
+// between the small-T GEMV path and the grouped-GEMM path, per-kernel
+// profiling events and the debug switches.
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "moe.h"
+#include "moe_internal.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 16;
+
+std::mutex g_mu;  // guards the per-device state and the profiler
+
+struct DeviceState {
+  bool checked = false;
+  bool usable = false;
+  int num_sms = 0;
+  uint32_t *status = nullptr;  // device status word (never reallocated)
+  void *ws = nullptr;          // grow-only workspace
+  size_t ws_bytes = 0;
+};
+DeviceState g_dev[kMaxDevices];
+
+int g_small_t_max = -1;  // -1: not read from the environment yet
+int g_sync_each = -1;
+int64_t g_wait_limit_ns = 2000000000LL;
+thread_local const char *g_failed_stage = "";
+
+// ---- profiler
+struct ProfEvent {
+  const char *name;
+  cudaEvent_t a, b;
+};
+bool g_prof = false;
+std::vector<ProfEvent> g_prof_pending;
+std::vector<std::string> g_prof_names;
+std::vector<int64_t> g_prof_count;
+std::vector<double> g_prof_ms;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t get_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+int small_t_max() {
+  if (g_small_t_max < 0) {
+    const char *v = std::getenv("MOE_SMALL_T_MAX");
+    g_small_t_max = v ? std::max(0, std::atoi(v)) : 16;
+    if (g_small_t_max > 16) g_small_t_max = 16;
+  }
+  return g_small_t_max;
+}
+
+bool sync_each() {
+  if (g_sync_each < 0) {
+    const char *v = std::getenv("MOE_SYNC_EACH_STAGE");
+    g_sync_each = (v && std::atoi(v) != 0) ? 1 : 0;
+  }
+  return g_sync_each != 0;
+}
+
+struct CallCtx {
+  cudaStream_t stream;
+  const char *cur;
+  cudaEvent_t ev0;
+};
+
+void hook_begin(void *c, const char *name) {
+  CallCtx *ctx = static_cast<CallCtx *>(c);
+  ctx->cur = name;
+  ctx->ev0 = nullptr;
+  if (g_prof) {
+    ctx->ev0 = get_event();
+    cudaEventRecord(ctx->ev0, ctx->stream);
+  }
+}
+
+cudaError_t hook_end(void *c, cudaError_t err) {
+  CallCtx *ctx = static_cast<CallCtx *>(c);
+  if (err == cudaSuccess && g_prof && ctx->ev0 != nullptr) {
+    cudaEvent_t ev1 = get_event();
+    cudaEventRecord(ev1, ctx->stream);
+    g_prof_pending.push_back({ctx->cur, ctx->ev0, ev1});
+  }
+  if (err == cudaSuccess && sync_each()) {
+    err = cudaStreamSynchronize(ctx->stream);
+    if (err == cudaSuccess) err = cudaGetLastError();
+  }
+  if (err != cudaSuccess) g_failed_stage = ctx->cur;
+  return err;
+}
+
+moe::StageHook make_hook(CallCtx *ctx) {
+  moe::StageHook h;
+  h.ctx = ctx;
+  h.on_begin = hook_begin;
+  h.on_end = hook_end;
+  // event records between launches would break programmatic serialisation
+  h.pdl = !g_prof && !sync_each();
+  return h;
+}
+
+// Current device, checked once for sm_100 and given its status word.
+int current_device(DeviceState **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return MOE_ERR_NO_DEVICE;
+  }
+  DeviceState &d = g_dev[dev];
+  if (!d.checked) {
+    d.checked = true;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_NO_DEVICE;
+    }
+    if (prop.major != 10 || prop.minor != 0) return MOE_ERR_NO_DEVICE;
+    d.num_sms = prop.multiProcessorCount;
+    if (cudaMalloc(&d.status, 256) != cudaSuccess || cudaMemset(d.status, 0, 256) != cudaSuccess ||
+        moe::grouped_gemm_setup(dev) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    d.usable = true;
+  }
+  if (!d.usable) return MOE_ERR_NO_DEVICE;
+  *out = &d;
+  return MOE_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Make the workspace at least `bytes` large.
+int ensure_workspace(DeviceState &d, size_t bytes) {
+  if (bytes <= d.ws_bytes) return MOE_OK;
+  if (d.ws != nullptr) {
+    cudaFree(d.ws);  // synchronises the device
+    d.ws = nullptr;
+    d.ws_bytes = 0;
+  }
+  const size_t want = align256(bytes);
+  if (cudaMalloc(&d.ws, want) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_OOM;
+  }
+  d.ws_bytes = want;
+  return MOE_OK;
+}
+
+struct Carver {
+  char *base;
+  size_t off = 0;
+  template <typename T>
+  T *take(size_t count) {
+    T *p = reinterpret_cast<T *>(base + off);
+    off = align256(off + count * sizeof(T));
+    return p;
+  }
+};
+
+size_t permute_ws_bytes(int64_t n, int E) {
+  const size_t chunks = static_cast<size_t>(moe::permute_num_chunks(n));
+  return align256(std::max<size_t>(chunks, 1) * E * sizeof(int32_t)) +
+         2 * align256((E + 1) * sizeof(int32_t)) + align256(std::max<int64_t>(n, 1) * 4);
+}
+
+int to_code(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  cudaGetLastError();
+  return MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_error_string(int code) {
+  switch (code) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size or k outside [1, E])";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape (needs H % 128 == 0, I % 128 == 0, E <= 1024, k <= 16)";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "a bounded device-side wait expired";
+    case MOE_ERR_NO_DEVICE: return "no usable sm_100 device is current";
+    case MOE_ERR_OOM: return "workspace allocation failed";
+    default: return "unknown error code";
+  }
+}
+
+int moe_route(const float *logits, int64_t T, int E, int k, int renorm, int32_t *topk_ids,
+              float *topk_weights, void *stream) {
+  if (T < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (logits == nullptr || topk_ids == nullptr || topk_weights == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (T / 8 >= (static_cast<int64_t>(1) << 31) - 1) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState *d = nullptr;
+  int rc = current_device(&d);
+  if (rc != MOE_OK) return rc;
+  CallCtx ctx{static_cast<cudaStream_t>(stream), "", nullptr};
+  moe::StageHook hook = make_hook(&ctx);
+  hook.begin("route");
+  cudaError_t e = moe::launch_route(logits, T, E, k, renorm, topk_ids, topk_weights, ctx.stream);
+  return to_code(hook.end(e));
+}
+
+int moe_permute(const int32_t *topk_ids, int64_t T, int k, int E, int32_t *sorted_rows,
+                int32_t *expert_offsets, void *stream) {
+  if (T < 0 || k < 1 || E < 1) return MOE_ERR_INVALID_ARG;
+  if (expert_offsets == nullptr || (T > 0 && (topk_ids == nullptr || sorted_rows == nullptr)))
+    return MOE_ERR_INVALID_ARG;
+  if (E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+  const int64_t n = T * k;
+  if (n >= (static_cast<int64_t>(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState *d = nullptr;
+  int rc = current_device(&d);
+  if (rc != MOE_OK) return rc;
+  if ((rc = ensure_workspace(*d, permute_ws_bytes(n, E))) != MOE_OK) return rc;
+  Carver cv{static_cast<char *>(d->ws)};
+  int32_t *chunk_counts = cv.take<int32_t>(std::max(moe::permute_num_chunks(n), 1) * static_cast<size_t>(E));
+  int32_t *tile_offsets = cv.take<int32_t>(E + 1);
+  CallCtx ctx{static_cast<cudaStream_t>(stream), "", nullptr};
+  moe::StageHook hook = make_hook(&ctx);
+  cudaError_t e = moe::launch_permute(topk_ids, n, E, moe::kGemmTileM, chunk_counts,
+                                      expert_offsets, tile_offsets, sorted_rows, ctx.stream, hook);
+  return to_code(e);
+}
+
+int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
+                const float *topk_weights, const int32_t *topk_ids, float *out, int64_t T, int H,
+                int I, int E, int k, void *stream) {
+  if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (hidden == nullptr || w1 == nullptr || w2 == nullptr || topk_weights == nullptr ||
+                topk_ids == nullptr || out == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (H % 128 != 0 || I % 128 != 0 || E > kMaxExperts || k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+  const int64_t n = T * k;
+  if (n >= (static_cast<int64_t>(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState *d = nullptr;
+  int rc = current_device(&d);
+  if (rc != MOE_OK) return rc;
+  CallCtx ctx{static_cast<cudaStream_t>(stream), "", nullptr};
+  moe::StageHook hook = make_hook(&ctx);
+
+  if (T <= small_t_max()) {
+    const size_t need = align256(static_cast<size_t>(n) * I * sizeof(float));
+    if ((rc = ensure_workspace(*d, need)) != MOE_OK) return rc;
+    Carver cv{static_cast<char *>(d->ws)};
+    float *act = cv.take<float>(static_cast<size_t>(n) * I);
+    return to_code(moe::launch_small_t(hidden, w1, w2, topk_weights, topk_ids, act, out, T, H, I,
+                                       E, k, d->status, ctx.stream, hook));
+  }
+
+  const size_t need = permute_ws_bytes(n, E) + align256((E + 1) * sizeof(int32_t)) +
+                      align256(static_cast<size_t>(n) * I * 2) +
+                      align256(static_cast<size_t>(n) * H * sizeof(float));
+  if ((rc = ensure_workspace(*d, need)) != MOE_OK) return rc;
+  Carver cv{static_cast<char *>(d->ws)};
+  int32_t *chunk_counts =
+      cv.take<int32_t>(std::max(moe::permute_num_chunks(n), 1) * static_cast<size_t>(E));
+  int32_t *tile_offsets = cv.take<int32_t>(E + 1);
+  int32_t *sorted_rows = cv.take<int32_t>(std::max<int64_t>(n, 1));
+  int32_t *expert_offsets = cv.take<int32_t>(E + 1);
+  uint16_t *act = cv.take<uint16_t>(static_cast<size_t>(n) * I);
+  float *P = cv.take<float>(static_cast<size_t>(n) * H);
+
+  cudaError_t e = moe::launch_permute(topk_ids, n, E, moe::kGemmTileM, chunk_counts,
+                                      expert_offsets, tile_offsets, sorted_rows, ctx.stream, hook);
+  if (e != cudaSuccess) return to_code(e);
+  moe::GroupedGemmArgs ga;
+  ga.hidden = hidden;
+  ga.w1 = w1;
+  ga.w2 = w2;
+  ga.sorted_rows = sorted_rows;
+  ga.expert_offsets = expert_offsets;
+  ga.tile_offsets = tile_offsets;
+  ga.act = act;
+  ga.P = P;
+  ga.T = T;
+  ga.H = H;
+  ga.I = I;
+  ga.E = E;
+  ga.k = k;
+  ga.num_sms = d->num_sms;
+  ga.status = d->status;
+  ga.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns);
+  if ((e = moe::launch_gemm1_swiglu(ga, ctx.stream, hook)) != cudaSuccess) return to_code(e);
+  if ((e = moe::launch_gemm2(ga, ctx.stream, hook)) != cudaSuccess) return to_code(e);
+  e = moe::launch_combine(P, topk_weights, topk_ids, out, T, H, E, k, d->status, ctx.stream, hook);
+  return to_code(e);
+}
+
+int moe_get_device_status(void *stream, uint32_t *status) {
+  if (status == nullptr) return MOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState *d = nullptr;
+  int rc = current_device(&d);
+  if (rc != MOE_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(&v, d->status, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(d->status, 0, sizeof(v));
+  if (e != cudaSuccess) return to_code(e);
+  *status = v;
+  return MOE_OK;
+}
+
+int moe_set_small_t_max(int n) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  const int prev = small_t_max();
+  g_small_t_max = std::min(16, std::max(0, n));
+  return prev;
+}
+
+int moe_set_sync_each_stage(int on) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  const int prev = sync_each() ? 1 : 0;
+  g_sync_each = on ? 1 : 0;
+  return prev;
+}
+
+int64_t moe_set_wait_limit_ns(int64_t ns) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  const int64_t prev = g_wait_limit_ns;
+  g_wait_limit_ns = ns > 0 ? ns : 2000000000LL;
+  return prev;
+}
+
+const char *moe_last_failed_stage(void) { return g_failed_stage; }
+
+int moe_debug_wait_timeout(int64_t limit_ns, void *stream) {
+  if (limit_ns <= 0 || limit_ns > 10000000000LL) return MOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState *d = nullptr;
+  int rc = current_device(&d);
+  if (rc != MOE_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = moe::launch_wait_probe(d->status, static_cast<uint64_t>(limit_ns), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  uint32_t v = 0;
+  if (e == cudaSuccess) e = cudaMemcpy(&v, d->status, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return to_code(e);
+  return (v & MOE_STATUS_TIMEOUT) ? MOE_ERR_TIMEOUT : MOE_OK;
+}
+
+int moe_profile_enable(int on) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  const int prev = g_prof ? 1 : 0;
+  g_prof = on != 0;
+  return prev;
+}
+
+static void profile_collect() {
+  if (g_prof_pending.empty()) return;
+  cudaDeviceSynchronize();
+  for (const ProfEvent &pe : g_prof_pending) {
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, pe.a, pe.b);
+    size_t i = 0;
+    while (i < g_prof_names.size() && g_prof_names[i] != pe.name) ++i;
+    if (i == g_prof_names.size()) {
+      g_prof_names.emplace_back(pe.name);
+      g_prof_count.push_back(0);
+      g_prof_ms.push_back(0.0);
+    }
+    g_prof_count[i] += 1;
+    g_prof_ms[i] += ms;
+    g_event_pool.push_back(pe.a);
+    g_event_pool.push_back(pe.b);
+  }
+  g_prof_pending.clear();
+  cudaGetLastError();
+}
+
+int moe_profile_reset(void) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  profile_collect();
+  g_prof_names.clear();
+  g_prof_count.clear();
+  g_prof_ms.clear();
+  return MOE_OK;
+}
+
+int moe_profile_read(int max_names, char (*names)[64], int64_t *launches, double *total_ms) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  profile_collect();
+  const int n = static_cast<int>(g_prof_names.size());
+  for (int i = 0; i < n && i < max_names; ++i) {
+    if (names != nullptr) {
+      std::strncpy(names[i], g_prof_names[i].c_str(), 63);
+      names[i][63] = '\0';
+    }
+    if (launches != nullptr) launches[i] = g_prof_count[i];
+    if (total_ms != nullptr) total_ms[i] = g_prof_ms[i];
+  }
+  return n;
+}
+
+}  // extern "C"

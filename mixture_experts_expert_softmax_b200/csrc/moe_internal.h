@@ -1,0 +1,84 @@
+// moe_internal.h -- launchers of the kernels of libmoe.so (host side), used
+// by moe_api.cu.  Not part of the public ABI.
+#pragma once
+
+#include <utility>
+
+#include "common.cuh"
+
+namespace moe {
+
+// Hooks called around every kernel launch: profiling events, the
+// synchronise-after-each-stage debug mode, and whether launches may use
+// programmatic dependent launch (PDL).
+struct StageHook {
+  bool pdl = false;
+  void *ctx = nullptr;
+  void (*on_begin)(void *, const char *) = nullptr;
+  cudaError_t (*on_end)(void *, cudaError_t) = nullptr;
+  void begin(const char *name) const {
+    if (on_begin) on_begin(ctx, name);
+  }
+  cudaError_t end(cudaError_t e) const { return on_end ? on_end(ctx, e) : e; }
+};
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, bool pdl, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// route.cu
+cudaError_t launch_route(const float *logits, int64_t T, int E, int k, int renorm, int32_t *ids,
+                         float *weights, cudaStream_t s);
+
+// permute.cu
+int permute_num_chunks(int64_t n);
+cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int tile_m,
+                           int32_t *chunk_counts, int32_t *expert_offsets, int32_t *tile_offsets,
+                           int32_t *sorted_rows, cudaStream_t s, const StageHook &hook);
+
+// grouped_gemm.cu
+constexpr int kGemmTileM = 128;
+struct GroupedGemmArgs {
+  const uint16_t *hidden;  // [T, H] bf16
+  const uint16_t *w1;      // [E, 2I, H] bf16
+  const uint16_t *w2;      // [E, H, I] bf16
+  const int32_t *sorted_rows;
+  const int32_t *expert_offsets;
+  const int32_t *tile_offsets;
+  uint16_t *act;  // [T*k, I] bf16, expert-sorted rows
+  float *P;       // [T*k, H] fp32, flat (t*k + j) rows
+  int64_t T;
+  int H, I, E, k;
+  int num_sms;
+  uint32_t *status;
+  uint64_t wait_limit_ns;
+};
+cudaError_t grouped_gemm_setup(int device);
+cudaError_t launch_gemm1_swiglu(const GroupedGemmArgs &a, cudaStream_t s, const StageHook &hook);
+cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s, const StageHook &hook);
+cudaError_t launch_wait_probe(uint32_t *status, uint64_t limit_ns, cudaStream_t s);
+
+// combine.cu
+cudaError_t launch_combine(const float *P, const float *topk_weights, const int32_t *topk_ids,
+                           float *out, int64_t T, int H, int E, int k, uint32_t *status,
+                           cudaStream_t s, const StageHook &hook);
+
+// small_t.cu
+cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
+                           const float *topk_weights, const int32_t *topk_ids, float *act,
+                           float *out, int64_t T, int H, int I, int E, int k, uint32_t *status,
+                           cudaStream_t s, const StageHook &hook);
+
+}  // namespace moe

@@ -1,0 +1,197 @@
+// permute.cu -- grouping of the flat (token, slot) indices i = t*k + j by
+// expert: histogram -> exclusive scan -> stable scatter.  Integer only; the
+// result is unique (ascending i inside each expert), which is the (token, k)
+// order in which the TPU kernel of "tpu_inference/kernels/fused_moe/v1/
+// kernel.py" hands rows to each expert and the ascending token order of
+// nonzero() in atrex-bench #009 Model.forward.
+//
+// The flat index range is cut into chunks of kChunk entries; each chunk is
+// split between kPermWarps warps, kChunk / kPermWarps consecutive entries
+// each.  Stability comes from (chunk, warp, lane) order: a chunk's base for
+// expert e counts the entries of e in all earlier chunks, a warp's base adds
+// the earlier warps of its chunk, and inside a warp step lanes are ranked
+// with __match_any_sync.
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kPermWarps = 8;
+constexpr int kPermThreads = kPermWarps * 32;
+constexpr int kChunk = 2048;
+constexpr int kPerWarp = kChunk / kPermWarps;
+
+// counts[c * E + e] = number of entries of expert e in chunk c.
+__global__ void __launch_bounds__(kPermThreads)
+    permute_count_kernel(const int32_t *__restrict__ ids, int64_t n, int E,
+                         int32_t *__restrict__ chunk_counts) {
+  extern __shared__ int32_t hist[];
+  grid_dep_wait();
+  grid_dep_launch();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kChunk;
+  for (int r = threadIdx.x; r < kChunk; r += blockDim.x) {
+    const int64_t i = c0 + r;
+    if (i < n) {
+      const int e = __ldg(ids + i);
+      if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+    }
+  }
+  __syncthreads();
+  int32_t *dst = chunk_counts + static_cast<int64_t>(blockIdx.x) * E;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) dst[e] = hist[e];
+}
+
+// One CTA of 1024 threads.  Turns chunk_counts into per-chunk exclusive
+// bases (in place), writes expert_offsets[E+1] (exclusive scan of the
+// totals) and tile_offsets[E+1] (exclusive scan of ceil(count / tile_m),
+// the m-tiles of each expert in the grouped GEMMs).
+__global__ void __launch_bounds__(1024)
+    permute_scan_kernel(int32_t *__restrict__ chunk_counts, int n_chunks, int E, int tile_m,
+                        int32_t *__restrict__ expert_offsets,
+                        int32_t *__restrict__ tile_offsets) {
+  __shared__ int32_t s_warp_cnt[32];
+  __shared__ int32_t s_warp_tiles[32];
+  grid_dep_wait();
+  grid_dep_launch();
+  const int e = threadIdx.x;
+  int32_t total = 0;
+  if (e < E) {
+    for (int c = 0; c < n_chunks; ++c) {
+      int32_t *p = chunk_counts + static_cast<int64_t>(c) * E + e;
+      const int32_t x = *p;
+      *p = total;
+      total += x;
+    }
+  }
+  const int32_t tiles = (total + tile_m - 1) / tile_m;
+  // block-wide inclusive scans of (total, tiles)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t a = total, b = tiles;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t xa = __shfl_up_sync(0xffffffffu, a, o);
+    const int32_t xb = __shfl_up_sync(0xffffffffu, b, o);
+    if (lane >= o) {
+      a += xa;
+      b += xb;
+    }
+  }
+  if (lane == 31) {
+    s_warp_cnt[warp] = a;
+    s_warp_tiles[warp] = b;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int32_t wa = s_warp_cnt[lane], wb = s_warp_tiles[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t xa = __shfl_up_sync(0xffffffffu, wa, o);
+      const int32_t xb = __shfl_up_sync(0xffffffffu, wb, o);
+      if (lane >= o) {
+        wa += xa;
+        wb += xb;
+      }
+    }
+    s_warp_cnt[lane] = wa;
+    s_warp_tiles[lane] = wb;
+  }
+  __syncthreads();
+  const int32_t incl_a = a + (warp > 0 ? s_warp_cnt[warp - 1] : 0);
+  const int32_t incl_b = b + (warp > 0 ? s_warp_tiles[warp - 1] : 0);
+  if (e < E) {
+    expert_offsets[e] = incl_a - total;
+    tile_offsets[e] = incl_b - tiles;
+  }
+  if (e == E - 1) {
+    expert_offsets[E] = incl_a;
+    tile_offsets[E] = incl_b;
+  }
+}
+
+// Writes sorted_rows[pos] = i for every valid entry.  Shared memory holds
+// one running base per (warp, expert).
+__global__ void __launch_bounds__(kPermThreads)
+    permute_scatter_kernel(const int32_t *__restrict__ ids, int64_t n, int E,
+                           const int32_t *__restrict__ chunk_bases,
+                           const int32_t *__restrict__ expert_offsets,
+                           int32_t *__restrict__ sorted_rows) {
+  extern __shared__ int32_t wbase[];  // [kPermWarps][E]
+  grid_dep_wait();
+  grid_dep_launch();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int x = threadIdx.x; x < kPermWarps * E; x += blockDim.x) wbase[x] = 0;
+  __syncthreads();
+  const int64_t w0 = static_cast<int64_t>(blockIdx.x) * kChunk + warp * kPerWarp;
+  int32_t *mine = wbase + warp * E;
+  for (int r = lane; r < kPerWarp; r += 32) {
+    const int64_t i = w0 + r;
+    if (i < n) {
+      const int e = __ldg(ids + i);
+      if (e >= 0 && e < E) atomicAdd(&mine[e], 1);
+    }
+  }
+  __syncthreads();
+  const int32_t *cb = chunk_bases + static_cast<int64_t>(blockIdx.x) * E;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int32_t run = expert_offsets[e] + cb[e];
+    for (int w = 0; w < kPermWarps; ++w) {
+      const int32_t x = wbase[w * E + e];
+      wbase[w * E + e] = run;
+      run += x;
+    }
+  }
+  __syncthreads();
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int r0 = 0; r0 < kPerWarp; r0 += 32) {
+    const int64_t i = w0 + r0 + lane;
+    int e = -1;
+    if (i < n) {
+      e = __ldg(ids + i);
+      if (e < 0 || e >= E) e = -1;
+    }
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0) {
+      const int32_t pos = mine[e] + __popc(peers & lt_mask);
+      sorted_rows[pos] = static_cast<int32_t>(i);
+    }
+    __syncwarp();
+    if (e >= 0 && (peers & lt_mask) == 0) mine[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+int permute_num_chunks(int64_t n) { return static_cast<int>((n + kChunk - 1) / kChunk); }
+
+cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int tile_m,
+                           int32_t *chunk_counts, int32_t *expert_offsets, int32_t *tile_offsets,
+                           int32_t *sorted_rows, cudaStream_t s, const StageHook &hook) {
+  const int n_chunks = permute_num_chunks(n);
+  cudaError_t err;
+  if (n_chunks > 0) {
+    hook.begin("permute_count");
+    // first kernel of the call: ordinary stream order after earlier work
+    err = launch_pdl(permute_count_kernel, dim3(n_chunks), dim3(kPermThreads),
+                     static_cast<size_t>(E) * sizeof(int32_t), s, false, ids, n, E,
+                     chunk_counts);
+    if ((err = hook.end(err)) != cudaSuccess) return err;
+  }
+  hook.begin("permute_scan");
+  err = launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, s, hook.pdl, chunk_counts,
+                   n_chunks, E, tile_m, expert_offsets, tile_offsets);
+  if ((err = hook.end(err)) != cudaSuccess) return err;
+  if (n_chunks > 0) {
+    hook.begin("permute_scatter");
+    err = launch_pdl(permute_scatter_kernel, dim3(n_chunks), dim3(kPermThreads),
+                     static_cast<size_t>(kPermWarps) * E * sizeof(int32_t), s, hook.pdl, ids, n,
+                     E, static_cast<const int32_t *>(chunk_counts),
+                     static_cast<const int32_t *>(expert_offsets), sorted_rows);
+    if ((err = hook.end(err)) != cudaSuccess) return err;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace moe

@@ -8,8 +8,11 @@ w1 ``randn * H**-0.5`` and w2 ``randn * I**-0.5`` in bf16, and fp32 ``randn``
 router logits.  Routing (softmax / top-k / renormalisation) is NOT done here;
 each side computes it from the logits with its own code.
 
-The draws use torch's CPU generator so that the CPU oracle and the GPU path
-see bit-identical inputs; callers move tensors to the GPU themselves.
+The draws come from one seeded torch generator on the requested device (CPU
+by default).  Both sides always see the same tensors: GPU draws are copied to
+the host for the oracle, CPU draws are copied to the GPU for the kernels.
+Large shapes draw on the GPU because the CPU generator needs tens of seconds
+for the biggest weight sets.
 """
 from __future__ import annotations
 
@@ -53,17 +56,18 @@ SHAPES = {
 
 
 def make_inputs(T: int, H: int, I: int, E: int, seed: int = 0,
-                hidden_scale: float = 0.1):
+                hidden_scale: float = 0.1, device: str = "cpu"):
     """Draw (hidden [T,H] bf16, w1 [E,2I,H] bf16, w2 [E,H,I] bf16,
-    logits [T,E] fp32) on the CPU, in that order, from one seeded generator."""
-    g = torch.Generator(device="cpu")
+    logits [T,E] fp32) on `device`, in that order, from one seeded generator."""
+    g = torch.Generator(device=device)
     g.manual_seed(seed)
-    hidden = torch.randn(T, H, dtype=torch.bfloat16, generator=g) * hidden_scale
-    w1 = torch.randn(E, 2 * I, H, dtype=torch.bfloat16, generator=g) * (H ** -0.5)
-    w2 = torch.randn(E, H, I, dtype=torch.bfloat16, generator=g) * (I ** -0.5)
-    logits = torch.randn(T, E, dtype=torch.float32, generator=g)
+    kw = dict(generator=g, device=device)
+    hidden = torch.randn(T, H, dtype=torch.bfloat16, **kw) * hidden_scale
+    w1 = torch.randn(E, 2 * I, H, dtype=torch.bfloat16, **kw) * (H ** -0.5)
+    w2 = torch.randn(E, H, I, dtype=torch.bfloat16, **kw) * (I ** -0.5)
+    logits = torch.randn(T, E, dtype=torch.float32, **kw)
     return hidden, w1, w2, logits
 
 
-def make_shape_inputs(shape: MoEShape, seed: int = 0):
-    return make_inputs(shape.T, shape.H, shape.I, shape.E, seed=seed)
+def make_shape_inputs(shape: MoEShape, seed: int = 0, device: str = "cpu"):
+    return make_inputs(shape.T, shape.H, shape.I, shape.E, seed=seed, device=device)

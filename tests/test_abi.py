@@ -1,0 +1,105 @@
+"""The C-ABI library loads, exports every symbol include/moe.h declares, and
+rejects bad arguments before touching a GPU (runs on a CPU-only host)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixture_experts_expert_softmax_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_exports():
+    declared = header_functions()
+    assert "moe_route" in declared and "moe_forward" in declared
+    assert sorted(moe.EXPORTED) == declared
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(moe.LIB_PATH)
+    for name in header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_error_strings():
+    for code in range(0, -7, -1):
+        s = moe.error_string(code)
+        assert s and "unknown" not in s
+    assert "unknown" in moe.error_string(-99)
+
+
+L = moe._lib
+NULL = None
+
+
+@pytest.mark.parametrize("args,code", [
+    ((NULL, 4, 8, 2, 1, NULL, NULL, NULL), moe.MOE_ERR_INVALID_ARG),   # null pointers
+    ((1, -1, 8, 2, 1, 1, 1, NULL), moe.MOE_ERR_INVALID_ARG),          # T < 0
+    ((1, 4, 8, 9, 1, 1, 1, NULL), moe.MOE_ERR_INVALID_ARG),           # k > E
+    ((1, 4, 8, 0, 1, 1, 1, NULL), moe.MOE_ERR_INVALID_ARG),           # k < 1
+    ((1, 4, 0, 1, 1, 1, 1, NULL), moe.MOE_ERR_INVALID_ARG),           # E < 1
+    ((1, 4, 2048, 2, 1, 1, 1, NULL), moe.MOE_ERR_UNSUPPORTED),        # E > 1024
+    ((NULL, 0, 8, 2, 1, NULL, NULL, NULL), moe.MOE_OK),               # T == 0: nothing to do
+])
+def test_route_argument_checks(args, code):
+    assert L.moe_route(*args) == code
+
+
+FWD_OK = dict(h=1, w1=1, w2=1, w=1, ids=1, out=1, T=4, H=256, I=128, E=8, k=2)
+
+
+def fwd(**kw):
+    a = dict(FWD_OK, **kw)
+    return L.moe_forward(a["h"], a["w1"], a["w2"], a["w"], a["ids"], a["out"], a["T"], a["H"],
+                         a["I"], a["E"], a["k"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(h=NULL), moe.MOE_ERR_INVALID_ARG),
+    (dict(out=NULL), moe.MOE_ERR_INVALID_ARG),
+    (dict(T=-1), moe.MOE_ERR_INVALID_ARG),
+    (dict(k=9), moe.MOE_ERR_INVALID_ARG),
+    (dict(k=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(H=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(H=200), moe.MOE_ERR_UNSUPPORTED),       # H % 128
+    (dict(I=96), moe.MOE_ERR_UNSUPPORTED),        # I % 128
+    (dict(E=2000, k=2), moe.MOE_ERR_UNSUPPORTED),  # E > 1024
+    (dict(E=64, k=17), moe.MOE_ERR_UNSUPPORTED),   # k > 16
+    (dict(T=0, h=NULL, out=NULL), moe.MOE_OK),    # empty batch
+])
+def test_forward_argument_checks(kw, code):
+    assert fwd(**kw) == code
+
+
+def test_permute_argument_checks():
+    assert L.moe_permute(NULL, 4, 2, 8, NULL, NULL, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_permute(1, 4, 0, 8, 1, 1, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_permute(1, 4, 2, 4096, 1, 1, None) == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_debug_switches_roundtrip():
+    prev = moe.set_small_t_max(5)
+    assert moe.set_small_t_max(prev) == 5
+    prev = moe.set_sync_each_stage(True)
+    assert moe.set_sync_each_stage(prev) == 1
+    prev = moe.set_wait_limit_ns(12345)
+    assert moe.set_wait_limit_ns(prev) == 12345
+    assert moe.debug_wait_timeout(0) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_no_gpu_fails_loudly():
+    """Without a usable sm_100 device the library reports it; it never falls back."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert L.moe_route(1, 4, 8, 2, 1, 1, 1, None) == moe.MOE_ERR_NO_DEVICE
+    assert fwd() == moe.MOE_ERR_NO_DEVICE

@@ -1,0 +1,300 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Gates: routing ids, permutation indices and expert offsets bit-exact;
+routing weights within 1e-6 + 1e-5*|w|; forward output within
+1e-2 + 1e-2*|ref| elementwise plus the diagnostic gates of moe_testutil.
+Shapes span several 128-row tiles with ragged tails, empty experts, the
+small-T path and both GEMM paths; the five named workloads run at full size
+(all tokens for the tiny and decode workloads, sampled tokens that the
+oracle computes one by one for the three prefill workloads).
+"""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_expert_softmax_b200 as moe
+import oracle
+from moe_inputs import SHAPES, make_inputs, make_shape_inputs
+from moe_testutil import assert_output_close, assert_weights_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_device():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    torch.cuda.set_device(0)
+    moe.set_small_t_max(16)
+    yield
+    moe.set_small_t_max(16)
+
+
+def gpu_route(logits_cpu, k, renorm=True):
+    ids, w = moe.moe_route(logits_cpu.cuda(), k, renorm)
+    torch.cuda.synchronize()
+    return ids.cpu().numpy(), w.cpu().numpy()
+
+
+def gpu_forward(hidden, w1, w2, w, ids):
+    """Inputs may live on CPU or GPU; routing comes in as numpy."""
+    dev = torch.device("cuda")
+    out = moe.moe_forward(hidden.to(dev), w1.to(dev), w2.to(dev),
+                          torch.as_tensor(np.asarray(w, np.float32)).to(dev),
+                          torch.as_tensor(np.asarray(ids, np.int32)).to(dev))
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def check_status_clean():
+    assert moe.get_device_status() == 0
+
+
+# ------------------------------------------------------------------ routing
+@pytest.mark.parametrize("name", sorted(SHAPES))
+def test_route_workloads(name):
+    s = SHAPES[name]
+    logits = torch.randn(s.T, s.E, generator=torch.Generator().manual_seed(0))
+    for renorm in (True, False):
+        ids_r, w_r = oracle.route(logits.numpy(), s.k, renorm)
+        ids_g, w_g = gpu_route(logits, s.k, renorm)
+        assert np.array_equal(ids_g, ids_r)
+        assert_weights_close(w_g, w_r, name)
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 1, 1), (3, 2, 2), (257, 37, 5), (100, 100, 16),
+                                   (64, 256, 8), (33, 512, 3), (17, 1024, 16), (9, 8, 8)])
+def test_route_shapes(T, E, k):
+    g = torch.Generator().manual_seed(T * 1000 + E)
+    logits = torch.randn(T, E, generator=g)
+    ids_r, w_r = oracle.route(logits.numpy(), k, True)
+    ids_g, w_g = gpu_route(logits, k, True)
+    assert np.array_equal(ids_g, ids_r)
+    assert_weights_close(w_g, w_r)
+
+
+def test_route_ties_and_neg_inf():
+    g = torch.Generator().manual_seed(5)
+    logits = torch.randint(-2, 3, (300, 40), generator=g).float()
+    logits[::7, 3:30] = -float("inf")
+    logits[1, :] = 0.0
+    for k in (1, 4, 40):
+        ids_r, w_r = oracle.route(logits.numpy(), k, False)
+        ids_g, w_g = gpu_route(logits, k, False)
+        assert np.array_equal(ids_g, ids_r)
+        assert_weights_close(w_g, w_r)
+
+
+def test_route_empty():
+    ids, w = moe.moe_route(torch.empty(0, 8, device="cuda"), 2)
+    assert ids.shape == (0, 2)
+
+
+# ------------------------------------------------------------------ permutation
+@pytest.mark.parametrize("T,k,E", [(1, 1, 1), (5, 2, 3), (1024, 2, 8), (1025, 2, 8),
+                                   (4096, 8, 128), (3000, 7, 1024), (8192, 8, 128),
+                                   (15381, 2, 8), (100, 16, 1000)])
+def test_permute_bit_exact(T, k, E):
+    g = torch.Generator().manual_seed(T + 7 * E)
+    ids = torch.randint(-1, E + 1, (T, k), generator=g, dtype=torch.int32)
+    rows_r, offs_r = oracle.permute(ids.numpy(), E)
+    rows_g, offs_g = moe.moe_permute(ids.cuda(), E)
+    torch.cuda.synchronize()
+    offs_g = offs_g.cpu().numpy()
+    assert np.array_equal(offs_g, offs_r)
+    nv = int(offs_r[-1])
+    assert np.array_equal(rows_g.cpu().numpy()[:nv], rows_r[:nv])
+
+
+def test_permute_of_routed_workload():
+    s = SHAPES["prefill_thin"]
+    logits = torch.randn(s.T, s.E, generator=torch.Generator().manual_seed(0))
+    ids, _ = oracle.route(logits.numpy(), s.k, True)
+    rows_r, offs_r = oracle.permute(ids, s.E)
+    rows_g, offs_g = moe.moe_permute(torch.as_tensor(ids).cuda(), s.E)
+    assert np.array_equal(offs_g.cpu().numpy(), offs_r)
+    assert np.array_equal(rows_g.cpu().numpy(), rows_r)
+
+
+# ------------------------------------------------------------------ forward
+CASES = [
+    # (T, H, I, E, k)            what it covers
+    (64, 256, 128, 8, 2),      # the tiny workload
+    (300, 512, 256, 8, 2),     # several m-tiles per expert, ragged tails
+    (333, 384, 384, 16, 4),    # H = 3*128: GEMM2's last n-tile is half valid
+    (100, 256, 128, 128, 8),   # most experts hold < 1 tile, many empty
+    (17, 256, 256, 4, 4),      # k = E
+    (129, 128, 128, 1, 1),     # one expert, one slot
+    (257, 640, 512, 32, 6),    # odd k, E not a power of two multiple of tiles
+]
+
+
+@pytest.mark.parametrize("T,H,I,E,k", CASES)
+@pytest.mark.parametrize("path", ["auto", "gemm"])
+def test_forward_parity(T, H, I, E, k, path):
+    hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=T + H)
+    ids, w = oracle.route(logits.numpy(), k, True)
+    ref = oracle.moe_token_loop(hidden, w1, w2, w, ids)
+    prev = moe.set_small_t_max(0 if path == "gemm" else 16)
+    try:
+        out = gpu_forward(hidden, w1, w2, w, ids)
+    finally:
+        moe.set_small_t_max(prev)
+    assert_output_close(out, ref, f"T={T} H={H} I={I} E={E} k={k} {path}")
+    check_status_clean()
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 8, 16])
+@pytest.mark.parametrize("path", ["small_t", "gemm"])
+def test_forward_small_batches(T, path):
+    H, I, E, k = 2048, 768, 128, 8
+    hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=40 + T)
+    ids, w = oracle.route(logits.numpy(), k, True)
+    ref = oracle.moe_token_loop(hidden, w1, w2, w, ids)
+    prev = moe.set_small_t_max(16 if path == "small_t" else 0)
+    try:
+        out = gpu_forward(hidden, w1, w2, w, ids)
+    finally:
+        moe.set_small_t_max(prev)
+    assert_output_close(out, ref, f"T={T} {path}")
+    check_status_clean()
+
+
+def test_forward_small_t_shared_and_duplicate_experts():
+    """Several tokens on one expert, and one token routed twice to an expert."""
+    T, H, I, E, k = 6, 512, 256, 4, 3
+    hidden, w1, w2, _ = make_inputs(T, H, I, E, seed=3)
+    ids = np.array([[0, 1, 2], [0, 1, 2], [2, 2, 0], [3, 3, 3], [1, 0, 3], [0, 0, 1]], np.int32)
+    w = np.random.default_rng(0).uniform(0.1, 1.0, (T, k))
+    ref = oracle.moe_token_loop(hidden, w1, w2, w, ids)
+    for small in (16, 0):
+        prev = moe.set_small_t_max(small)
+        try:
+            out = gpu_forward(hidden, w1, w2, w, ids)
+        finally:
+            moe.set_small_t_max(prev)
+        assert_output_close(out, ref, f"small_t_max={small}")
+
+
+@pytest.mark.parametrize("small", [16, 0])
+def test_forward_invalid_ids_are_skipped_and_flagged(small):
+    T, H, I, E, k = 12, 256, 128, 8, 2
+    hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=11)
+    ids, w = oracle.route(logits.numpy(), k, True)
+    ids[3, 1] = -1
+    ids[7, 0] = E
+    ids[9, :] = 99  # no valid slot -> zero row
+    ref = oracle.moe_token_loop(hidden, w1, w2, w, ids)
+    moe.get_device_status()
+    prev = moe.set_small_t_max(small)
+    try:
+        out = gpu_forward(hidden, w1, w2, w, ids)
+    finally:
+        moe.set_small_t_max(prev)
+    assert_output_close(out, ref)
+    assert np.all(out[9] == 0.0)
+    assert moe.get_device_status() & moe.MOE_STATUS_BAD_ID
+
+
+@pytest.mark.parametrize("small", [16, 0])
+def test_forward_zero_token_gives_zero_row(small):
+    T, H, I, E, k = 20, 256, 128, 8, 2
+    hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=12)
+    hidden[4] = 0
+    ids, w = oracle.route(logits.numpy(), k, True)
+    prev = moe.set_small_t_max(small)
+    try:
+        out = gpu_forward(hidden, w1, w2, w, ids)
+    finally:
+        moe.set_small_t_max(prev)
+    assert np.all(out[4] == 0.0)
+
+
+def test_forward_deterministic():
+    s = SHAPES["tiny"]
+    hidden, w1, w2, logits = make_shape_inputs(s)
+    ids, w = oracle.route(logits.numpy(), s.k, True)
+    a = gpu_forward(hidden, w1, w2, w, ids)
+    b = gpu_forward(hidden, w1, w2, w, ids)
+    assert np.array_equal(a, b)
+
+
+def test_forward_empty_batch():
+    out = moe.moe_forward(torch.empty(0, 256, dtype=torch.bfloat16, device="cuda"),
+                          torch.zeros(8, 256, 256, dtype=torch.bfloat16, device="cuda"),
+                          torch.zeros(8, 256, 128, dtype=torch.bfloat16, device="cuda"),
+                          torch.empty(0, 2, device="cuda"),
+                          torch.empty(0, 2, dtype=torch.int32, device="cuda"))
+    assert out.shape == (0, 256)
+
+
+def test_end_to_end_route_then_forward():
+    """GPU routing feeds the GPU forward; the oracle routes for itself."""
+    for name in ("tiny",):
+        s = SHAPES[name]
+        hidden, w1, w2, logits = make_shape_inputs(s)
+        ids_r, w_r = oracle.route(logits.numpy(), s.k, True)
+        ref = oracle.moe_token_loop(hidden, w1, w2, w_r, ids_r)
+        ids_g, w_g = moe.moe_route(logits.cuda(), s.k, True)
+        out = moe.moe_forward(hidden.cuda(), w1.cuda(), w2.cuda(), w_g, ids_g)
+        torch.cuda.synchronize()
+        assert np.array_equal(ids_g.cpu().numpy(), ids_r)
+        assert_output_close(out.cpu().numpy(), ref, name)
+
+
+# ------------------------------------------------------------------ full-size workloads
+def _sample_rows(T, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = {0, T - 1} | set(rng.choice(T, size=min(n, T), replace=False).tolist())
+    return np.array(sorted(rows), np.int64)
+
+
+@pytest.mark.parametrize("name", ["decode", "prefill_8e", "prefill_thin", "prefill_big"])
+def test_forward_full_size_workloads(name):
+    s = SHAPES[name]
+    hidden, w1, w2, logits = make_shape_inputs(s, device="cuda")
+    logits_c = logits.cpu()
+    ids_r, w_r = oracle.route(logits_c.numpy(), s.k, True)
+    ids_g, w_g = moe.moe_route(logits, s.k, True)
+    torch.cuda.synchronize()
+    assert np.array_equal(ids_g.cpu().numpy(), ids_r)
+    # the forward takes the oracle's routing so both sides compute the same sum
+    out = moe.moe_forward(hidden, w1, w2, torch.as_tensor(w_r.astype(np.float32)).cuda(),
+                          torch.as_tensor(ids_r).cuda())
+    torch.cuda.synchronize()
+    rows = np.arange(s.T) if s.T <= 64 else _sample_rows(s.T, 14, 1)
+    ref = oracle.moe_token_loop(hidden.cpu(), w1.cpu(), w2.cpu(), w_r, ids_r, rows=rows)
+    assert_output_close(out.cpu().numpy()[rows], ref, name)
+    check_status_clean()
+    # properties that hold at any size: every row written and finite
+    assert torch.isfinite(out).all()
+
+
+# ------------------------------------------------------------------ failure paths
+def test_bounded_wait_times_out_without_hanging():
+    moe.get_device_status()
+    assert moe.debug_wait_timeout(2_000_000) == moe.MOE_ERR_TIMEOUT  # 2 ms
+    assert moe.get_device_status() & moe.MOE_STATUS_TIMEOUT
+    # the context is still usable afterwards
+    test_forward_deterministic()
+    check_status_clean()
+
+
+def test_sync_each_stage_mode_and_profiler():
+    s = SHAPES["tiny"]
+    hidden, w1, w2, logits = make_shape_inputs(s)
+    ids, w = oracle.route(logits.numpy(), s.k, True)
+    prev = moe.set_sync_each_stage(True)
+    moe.profile_reset()
+    moe.profile_enable(True)
+    try:
+        out = gpu_forward(hidden, w1, w2, w, ids)
+    finally:
+        moe.profile_enable(False)
+        moe.set_sync_each_stage(prev)
+    prof = moe.profile_read()
+    for kname in ("permute_count", "permute_scan", "permute_scatter", "gemm1_swiglu", "gemm2",
+                  "combine"):
+        assert prof[kname][0] == 1 and prof[kname][1] > 0
+    ref = oracle.moe_token_loop(hidden, w1, w2, w, ids)
+    assert_output_close(out, ref)
