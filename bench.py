@@ -88,6 +88,12 @@ def max_over_ranks(x: float, device) -> float:
     return float(t.item())
 
 
+def whole_job_tflops(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Throughput of all replicas: every rank did `steps` steps; the job took
+    the slowest rank's time."""
+    return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
+
+
 def barrier():
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized():
@@ -223,7 +229,7 @@ def run_ours(args, ws, rank, local):
     total_ms = sum(a + b for a, b in t)
     total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
-    value = s.flops * args.steps * ws / (total_ms * 1e-3) / 1e12
+    value = whole_job_tflops(s.flops, args.steps, ws, total_ms)
     n_active = int(torch.unique(ids).numel())
 
     # per-kernel durations: the same K steps again with the library's event
@@ -276,7 +282,7 @@ def run_ours(args, ws, rank, local):
 
     te = time_steps(step_e2e, args.steps, args.warmup, flush, stream, marks=1)
     e2e_ms = max_over_ranks(sum(x[0] for x in te), dev)
-    e2e_value = s.flops * args.steps * ws / (e2e_ms * 1e-3) / 1e12
+    e2e_value = whole_job_tflops(s.flops, args.steps, ws, e2e_ms)
     h2d = h_hidden.numel() * 2 + h_logits.numel() * 4
     d2h = h_out.numel() * 4
 

@@ -5,7 +5,7 @@ of torch tensors, passes raw device pointers, sizes and the current CUDA
 stream to the C ABI of ``include/moe.h`` and raises ``MoEError`` on a
 non-zero return code.  All arithmetic runs in the library's CUDA kernels;
 there is no CPU or PyTorch fallback, and importing this package fails if
-libmoe.so has not been built (``python -m mixture_experts_expert_softmax_b200.build``).
+libmoe.so has not been built (``python mixture_experts_expert_softmax_b200/build.py``).
 
     ids, w = moe_route(logits, k=8, renorm=True)          # [T,k] int32, fp32
     out = moe_forward(hidden, w1, w2, w, ids)              # [T,H] fp32
@@ -49,7 +49,7 @@ def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"{LIB_PATH} is missing: build it with "
-            "`python -m mixture_experts_expert_softmax_b200.build` (nvcc, sm_100a)")
+            "`python mixture_experts_expert_softmax_b200/build.py` (nvcc, sm_100a)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
     sig = {

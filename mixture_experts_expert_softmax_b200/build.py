@@ -1,6 +1,6 @@
 """Build libmoe.so (the CUDA library behind include/moe.h) for sm_100a.
 
-    python -m mixture_experts_expert_softmax_b200.build [--force] [--verbose]
+    python mixture_experts_expert_softmax_b200/build.py [--force] [--verbose]
 
 Each csrc/*.cu file is compiled with nvcc for sm_100a into _build/, in
 parallel, then linked (static CUDA runtime) into
