@@ -45,6 +45,7 @@ extern "C" {
 #define MOE_ERR_TIMEOUT -4     /* a bounded device-side wait expired */
 #define MOE_ERR_NO_DEVICE -5   /* no usable sm_100 device is current */
 #define MOE_ERR_OOM -6         /* workspace allocation failed */
+#define MOE_ERR_SCRATCH_LIMIT -7 /* request larger than the fixed scratch of moe_forward_small_noalloc */
 
 /* Bits of the device status word (moe_get_device_status). */
 #define MOE_STATUS_TIMEOUT 0x1u  /* a pipeline wait gave up; that launch's output is invalid */
@@ -101,6 +102,38 @@ int moe_route(const float *logits, int64_t T, int E, int k, int renorm,
 int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
                 const float *topk_weights, const int32_t *topk_ids, float *out,
                 int64_t T, int H, int I, int E, int k, void *stream);
+
+/*
+ * moe_forward_small_noalloc -- the small-batch path of moe_forward (the two
+ * GEMV kernels) in a form that never allocates device memory.  The pages
+ * have no counterpart: it exists for callers that cannot allocate once they
+ * are running, such as a serving runtime that reserves all of its device
+ * memory at start-up, or a decode loop that must not pay the device-wide
+ * synchronisation of cudaFree when a workspace grows.
+ *
+ * Arguments, layouts, numerics and the result are those of moe_forward on
+ * its small-T path (fp32 SwiGLU intermediate, fixed-order fp32 combine).
+ * Its only scratch is a fixed __device__ array of this library:
+ * 256 bytes + MOE_NOALLOC_MAX_ACT fp32 values (1 MiB), which every GPU that
+ * loads the library holds until the process exits.
+ *   - Limits: T <= MOE_NOALLOC_MAX_T and T*k*I <= MOE_NOALLOC_MAX_ACT, else
+ *     MOE_ERR_SCRATCH_LIMIT and nothing is launched.  Other checks and
+ *     codes as in moe_forward.
+ *   - The first call on each device, with that device current, looks up
+ *     the array's device address (cudaGetSymbolAddress) and caches it; make
+ *     that first call before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents:
+ *     calls whose kernels overlap on the GPU (e.g. on two streams without
+ *     ordering) race on it.  Nothing in it has to start at zero.
+ *   - Expert ids outside [0, E) are skipped as in moe_forward, but the bad-id
+ *     flag is not reported through moe_get_device_status.
+ *   - Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define MOE_NOALLOC_MAX_T 16
+#define MOE_NOALLOC_MAX_ACT 262144
+int moe_forward_small_noalloc(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
+                              const float *topk_weights, const int32_t *topk_ids, float *out,
+                              int64_t T, int H, int I, int E, int k, void *stream);
 
 /*
  * moe_permute -- the expert grouping that moe_forward uses internally,

@@ -27,6 +27,9 @@ MOE_ERR_CUDA = -3
 MOE_ERR_TIMEOUT = -4
 MOE_ERR_NO_DEVICE = -5
 MOE_ERR_OOM = -6
+MOE_ERR_SCRATCH_LIMIT = -7
+MOE_NOALLOC_MAX_T = 16
+MOE_NOALLOC_MAX_ACT = 262144
 MOE_STATUS_TIMEOUT = 0x1
 MOE_STATUS_BAD_ID = 0x2
 
@@ -36,6 +39,7 @@ EXPORTED = (
     "moe_get_device_status", "moe_set_small_t_max", "moe_set_sync_each_stage",
     "moe_set_wait_limit_ns", "moe_last_failed_stage", "moe_debug_wait_timeout",
     "moe_profile_enable", "moe_profile_reset", "moe_profile_read",
+    "moe_forward_small_noalloc",
 )
 
 
@@ -66,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "moe_profile_enable": ([I32], I32),
         "moe_profile_reset": ([], I32),
         "moe_profile_read": ([I32, P, P, P], I32),
+        "moe_forward_small_noalloc": ([P, P, P, P, P, P, I64, I32, I32, I32, I32, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -150,6 +155,29 @@ def moe_forward(hidden: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
     return out
 
 
+def moe_forward_small_noalloc(hidden: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
+                              topk_weights: torch.Tensor, topk_ids: torch.Tensor,
+                              out: torch.Tensor, stream=None) -> torch.Tensor:
+    """Small-batch forward that allocates nothing on the device: for callers
+    that reserve all device memory up front.  `out` must be given; limits
+    T <= MOE_NOALLOC_MAX_T and T*k*I <= MOE_NOALLOC_MAX_ACT."""
+    _need(hidden, "hidden", torch.bfloat16)
+    T, H = hidden.shape
+    E, twoI, _ = w1.shape
+    I = twoI // 2
+    _need(w1, "w1", torch.bfloat16, (E, 2 * I, H))
+    _need(w2, "w2", torch.bfloat16, (E, H, I))
+    k = topk_ids.shape[1] if topk_ids.dim() == 2 else 0
+    _need(topk_ids, "topk_ids", torch.int32, (T, k))
+    _need(topk_weights, "topk_weights", torch.float32, (T, k))
+    _need(out, "out", torch.float32, (T, H))
+    _check(_lib.moe_forward_small_noalloc(hidden.data_ptr(), w1.data_ptr(), w2.data_ptr(),
+                                          topk_weights.data_ptr(), topk_ids.data_ptr(),
+                                          out.data_ptr(), T, H, I, E, k, _stream(stream)),
+           "moe_forward_small_noalloc")
+    return out
+
+
 def moe_permute(topk_ids: torch.Tensor, E: int, sorted_rows: torch.Tensor | None = None,
                 expert_offsets: torch.Tensor | None = None, stream=None):
     """Stable grouping of the flat (token, slot) indices by expert.
@@ -217,7 +245,7 @@ def profile_read() -> dict[str, tuple[int, float]]:
 
 
 __all__ = [
-    "moe_route", "moe_forward", "moe_permute", "get_device_status", "set_small_t_max",
+    "moe_route", "moe_forward", "moe_forward_small_noalloc", "moe_permute", "get_device_status", "set_small_t_max",
     "set_sync_each_stage", "set_wait_limit_ns", "last_failed_stage", "debug_wait_timeout",
     "profile_enable", "profile_reset", "profile_read", "error_string", "MoEError",
     "LIB_PATH", "EXPORTED",

@@ -200,6 +200,9 @@ const char *moe_error_string(int code) {
     case MOE_ERR_TIMEOUT: return "a bounded device-side wait expired";
     case MOE_ERR_NO_DEVICE: return "no usable sm_100 device is current";
     case MOE_ERR_OOM: return "workspace allocation failed";
+    case MOE_ERR_SCRATCH_LIMIT:
+      return "request exceeds the fixed scratch of moe_forward_small_noalloc "
+             "(T <= MOE_NOALLOC_MAX_T, T*k*I <= MOE_NOALLOC_MAX_ACT)";
     default: return "unknown error code";
   }
 }

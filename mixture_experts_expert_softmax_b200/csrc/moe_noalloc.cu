@@ -1,0 +1,89 @@
+// moe_noalloc.cu -- moe_forward_small_noalloc: the small-batch (GEMV) form
+// of moe_forward that never allocates device memory.
+//
+// Who needs it: callers whose device memory is planned up front and must not
+// change afterwards -- a serving runtime that carves every buffer out of one
+// reservation at start-up, or a latency-critical decode loop that cannot
+// afford the device-wide synchronisation that cudaFree performs when the
+// regular entry points grow their workspace.  Such callers pass inputs and
+// outputs as usual; the only scratch this path needs (the fp32 SwiGLU
+// intermediate of at most MOE_NOALLOC_MAX_ACT values, plus a status word)
+// lives in a fixed __device__ array of this file, which every GPU that loads
+// the library keeps until the process exits.
+//
+// Host code cannot use the array's name as a device address (on the host it
+// names a stand-in object), so the first call on each device looks the
+// address up with cudaGetSymbolAddress while that device is current and
+// caches it; later calls reuse the cached address.
+#include <mutex>
+
+#include "moe.h"
+#include "moe_internal.h"
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+constexpr size_t kStatusBytes = 256;
+constexpr size_t kScratchBytes =
+    kStatusBytes + static_cast<size_t>(MOE_NOALLOC_MAX_ACT) * sizeof(float);
+
+// [0, 256): status word the kernels may raise bits in (not reported back);
+// [256, ...): the act scratch, T*k*I fp32 values.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+}  // namespace
+
+extern "C" int moe_forward_small_noalloc(const uint16_t *hidden, const uint16_t *w1,
+                                         const uint16_t *w2, const float *topk_weights,
+                                         const int32_t *topk_ids, float *out, int64_t T, int H,
+                                         int I, int E, int k, void *stream) {
+  if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (hidden == nullptr || w1 == nullptr || w2 == nullptr || topk_weights == nullptr ||
+                topk_ids == nullptr || out == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (H % 128 != 0 || I % 128 != 0 || E > 1024 || k > 16) return MOE_ERR_UNSUPPORTED;
+  if (T > MOE_NOALLOC_MAX_T ||
+      T * static_cast<int64_t>(k) * static_cast<int64_t>(I) > MOE_NOALLOC_MAX_ACT)
+    return MOE_ERR_SCRATCH_LIMIT;
+  if (T == 0) return MOE_OK;
+
+  int dev = -1, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_NO_DEVICE;
+  }
+  if (major != 10 || minor != 0) return MOE_ERR_NO_DEVICE;
+
+  void *base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+      void *p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+      }
+      g_noalloc_addr[dev] = p;
+    }
+    base = g_noalloc_addr[dev];
+  }
+  // Nothing here has to start at zero: every act value the second kernel
+  // reads is written by the first kernel of the same call.
+  uint32_t *status = static_cast<uint32_t *>(base);
+  float *act = reinterpret_cast<float *>(static_cast<char *>(base) + kStatusBytes);
+  moe::StageHook hook;
+  hook.pdl = true;
+  const cudaError_t e =
+      moe::launch_small_t(hidden, w1, w2, topk_weights, topk_ids, act, out, T, H, I, E, k, status,
+                          static_cast<cudaStream_t>(stream), hook);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}

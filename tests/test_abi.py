@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_error_strings():
-    for code in range(0, -7, -1):
+    for code in range(0, -8, -1):
         s = moe.error_string(code)
         assert s and "unknown" not in s
     assert "unknown" in moe.error_string(-99)
