@@ -91,7 +91,8 @@ int moe_route(const float *logits, int64_t T, int E, int k, int renorm,
  *                 accumulated in fp32; a row with no valid id is 0.
  * Numerics: bf16 inputs, fp32 accumulation; the SwiGLU intermediate is
  * rounded to bf16 before the second projection on the grouped-GEMM path
- * (T > small-T limit) and kept in fp32 on the small-T path.  The combine is
+ * and kept in fp32 on the small-T path (T <= the small-T limit, H <= 6144
+ * and I <= 12288).  The combine is
  * deterministic (fixed j order, no atomics): repeated calls give identical
  * bits.
  * Errors: INVALID_ARG for null pointers, T < 0, H/I/E < 1, k < 1 or k > E;
@@ -118,7 +119,8 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
  * loads the library holds until the process exits.
  *   - Limits: T <= MOE_NOALLOC_MAX_T and T*k*I <= MOE_NOALLOC_MAX_ACT, else
  *     MOE_ERR_SCRATCH_LIMIT and nothing is launched.  Other checks and
- *     codes as in moe_forward.
+ *     codes as in moe_forward, plus UNSUPPORTED when H > 6144 or I > 12288
+ *     (the largest rows the small-T kernels stage).
  *   - The first call on each device, with that device current, looks up
  *     the array's device address (cudaGetSymbolAddress) and caches it; make
  *     that first call before any stream capture.

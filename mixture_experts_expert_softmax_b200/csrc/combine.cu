@@ -1,20 +1,20 @@
 // combine.cu -- the top-k weighted sum of ref_moe ("tpu_inference/kernels/
 // fused_moe/v1/kernel.py": sum over the chosen experts of w_j * y_j) from
-// the per-(token, slot) expert outputs P[t*k + j, :] that GEMM2 stores.
-// out[t, h] = sum_{j=0..k-1} w[t, j] * P[t*k + j, h], accumulated in fp32
-// with one FMA per term in ascending j, so the result does not depend on
-// scheduling.  Slots whose id is outside [0, E) are skipped (their P row was
-// never written) and raise the bad-id status bit; a token with no valid slot
-// gets a zero row.  HBM-bound: reads T*k*H*4 bytes, writes T*H*4.
+// the expert outputs that GEMM2 stores in expert-sorted row order:
+// out[t, h] = sum_{j=0..k-1} w[t, j] * P[inv[t*k + j], h], accumulated in
+// fp32 with one FMA per term in ascending j, so the result does not depend
+// on scheduling.  Slots whose id is outside [0, E) have inv = -1: they are
+// skipped and raise the bad-id status bit; a token with no valid slot gets a
+// zero row.  HBM-bound: reads T*k*H*4 bytes of P (whole rows), writes T*H*4.
 #include "moe_internal.h"
 
 namespace moe {
 namespace {
 
 __global__ void __launch_bounds__(256)
-    combine_kernel(const float4 *__restrict__ P, const float *__restrict__ w,
-                   const int32_t *__restrict__ ids, float4 *__restrict__ out, int64_t T, int H4,
-                   int E, int k, uint32_t *status) {
+    combine_kernel(const float4 *__restrict__ P, const int32_t *__restrict__ inv,
+                   const float *__restrict__ w, float4 *__restrict__ out, int64_t T, int H4, int k,
+                   uint32_t *status) {
   grid_dep_wait();
   grid_dep_launch();
   const int64_t n = T * H4;
@@ -26,13 +26,13 @@ __global__ void __launch_bounds__(256)
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     bool bad = false;
     for (int j = 0; j < k; ++j) {
-      const int e = __ldg(ids + t * k + j);
-      if (e < 0 || e >= E) {
+      const int r = __ldg(inv + t * k + j);
+      if (r < 0) {
         bad = true;
         continue;
       }
       const float wj = __ldg(w + t * k + j);
-      const float4 y = __ldcs(P + (t * k + j) * H4 + h4);
+      const float4 y = __ldcs(P + static_cast<int64_t>(r) * H4 + h4);
       acc.x = fmaf(wj, y.x, acc.x);
       acc.y = fmaf(wj, y.y, acc.y);
       acc.z = fmaf(wj, y.z, acc.z);
@@ -45,9 +45,9 @@ __global__ void __launch_bounds__(256)
 
 }  // namespace
 
-cudaError_t launch_combine(const float *P, const float *topk_weights, const int32_t *topk_ids,
-                           float *out, int64_t T, int H, int E, int k, uint32_t *status,
-                           cudaStream_t s, const StageHook &hook) {
+cudaError_t launch_combine(const float *P, const int32_t *inv, const float *topk_weights,
+                           float *out, int64_t T, int H, int k, uint32_t *status, cudaStream_t s,
+                           const StageHook &hook) {
   const int H4 = H / 4;
   const int64_t n = T * H4;
   int dev = 0, sms = 148;
@@ -58,8 +58,8 @@ cudaError_t launch_combine(const float *P, const float *topk_weights, const int3
   const int blocks = static_cast<int>(want < cap ? want : cap);
   hook.begin("combine");
   cudaError_t e = launch_pdl(combine_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, s,
-                             hook.pdl, reinterpret_cast<const float4 *>(P), topk_weights,
-                             topk_ids, reinterpret_cast<float4 *>(out), T, H4, E, k, status);
+                             hook.pdl, reinterpret_cast<const float4 *>(P), inv, topk_weights,
+                             reinterpret_cast<float4 *>(out), T, H4, k, status);
   return hook.end(e);
 }
 

@@ -4,33 +4,46 @@
 //   GEMM1 (+SwiGLU): for the rows of expert e in expert-sorted order,
 //     g = x . w1[e, 0:I, :]^T, u = x . w1[e, I:2I, :]^T  (fp32 in TMEM),
 //     act = silu(g) * u, stored as bf16 [rows, I].
-//   GEMM2: y = act . w2[e]^T (fp32 in TMEM), stored to the per-(token, slot)
-//     buffer P at row t*k + j; combine.cu then forms sum_j w_j * y_j.
+//   GEMM2: y = act . w2[e]^T (fp32 in TMEM), stored as fp32 rows of P in the
+//     same expert-sorted order; combine.cu then forms sum_j w_j * y_j.
 // This is the expert FFN of ref_moe on the page "tpu_inference/kernels/
 // fused_moe/v1/kernel.py" (gate = w1, up = w3, then act . w2) in the weight
 // layout of atrex-bench #009 (w1 [E, 2I, H], w2 [E, H, I], both applied as
 // F.linear, i.e. K-major).
 //
-// Work unit: a 128-row m-tile of one expert's rows times one n-tile (GEMM1:
-// 128 act columns = 256 accumulator columns, gate and up side by side;
-// GEMM2: 256 output columns).  Tiles are ordered expert-major, then n-tile,
-// then m-tile, so CTAs that run together share an expert's weight tile in
-// L2.  Each CTA loops over tiles with a stride of the grid size.
+// Work unit: an m-tile of one expert's rows times one 256-column n-tile of
+// the accumulator.  Tiles run expert-major, then n-tile, then m-tile, so
+// CTAs working together share a weight tile through L2; the grid is
+// persistent and loops over tiles.
 //
-// Warp roles (288 threads):
-//   warps 0-3  producers.  GEMM1: the 128 threads gather the A rows (hidden
-//              rows of the tile's tokens) with 16-byte cp.async into the
-//              128-byte-swizzled K-major layout, and thread 0 issues the two
-//              TMA boxes of w1 (gate rows, up rows).  GEMM2: thread 0 issues
-//              TMA for the act tile and the w2 tile.
-//   warp 4     allocates 512 TMEM columns (two 128x256 fp32 accumulators)
-//              and one thread issues tcgen05.mma (M=128, N=256, K=16).
-//   warps 5-8  epilogue: tcgen05.ld of their 32-lane quarter, SwiGLU or
-//              plain store, then release the accumulator.
-// Pipelines: kStages smem stages (full/empty mbarriers) between producers
-// and MMA; two accumulators (acc_full/acc_empty) between MMA and epilogue.
+//   GEMM1 runs on single CTAs (M = 128, tcgen05.mma.cta_group::1): its A rows
+//   are gathered by token index with cp.async, whose completion can only be
+//   signalled to the CTA's own barriers.  The B tile is the n-tile's 128 gate
+//   rows and the matching 128 up rows, so one accumulator holds gate and up
+//   side by side and the epilogue applies SwiGLU.
+//   GEMM2 runs on CTA pairs (a cluster of 2, M = 256, cta_group::2): rank r
+//   loads A rows 128r..128r+127 and B rows 128r..128r+127 of the pair's tile
+//   with TMA into its own shared memory, rank 0 issues the MMAs, and each
+//   CTA receives its 128 accumulator rows in its own TMEM.  Splitting B
+//   between the pair halves the weight bytes each SM must fetch.  Its
+//   epilogue stages each 32x32 fp32 block in shared memory and writes it
+//   with a TMA store (coalesced, asynchronous); a block that straddles the
+//   end of an expert's rows is written row by row instead.
+//
+// Warp roles (288 threads per CTA):
+//   warps 0-3  producers.  GEMM1: the 128 threads gather the A rows with
+//              16-byte cp.async into the 128-byte-swizzled K-major layout and
+//              arrive on the stage barrier asynchronously when they land;
+//              thread 0 issues the two TMA boxes of w1.  GEMM2: thread 0 of
+//              each CTA issues TMA for its act rows and half of B, counted on
+//              rank 0's barrier.
+//   warp 4     allocates 512 TMEM columns (two accumulators); one thread (on
+//              rank 0) issues the MMAs and commits each stage back to the
+//              producers and each finished tile to the epilogues.
+//   warps 5-8  epilogue: tcgen05.ld of their 32-lane quarter, SwiGLU + bf16
+//              store, or the fp32 TMA store, then release the accumulator.
 // Every wait is bounded; a wait that gives up raises the timeout bit of the
-// status word and makes every role leave its loop.
+// status word and makes every role of the CTA leave its loop.
 #include <mutex>
 
 #include "moe_internal.h"
@@ -38,40 +51,68 @@
 namespace moe {
 namespace {
 
-constexpr int BM = kGemmTileM;  // 128 rows per tile (UMMA M)
-constexpr int BK = 64;          // K per stage: one 128-byte swizzle row of bf16
-constexpr int kStages = 4;
-constexpr int kLag = kStages - 1;  // cp.async groups in flight before a stage is signalled
+constexpr int BM = 128;  // rows per CTA
+constexpr int BK = 64;   // K per stage: one 128-byte swizzle row of bf16
 constexpr int kProducerThreads = 128;
 constexpr int kMmaWarp = 4;
 constexpr int kThreads = 9 * 32;
-constexpr int kAccN = 256;               // UMMA N = accumulator columns per tile
-constexpr int kTmemCols = 2 * kAccN;     // double-buffered accumulator
-constexpr int kABytes = BM * BK * 2;     // 16 KB
-constexpr int kBBytes = kAccN * BK * 2;  // 32 KB
+constexpr int kAccN = 256;            // UMMA N = accumulator columns per tile
+constexpr int kTmemCols = 2 * kAccN;  // double-buffered accumulator
+constexpr int kABytes = BM * BK * 2;  // 16 KB
 constexpr int kMaxE = 1024;
+constexpr int kMaxStages = 6;
+constexpr uint16_t kBothCtas = 0x3;
+constexpr int kEpiBlock = 32 * 32 * 4;  // one 32-row x 32-column fp32 block
 
 enum { kModeGemm1 = 0, kModeGemm2 = 1 };
 
-struct __align__(8) Bars {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
-  uint64_t drain;
-  uint32_t tmem_base;
-  int abort_flag;
+template <int MODE>
+struct Cfg;
+template <>
+struct Cfg<kModeGemm1> {
+  static constexpr int CG = 1;        // CTAs per MMA
+  static constexpr int kStages = 4;
+  static constexpr int kBRows = 256;  // B rows this CTA loads per stage
+  static constexpr int kEpiBytes = 0;
+};
+template <>
+struct Cfg<kModeGemm2> {
+  static constexpr int CG = 2;
+  static constexpr int kStages = 5;
+  static constexpr int kBRows = 128;
+  static constexpr int kEpiBytes = 4 * 2 * kEpiBlock;  // 4 warps x double buffer
 };
 
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kStages) * (kABytes + kBBytes) +
-                              sizeof(Bars) + 2 * (kMaxE + 1) * sizeof(int32_t);
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+template <int MODE>
+constexpr int tile_m() { return BM * Cfg<MODE>::CG; }
+template <int MODE>
+constexpr int b_bytes() { return Cfg<MODE>::kBRows * BK * 2; }
+template <int MODE>
+constexpr size_t smem_bytes();
+
+struct __align__(8) Bars {
+  uint64_t full[kMaxStages];   // stage landed (rank 0's counts both CTAs)
+  uint64_t empty[kMaxStages];  // the MMAs finished reading the stage
+  uint64_t acc_full[2];        // accumulator ready for the epilogue
+  uint64_t acc_empty[2];       // epilogues (of both CTAs) drained the accumulator
+  uint64_t drain;              // every MMA has completed
+  uint32_t tmem_base;
+  int abort_flag;
+  int32_t scan[32];            // per-warp partial sums of build_tile_offsets
+};
+
+template <int MODE>
+constexpr size_t smem_bytes() {
+  return 1024 + static_cast<size_t>(Cfg<MODE>::kStages) * (kABytes + b_bytes<MODE>()) +
+         Cfg<MODE>::kEpiBytes + sizeof(Bars) + 2 * (kMaxE + 1) * sizeof(int32_t);
+}
+static_assert(smem_bytes<kModeGemm1>() <= 232448, "shared memory budget");
+static_assert(smem_bytes<kModeGemm2>() <= 232448, "shared memory budget");
 
 struct Params {
   const __nv_bfloat16 *hidden;
   const int32_t *sorted_rows;
   const int32_t *expert_offsets;
-  const int32_t *tile_offsets;
   __nv_bfloat16 *act;
   float *P;
   int H, I, E, k;
@@ -83,11 +124,12 @@ struct Params {
 };
 
 struct Tile {
-  int e, mt, nt, row0, rows;
+  int e, mt, nt, row0, rows;  // row0/rows: the whole m-tile (both CTAs of a pair)
 };
 
 // Tile t -> (expert, m-tile, n-tile).  tile_off[e] counts the m-tiles of
 // experts < e, so expert e owns tiles [tile_off[e] * NT, tile_off[e+1] * NT).
+template <int TM>
 __device__ __forceinline__ Tile decode_tile(int t, int NT, int E, const int32_t *tile_off,
                                             const int32_t *exp_off) {
   const int q = t / NT;
@@ -105,9 +147,43 @@ __device__ __forceinline__ Tile decode_tile(int t, int NT, int E, const int32_t 
   const int local = t - tile_off[lo] * NT;
   tl.nt = local / mt_cnt;
   tl.mt = local - tl.nt * mt_cnt;
-  tl.row0 = exp_off[lo] + tl.mt * BM;
-  tl.rows = min(BM, exp_off[lo + 1] - tl.row0);
+  tl.row0 = exp_off[lo] + tl.mt * TM;
+  tl.rows = min(TM, exp_off[lo + 1] - tl.row0);
   return tl;
+}
+
+// exp_off[0..E] -> tile_off[0..E]: exclusive prefix sum of ceil(count / TM),
+// computed by the whole CTA (E <= 1024, kThreads threads).
+template <int TM>
+__device__ void build_tile_offsets(const int32_t *exp_off, int32_t *tile_off, int E,
+                                   int32_t *scratch /* >= 32 ints */) {
+  constexpr int kPer = (kMaxE + kThreads - 1) / kThreads;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int local[kPer];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = tid * kPer + i;
+    local[i] = e < E ? (exp_off[e + 1] - exp_off[e] + TM - 1) / TM : 0;
+    sum += local[i];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  int before = 0;
+  for (int w = 0; w < warp; ++w) before += scratch[w];
+  int run = before + incl - sum;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = tid * kPer + i;
+    if (e <= E) tile_off[e] = run;  // e == E receives the total
+    run += local[i];
+  }
 }
 
 __device__ __forceinline__ void give_up(const Params &p, volatile int *abort_flag) {
@@ -120,44 +196,64 @@ __device__ __forceinline__ float as_f32(uint32_t u) { return __uint_as_float(u);
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
-                        const __grid_constant__ CUtensorMap tm_b, const Params p) {
+                        const __grid_constant__ CUtensorMap tm_b,
+                        const __grid_constant__ CUtensorMap tm_out, const Params p) {
+  using C = Cfg<MODE>;
+  constexpr int CG = C::CG;
+  constexpr int kStages = C::kStages;
+  constexpr int TM = tile_m<MODE>();
+  constexpr int kBBytes = b_bytes<MODE>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *sA = smem;
-  uint8_t *sB = smem + kStages * kABytes;
-  Bars *bars = reinterpret_cast<Bars *>(sB + kStages * kBBytes);
+  uint8_t *sB = sA + kStages * kABytes;
+  uint8_t *sEpi = sB + kStages * kBBytes;
+  Bars *bars = reinterpret_cast<Bars *>(sEpi + C::kEpiBytes);
   int32_t *s_tile_off = reinterpret_cast<int32_t *>(bars + 1);
   int32_t *s_exp_off = s_tile_off + (kMaxE + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 2 ? cluster_rank() : 0;
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
+      // GEMM1: 128 cp.async arrivals + the expect_tx arrival; GEMM2: rank 0's
+      // expect_tx arrival (both CTAs' TMA bytes are counted on it)
       mbar_init(&bars->full[s], MODE == kModeGemm1 ? kProducerThreads + 1 : 1);
       mbar_init(&bars->empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&bars->acc_full[a], 1);
-      mbar_init(&bars->acc_empty[a], 4);
+      mbar_init(&bars->acc_empty[a], 4 * CG);  // 4 epilogue warps per CTA
     }
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
-    if (MODE == kModeGemm2) prefetch_tmap(&tm_a);
+    if (MODE == kModeGemm2) {
+      prefetch_tmap(&tm_a);
+      prefetch_tmap(&tm_out);
+    }
     prefetch_tmap(&tm_b);
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&bars->tmem_base, kTmemCols);
-    tmem_relinquish();
+    if (CG == 2) {
+      tmem_alloc_pair(&bars->tmem_base, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&bars->tmem_base, kTmemCols);
+      tmem_relinquish();
+    }
   }
+  // both CTAs' barriers exist before any traffic crosses the pair
+  if (CG == 2) cluster_sync();
   // Everything above overlaps the previous kernel under PDL; the routing
   // permutation (and, for GEMM2, act) is read only after this point.
   grid_dep_wait();
   grid_dep_launch();
-  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
-    s_tile_off[i] = p.tile_offsets[i];
-    s_exp_off[i] = p.expert_offsets[i];
-  }
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_exp_off[i] = p.expert_offsets[i];
+  __syncthreads();
+  build_tile_offsets<TM>(s_exp_off, s_tile_off, p.E, bars->scan);
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -166,8 +262,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int NT = p.n_tiles_n;
   const int total = s_tile_off[p.E] * NT;
   const int KB = p.K / BK;
+  const int unit = CG == 2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int nunits = CG == 2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   volatile int *abort_flag = &bars->abort_flag;
   const uint64_t limit = p.wait_limit_ns;
+  // rank 0's barriers as seen from this CTA
+  const uint32_t full0 = CG == 2 ? map_to_rank(smem_addr(&bars->full[0]), 0) : 0u;
+  const uint32_t acc_empty0 = CG == 2 ? map_to_rank(smem_addr(&bars->acc_empty[0]), 0) : 0u;
 
   if (warp < 4) {
     // ------------------------------------------------------------ producers
@@ -176,8 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rsub = threadIdx.x >> 3;  // rows rsub, rsub+16, ..., rsub+112
       int it = 0;
       bool stop = false;
-      for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
-        const Tile tl = decode_tile(t, NT, p.E, s_tile_off, s_exp_off);
+      for (int t = unit; t < total && !stop; t += nunits) {
+        const Tile tl = decode_tile<TM>(t, NT, p.E, s_tile_off, s_exp_off);
         const __nv_bfloat16 *src[8];
         uint32_t nbytes[8];
 #pragma unroll
@@ -204,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (threadIdx.x == 0) {
             mbar_arrive_expect_tx(&bars->full[s], kBBytes);
             uint8_t *b = sB + s * kBBytes;
-            tma_load_2d(b, &tm_b, &bars->full[s], kb * BK, b_row);                   // gate
+            tma_load_2d(b, &tm_b, &bars->full[s], kb * BK, b_row);                       // gate
             tma_load_2d(b + kBBytes / 2, &tm_b, &bars->full[s], kb * BK, b_row + p.I);  // up
           }
           const uint32_t a_base = smem_addr(sA + s * kABytes);
@@ -213,17 +314,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int r = rsub + 16 * i;
             cp_async_16(a_base + r * 128 + ((c ^ (r & 7)) << 4), src[i] + kb * BK, nbytes[i]);
           }
-          cp_async_commit();
-          if (it >= kLag) {
-            cp_async_wait_group<kLag>();
-            fence_proxy_async_smem();
-            mbar_arrive(&bars->full[(it - kLag) % kStages]);
-          }
+          // counts as this thread's arrival on full[s] once its copies land
+          cp_async_arrive_noinc(&bars->full[s]);
         }
       }
       cp_async_wait_all();
-      fence_proxy_async_smem();
-      for (int j = it - kLag > 0 ? it - kLag : 0; j < it; ++j) mbar_arrive(&bars->full[j % kStages]);
       if (stop && threadIdx.x == 0) {
         // let TMA copies already issued land before the CTA can exit
         const uint64_t t0 = global_timer_ns();
@@ -233,9 +328,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (threadIdx.x == 0) {
       int it = 0;
       bool stop = false;
-      for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
-        const Tile tl = decode_tile(t, NT, p.E, s_tile_off, s_exp_off);
-        const int b_row = tl.e * p.b_rows_per_expert + tl.nt * kAccN;
+      for (int t = unit; t < total && !stop; t += nunits) {
+        const Tile tl = decode_tile<TM>(t, NT, p.E, s_tile_off, s_exp_off);
+        const int a_row = tl.row0 + static_cast<int>(rank) * BM;
+        const int b_row =
+            tl.e * p.b_rows_per_expert + tl.nt * kAccN + static_cast<int>(rank) * C::kBRows;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
@@ -244,9 +341,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             stop = true;
             break;
           }
-          mbar_arrive_expect_tx(&bars->full[s], kABytes + kBBytes);
-          tma_load_2d(sA + s * kABytes, &tm_a, &bars->full[s], kb * BK, tl.row0);
-          tma_load_2d(sB + s * kBBytes, &tm_b, &bars->full[s], kb * BK, b_row);
+          if (leader) mbar_arrive_expect_tx(&bars->full[s], CG * (kABytes + kBBytes));
+          tma_load_2d_pair(sA + s * kABytes, &tm_a, full0 + 8u * s, kb * BK, a_row);
+          tma_load_2d_pair(sB + s * kBBytes, &tm_b, full0 + 8u * s, kb * BK, b_row);
         }
       }
       if (stop) {
@@ -256,12 +353,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(BM, kAccN);
+    if (lane == 0 && leader) {
+      // ---------------------------------------------------------- MMA issuer
+      const uint32_t idesc = idesc_bf16_f32(TM, kAccN);
       int it = 0, acc_it = 0;
       bool stop = false;
-      for (int t = blockIdx.x; t < total && !stop; t += gridDim.x, ++acc_it) {
+      for (int t = unit; t < total && !stop; t += nunits, ++acc_it) {
         const int a = acc_it & 1;
         const uint32_t aph = (acc_it >> 1) & 1;
         if (!mbar_wait(&bars->acc_empty[a], aph ^ 1, limit, abort_flag)) {
@@ -279,19 +376,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after_sync();
+          // A rows may have been written by cp.async: order them before the
+          // tensor core's (async-proxy) reads
+          if (MODE == kModeGemm1) fence_proxy_async_smem();
           const uint64_t a_desc = smem_desc_sw128(smem_addr(sA + s * kABytes));
           const uint64_t b_desc = smem_desc_sw128(smem_addr(sB + s * kBBytes));
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             // +32 bytes of K per step, in 16-byte units of the start address
-            umma_f16(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, idesc, (kb | kk) != 0);
+            if (CG == 2)
+              umma_f16_pair(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, idesc, (kb | kk) != 0);
+            else
+              umma_f16(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, idesc, (kb | kk) != 0);
           }
-          umma_commit(&bars->empty[s]);
+          if (CG == 2)
+            umma_commit_pair(&bars->empty[s], kBothCtas);
+          else
+            umma_commit(&bars->empty[s]);
         }
-        if (!stop) umma_commit(&bars->acc_full[a]);
+        if (!stop) {
+          if (CG == 2)
+            umma_commit_pair(&bars->acc_full[a], kBothCtas);
+          else
+            umma_commit(&bars->acc_full[a]);
+        }
       }
       // every MMA must be complete before TMEM is released
-      umma_commit(&bars->drain);
+      if (CG == 2)
+        umma_commit_pair(&bars->drain, kBothCtas);
+      else
+        umma_commit(&bars->drain);
+      if (!mbar_wait(&bars->drain, 0, limit)) give_up(p, abort_flag);
+    } else if (lane == 0) {
+      // rank 1 of a pair: wait for the pair's MMAs to finish with this TMEM
       if (!mbar_wait(&bars->drain, 0, limit)) give_up(p, abort_flag);
     }
     __syncwarp();
@@ -299,8 +416,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter accessible to this warp
     const int row = q * 32 + lane;
-    int acc_it = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++acc_it) {
+    uint8_t *ebuf = sEpi + q * 2 * kEpiBlock;  // GEMM2: this warp's two staging blocks
+    int acc_it = 0, nstore = 0;
+    for (int t = unit; t < total; t += nunits, ++acc_it) {
       const int a = acc_it & 1;
       const uint32_t aph = (acc_it >> 1) & 1;
       if (!mbar_wait(&bars->acc_full[a], aph, limit, abort_flag)) {
@@ -308,12 +426,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after_sync();
-      const Tile tl = decode_tile(t, NT, p.E, s_tile_off, s_exp_off);
-      const bool valid = row < tl.rows;
+      const Tile tl = decode_tile<TM>(t, NT, p.E, s_tile_off, s_exp_off);
+      const int my_row0 = tl.row0 + static_cast<int>(rank) * BM;
+      const int my_rows = min(BM, max(0, tl.rows - static_cast<int>(rank) * BM));
+      const bool valid = row < my_rows;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kAccN;
       if (MODE == kModeGemm1) {
         __nv_bfloat16 *dst =
-            p.act + static_cast<size_t>(tl.row0 + (valid ? row : 0)) * p.I + tl.nt * (kAccN / 2);
+            p.act + static_cast<size_t>(my_row0 + (valid ? row : 0)) * p.I + tl.nt * (kAccN / 2);
 #pragma unroll 1
         for (int c0 = 0; c0 < kAccN / 2; c0 += 32) {
           uint32_t g[32], u[32];
@@ -335,15 +455,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        const int32_t flat = valid ? p.sorted_rows[tl.row0 + row] : 0;
-        float *dst = p.P + static_cast<size_t>(flat) * p.H + tl.nt * kAccN;
+        // this warp's 32 rows: whole blocks go out through TMA stores
+        const bool whole = q * 32 + 32 <= my_rows;
 #pragma unroll 1
         for (int c0 = 0; c0 < kAccN; c0 += 32) {
           uint32_t v[32];
           tmem_ld_32cols(tbase + c0, v);
           tmem_ld_wait();
-          if (valid && tl.nt * kAccN + c0 < p.H) {
-            float4 *d4 = reinterpret_cast<float4 *>(dst + c0);
+          const int col = tl.nt * kAccN + c0;
+          if (whole) {
+            uint8_t *blk = ebuf + (nstore & 1) * kEpiBlock;
+            // the store issued two blocks ago from this buffer must have read it
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+            // row `lane` as 8 chunks of 16 bytes, 128-byte swizzle
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4 *>(blk + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                  make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tm_out, blk, col, my_row0 + q * 32);
+              bulk_commit_group();
+            }
+            ++nstore;
+          } else if (valid && col < p.H) {
+            // the block crosses the end of the expert's rows: plain stores
+            float4 *d4 = reinterpret_cast<float4 *>(
+                p.P + static_cast<size_t>(my_row0 + row) * p.H + col);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               d4[i] = make_float4(as_f32(v[4 * i]), as_f32(v[4 * i + 1]), as_f32(v[4 * i + 2]),
@@ -353,15 +493,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->acc_empty[a]);
+      if (lane == 0) {
+        if (CG == 2)
+          mbar_arrive_cluster(acc_empty0 + 8u * a);
+        else
+          mbar_arrive(&bars->acc_empty[a]);
+      }
     }
+    if (MODE == kModeGemm2 && lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before_sync();
   __syncthreads();
+  // neither CTA may leave (or free TMEM) while its peer can still reach it
+  if (CG == 2) cluster_sync();
   if (warp == kMmaWarp) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if (CG == 2)
+      tmem_dealloc_pair(tmem_base, kTmemCols);
+    else
+      tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -397,25 +548,37 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major bf16 matrix [outer, inner] as a 2-D tensor map with a
-// (64 x box_rows) box and the 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
-              uint32_t box_rows) {
+// Row-major matrix [outer, inner] as a 2-D tensor map with a
+// (box_inner x box_rows) box and the 128-byte swizzle.
+bool make_map(CUtensorMap *m, CUtensorMapDataType dtype, int elem_bytes, const void *base,
+              uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {inner * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
+  const cuuint64_t strides[1] = {inner * elem_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return enc(m, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int grid_for(const GroupedGemmArgs &a, int n_tiles_n) {
+bool make_bf16_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
+                   uint32_t box_rows) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, inner, outer, BK, box_rows);
+}
+
+int g_max_pairs[64] = {};  // 2-CTA clusters of GEMM2 resident at once, per device
+
+template <int MODE>
+int grid_for(const GroupedGemmArgs &a, int n_tiles_n, int device) {
+  constexpr int CG = Cfg<MODE>::CG;
   const int64_t rows = a.T * a.k;
-  const int64_t max_tiles = ((rows + BM - 1) / BM + a.E) * n_tiles_n;
-  return static_cast<int>(max_tiles < a.num_sms ? max_tiles : a.num_sms);
+  const int64_t max_tiles = ((rows + tile_m<MODE>() - 1) / tile_m<MODE>() + a.E) * n_tiles_n;
+  int units = a.num_sms / CG;
+  if (CG == 2 && device >= 0 && device < 64 && g_max_pairs[device] > 0) units = g_max_pairs[device];
+  if (max_tiles < units) units = static_cast<int>(max_tiles);
+  return CG * (units > 0 ? units : 1);
 }
 
 Params base_params(const GroupedGemmArgs &a) {
@@ -423,7 +586,6 @@ Params base_params(const GroupedGemmArgs &a) {
   p.hidden = reinterpret_cast<const __nv_bfloat16 *>(a.hidden);
   p.sorted_rows = a.sorted_rows;
   p.expert_offsets = a.expert_offsets;
-  p.tile_offsets = a.tile_offsets;
   p.act = reinterpret_cast<__nv_bfloat16 *>(a.act);
   p.P = a.P;
   p.H = a.H;
@@ -435,6 +597,31 @@ Params base_params(const GroupedGemmArgs &a) {
   return p;
 }
 
+template <int MODE>
+cudaLaunchConfig_t launch_config(int grid, cudaStream_t s, bool pdl, cudaLaunchAttribute (&attr)[2]) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem_bytes<MODE>();
+  cfg.stream = s;
+  int n = 0;
+  if (Cfg<MODE>::CG == 2) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = 2;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cfg;
+}
+
 }  // namespace
 
 cudaError_t grouped_gemm_setup(int device) {
@@ -444,45 +631,68 @@ cudaError_t grouped_gemm_setup(int device) {
   if (device >= 0 && device < 64 && (done_mask >> device) & 1) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<kModeGemm1>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes));
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(grouped_gemm_kernel<kModeGemm2>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kSmemBytes));
+                                       static_cast<int>(smem_bytes<kModeGemm1>()));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(grouped_gemm_kernel<kModeGemm2>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_bytes<kModeGemm2>()));
   if (e != cudaSuccess) return e;
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
-  if (device >= 0 && device < 64) done_mask |= 1ull << device;
+  // how many 2-CTA clusters of GEMM2 can be resident at once
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = launch_config<kModeGemm2>(2, nullptr, false, attr);
+  int clusters = 0;
+  e = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<kModeGemm2>, &cfg);
+  if (e != cudaSuccess || clusters < 1) {
+    cudaGetLastError();
+    return e != cudaSuccess ? e : cudaErrorNotSupported;
+  }
+  if (device >= 0 && device < 64) {
+    g_max_pairs[device] = clusters;
+    done_mask |= 1ull << device;
+  }
   return cudaSuccess;
 }
 
 cudaError_t launch_gemm1_swiglu(const GroupedGemmArgs &a, cudaStream_t s, const StageHook &hook) {
   CUtensorMap tm_w1;
-  if (!make_map(&tm_w1, a.w1, static_cast<uint64_t>(a.H), static_cast<uint64_t>(a.E) * 2 * a.I,
-                kAccN / 2))
+  if (!make_bf16_map(&tm_w1, a.w1, static_cast<uint64_t>(a.H),
+                     static_cast<uint64_t>(a.E) * 2 * a.I, kAccN / 2))
     return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaGetDevice(&dev);
   Params p = base_params(a);
   p.K = a.H;
   p.n_tiles_n = a.I / (kAccN / 2);
   p.b_rows_per_expert = 2 * a.I;
+  cudaLaunchAttribute attr[2];
+  const cudaLaunchConfig_t cfg =
+      launch_config<kModeGemm1>(grid_for<kModeGemm1>(a, p.n_tiles_n, dev), s, hook.pdl, attr);
   hook.begin("gemm1_swiglu");
-  cudaError_t e = launch_pdl(grouped_gemm_kernel<kModeGemm1>, dim3(grid_for(a, p.n_tiles_n)),
-                             dim3(kThreads), kSmemBytes, s, hook.pdl, tm_w1, tm_w1, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm1>, tm_w1, tm_w1, tm_w1, p);
   return hook.end(e);
 }
 
 cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s, const StageHook &hook) {
-  CUtensorMap tm_act, tm_w2;
-  if (!make_map(&tm_act, a.act, static_cast<uint64_t>(a.I), static_cast<uint64_t>(a.T) * a.k, BM))
+  CUtensorMap tm_act, tm_w2, tm_p;
+  const uint64_t rows = static_cast<uint64_t>(a.T) * a.k;
+  if (!make_bf16_map(&tm_act, a.act, static_cast<uint64_t>(a.I), rows, BM) ||
+      !make_bf16_map(&tm_w2, a.w2, static_cast<uint64_t>(a.I), static_cast<uint64_t>(a.E) * a.H,
+                     Cfg<kModeGemm2>::kBRows) ||
+      !make_map(&tm_p, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.P, static_cast<uint64_t>(a.H), rows,
+                32, 32))
     return cudaErrorInvalidValue;
-  if (!make_map(&tm_w2, a.w2, static_cast<uint64_t>(a.I), static_cast<uint64_t>(a.E) * a.H, kAccN))
-    return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaGetDevice(&dev);
   Params p = base_params(a);
   p.K = a.I;
   p.n_tiles_n = (a.H + kAccN - 1) / kAccN;  // H % 128 == 0: a last half tile is masked
   p.b_rows_per_expert = a.H;
+  cudaLaunchAttribute attr[2];
+  const cudaLaunchConfig_t cfg =
+      launch_config<kModeGemm2>(grid_for<kModeGemm2>(a, p.n_tiles_n, dev), s, hook.pdl, attr);
   hook.begin("gemm2");
-  cudaError_t e = launch_pdl(grouped_gemm_kernel<kModeGemm2>, dim3(grid_for(a, p.n_tiles_n)),
-                             dim3(kThreads), kSmemBytes, s, hook.pdl, tm_act, tm_w2, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm2>, tm_act, tm_w2, tm_p, p);
   return hook.end(e);
 }
 

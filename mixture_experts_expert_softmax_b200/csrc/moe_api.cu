@@ -241,11 +241,10 @@ int moe_permute(const int32_t *topk_ids, int64_t T, int k, int E, int32_t *sorte
   if ((rc = ensure_workspace(*d, permute_ws_bytes(n, E))) != MOE_OK) return rc;
   Carver cv{static_cast<char *>(d->ws)};
   int32_t *chunk_counts = cv.take<int32_t>(std::max(moe::permute_num_chunks(n), 1) * static_cast<size_t>(E));
-  int32_t *tile_offsets = cv.take<int32_t>(E + 1);
   CallCtx ctx{static_cast<cudaStream_t>(stream), "", nullptr};
   moe::StageHook hook = make_hook(&ctx);
-  cudaError_t e = moe::launch_permute(topk_ids, n, E, moe::kGemmTileM, chunk_counts,
-                                      expert_offsets, tile_offsets, sorted_rows, ctx.stream, hook);
+  cudaError_t e = moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets, sorted_rows,
+                                      nullptr, ctx.stream, hook);
   return to_code(e);
 }
 
@@ -267,30 +266,31 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
   CallCtx ctx{static_cast<cudaStream_t>(stream), "", nullptr};
   moe::StageHook hook = make_hook(&ctx);
 
-  if (T <= small_t_max()) {
+  if (T <= small_t_max() && moe::small_t_supported(H, I)) {
     const size_t need = align256(static_cast<size_t>(n) * I * sizeof(float));
     if ((rc = ensure_workspace(*d, need)) != MOE_OK) return rc;
     Carver cv{static_cast<char *>(d->ws)};
     float *act = cv.take<float>(static_cast<size_t>(n) * I);
     return to_code(moe::launch_small_t(hidden, w1, w2, topk_weights, topk_ids, act, out, T, H, I,
-                                       E, k, d->status, ctx.stream, hook));
+                                       E, k, d->status,
+                                       static_cast<uint64_t>(g_wait_limit_ns), ctx.stream, hook));
   }
 
-  const size_t need = permute_ws_bytes(n, E) + align256((E + 1) * sizeof(int32_t)) +
+  const size_t need = permute_ws_bytes(n, E) + align256(static_cast<size_t>(n) * 4) +
                       align256(static_cast<size_t>(n) * I * 2) +
                       align256(static_cast<size_t>(n) * H * sizeof(float));
   if ((rc = ensure_workspace(*d, need)) != MOE_OK) return rc;
   Carver cv{static_cast<char *>(d->ws)};
   int32_t *chunk_counts =
       cv.take<int32_t>(std::max(moe::permute_num_chunks(n), 1) * static_cast<size_t>(E));
-  int32_t *tile_offsets = cv.take<int32_t>(E + 1);
   int32_t *sorted_rows = cv.take<int32_t>(std::max<int64_t>(n, 1));
+  int32_t *inv = cv.take<int32_t>(std::max<int64_t>(n, 1));
   int32_t *expert_offsets = cv.take<int32_t>(E + 1);
   uint16_t *act = cv.take<uint16_t>(static_cast<size_t>(n) * I);
   float *P = cv.take<float>(static_cast<size_t>(n) * H);
 
-  cudaError_t e = moe::launch_permute(topk_ids, n, E, moe::kGemmTileM, chunk_counts,
-                                      expert_offsets, tile_offsets, sorted_rows, ctx.stream, hook);
+  cudaError_t e = moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets, sorted_rows,
+                                      inv, ctx.stream, hook);
   if (e != cudaSuccess) return to_code(e);
   moe::GroupedGemmArgs ga;
   ga.hidden = hidden;
@@ -298,7 +298,6 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
   ga.w2 = w2;
   ga.sorted_rows = sorted_rows;
   ga.expert_offsets = expert_offsets;
-  ga.tile_offsets = tile_offsets;
   ga.act = act;
   ga.P = P;
   ga.T = T;
@@ -311,7 +310,7 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
   ga.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns);
   if ((e = moe::launch_gemm1_swiglu(ga, ctx.stream, hook)) != cudaSuccess) return to_code(e);
   if ((e = moe::launch_gemm2(ga, ctx.stream, hook)) != cudaSuccess) return to_code(e);
-  e = moe::launch_combine(P, topk_weights, topk_ids, out, T, H, E, k, d->status, ctx.stream, hook);
+  e = moe::launch_combine(P, inv, topk_weights, out, T, H, k, d->status, ctx.stream, hook);
   return to_code(e);
 }
 

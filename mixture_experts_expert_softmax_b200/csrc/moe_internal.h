@@ -44,21 +44,19 @@ cudaError_t launch_route(const float *logits, int64_t T, int E, int k, int renor
 
 // permute.cu
 int permute_num_chunks(int64_t n);
-cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int tile_m,
-                           int32_t *chunk_counts, int32_t *expert_offsets, int32_t *tile_offsets,
-                           int32_t *sorted_rows, cudaStream_t s, const StageHook &hook);
+cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int32_t *chunk_counts,
+                           int32_t *expert_offsets, int32_t *sorted_rows, int32_t *inv,
+                           cudaStream_t s, const StageHook &hook);
 
 // grouped_gemm.cu
-constexpr int kGemmTileM = 128;
 struct GroupedGemmArgs {
   const uint16_t *hidden;  // [T, H] bf16
   const uint16_t *w1;      // [E, 2I, H] bf16
   const uint16_t *w2;      // [E, H, I] bf16
   const int32_t *sorted_rows;
   const int32_t *expert_offsets;
-  const int32_t *tile_offsets;
   uint16_t *act;  // [T*k, I] bf16, expert-sorted rows
-  float *P;       // [T*k, H] fp32, flat (t*k + j) rows
+  float *P;       // [T*k, H] fp32, expert-sorted rows
   int64_t T;
   int H, I, E, k;
   int num_sms;
@@ -71,14 +69,15 @@ cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s, const StageHo
 cudaError_t launch_wait_probe(uint32_t *status, uint64_t limit_ns, cudaStream_t s);
 
 // combine.cu
-cudaError_t launch_combine(const float *P, const float *topk_weights, const int32_t *topk_ids,
-                           float *out, int64_t T, int H, int E, int k, uint32_t *status,
-                           cudaStream_t s, const StageHook &hook);
+cudaError_t launch_combine(const float *P, const int32_t *inv, const float *topk_weights,
+                           float *out, int64_t T, int H, int k, uint32_t *status, cudaStream_t s,
+                           const StageHook &hook);
 
 // small_t.cu
+bool small_t_supported(int H, int I);
 cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
                            const float *topk_weights, const int32_t *topk_ids, float *act,
                            float *out, int64_t T, int H, int I, int E, int k, uint32_t *status,
-                           cudaStream_t s, const StageHook &hook);
+                           uint64_t wait_limit_ns, cudaStream_t s, const StageHook &hook);
 
 }  // namespace moe

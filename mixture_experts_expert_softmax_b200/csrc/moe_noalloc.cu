@@ -44,7 +44,8 @@ extern "C" int moe_forward_small_noalloc(const uint16_t *hidden, const uint16_t 
   if (T > 0 && (hidden == nullptr || w1 == nullptr || w2 == nullptr || topk_weights == nullptr ||
                 topk_ids == nullptr || out == nullptr))
     return MOE_ERR_INVALID_ARG;
-  if (H % 128 != 0 || I % 128 != 0 || E > 1024 || k > 16) return MOE_ERR_UNSUPPORTED;
+  if (H % 128 != 0 || I % 128 != 0 || E > 1024 || k > 16 || !moe::small_t_supported(H, I))
+    return MOE_ERR_UNSUPPORTED;
   if (T > MOE_NOALLOC_MAX_T ||
       T * static_cast<int64_t>(k) * static_cast<int64_t>(I) > MOE_NOALLOC_MAX_ACT)
     return MOE_ERR_SCRATCH_LIMIT;
@@ -80,7 +81,7 @@ extern "C" int moe_forward_small_noalloc(const uint16_t *hidden, const uint16_t 
   hook.pdl = true;
   const cudaError_t e =
       moe::launch_small_t(hidden, w1, w2, topk_weights, topk_ids, act, out, T, H, I, E, k, status,
-                          static_cast<cudaStream_t>(stream), hook);
+                          2000000000ull, static_cast<cudaStream_t>(stream), hook);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;

@@ -44,15 +44,12 @@ __global__ void __launch_bounds__(kPermThreads)
 }
 
 // One CTA of 1024 threads.  Turns chunk_counts into per-chunk exclusive
-// bases (in place), writes expert_offsets[E+1] (exclusive scan of the
-// totals) and tile_offsets[E+1] (exclusive scan of ceil(count / tile_m),
-// the m-tiles of each expert in the grouped GEMMs).
+// bases (in place) and writes expert_offsets[E+1] (exclusive scan of the
+// per-expert totals).
 __global__ void __launch_bounds__(1024)
-    permute_scan_kernel(int32_t *__restrict__ chunk_counts, int n_chunks, int E, int tile_m,
-                        int32_t *__restrict__ expert_offsets,
-                        int32_t *__restrict__ tile_offsets) {
+    permute_scan_kernel(int32_t *__restrict__ chunk_counts, int n_chunks, int E,
+                        int32_t *__restrict__ expert_offsets) {
   __shared__ int32_t s_warp_cnt[32];
-  __shared__ int32_t s_warp_tiles[32];
   grid_dep_wait();
   grid_dep_launch();
   const int e = threadIdx.x;
@@ -65,58 +62,39 @@ __global__ void __launch_bounds__(1024)
       total += x;
     }
   }
-  const int32_t tiles = (total + tile_m - 1) / tile_m;
-  // block-wide inclusive scans of (total, tiles)
+  // block-wide inclusive scan of the totals
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int32_t a = total, b = tiles;
+  int32_t a = total;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int32_t xa = __shfl_up_sync(0xffffffffu, a, o);
-    const int32_t xb = __shfl_up_sync(0xffffffffu, b, o);
-    if (lane >= o) {
-      a += xa;
-      b += xb;
-    }
+    if (lane >= o) a += xa;
   }
-  if (lane == 31) {
-    s_warp_cnt[warp] = a;
-    s_warp_tiles[warp] = b;
-  }
+  if (lane == 31) s_warp_cnt[warp] = a;
   __syncthreads();
   if (warp == 0) {
-    int32_t wa = s_warp_cnt[lane], wb = s_warp_tiles[lane];
+    int32_t wa = s_warp_cnt[lane];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int32_t xa = __shfl_up_sync(0xffffffffu, wa, o);
-      const int32_t xb = __shfl_up_sync(0xffffffffu, wb, o);
-      if (lane >= o) {
-        wa += xa;
-        wb += xb;
-      }
+      if (lane >= o) wa += xa;
     }
     s_warp_cnt[lane] = wa;
-    s_warp_tiles[lane] = wb;
   }
   __syncthreads();
   const int32_t incl_a = a + (warp > 0 ? s_warp_cnt[warp - 1] : 0);
-  const int32_t incl_b = b + (warp > 0 ? s_warp_tiles[warp - 1] : 0);
-  if (e < E) {
-    expert_offsets[e] = incl_a - total;
-    tile_offsets[e] = incl_b - tiles;
-  }
-  if (e == E - 1) {
-    expert_offsets[E] = incl_a;
-    tile_offsets[E] = incl_b;
-  }
+  if (e < E) expert_offsets[e] = incl_a - total;
+  if (e == E - 1) expert_offsets[E] = incl_a;
 }
 
-// Writes sorted_rows[pos] = i for every valid entry.  Shared memory holds
-// one running base per (warp, expert).
+// Writes sorted_rows[pos] = i for every valid entry and, when inv is given,
+// its inverse inv[i] = pos (-1 for an id outside [0, E)).  Shared memory
+// holds one running base per (warp, expert).
 __global__ void __launch_bounds__(kPermThreads)
     permute_scatter_kernel(const int32_t *__restrict__ ids, int64_t n, int E,
                            const int32_t *__restrict__ chunk_bases,
                            const int32_t *__restrict__ expert_offsets,
-                           int32_t *__restrict__ sorted_rows) {
+                           int32_t *__restrict__ sorted_rows, int32_t *__restrict__ inv) {
   extern __shared__ int32_t wbase[];  // [kPermWarps][E]
   grid_dep_wait();
   grid_dep_launch();
@@ -152,10 +130,12 @@ __global__ void __launch_bounds__(kPermThreads)
       if (e < 0 || e >= E) e = -1;
     }
     const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    int32_t pos = -1;
     if (e >= 0) {
-      const int32_t pos = mine[e] + __popc(peers & lt_mask);
+      pos = mine[e] + __popc(peers & lt_mask);
       sorted_rows[pos] = static_cast<int32_t>(i);
     }
+    if (inv != nullptr && i < n) inv[i] = pos;
     __syncwarp();
     if (e >= 0 && (peers & lt_mask) == 0) mine[e] += __popc(peers);
     __syncwarp();
@@ -166,9 +146,9 @@ __global__ void __launch_bounds__(kPermThreads)
 
 int permute_num_chunks(int64_t n) { return static_cast<int>((n + kChunk - 1) / kChunk); }
 
-cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int tile_m,
-                           int32_t *chunk_counts, int32_t *expert_offsets, int32_t *tile_offsets,
-                           int32_t *sorted_rows, cudaStream_t s, const StageHook &hook) {
+cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int32_t *chunk_counts,
+                           int32_t *expert_offsets, int32_t *sorted_rows, int32_t *inv,
+                           cudaStream_t s, const StageHook &hook) {
   const int n_chunks = permute_num_chunks(n);
   cudaError_t err;
   if (n_chunks > 0) {
@@ -181,14 +161,14 @@ cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int tile_m,
   }
   hook.begin("permute_scan");
   err = launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, s, hook.pdl, chunk_counts,
-                   n_chunks, E, tile_m, expert_offsets, tile_offsets);
+                   n_chunks, E, expert_offsets);
   if ((err = hook.end(err)) != cudaSuccess) return err;
   if (n_chunks > 0) {
     hook.begin("permute_scatter");
     err = launch_pdl(permute_scatter_kernel, dim3(n_chunks), dim3(kPermThreads),
                      static_cast<size_t>(kPermWarps) * E * sizeof(int32_t), s, hook.pdl, ids, n,
                      E, static_cast<const int32_t *>(chunk_counts),
-                     static_cast<const int32_t *>(expert_offsets), sorted_rows);
+                     static_cast<const int32_t *>(expert_offsets), sorted_rows, inv);
     if ((err = hook.end(err)) != cudaSuccess) return err;
   }
   return cudaSuccess;
