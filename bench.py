@@ -13,7 +13,9 @@ top-k 2); the other shapes are reported under "per_shape".
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
 device synchronise on both sides; each step is timed with CUDA events on the
 launching stream, and a 256 MiB buffer is written between steps (untimed) so
-that every step starts with a cold L2.  Multi-GPU (torchrun): one independent
+that every step starts with a cold L2 (then 256 MiB are read, so
+that L2 holds clean lines only: the step does not pay for writing back the
+flush's dirty lines).  Multi-GPU (torchrun): one independent
 replica per GPU, no collective in the data path; the time is the max over
 ranks and `value` counts the work of all ranks.
 
@@ -205,12 +207,16 @@ def run_ours(args, ws, rank, local):
     hidden, w1, w2, logits = make_shape_inputs(s, seed=0, device=str(dev))
     stream = torch.cuda.current_stream()
     flush_buf = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_read = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     ids = torch.empty(s.T, s.k, dtype=torch.int32, device=dev)
     wts = torch.empty(s.T, s.k, dtype=torch.float32, device=dev)
     out = torch.empty(s.T, s.H, dtype=torch.float32, device=dev)
 
     def flush():
+        # evict everything: write 256 MiB (twice L2), then read another
+        # 256 MiB so that L2 holds only clean lines when the step starts
         flush_buf.zero_()
+        flush_read.sum()
 
     def step(ev):
         if ev is not None:
@@ -307,7 +313,7 @@ def run_ours(args, ws, rank, local):
         "data": "synthetic (seeded randn, shapes and scales of atrex-bench #009 input.py)",
         "config": {"workload": s.name, "T": s.T, "H": s.H, "I": s.I, "E": s.E, "top_k": s.k,
                    "renorm": True, "active_experts": n_active,
-                   "l2": "flushed between steps (256 MiB write, untimed)",
+                   "l2": "flushed between steps (256 MiB write + 256 MiB read, untimed)",
                    "step": "moe_route + moe_forward", "parallelism": f"replicas x{ws}"},
         "roofline": roof,
         "kernels": {k: {"launches": v["launches"], "avg_us": round(v["avg_us"], 2)}

@@ -86,14 +86,17 @@ int moe_route(const float *logits, int64_t T, int E, int k, int renorm,
  *   topk_ids      [T, k] int32; ids outside [0, E) are skipped and flagged
  *                 with MOE_STATUS_BAD_ID in the device status word
  *   out           [T, H] fp32, every element overwritten:
- *                 out[t] = sum over j = 0..k-1 (in that order) of
+ *                 out[t] = sum over j = 0..k-1 of
  *                          topk_weights[t, j] * FFN_{topk_ids[t, j]}(hidden[t]),
- *                 accumulated in fp32; a row with no valid id is 0.
+ *                 accumulated in fp32 in a fixed order (grouped-GEMM path:
+ *                 ascending j; small-T path: per column slice in ascending
+ *                 expert order, then a fixed tree); a row with no valid id
+ *                 is 0.
  * Numerics: bf16 inputs, fp32 accumulation; the SwiGLU intermediate is
  * rounded to bf16 before the second projection on the grouped-GEMM path
- * and kept in fp32 on the small-T path (T <= the small-T limit, H <= 6144
+ * and kept in fp32 on the small-T path (T <= the small-T limit, H <= 4096
  * and I <= 12288).  The combine is
- * deterministic (fixed j order, no atomics): repeated calls give identical
+ * deterministic (fixed order, no atomics): repeated calls give identical
  * bits.
  * Errors: INVALID_ARG for null pointers, T < 0, H/I/E < 1, k < 1 or k > E;
  *         UNSUPPORTED unless H % 128 == 0 and I % 128 == 0 (the alignment
@@ -119,14 +122,16 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
  * loads the library holds until the process exits.
  *   - Limits: T <= MOE_NOALLOC_MAX_T and T*k*I <= MOE_NOALLOC_MAX_ACT, else
  *     MOE_ERR_SCRATCH_LIMIT and nothing is launched.  Other checks and
- *     codes as in moe_forward, plus UNSUPPORTED when H > 6144 or I > 12288
+ *     codes as in moe_forward, plus UNSUPPORTED when H > 4096 or I > 12288
  *     (the largest rows the small-T kernels stage).
  *   - The first call on each device, with that device current, looks up
  *     the array's device address (cudaGetSymbolAddress) and caches it; make
  *     that first call before any stream capture.
  *   - All calls share the one array, which keeps the last call's contents:
  *     calls whose kernels overlap on the GPU (e.g. on two streams without
- *     ordering) race on it.  Nothing in it has to start at zero.
+ *     ordering) race on it.  Nothing in it has to be cleared between calls
+ *     (its grid-barrier counter starts at zero when the library loads and
+ *     every call advances it).
  *   - Expert ids outside [0, E) are skipped as in moe_forward, but the bad-id
  *     flag is not reported through moe_get_device_status.
  *   - Calls no cudaMalloc, cudaFree or other allocating routine.

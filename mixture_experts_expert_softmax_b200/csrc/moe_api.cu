@@ -24,7 +24,8 @@ struct DeviceState {
   bool checked = false;
   bool usable = false;
   int num_sms = 0;
-  uint32_t *status = nullptr;  // device status word (never reallocated)
+  uint32_t *status = nullptr;  // 256 B: status word at 0, small-T grid counter at 64
+  unsigned long long small_t_launches = 0;
   void *ws = nullptr;          // grow-only workspace
   size_t ws_bytes = 0;
 };
@@ -271,9 +272,10 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
     if ((rc = ensure_workspace(*d, need)) != MOE_OK) return rc;
     Carver cv{static_cast<char *>(d->ws)};
     float *act = cv.take<float>(static_cast<size_t>(n) * I);
-    return to_code(moe::launch_small_t(hidden, w1, w2, topk_weights, topk_ids, act, out, T, H, I,
-                                       E, k, d->status,
-                                       static_cast<uint64_t>(g_wait_limit_ns), ctx.stream, hook));
+    return to_code(moe::launch_small_t(
+        hidden, w1, w2, topk_weights, topk_ids, act, out, T, H, I, E, k, d->status,
+        reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(d->status) + 64),
+        &d->small_t_launches, static_cast<uint64_t>(g_wait_limit_ns), ctx.stream, hook));
   }
 
   const size_t need = permute_ws_bytes(n, E) + align256(static_cast<size_t>(n) * 4) +
@@ -289,8 +291,13 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
   uint16_t *act = cv.take<uint16_t>(static_cast<size_t>(n) * I);
   float *P = cv.take<float>(static_cast<size_t>(n) * H);
 
-  cudaError_t e = moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets, sorted_rows,
-                                      inv, ctx.stream, hook);
+  // the forward's result does not depend on the order of rows inside an
+  // expert, so a single-CTA grouping replaces the stable three-kernel one
+  cudaError_t e = moe::permute_fused_supported(n)
+                      ? moe::launch_permute_fused(topk_ids, n, E, expert_offsets, sorted_rows,
+                                                  inv, ctx.stream, hook)
+                      : moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets,
+                                            sorted_rows, inv, ctx.stream, hook);
   if (e != cudaSuccess) return to_code(e);
   moe::GroupedGemmArgs ga;
   ga.hidden = hidden;

@@ -48,6 +48,11 @@ cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int32_t *chunk_
                            int32_t *expert_offsets, int32_t *sorted_rows, int32_t *inv,
                            cudaStream_t s, const StageHook &hook);
 
+bool permute_fused_supported(int64_t n);
+cudaError_t launch_permute_fused(const int32_t *ids, int64_t n, int E, int32_t *expert_offsets,
+                                 int32_t *sorted_rows, int32_t *inv, cudaStream_t s,
+                                 const StageHook &hook);
+
 // grouped_gemm.cu
 struct GroupedGemmArgs {
   const uint16_t *hidden;  // [T, H] bf16
@@ -75,9 +80,13 @@ cudaError_t launch_combine(const float *P, const int32_t *inv, const float *topk
 
 // small_t.cu
 bool small_t_supported(int H, int I);
+// grid_sync: a 64-bit device counter that only this launcher's kernels
+// touch, 0 before the first launch; launches: host count of launches made
+// with it (advanced by the call).
 cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
                            const float *topk_weights, const int32_t *topk_ids, float *act,
                            float *out, int64_t T, int H, int I, int E, int k, uint32_t *status,
+                           unsigned long long *grid_sync, unsigned long long *launches,
                            uint64_t wait_limit_ns, cudaStream_t s, const StageHook &hook);
 
 }  // namespace moe

@@ -27,12 +27,15 @@ constexpr size_t kStatusBytes = 256;
 constexpr size_t kScratchBytes =
     kStatusBytes + static_cast<size_t>(MOE_NOALLOC_MAX_ACT) * sizeof(float);
 
-// [0, 256): status word the kernels may raise bits in (not reported back);
+// [0, 256): status word the kernel may raise bits in (not reported back) at
+// byte 0, and at byte 64 the kernel's grid-barrier counter, which starts at
+// zero when the module loads and is advanced by every call;
 // [256, ...): the act scratch, T*k*I fp32 values.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 std::mutex g_noalloc_mu;
 void *g_noalloc_addr[kNoAllocMaxDevices] = {};
+unsigned long long g_noalloc_launches[kNoAllocMaxDevices] = {};
 
 }  // namespace
 
@@ -61,8 +64,8 @@ extern "C" int moe_forward_small_noalloc(const uint16_t *hidden, const uint16_t 
   if (major != 10 || minor != 0) return MOE_ERR_NO_DEVICE;
 
   void *base = nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
   {
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
     if (g_noalloc_addr[dev] == nullptr) {
       void *p = nullptr;
       if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
@@ -73,15 +76,19 @@ extern "C" int moe_forward_small_noalloc(const uint16_t *hidden, const uint16_t 
     }
     base = g_noalloc_addr[dev];
   }
-  // Nothing here has to start at zero: every act value the second kernel
-  // reads is written by the first kernel of the same call.
+  // Nothing has to be cleared between calls: every act value the second
+  // phase reads is written by the first phase of the same call, and the
+  // grid-barrier counter only ever advances.
   uint32_t *status = static_cast<uint32_t *>(base);
+  unsigned long long *grid_sync =
+      reinterpret_cast<unsigned long long *>(static_cast<char *>(base) + 64);
   float *act = reinterpret_cast<float *>(static_cast<char *>(base) + kStatusBytes);
   moe::StageHook hook;
   hook.pdl = true;
   const cudaError_t e =
       moe::launch_small_t(hidden, w1, w2, topk_weights, topk_ids, act, out, T, H, I, E, k, status,
-                          2000000000ull, static_cast<cudaStream_t>(stream), hook);
+                          grid_sync, &g_noalloc_launches[dev], 2000000000ull,
+                          static_cast<cudaStream_t>(stream), hook);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;

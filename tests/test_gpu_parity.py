@@ -293,8 +293,7 @@ def test_sync_each_stage_mode_and_profiler():
         moe.profile_enable(False)
         moe.set_sync_each_stage(prev)
     prof = moe.profile_read()
-    for kname in ("permute_count", "permute_scan", "permute_scatter", "gemm1_swiglu", "gemm2",
-                  "combine"):
+    for kname in ("permute", "gemm1_swiglu", "gemm2", "combine"):
         assert prof[kname][0] == 1 and prof[kname][1] > 0
     ref = oracle.moe_token_loop(hidden, w1, w2, w, ids)
     assert_output_close(out, ref)
