@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(kPermThreads)
 // the fixed-order combine do not depend on where a row sits), and the
 // exported stable grouping uses the three kernels above.
 constexpr int kFusedThreads = 1024;
-constexpr int64_t kFusedMaxN = 1 << 17;
+constexpr int64_t kFusedMaxN = 8192;  // above this the multi-CTA kernels are faster
 
 __global__ void __launch_bounds__(kFusedThreads)
     permute_fused_kernel(const int32_t *__restrict__ ids, int n, int E,
