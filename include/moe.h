@@ -88,17 +88,20 @@ int moe_route(const float *logits, int64_t T, int E, int k, int renorm,
  *   out           [T, H] fp32, every element overwritten:
  *                 out[t] = sum over j = 0..k-1 of
  *                          topk_weights[t, j] * FFN_{topk_ids[t, j]}(hidden[t]),
- *                 accumulated in fp32 in a fixed order (grouped-GEMM path:
+ *                 accumulated in fp32 (grouped-GEMM path, k <= 2: out is
+ *                 zeroed and each rounded product w_j * y_j is added at L2,
+ *                 which gives the same bits in either order; k > 2:
  *                 ascending j; small-T path: per column slice in ascending
  *                 expert order, then a fixed tree); a row with no valid id
  *                 is 0.
  * Numerics: bf16 inputs, fp32 accumulation; the SwiGLU intermediate is
  * rounded to bf16 before the second projection on the grouped-GEMM path
  * and kept in fp32 on the small-T path (T <= the small-T limit, H <= 4096
- * and I <= 12288).  The combine is
- * deterministic (fixed order, no atomics): repeated calls give identical
- * bits.
- * Errors: INVALID_ARG for null pointers, T < 0, H/I/E < 1, k < 1 or k > E;
+ * and I <= 12288).  The combine is deterministic: repeated calls give
+ * identical bits.
+ * hidden, w1, w2 and out must start on a 16-byte boundary.
+ * Errors: INVALID_ARG for null pointers, hidden/w1/w2/out not 16-byte
+ *         aligned, T < 0, H/I/E < 1, k < 1 or k > E;
  *         UNSUPPORTED unless H % 128 == 0 and I % 128 == 0 (the alignment
  *         the TPU page also demands), E <= 1024 and k <= 16;
  *         OOM if the workspace cannot grow.  T == 0 launches nothing.

@@ -116,6 +116,16 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *s
                : "memory");
 }
 
+// 1-D bulk reduction shared -> global: dst[i] += src[i] for bytes / 4 fp32
+// values, performed at L2 (bulk-group completion).  Both addresses 16-byte
+// aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_reduce_add_f32(float *dst, const void *src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(dst)),
+               "r"(smem_addr(src)), "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

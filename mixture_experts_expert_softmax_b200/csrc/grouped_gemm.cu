@@ -4,8 +4,12 @@
 //   GEMM1 (+SwiGLU): for the rows of expert e in expert-sorted order,
 //     g = x . w1[e, 0:I, :]^T, u = x . w1[e, I:2I, :]^T  (fp32 in TMEM),
 //     act = silu(g) * u, stored as bf16 [rows, I].
-//   GEMM2: y = act . w2[e]^T (fp32 in TMEM), stored as fp32 rows of P in the
-//     same expert-sorted order; combine.cu then forms sum_j w_j * y_j.
+//   GEMM2: y = act . w2[e]^T (fp32 in TMEM).  For top-k <= 2 the epilogue
+//     adds w_j * y_j of each row straight into out[token] with bulk
+//     reductions at L2 (GEMM1 has zeroed out); out[t] = 0 + a + b is the same
+//     in either arrival order, so the result is still deterministic.  For
+//     larger k it stores y as fp32 rows of P in the same expert-sorted order
+//     and combine.cu forms sum_j w_j * y_j in fixed j order.
 // This is the expert FFN of ref_moe on the page "tpu_inference/kernels/
 // fused_moe/v1/kernel.py" (gate = w1, up = w3, then act . w2) in the weight
 // layout of atrex-bench #009 (w1 [E, 2I, H], w2 [E, H, I], both applied as
@@ -27,10 +31,12 @@
 //   CTA receives its 128 accumulator rows in its own TMEM.  Splitting B
 //   between the pair halves the weight bytes each SM must fetch.  Its
 //   epilogue stages each 32x32 fp32 block in shared memory and writes it
-//   with a TMA store (coalesced, asynchronous); a block that straddles the
-//   end of an expert's rows is written row by row instead.
+//   with a TMA store (coalesced, asynchronous; a block that straddles the
+//   end of an expert's rows is written row by row instead), or, fused with
+//   the combine, scales row r by its top-k weight and issues one 128-byte
+//   bulk reduce-add per row into out.
 //
-// Warp roles (288 threads per CTA):
+// Warp roles (416 threads per CTA):
 //   warps 0-3  producers.  GEMM1: the 128 threads gather the A rows with
 //              16-byte cp.async into the 128-byte-swizzled K-major layout and
 //              arrive on the stage barrier asynchronously when they land;
@@ -40,8 +46,10 @@
 //   warp 4     allocates 512 TMEM columns (two accumulators); one thread (on
 //              rank 0) issues the MMAs and commits each stage back to the
 //              producers and each finished tile to the epilogues.
-//   warps 5-8  epilogue: tcgen05.ld of their 32-lane quarter, SwiGLU + bf16
-//              store, or the fp32 TMA store, then release the accumulator.
+//   warps 5-12 epilogue, two warps per 32-lane TMEM quarter (a warp can only
+//              read the quarter warp_id % 4), each taking half of the tile's
+//              columns: tcgen05.ld, SwiGLU + bf16 store, or the fp32 TMA
+//              store, then release the accumulator.
 // Every wait is bounded; a wait that gives up raises the timeout bit of the
 // status word and makes every role of the CTA leave its loop.
 #include <mutex>
@@ -55,7 +63,8 @@ constexpr int BM = 128;  // rows per CTA
 constexpr int BK = 64;   // K per stage: one 128-byte swizzle row of bf16
 constexpr int kProducerThreads = 128;
 constexpr int kMmaWarp = 4;
-constexpr int kThreads = 9 * 32;
+constexpr int kEpiWarps = 8;  // warps 5..12
+constexpr int kThreads = (5 + kEpiWarps) * 32;
 constexpr int kAccN = 256;            // UMMA N = accumulator columns per tile
 constexpr int kTmemCols = 2 * kAccN;  // double-buffered accumulator
 constexpr int kABytes = BM * BK * 2;  // 16 KB
@@ -63,6 +72,12 @@ constexpr int kMaxE = 1024;
 constexpr int kMaxStages = 6;
 constexpr uint16_t kBothCtas = 0x3;
 constexpr int kEpiBlock = 32 * 32 * 4;  // one 32-row x 32-column fp32 block
+// Per-warp staging: a swizzled kEpiBlock for the P store, or 32 rows at a
+// 144-byte pitch (conflict-free 16-byte writes) for the bulk reductions;
+// 1024-byte multiple so every warp's buffer stays swizzle-aligned.
+constexpr int kRedPitch = 144;
+constexpr int kEpiWarpBytes = 5 * 1024;
+static_assert(32 * kRedPitch <= kEpiWarpBytes && kEpiBlock <= kEpiWarpBytes, "staging");
 
 enum { kModeGemm1 = 0, kModeGemm2 = 1 };
 
@@ -80,7 +95,7 @@ struct Cfg<kModeGemm2> {
   static constexpr int CG = 2;
   static constexpr int kStages = 5;
   static constexpr int kBRows = 128;
-  static constexpr int kEpiBytes = 4 * 2 * kEpiBlock;  // 4 warps x double buffer
+  static constexpr int kEpiBytes = kEpiWarps * kEpiWarpBytes;
 };
 
 template <int MODE>
@@ -121,6 +136,13 @@ struct Params {
   int b_rows_per_expert;  // 2I for w1, H for w2
   uint32_t *status;
   uint64_t wait_limit_ns;
+  // GEMM1: float4 count of out to zero before the first tile (0: none)
+  float4 *zero_out;
+  int64_t zero_n4;
+  // GEMM2 fused with the combine: out [T, H] and the top-k weights [T, k]
+  float *out;
+  const float *topk_weights;
+  int fuse_combine;
 };
 
 struct Tile {
@@ -225,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&bars->acc_full[a], 1);
-      mbar_init(&bars->acc_empty[a], 4 * CG);  // 4 epilogue warps per CTA
+      mbar_init(&bars->acc_empty[a], kEpiWarps * CG);  // every epilogue warp of the pair
     }
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
@@ -414,10 +436,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter accessible to this warp
+    const int ew = warp - (kMmaWarp + 1);  // 0..7
+    const int q = warp & 3;                 // TMEM lane quarter accessible to this warp
+    const int half = ew >> 2;               // which half of the tile's columns
     const int row = q * 32 + lane;
-    uint8_t *ebuf = sEpi + q * 2 * kEpiBlock;  // GEMM2: this warp's two staging blocks
-    int acc_it = 0, nstore = 0;
+    uint8_t *ebuf = sEpi + ew * kEpiWarpBytes;  // GEMM2: this warp's staging buffer
+    if (MODE == kModeGemm1 && p.zero_n4 > 0) {
+      // out must read zero before GEMM2 adds into it; this runs while the
+      // first tiles' MMAs are in flight
+      const int64_t nw = static_cast<int64_t>(gridDim.x) * kEpiWarps;
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int64_t i = (static_cast<int64_t>(blockIdx.x) * kEpiWarps + ew) * 32 + lane;
+           i < p.zero_n4; i += nw * 32)
+        p.zero_out[i] = z;
+    }
+    int acc_it = 0;
     for (int t = unit; t < total; t += nunits, ++acc_it) {
       const int a = acc_it & 1;
       const uint32_t aph = (acc_it >> 1) & 1;
@@ -435,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __nv_bfloat16 *dst =
             p.act + static_cast<size_t>(my_row0 + (valid ? row : 0)) * p.I + tl.nt * (kAccN / 2);
 #pragma unroll 1
-        for (int c0 = 0; c0 < kAccN / 2; c0 += 32) {
+        for (int c0 = half * (kAccN / 4); c0 < (half + 1) * (kAccN / 4); c0 += 32) {
           uint32_t g[32], u[32];
           tmem_ld_32cols(tbase + c0, g);
           tmem_ld_32cols(tbase + kAccN / 2 + c0, u);
@@ -453,20 +486,53 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int v = 0; v < 4; ++v)
               d4[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
           }
+          __syncwarp();
+        }
+      } else if (p.fuse_combine) {
+        // row -> (token, weight); each lane stages and reduces its own row,
+        // so the lanes need no synchronisation with one another
+        float wgt = 0.f;
+        float *orow = p.out;
+        if (valid) {
+          const int slot = p.sorted_rows[my_row0 + row];
+          wgt = p.topk_weights[slot];
+          orow = p.out + static_cast<size_t>(slot / p.k) * p.H;
+        }
+        uint8_t *srow = ebuf + lane * kRedPitch;
+#pragma unroll 1
+        for (int c0 = half * (kAccN / 2); c0 < (half + 1) * (kAccN / 2); c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32cols(tbase + c0, v);
+          tmem_ld_wait();
+          const int col = tl.nt * kAccN + c0;
+          if (col < p.H && valid) {
+            // the previous reduction from this row buffer must have read it
+            bulk_wait_group_read<0>();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<float4 *>(srow + 16 * j) =
+                  make_float4(wgt * as_f32(v[4 * j]), wgt * as_f32(v[4 * j + 1]),
+                              wgt * as_f32(v[4 * j + 2]), wgt * as_f32(v[4 * j + 3]));
+            fence_proxy_async_smem();
+            bulk_reduce_add_f32(orow + col, srow, 128);
+            bulk_commit_group();
+          }
+          __syncwarp();
         }
       } else {
         // this warp's 32 rows: whole blocks go out through TMA stores
         const bool whole = q * 32 + 32 <= my_rows;
 #pragma unroll 1
-        for (int c0 = 0; c0 < kAccN; c0 += 32) {
+        for (int c0 = half * (kAccN / 2); c0 < (half + 1) * (kAccN / 2); c0 += 32) {
           uint32_t v[32];
           tmem_ld_32cols(tbase + c0, v);
           tmem_ld_wait();
           const int col = tl.nt * kAccN + c0;
+          if (col >= p.H) continue;  // masked half of a last n-tile (H % 256 == 128)
           if (whole) {
-            uint8_t *blk = ebuf + (nstore & 1) * kEpiBlock;
-            // the store issued two blocks ago from this buffer must have read it
-            if (lane == 0) bulk_wait_group_read<1>();
+            uint8_t *blk = ebuf;
+            // the previous store from this buffer must have read it
+            if (lane == 0) bulk_wait_group_read<0>();
             __syncwarp();
             // row `lane` as 8 chunks of 16 bytes, 128-byte swizzle
 #pragma unroll
@@ -479,8 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_store_2d(&tm_out, blk, col, my_row0 + q * 32);
               bulk_commit_group();
             }
-            ++nstore;
-          } else if (valid && col < p.H) {
+          } else if (valid) {
             // the block crosses the end of the expert's rows: plain stores
             float4 *d4 = reinterpret_cast<float4 *>(
                 p.P + static_cast<size_t>(my_row0 + row) * p.H + col);
@@ -489,6 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               d4[i] = make_float4(as_f32(v[4 * i]), as_f32(v[4 * i + 1]), as_f32(v[4 * i + 2]),
                                   as_f32(v[4 * i + 3]));
           }
+          __syncwarp();
         }
       }
       tc_fence_before_sync();
@@ -500,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&bars->acc_empty[a]);
       }
     }
-    if (MODE == kModeGemm2 && lane == 0) bulk_wait_group_all();
+    if (MODE == kModeGemm2) bulk_wait_group_all();
   }
 
   tc_fence_before_sync();
@@ -594,6 +660,10 @@ Params base_params(const GroupedGemmArgs &a) {
   p.k = a.k;
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
+  if (a.fuse_combine) {
+    p.out = a.out;
+    p.topk_weights = a.topk_weights;
+  }
   return p;
 }
 
@@ -662,6 +732,10 @@ cudaError_t launch_gemm1_swiglu(const GroupedGemmArgs &a, cudaStream_t s, const 
   int dev = 0;
   cudaGetDevice(&dev);
   Params p = base_params(a);
+  if (a.fuse_combine) {
+    p.zero_out = reinterpret_cast<float4 *>(a.out);
+    p.zero_n4 = a.T * a.H / 4;
+  }
   p.K = a.H;
   p.n_tiles_n = a.I / (kAccN / 2);
   p.b_rows_per_expert = 2 * a.I;
@@ -685,6 +759,7 @@ cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s, const StageHo
   int dev = 0;
   cudaGetDevice(&dev);
   Params p = base_params(a);
+  p.fuse_combine = a.fuse_combine;
   p.K = a.I;
   p.n_tiles_n = (a.H + kAccN - 1) / kAccN;  // H % 128 == 0: a last half tile is masked
   p.b_rows_per_expert = a.H;

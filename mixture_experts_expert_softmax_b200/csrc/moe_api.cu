@@ -148,6 +148,8 @@ int current_device(DeviceState **out) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 // Make the workspace at least `bytes` large.
 int ensure_workspace(DeviceState &d, size_t bytes) {
   if (bytes <= d.ws_bytes) return MOE_OK;
@@ -245,7 +247,7 @@ int moe_permute(const int32_t *topk_ids, int64_t T, int k, int E, int32_t *sorte
   CallCtx ctx{static_cast<cudaStream_t>(stream), "", nullptr};
   moe::StageHook hook = make_hook(&ctx);
   cudaError_t e = moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets, sorted_rows,
-                                      nullptr, ctx.stream, hook);
+                                      nullptr, nullptr, ctx.stream, hook);
   return to_code(e);
 }
 
@@ -255,6 +257,8 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
   if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
   if (T > 0 && (hidden == nullptr || w1 == nullptr || w2 == nullptr || topk_weights == nullptr ||
                 topk_ids == nullptr || out == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(w1) || !aligned16(w2) || !aligned16(out))
     return MOE_ERR_INVALID_ARG;
   if (H % 128 != 0 || I % 128 != 0 || E > kMaxExperts || k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
   const int64_t n = T * k;
@@ -278,9 +282,11 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
         &d->small_t_launches, static_cast<uint64_t>(g_wait_limit_ns), ctx.stream, hook));
   }
 
+  // top-k <= 2: GEMM2 adds its rows straight into out and no P is needed
+  const bool fuse_combine = k <= 2;
   const size_t need = permute_ws_bytes(n, E) + align256(static_cast<size_t>(n) * 4) +
                       align256(static_cast<size_t>(n) * I * 2) +
-                      align256(static_cast<size_t>(n) * H * sizeof(float));
+                      (fuse_combine ? 0 : align256(static_cast<size_t>(n) * H * sizeof(float)));
   if ((rc = ensure_workspace(*d, need)) != MOE_OK) return rc;
   Carver cv{static_cast<char *>(d->ws)};
   int32_t *chunk_counts =
@@ -289,15 +295,15 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
   int32_t *inv = cv.take<int32_t>(std::max<int64_t>(n, 1));
   int32_t *expert_offsets = cv.take<int32_t>(E + 1);
   uint16_t *act = cv.take<uint16_t>(static_cast<size_t>(n) * I);
-  float *P = cv.take<float>(static_cast<size_t>(n) * H);
+  float *P = fuse_combine ? nullptr : cv.take<float>(static_cast<size_t>(n) * H);
 
   // the forward's result does not depend on the order of rows inside an
   // expert, so a single-CTA grouping replaces the stable three-kernel one
   cudaError_t e = moe::permute_fused_supported(n)
                       ? moe::launch_permute_fused(topk_ids, n, E, expert_offsets, sorted_rows,
-                                                  inv, ctx.stream, hook)
+                                                  inv, d->status, ctx.stream, hook)
                       : moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets,
-                                            sorted_rows, inv, ctx.stream, hook);
+                                            sorted_rows, inv, d->status, ctx.stream, hook);
   if (e != cudaSuccess) return to_code(e);
   moe::GroupedGemmArgs ga;
   ga.hidden = hidden;
@@ -315,8 +321,12 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
   ga.num_sms = d->num_sms;
   ga.status = d->status;
   ga.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns);
+  ga.out = out;
+  ga.topk_weights = topk_weights;
+  ga.fuse_combine = fuse_combine ? 1 : 0;
   if ((e = moe::launch_gemm1_swiglu(ga, ctx.stream, hook)) != cudaSuccess) return to_code(e);
   if ((e = moe::launch_gemm2(ga, ctx.stream, hook)) != cudaSuccess) return to_code(e);
+  if (fuse_combine) return MOE_OK;
   e = moe::launch_combine(P, inv, topk_weights, out, T, H, k, d->status, ctx.stream, hook);
   return to_code(e);
 }

@@ -46,12 +46,12 @@ cudaError_t launch_route(const float *logits, int64_t T, int E, int k, int renor
 int permute_num_chunks(int64_t n);
 cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int32_t *chunk_counts,
                            int32_t *expert_offsets, int32_t *sorted_rows, int32_t *inv,
-                           cudaStream_t s, const StageHook &hook);
+                           uint32_t *status, cudaStream_t s, const StageHook &hook);
 
 bool permute_fused_supported(int64_t n);
 cudaError_t launch_permute_fused(const int32_t *ids, int64_t n, int E, int32_t *expert_offsets,
-                                 int32_t *sorted_rows, int32_t *inv, cudaStream_t s,
-                                 const StageHook &hook);
+                                 int32_t *sorted_rows, int32_t *inv, uint32_t *status,
+                                 cudaStream_t s, const StageHook &hook);
 
 // grouped_gemm.cu
 struct GroupedGemmArgs {
@@ -61,7 +61,12 @@ struct GroupedGemmArgs {
   const int32_t *sorted_rows;
   const int32_t *expert_offsets;
   uint16_t *act;  // [T*k, I] bf16, expert-sorted rows
-  float *P;       // [T*k, H] fp32, expert-sorted rows
+  float *P;       // [T*k, H] fp32, expert-sorted rows (unused when fuse_combine)
+  // fuse_combine (k <= 2): GEMM1 zeroes out, and GEMM2 adds w * y of each
+  // row straight into out[token] instead of writing P.
+  float *out;                 // [T, H] fp32
+  const float *topk_weights;  // [T, k] fp32
+  int fuse_combine;
   int64_t T;
   int H, I, E, k;
   int num_sms;

@@ -47,6 +47,11 @@ extern "C" int moe_forward_small_noalloc(const uint16_t *hidden, const uint16_t 
   if (T > 0 && (hidden == nullptr || w1 == nullptr || w2 == nullptr || topk_weights == nullptr ||
                 topk_ids == nullptr || out == nullptr))
     return MOE_ERR_INVALID_ARG;
+  // the kernel moves rows with 16-byte bulk copies and vector accesses
+  if (((reinterpret_cast<uintptr_t>(hidden) | reinterpret_cast<uintptr_t>(w1) |
+        reinterpret_cast<uintptr_t>(w2) | reinterpret_cast<uintptr_t>(out)) &
+       15u) != 0)
+    return MOE_ERR_INVALID_ARG;
   if (H % 128 != 0 || I % 128 != 0 || E > 1024 || k > 16 || !moe::small_t_supported(H, I))
     return MOE_ERR_UNSUPPORTED;
   if (T > MOE_NOALLOC_MAX_T ||

@@ -89,12 +89,14 @@ __global__ void __launch_bounds__(1024)
 
 // Writes sorted_rows[pos] = i for every valid entry and, when inv is given,
 // its inverse inv[i] = pos (-1 for an id outside [0, E)).  Shared memory
-// holds one running base per (warp, expert).
+// holds one running base per (warp, expert).  An id outside [0, E) raises
+// the bad-id bit of *status when status is given.
 __global__ void __launch_bounds__(kPermThreads)
     permute_scatter_kernel(const int32_t *__restrict__ ids, int64_t n, int E,
                            const int32_t *__restrict__ chunk_bases,
                            const int32_t *__restrict__ expert_offsets,
-                           int32_t *__restrict__ sorted_rows, int32_t *__restrict__ inv) {
+                           int32_t *__restrict__ sorted_rows, int32_t *__restrict__ inv,
+                           uint32_t *status) {
   extern __shared__ int32_t wbase[];  // [kPermWarps][E]
   grid_dep_wait();
   grid_dep_launch();
@@ -130,6 +132,8 @@ __global__ void __launch_bounds__(kPermThreads)
       if (e < 0 || e >= E) e = -1;
     }
     const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    if (status != nullptr && __any_sync(0xffffffffu, i < n && e < 0) && lane == 0)
+      atomicOr(status, kStatusBadId);
     int32_t pos = -1;
     if (e >= 0) {
       pos = mine[e] + __popc(peers & lt_mask);
@@ -155,7 +159,7 @@ constexpr int64_t kFusedMaxN = 8192;  // above this the multi-CTA kernels are fa
 __global__ void __launch_bounds__(kFusedThreads)
     permute_fused_kernel(const int32_t *__restrict__ ids, int n, int E,
                          int32_t *__restrict__ expert_offsets, int32_t *__restrict__ sorted_rows,
-                         int32_t *__restrict__ inv) {
+                         int32_t *__restrict__ inv, uint32_t *status) {
   __shared__ int32_t cnt[1024];
   __shared__ int32_t warp_tot[32];
   grid_dep_wait();
@@ -205,6 +209,8 @@ __global__ void __launch_bounds__(kFusedThreads)
     int e = i < n ? __ldg(ids + i) : -1;
     if (e >= E) e = -1;
     const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    if (status != nullptr && __any_sync(0xffffffffu, i < n && e < 0) && lane == 0)
+      atomicOr(status, kStatusBadId);
     const int leader = __ffs(static_cast<int>(peers)) - 1;
     int pos0 = 0;
     if (e >= 0 && lane == leader) pos0 = atomicAdd(&cnt[e], __popc(peers));
@@ -224,18 +230,19 @@ int permute_num_chunks(int64_t n) { return static_cast<int>((n + kChunk - 1) / k
 bool permute_fused_supported(int64_t n) { return n <= kFusedMaxN; }
 
 cudaError_t launch_permute_fused(const int32_t *ids, int64_t n, int E, int32_t *expert_offsets,
-                                 int32_t *sorted_rows, int32_t *inv, cudaStream_t s,
-                                 const StageHook &hook) {
+                                 int32_t *sorted_rows, int32_t *inv, uint32_t *status,
+                                 cudaStream_t s, const StageHook &hook) {
   hook.begin("permute");
   // first kernel of the call: ordinary stream order after earlier work
   cudaError_t err = launch_pdl(permute_fused_kernel, dim3(1), dim3(kFusedThreads), 0, s, false,
-                               ids, static_cast<int>(n), E, expert_offsets, sorted_rows, inv);
+                               ids, static_cast<int>(n), E, expert_offsets, sorted_rows, inv,
+                               status);
   return hook.end(err);
 }
 
 cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int32_t *chunk_counts,
                            int32_t *expert_offsets, int32_t *sorted_rows, int32_t *inv,
-                           cudaStream_t s, const StageHook &hook) {
+                           uint32_t *status, cudaStream_t s, const StageHook &hook) {
   const int n_chunks = permute_num_chunks(n);
   cudaError_t err;
   if (n_chunks > 0) {
@@ -255,7 +262,7 @@ cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int32_t *chunk_
     err = launch_pdl(permute_scatter_kernel, dim3(n_chunks), dim3(kPermThreads),
                      static_cast<size_t>(kPermWarps) * E * sizeof(int32_t), s, hook.pdl, ids, n,
                      E, static_cast<const int32_t *>(chunk_counts),
-                     static_cast<const int32_t *>(expert_offsets), sorted_rows, inv);
+                     static_cast<const int32_t *>(expert_offsets), sorted_rows, inv, status);
     if ((err = hook.end(err)) != cudaSuccess) return err;
   }
   return cudaSuccess;

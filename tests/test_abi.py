@@ -54,7 +54,8 @@ def test_route_argument_checks(args, code):
     assert L.moe_route(*args) == code
 
 
-FWD_OK = dict(h=1, w1=1, w2=1, w=1, ids=1, out=1, T=4, H=256, I=128, E=8, k=2)
+# non-null stand-ins for device pointers, 16-byte aligned like real arrays
+FWD_OK = dict(h=256, w1=256, w2=256, w=256, ids=256, out=256, T=4, H=256, I=128, E=8, k=2)
 
 
 def fwd(**kw):
@@ -75,6 +76,9 @@ def fwd(**kw):
     (dict(E=2000, k=2), moe.MOE_ERR_UNSUPPORTED),  # E > 1024
     (dict(E=64, k=17), moe.MOE_ERR_UNSUPPORTED),   # k > 16
     (dict(T=0, h=NULL, out=NULL), moe.MOE_OK),    # empty batch
+    (dict(h=264), moe.MOE_ERR_INVALID_ARG),        # hidden not 16-byte aligned
+    (dict(w2=260), moe.MOE_ERR_INVALID_ARG),       # w2 not 16-byte aligned
+    (dict(out=258), moe.MOE_ERR_INVALID_ARG),      # out not 16-byte aligned
 ])
 def test_forward_argument_checks(kw, code):
     assert fwd(**kw) == code

@@ -39,9 +39,11 @@ def gpu_route(logits_cpu, k, renorm=True):
 def gpu_forward(hidden, w1, w2, w, ids):
     """Inputs may live on CPU or GPU; routing comes in as numpy."""
     dev = torch.device("cuda")
+    # NaN-filled: every element of out must be written by the call
+    out = torch.full((hidden.shape[0], hidden.shape[1]), float("nan"), device=dev)
     out = moe.moe_forward(hidden.to(dev), w1.to(dev), w2.to(dev),
                           torch.as_tensor(np.asarray(w, np.float32)).to(dev),
-                          torch.as_tensor(np.asarray(ids, np.int32)).to(dev))
+                          torch.as_tensor(np.asarray(ids, np.int32)).to(dev), out=out)
     torch.cuda.synchronize()
     return out.cpu().numpy()
 
@@ -176,9 +178,11 @@ def test_forward_small_t_shared_and_duplicate_experts():
         assert_output_close(out, ref, f"small_t_max={small}")
 
 
-@pytest.mark.parametrize("small", [16, 0])
-def test_forward_invalid_ids_are_skipped_and_flagged(small):
-    T, H, I, E, k = 12, 256, 128, 8, 2
+@pytest.mark.parametrize("small,k", [(16, 2), (0, 2), (0, 4)])
+def test_forward_invalid_ids_are_skipped_and_flagged(small, k):
+    """k = 2 on the GEMM path flags bad ids in the grouping (GEMM2 adds into
+    out); k = 4 also goes through the separate combine."""
+    T, H, I, E = 12, 256, 128, 8
     hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=11)
     ids, w = oracle.route(logits.numpy(), k, True)
     ids[3, 1] = -1
@@ -210,13 +214,41 @@ def test_forward_zero_token_gives_zero_row(small):
     assert np.all(out[4] == 0.0)
 
 
-def test_forward_deterministic():
-    s = SHAPES["tiny"]
-    hidden, w1, w2, logits = make_shape_inputs(s)
-    ids, w = oracle.route(logits.numpy(), s.k, True)
-    a = gpu_forward(hidden, w1, w2, w, ids)
-    b = gpu_forward(hidden, w1, w2, w, ids)
-    assert np.array_equal(a, b)
+@pytest.mark.parametrize("T,H,I,E,k", [(64, 256, 128, 8, 2), (600, 512, 256, 8, 2),
+                                        (600, 512, 256, 8, 1), (300, 384, 256, 16, 4)])
+def test_forward_deterministic(T, H, I, E, k):
+    """Identical bits on repeated calls: with k <= 2 GEMM2 adds two rounded
+    products onto zero in whatever order the tiles finish (a commutative
+    sum), with k > 2 the combine sums in fixed order."""
+    hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=5)
+    ids, w = oracle.route(logits.numpy(), k, True)
+    prev = moe.set_small_t_max(0)
+    try:
+        a = gpu_forward(hidden, w1, w2, w, ids)
+        b = gpu_forward(hidden, w1, w2, w, ids)
+        c = gpu_forward(hidden, w1, w2, w, ids)
+    finally:
+        moe.set_small_t_max(prev)
+    assert np.array_equal(a, b) and np.array_equal(a, c)
+
+
+def test_forward_gemm_duplicate_slots_top2():
+    """A token routed twice to one expert: two rows of that expert's group
+    added into the same output row (summed weight in atrex-bench #009)."""
+    T, H, I, E, k = 40, 256, 256, 4, 2
+    hidden, w1, w2, _ = make_inputs(T, H, I, E, seed=21)
+    rng = np.random.default_rng(1)
+    ids = rng.integers(0, E, (T, k)).astype(np.int32)
+    ids[::3, 1] = ids[::3, 0]
+    w = rng.uniform(0.1, 1.0, (T, k))
+    ref = oracle.moe_token_loop(hidden, w1, w2, w, ids)
+    prev = moe.set_small_t_max(0)
+    try:
+        out = gpu_forward(hidden, w1, w2, w, ids)
+    finally:
+        moe.set_small_t_max(prev)
+    assert_output_close(out, ref)
+    check_status_clean()
 
 
 def test_forward_empty_batch():
@@ -276,7 +308,7 @@ def test_bounded_wait_times_out_without_hanging():
     assert moe.debug_wait_timeout(2_000_000) == moe.MOE_ERR_TIMEOUT  # 2 ms
     assert moe.get_device_status() & moe.MOE_STATUS_TIMEOUT
     # the context is still usable afterwards
-    test_forward_deterministic()
+    test_forward_deterministic(64, 256, 128, 8, 2)
     check_status_clean()
 
 
@@ -293,7 +325,25 @@ def test_sync_each_stage_mode_and_profiler():
         moe.profile_enable(False)
         moe.set_sync_each_stage(prev)
     prof = moe.profile_read()
-    for kname in ("permute", "gemm1_swiglu", "gemm2", "combine"):
+    # top-2: GEMM2 adds into out, no separate combine
+    for kname in ("permute", "gemm1_swiglu", "gemm2"):
         assert prof[kname][0] == 1 and prof[kname][1] > 0
+    assert "combine" not in prof
     ref = oracle.moe_token_loop(hidden, w1, w2, w, ids)
     assert_output_close(out, ref)
+
+    T, H, I, E, k = 64, 256, 128, 8, 4
+    hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=8)
+    ids, w = oracle.route(logits.numpy(), k, True)
+    prev = moe.set_sync_each_stage(True)
+    moe.profile_reset()
+    moe.profile_enable(True)
+    try:
+        out = gpu_forward(hidden, w1, w2, w, ids)
+    finally:
+        moe.profile_enable(False)
+        moe.set_sync_each_stage(prev)
+    prof = moe.profile_read()
+    for kname in ("permute", "gemm1_swiglu", "gemm2", "combine"):
+        assert prof[kname][0] == 1 and prof[kname][1] > 0
+    assert_output_close(out, oracle.moe_token_loop(hidden, w1, w2, w, ids))
