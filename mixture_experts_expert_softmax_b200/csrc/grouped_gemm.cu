@@ -20,11 +20,15 @@
 // CTAs working together share a weight tile through L2; the grid is
 // persistent and loops over tiles.
 //
-//   GEMM1 runs on single CTAs (M = 128, tcgen05.mma.cta_group::1): its A rows
-//   are gathered by token index with cp.async, whose completion can only be
-//   signalled to the CTA's own barriers.  The B tile is the n-tile's 128 gate
-//   rows and the matching 128 up rows, so one accumulator holds gate and up
-//   side by side and the epilogue applies SwiGLU.
+//   GEMM1 has two forms.  When the hidden rows have been copied into
+//   expert-sorted order beforehand (gather_rows_kernel), it runs on CTA
+//   pairs like GEMM2 below, rank 0 loading the n-tile's 128 gate rows of w1
+//   and rank 1 the matching 128 up rows.  Otherwise it runs on single CTAs
+//   (M = 128, tcgen05.mma.cta_group::1) that gather their A rows by token
+//   index with cp.async, whose completion can only be signalled to the CTA's
+//   own barriers, and load gate and up rows themselves.  Either way one
+//   accumulator holds gate and up side by side and the epilogue applies
+//   SwiGLU.
 //   GEMM2 runs on CTA pairs (a cluster of 2, M = 256, cta_group::2): rank r
 //   loads A rows 128r..128r+127 and B rows 128r..128r+127 of the pair's tile
 //   with TMA into its own shared memory, rank 0 issues the MMAs, and each
@@ -40,9 +44,9 @@
 //   warps 0-3  producers.  GEMM1: the 128 threads gather the A rows with
 //              16-byte cp.async into the 128-byte-swizzled K-major layout and
 //              arrive on the stage barrier asynchronously when they land;
-//              thread 0 issues the two TMA boxes of w1.  GEMM2: thread 0 of
-//              each CTA issues TMA for its act rows and half of B, counted on
-//              rank 0's barrier.
+//              thread 0 issues the two TMA boxes of w1.  CTA pairs: thread 0
+//              of each CTA issues TMA for its A rows and half of B, counted
+//              on rank 0's barrier.
 //   warp 4     allocates 512 TMEM columns (two accumulators); one thread (on
 //              rank 0) issues the MMAs and commits each stage back to the
 //              producers and each finished tile to the epilogues.
@@ -52,6 +56,7 @@
 //              store, then release the accumulator.
 // Every wait is bounded; a wait that gives up raises the timeout bit of the
 // status word and makes every role of the CTA leave its loop.
+#include <algorithm>
 #include <mutex>
 
 #include "moe_internal.h"
@@ -79,7 +84,7 @@ constexpr int kRedPitch = 144;
 constexpr int kEpiWarpBytes = 5 * 1024;
 static_assert(32 * kRedPitch <= kEpiWarpBytes && kEpiBlock <= kEpiWarpBytes, "staging");
 
-enum { kModeGemm1 = 0, kModeGemm2 = 1 };
+enum { kModeGemm1 = 0, kModeGemm2 = 1, kModeGemm1Pair = 2 };
 
 template <int MODE>
 struct Cfg;
@@ -88,6 +93,13 @@ struct Cfg<kModeGemm1> {
   static constexpr int CG = 1;        // CTAs per MMA
   static constexpr int kStages = 4;
   static constexpr int kBRows = 256;  // B rows this CTA loads per stage
+  static constexpr int kEpiBytes = 0;
+};
+template <>
+struct Cfg<kModeGemm1Pair> {
+  static constexpr int CG = 2;
+  static constexpr int kStages = 6;
+  static constexpr int kBRows = 128;  // gate rows on rank 0, up rows on rank 1
   static constexpr int kEpiBytes = 0;
 };
 template <>
@@ -123,6 +135,7 @@ constexpr size_t smem_bytes() {
 }
 static_assert(smem_bytes<kModeGemm1>() <= 232448, "shared memory budget");
 static_assert(smem_bytes<kModeGemm2>() <= 232448, "shared memory budget");
+static_assert(smem_bytes<kModeGemm1Pair>() <= 232448, "shared memory budget");
 
 struct Params {
   const __nv_bfloat16 *hidden;
@@ -222,6 +235,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tm_out, const Params p) {
   using C = Cfg<MODE>;
   constexpr int CG = C::CG;
+  constexpr bool kGather = MODE == kModeGemm1;  // A rows by cp.async
+  constexpr bool kSwiglu = MODE != kModeGemm2;  // GEMM1 epilogue
   constexpr int kStages = C::kStages;
   constexpr int TM = tile_m<MODE>();
   constexpr int kBBytes = b_bytes<MODE>();
@@ -242,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       // GEMM1: 128 cp.async arrivals + the expect_tx arrival; GEMM2: rank 0's
       // expect_tx arrival (both CTAs' TMA bytes are counted on it)
-      mbar_init(&bars->full[s], MODE == kModeGemm1 ? kProducerThreads + 1 : 1);
+      mbar_init(&bars->full[s], kGather ? kProducerThreads + 1 : 1);
       mbar_init(&bars->empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -252,10 +267,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
-    if (MODE == kModeGemm2) {
-      prefetch_tmap(&tm_a);
-      prefetch_tmap(&tm_out);
-    }
+    if (!kGather) prefetch_tmap(&tm_a);
+    if (MODE == kModeGemm2) prefetch_tmap(&tm_out);
     prefetch_tmap(&tm_b);
   }
   if (warp == kMmaWarp) {
@@ -294,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
     // ------------------------------------------------------------ producers
-    if (MODE == kModeGemm1) {
+    if (kGather) {
       const int c = threadIdx.x & 7;      // 16-byte chunk of the 128-byte row
       const int rsub = threadIdx.x >> 3;  // rows rsub, rsub+16, ..., rsub+112
       int it = 0;
@@ -353,8 +366,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = unit; t < total && !stop; t += nunits) {
         const Tile tl = decode_tile<TM>(t, NT, p.E, s_tile_off, s_exp_off);
         const int a_row = tl.row0 + static_cast<int>(rank) * BM;
-        const int b_row =
-            tl.e * p.b_rows_per_expert + tl.nt * kAccN + static_cast<int>(rank) * C::kBRows;
+        // GEMM1: rank 0 the n-tile's gate rows, rank 1 its up rows;
+        // GEMM2: rank r rows 128r.. of the n-tile's 256 rows of w2
+        const int b_row = tl.e * p.b_rows_per_expert +
+                          (kSwiglu ? static_cast<int>(rank) * p.I + tl.nt * (kAccN / 2)
+                                   : tl.nt * kAccN + static_cast<int>(rank) * C::kBRows);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
@@ -400,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after_sync();
           // A rows may have been written by cp.async: order them before the
           // tensor core's (async-proxy) reads
-          if (MODE == kModeGemm1) fence_proxy_async_smem();
+          if (kGather) fence_proxy_async_smem();
           const uint64_t a_desc = smem_desc_sw128(smem_addr(sA + s * kABytes));
           const uint64_t b_desc = smem_desc_sw128(smem_addr(sB + s * kBBytes));
 #pragma unroll
@@ -441,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = ew >> 2;               // which half of the tile's columns
     const int row = q * 32 + lane;
     uint8_t *ebuf = sEpi + ew * kEpiWarpBytes;  // GEMM2: this warp's staging buffer
-    if (MODE == kModeGemm1 && p.zero_n4 > 0) {
+    if (kSwiglu && p.zero_n4 > 0) {
       // out must read zero before GEMM2 adds into it; this runs while the
       // first tiles' MMAs are in flight
       const int64_t nw = static_cast<int64_t>(gridDim.x) * kEpiWarps;
@@ -464,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int my_rows = min(BM, max(0, tl.rows - static_cast<int>(rank) * BM));
       const bool valid = row < my_rows;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kAccN;
-      if (MODE == kModeGemm1) {
+      if (kSwiglu) {
         __nv_bfloat16 *dst =
             p.act + static_cast<size_t>(my_row0 + (valid ? row : 0)) * p.I + tl.nt * (kAccN / 2);
 #pragma unroll 1
@@ -706,13 +722,23 @@ cudaError_t grouped_gemm_setup(int device) {
     e = cudaFuncSetAttribute(grouped_gemm_kernel<kModeGemm2>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem_bytes<kModeGemm2>()));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(grouped_gemm_kernel<kModeGemm1Pair>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_bytes<kModeGemm1Pair>()));
   if (e != cudaSuccess) return e;
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
-  // how many 2-CTA clusters of GEMM2 can be resident at once
+  // how many 2-CTA clusters can be resident at once (both pair kernels take
+  // one CTA per SM; the smaller count of the two is used for both)
   cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = launch_config<kModeGemm2>(2, nullptr, false, attr);
-  int clusters = 0;
+  int clusters = 0, clusters1 = 0;
   e = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<kModeGemm2>, &cfg);
+  if (e == cudaSuccess) {
+    cfg = launch_config<kModeGemm1Pair>(2, nullptr, false, attr);
+    e = cudaOccupancyMaxActiveClusters(&clusters1, grouped_gemm_kernel<kModeGemm1Pair>, &cfg);
+    clusters = std::min(clusters, clusters1);
+  }
   if (e != cudaSuccess || clusters < 1) {
     cudaGetLastError();
     return e != cudaSuccess ? e : cudaErrorNotSupported;
@@ -725,9 +751,12 @@ cudaError_t grouped_gemm_setup(int device) {
 }
 
 cudaError_t launch_gemm1_swiglu(const GroupedGemmArgs &a, cudaStream_t s, const StageHook &hook) {
-  CUtensorMap tm_w1;
+  CUtensorMap tm_w1, tm_xs;
   if (!make_bf16_map(&tm_w1, a.w1, static_cast<uint64_t>(a.H),
                      static_cast<uint64_t>(a.E) * 2 * a.I, kAccN / 2))
+    return cudaErrorInvalidValue;
+  if (a.xs != nullptr && !make_bf16_map(&tm_xs, a.xs, static_cast<uint64_t>(a.H),
+                                        static_cast<uint64_t>(a.T) * a.k, BM))
     return cudaErrorInvalidValue;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -740,10 +769,17 @@ cudaError_t launch_gemm1_swiglu(const GroupedGemmArgs &a, cudaStream_t s, const 
   p.n_tiles_n = a.I / (kAccN / 2);
   p.b_rows_per_expert = 2 * a.I;
   cudaLaunchAttribute attr[2];
-  const cudaLaunchConfig_t cfg =
-      launch_config<kModeGemm1>(grid_for<kModeGemm1>(a, p.n_tiles_n, dev), s, hook.pdl, attr);
   hook.begin("gemm1_swiglu");
-  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm1>, tm_w1, tm_w1, tm_w1, p);
+  cudaError_t e;
+  if (a.xs != nullptr) {
+    const cudaLaunchConfig_t cfg = launch_config<kModeGemm1Pair>(
+        grid_for<kModeGemm1Pair>(a, p.n_tiles_n, dev), s, hook.pdl, attr);
+    e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm1Pair>, tm_xs, tm_w1, tm_xs, p);
+  } else {
+    const cudaLaunchConfig_t cfg =
+        launch_config<kModeGemm1>(grid_for<kModeGemm1>(a, p.n_tiles_n, dev), s, hook.pdl, attr);
+    e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm1>, tm_w1, tm_w1, tm_w1, p);
+  }
   return hook.end(e);
 }
 

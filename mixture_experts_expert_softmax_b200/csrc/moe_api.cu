@@ -284,8 +284,13 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
 
   // top-k <= 2: GEMM2 adds its rows straight into out and no P is needed
   const bool fuse_combine = k <= 2;
+  // Copying the hidden rows into expert-sorted order costs k row copies per
+  // token and lets GEMM1 run on CTA pairs with TMA operands; with few slots
+  // per token that pays off.
+  const bool gather_rows = k <= 2;
   const size_t need = permute_ws_bytes(n, E) + align256(static_cast<size_t>(n) * 4) +
                       align256(static_cast<size_t>(n) * I * 2) +
+                      (gather_rows ? align256(static_cast<size_t>(n) * H * 2) : 0) +
                       (fuse_combine ? 0 : align256(static_cast<size_t>(n) * H * sizeof(float)));
   if ((rc = ensure_workspace(*d, need)) != MOE_OK) return rc;
   Carver cv{static_cast<char *>(d->ws)};
@@ -296,6 +301,7 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
   int32_t *expert_offsets = cv.take<int32_t>(E + 1);
   uint16_t *act = cv.take<uint16_t>(static_cast<size_t>(n) * I);
   float *P = fuse_combine ? nullptr : cv.take<float>(static_cast<size_t>(n) * H);
+  uint16_t *xs = gather_rows ? cv.take<uint16_t>(static_cast<size_t>(n) * H) : nullptr;
 
   // the forward's result does not depend on the order of rows inside an
   // expert, so a single-CTA grouping replaces the stable three-kernel one
@@ -305,12 +311,17 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
                       : moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets,
                                             sorted_rows, inv, d->status, ctx.stream, hook);
   if (e != cudaSuccess) return to_code(e);
-  moe::GroupedGemmArgs ga;
+  if (gather_rows && (e = moe::launch_gather_rows(hidden, H, k, sorted_rows, expert_offsets, E, n,
+                                                  d->num_sms, xs, ctx.stream, hook)) !=
+                         cudaSuccess)
+    return to_code(e);
+  moe::GroupedGemmArgs ga = {};
   ga.hidden = hidden;
   ga.w1 = w1;
   ga.w2 = w2;
   ga.sorted_rows = sorted_rows;
   ga.expert_offsets = expert_offsets;
+  ga.xs = xs;
   ga.act = act;
   ga.P = P;
   ga.T = T;

@@ -53,6 +53,12 @@ cudaError_t launch_permute_fused(const int32_t *ids, int64_t n, int E, int32_t *
                                  int32_t *sorted_rows, int32_t *inv, uint32_t *status,
                                  cudaStream_t s, const StageHook &hook);
 
+// Expert-sorted copy of the hidden rows, xs[r] = hidden[sorted_rows[r] / k]
+// for r < expert_offsets[E] (device value); n = T*k bounds the grid.
+cudaError_t launch_gather_rows(const uint16_t *hidden, int H, int k, const int32_t *sorted_rows,
+                               const int32_t *expert_offsets, int E, int64_t n, int num_sms,
+                               uint16_t *xs, cudaStream_t s, const StageHook &hook);
+
 // grouped_gemm.cu
 struct GroupedGemmArgs {
   const uint16_t *hidden;  // [T, H] bf16
@@ -60,6 +66,9 @@ struct GroupedGemmArgs {
   const uint16_t *w2;      // [E, H, I] bf16
   const int32_t *sorted_rows;
   const int32_t *expert_offsets;
+  // [T*k, H] bf16 hidden rows in expert-sorted order (launch_gather_rows),
+  // or null: GEMM1 then runs on single CTAs and gathers its A rows itself
+  const uint16_t *xs;
   uint16_t *act;  // [T*k, I] bf16, expert-sorted rows
   float *P;       // [T*k, H] fp32, expert-sorted rows (unused when fuse_combine)
   // fuse_combine (k <= 2): GEMM1 zeroes out, and GEMM2 adds w * y of each
