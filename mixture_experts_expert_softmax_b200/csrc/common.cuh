@@ -70,9 +70,37 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
   return true;
 }
 
+// ---------------------------------------------------------------- global flags
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait until *p >= target (acquire at GPU scope): false when the
+// limit passes or *abort becomes non-zero first.
+__device__ __forceinline__ bool wait_geq(const int *p, int target, uint64_t limit_ns,
+                                         const volatile int *abort = nullptr) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (ld_acquire_gpu(p) < target) {
+    if (abort != nullptr && *abort != 0) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
+    __nanosleep(64);
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------- async copies
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Orders this thread's view of global memory (generic proxy, e.g. data
+// another CTA published with release/acquire) before its later TMA or bulk
+// (async proxy) accesses to global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m) {
@@ -113,6 +141,15 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *s
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
                    reinterpret_cast<uint64_t>(m)),
                "r"(smem_addr(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+
+// 1-D bulk copy shared -> global (bulk-group completion).  Both addresses
+// 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(dst)),
+               "r"(smem_addr(src)), "r"(bytes)
                : "memory");
 }
 

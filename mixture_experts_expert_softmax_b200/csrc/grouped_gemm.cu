@@ -6,10 +6,10 @@
 //     act = silu(g) * u, stored as bf16 [rows, I].
 //   GEMM2: y = act . w2[e]^T (fp32 in TMEM).  For top-k <= 2 the epilogue
 //     adds w_j * y_j of each row straight into out[token] with bulk
-//     reductions at L2 (GEMM1 has zeroed out); out[t] = 0 + a + b is the same
-//     in either arrival order, so the result is still deterministic.  For
-//     larger k it stores y as fp32 rows of P in the same expert-sorted order
-//     and combine.cu forms sum_j w_j * y_j in fixed j order.
+//     reductions at L2 (out was zeroed first); out[t] = 0 + a + b is the
+//     same in either arrival order, so the result is still deterministic.
+//     For larger k it stores y as fp32 rows of P in the same expert-sorted
+//     order and combine.cu forms sum_j w_j * y_j in fixed j order.
 // This is the expert FFN of ref_moe on the page "tpu_inference/kernels/
 // fused_moe/v1/kernel.py" (gate = w1, up = w3, then act . w2) in the weight
 // layout of atrex-bench #009 (w1 [E, 2I, H], w2 [E, H, I], both applied as
@@ -20,28 +20,42 @@
 // CTAs working together share a weight tile through L2; the grid is
 // persistent and loops over tiles.
 //
-//   GEMM1 has two forms.  When the hidden rows have been copied into
-//   expert-sorted order beforehand (gather_rows_kernel), it runs on CTA
-//   pairs like GEMM2 below, rank 0 loading the n-tile's 128 gate rows of w1
-//   and rank 1 the matching 128 up rows.  Otherwise it runs on single CTAs
-//   (M = 128, tcgen05.mma.cta_group::1) that gather their A rows by token
-//   index with cp.async, whose completion can only be signalled to the CTA's
-//   own barriers, and load gate and up rows themselves.  Either way one
-//   accumulator holds gate and up side by side and the epilogue applies
-//   SwiGLU.
-//   GEMM2 runs on CTA pairs (a cluster of 2, M = 256, cta_group::2): rank r
-//   loads A rows 128r..128r+127 and B rows 128r..128r+127 of the pair's tile
-//   with TMA into its own shared memory, rank 0 issues the MMAs, and each
-//   CTA receives its 128 accumulator rows in its own TMEM.  Splitting B
-//   between the pair halves the weight bytes each SM must fetch.  Its
-//   epilogue stages each 32x32 fp32 block in shared memory and writes it
-//   with a TMA store (coalesced, asynchronous; a block that straddles the
-//   end of an expert's rows is written row by row instead), or, fused with
-//   the combine, scales row r by its top-k weight and issues one 128-byte
-//   bulk reduce-add per row into out.
+// Three kernels share the code (MODE):
+//   kModeFused   one launch on CTA pairs (a cluster of 2, M = 256,
+//                cta_group::2) that runs every GEMM1 tile and then every
+//                GEMM2 tile.  Its A rows come from copies in expert-sorted
+//                order (hidden rows gathered by gather_rows_kernel, and act),
+//                so rank r of the pair loads A rows 128r..128r+127 and half
+//                of the B tile with TMA into its own shared memory; rank 0
+//                issues the MMAs and each CTA receives its 128 accumulator
+//                rows in its own TMEM.  For GEMM1 rank 0 loads the n-tile's
+//                128 gate rows of w1 and rank 1 the matching 128 up rows, so
+//                one accumulator holds gate and up side by side.  A GEMM2
+//                tile waits (bounded) until the epilogues of all GEMM1 tiles
+//                of its m-tile have published their act rows through a
+//                per-m-tile counter: the static tile order puts every GEMM1
+//                tile of a CTA before its GEMM2 tiles, so no wait can form a
+//                cycle, and GEMM2 tiles fill the last, partial wave of GEMM1.
+//   kModeGemm1   GEMM1 alone on single CTAs (M = 128, cta_group::1) that
+//                gather their A rows by token index with cp.async (whose
+//                completion can only be signalled to the CTA's own barriers)
+//                and load gate and up rows themselves: no row copy needed.
+//   kModeGemm2   GEMM2 alone on CTA pairs, after kModeGemm1.
+// The GEMM2 epilogue stages each warp's 32 rows x 32 columns in shared
+// memory and writes them with one asynchronous TMA tile store into P (a
+// block that straddles the end of an expert's rows is written row by row
+// instead), or, fused with the combine, scales row r by its top-k weight
+// and issues one 128-byte bulk reduce-add per row into out[token]: large
+// operations, because the TMA engine's cost per operation, not the bytes,
+// bounds this epilogue.
+//
+// Shared memory: the barriers and the expert / tile offset tables sit in
+// front, then (1024-byte aligned, as the 128-byte swizzle needs) the stage
+// ring and the epilogue staging.  The number of stages is chosen at launch:
+// as many as fit, up to kMaxStages, given the expert count.
 //
 // Warp roles (416 threads per CTA):
-//   warps 0-3  producers.  GEMM1: the 128 threads gather the A rows with
+//   warps 0-3  producers.  kModeGemm1: the 128 threads gather the A rows with
 //              16-byte cp.async into the 128-byte-swizzled K-major layout and
 //              arrive on the stage barrier asynchronously when they land;
 //              thread 0 issues the two TMA boxes of w1.  CTA pairs: thread 0
@@ -53,7 +67,7 @@
 //   warps 5-12 epilogue, two warps per 32-lane TMEM quarter (a warp can only
 //              read the quarter warp_id % 4), each taking half of the tile's
 //              columns: tcgen05.ld, SwiGLU + bf16 store, or the fp32 TMA
-//              store, then release the accumulator.
+//              store / bulk reductions, then release the accumulator.
 // Every wait is bounded; a wait that gives up raises the timeout bit of the
 // status word and makes every role of the CTA leave its loop.
 #include <algorithm>
@@ -76,37 +90,40 @@ constexpr int kABytes = BM * BK * 2;  // 16 KB
 constexpr int kMaxE = 1024;
 constexpr int kMaxStages = 6;
 constexpr uint16_t kBothCtas = 0x3;
-constexpr int kEpiBlock = 32 * 32 * 4;  // one 32-row x 32-column fp32 block
-// Per-warp staging: a swizzled kEpiBlock for the P store, or 32 rows at a
-// 144-byte pitch (conflict-free 16-byte writes) for the bulk reductions;
-// 1024-byte multiple so every warp's buffer stays swizzle-aligned.
+// Per-warp staging of the GEMM2 epilogue: one 32-row x 32-column fp32 block,
+// 128-byte swizzled for the TMA store, or 32 plain rows at a 144-byte pitch
+// for the reductions (16-byte writes of 8 consecutive lanes then hit 8
+// different bank groups: bank conflicts here would take shared-memory
+// bandwidth from the tensor core's operand reads).  A 1024-byte multiple
+// keeps every warp's block swizzle-aligned.
 constexpr int kRedPitch = 144;
 constexpr int kEpiWarpBytes = 5 * 1024;
-static_assert(32 * kRedPitch <= kEpiWarpBytes && kEpiBlock <= kEpiWarpBytes, "staging");
+static_assert(32 * kRedPitch <= kEpiWarpBytes, "staging");
+constexpr size_t kSmemMax = 232448;  // opt-in maximum per block on sm_100
+// act rows of an m-tile are complete when every epilogue warp of both CTAs
+// has published each of its n-tiles
+constexpr int kReadyPerTile = 2 * kEpiWarps;
 
-enum { kModeGemm1 = 0, kModeGemm2 = 1, kModeGemm1Pair = 2 };
+enum { kModeGemm1 = 0, kModeGemm2 = 1, kModeFused = 2 };
 
 template <int MODE>
 struct Cfg;
 template <>
 struct Cfg<kModeGemm1> {
   static constexpr int CG = 1;        // CTAs per MMA
-  static constexpr int kStages = 4;
   static constexpr int kBRows = 256;  // B rows this CTA loads per stage
-  static constexpr int kEpiBytes = 0;
-};
-template <>
-struct Cfg<kModeGemm1Pair> {
-  static constexpr int CG = 2;
-  static constexpr int kStages = 6;
-  static constexpr int kBRows = 128;  // gate rows on rank 0, up rows on rank 1
   static constexpr int kEpiBytes = 0;
 };
 template <>
 struct Cfg<kModeGemm2> {
   static constexpr int CG = 2;
-  static constexpr int kStages = 5;
   static constexpr int kBRows = 128;
+  static constexpr int kEpiBytes = kEpiWarps * kEpiWarpBytes;
+};
+template <>
+struct Cfg<kModeFused> {
+  static constexpr int CG = 2;
+  static constexpr int kBRows = 128;  // GEMM1: gate rows on rank 0, up rows on rank 1
   static constexpr int kEpiBytes = kEpiWarps * kEpiWarpBytes;
 };
 
@@ -114,8 +131,6 @@ template <int MODE>
 constexpr int tile_m() { return BM * Cfg<MODE>::CG; }
 template <int MODE>
 constexpr int b_bytes() { return Cfg<MODE>::kBRows * BK * 2; }
-template <int MODE>
-constexpr size_t smem_bytes();
 
 struct __align__(8) Bars {
   uint64_t full[kMaxStages];   // stage landed (rank 0's counts both CTAs)
@@ -128,14 +143,30 @@ struct __align__(8) Bars {
   int32_t scan[32];            // per-warp partial sums of build_tile_offsets
 };
 
-template <int MODE>
-constexpr size_t smem_bytes() {
-  return 1024 + static_cast<size_t>(Cfg<MODE>::kStages) * (kABytes + b_bytes<MODE>()) +
-         Cfg<MODE>::kEpiBytes + sizeof(Bars) + 2 * (kMaxE + 1) * sizeof(int32_t);
+// Bytes in front of the aligned region: barriers, then exp_off and tile_off
+// (E + 1 entries each).
+__host__ __device__ constexpr size_t front_bytes(int E) {
+  return sizeof(Bars) + 2 * static_cast<size_t>(E + 1) * sizeof(int32_t);
 }
-static_assert(smem_bytes<kModeGemm1>() <= 232448, "shared memory budget");
-static_assert(smem_bytes<kModeGemm2>() <= 232448, "shared memory budget");
-static_assert(smem_bytes<kModeGemm1Pair>() <= 232448, "shared memory budget");
+
+// Dynamic shared memory for `stages` stages (with the GEMM2 epilogue's
+// staging when `gemm2`); 1008 bytes cover the padding to the next 1024-byte
+// boundary from any 16-byte aligned base.
+template <int MODE>
+constexpr size_t smem_bytes(int E, int stages, bool gemm2 = true) {
+  return front_bytes(E) + 1008 + static_cast<size_t>(stages) * (kABytes + b_bytes<MODE>()) +
+         (gemm2 ? Cfg<MODE>::kEpiBytes : 0);
+}
+
+template <int MODE>
+int stages_for(int E, bool gemm2 = true) {
+  int st = kMaxStages;
+  while (st > 2 && smem_bytes<MODE>(E, st, gemm2) > kSmemMax) --st;
+  return st;
+}
+static_assert(smem_bytes<kModeGemm1>(kMaxE, 4) <= kSmemMax, "shared memory budget");
+static_assert(smem_bytes<kModeGemm2>(kMaxE, 5) <= kSmemMax, "shared memory budget");
+static_assert(smem_bytes<kModeFused>(kMaxE, 5) <= kSmemMax, "shared memory budget");
 
 struct Params {
   const __nv_bfloat16 *hidden;
@@ -144,18 +175,23 @@ struct Params {
   __nv_bfloat16 *act;
   float *P;
   int H, I, E, k;
-  int K;                  // contraction length (H for GEMM1, I for GEMM2)
-  int n_tiles_n;          // n-tiles per m-tile
-  int b_rows_per_expert;  // 2I for w1, H for w2
+  int nt1, nt2;  // n-tiles per m-tile of GEMM1 (I / 128) and GEMM2 (ceil(H / 256))
+  int stages;    // depth of the operand ring (<= kMaxStages)
+  int run_gemm2; // kModeFused: 0 runs the GEMM1 tiles only (GEMM2 follows as
+                 // its own kModeGemm2 launch)
   uint32_t *status;
   uint64_t wait_limit_ns;
-  // GEMM1: float4 count of out to zero before the first tile (0: none)
+  // float4 count of out to zero before GEMM2 adds into it (0: none)
   float4 *zero_out;
   int64_t zero_n4;
   // GEMM2 fused with the combine: out [T, H] and the top-k weights [T, k]
   float *out;
   const float *topk_weights;
   int fuse_combine;
+  // kModeFused: per-m-tile act counters and the count of epilogue warps
+  // that finished zeroing out (both zero at launch)
+  int *ready;
+  int *zero_done;
 };
 
 struct Tile {
@@ -228,35 +264,60 @@ __device__ __forceinline__ void give_up(const Params &p, volatile int *abort_fla
 
 __device__ __forceinline__ float as_f32(uint32_t u) { return __uint_as_float(u); }
 
+// What one tile of the static schedule is: GEMM1 or GEMM2 (phase 1 or 2),
+// its place, and its global m-tile index.
+struct Work {
+  int phase;
+  int mi;
+  Tile tl;
+};
+
+template <int MODE>
+__device__ __forceinline__ Work get_work(int t, int total1, const Params &p,
+                                         const int32_t *tile_off, const int32_t *exp_off) {
+  Work w;
+  int local = t, nt = p.nt1;
+  w.phase = 1;
+  if (MODE == kModeGemm2 || (MODE == kModeFused && t >= total1)) {
+    w.phase = 2;
+    nt = p.nt2;
+    if (MODE == kModeFused) local = t - total1;
+  }
+  w.tl = decode_tile<tile_m<MODE>()>(local, nt, p.E, tile_off, exp_off);
+  w.mi = tile_off[w.tl.e] + w.tl.mt;
+  return w;
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
-                        const __grid_constant__ CUtensorMap tm_b,
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a1,
+                        const __grid_constant__ CUtensorMap tm_b1,
+                        const __grid_constant__ CUtensorMap tm_a2,
+                        const __grid_constant__ CUtensorMap tm_b2,
                         const __grid_constant__ CUtensorMap tm_out, const Params p) {
   using C = Cfg<MODE>;
   constexpr int CG = C::CG;
-  constexpr bool kGather = MODE == kModeGemm1;  // A rows by cp.async
-  constexpr bool kSwiglu = MODE != kModeGemm2;  // GEMM1 epilogue
-  constexpr int kStages = C::kStages;
   constexpr int TM = tile_m<MODE>();
   constexpr int kBBytes = b_bytes<MODE>();
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *sA = smem;
+  constexpr bool kGather = MODE == kModeGemm1;  // A rows by cp.async
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const int kStages = p.stages;
+  Bars *bars = reinterpret_cast<Bars *>(smem_raw);
+  int32_t *s_tile_off = reinterpret_cast<int32_t *>(bars + 1);
+  int32_t *s_exp_off = s_tile_off + (p.E + 1);
+  uint8_t *sA = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + front_bytes(p.E) + 1023) &
+      ~static_cast<uintptr_t>(1023));
   uint8_t *sB = sA + kStages * kABytes;
   uint8_t *sEpi = sB + kStages * kBBytes;
-  Bars *bars = reinterpret_cast<Bars *>(sEpi + C::kEpiBytes);
-  int32_t *s_tile_off = reinterpret_cast<int32_t *>(bars + 1);
-  int32_t *s_exp_off = s_tile_off + (kMaxE + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = CG == 2 ? cluster_rank() : 0;
   const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      // GEMM1: 128 cp.async arrivals + the expect_tx arrival; GEMM2: rank 0's
-      // expect_tx arrival (both CTAs' TMA bytes are counted on it)
+      // kModeGemm1: 128 cp.async arrivals + the expect_tx arrival; pairs:
+      // rank 0's expect_tx arrival (both CTAs' TMA bytes are counted on it)
       mbar_init(&bars->full[s], kGather ? kProducerThreads + 1 : 1);
       mbar_init(&bars->empty[s], 1);
     }
@@ -267,9 +328,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
-    if (!kGather) prefetch_tmap(&tm_a);
-    if (MODE == kModeGemm2) prefetch_tmap(&tm_out);
-    prefetch_tmap(&tm_b);
+    if (MODE != kModeGemm2) prefetch_tmap(&tm_b1);
+    if (MODE == kModeFused) prefetch_tmap(&tm_a1);
+    if (MODE != kModeGemm1) {
+      prefetch_tmap(&tm_a2);
+      prefetch_tmap(&tm_b2);
+      if (!p.fuse_combine) prefetch_tmap(&tm_out);
+    }
   }
   if (warp == kMmaWarp) {
     if (CG == 2) {
@@ -283,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // both CTAs' barriers exist before any traffic crosses the pair
   if (CG == 2) cluster_sync();
   // Everything above overlaps the previous kernel under PDL; the routing
-  // permutation (and, for GEMM2, act) is read only after this point.
+  // permutation (and the A rows) are read only after this point.
   grid_dep_wait();
   grid_dep_launch();
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_exp_off[i] = p.expert_offsets[i];
@@ -294,9 +359,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
 
   const uint32_t tmem_base = bars->tmem_base;
-  const int NT = p.n_tiles_n;
-  const int total = s_tile_off[p.E] * NT;
-  const int KB = p.K / BK;
+  const int m_tiles = s_tile_off[p.E];
+  const int total1 = MODE == kModeGemm2 ? 0 : m_tiles * p.nt1;
+  const int total =
+      total1 + (MODE == kModeGemm1 || (MODE == kModeFused && !p.run_gemm2) ? 0 : m_tiles * p.nt2);
   const int unit = CG == 2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int nunits = CG == 2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   volatile int *abort_flag = &bars->abort_flag;
@@ -310,10 +376,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (kGather) {
       const int c = threadIdx.x & 7;      // 16-byte chunk of the 128-byte row
       const int rsub = threadIdx.x >> 3;  // rows rsub, rsub+16, ..., rsub+112
-      int it = 0;
+      const int KB = p.H / BK;
+      int s = 0;  // ring slot and its phase parity, advanced per k-block
+      uint32_t ph = 0;
       bool stop = false;
       for (int t = unit; t < total && !stop; t += nunits) {
-        const Tile tl = decode_tile<TM>(t, NT, p.E, s_tile_off, s_exp_off);
+        const Tile tl = get_work<MODE>(t, total1, p, s_tile_off, s_exp_off).tl;
         const __nv_bfloat16 *src[8];
         uint32_t nbytes[8];
 #pragma unroll
@@ -328,10 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             nbytes[i] = 0;
           }
         }
-        const int b_row = tl.e * p.b_rows_per_expert + tl.nt * (kAccN / 2);
-        for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
+        const int b_row = tl.e * 2 * p.I + tl.nt * (kAccN / 2);
+        for (int kb = 0; kb < KB; ++kb, s = s + 1 == kStages ? 0 : s + 1, ph ^= s == 0) {
           if (!mbar_wait(&bars->empty[s], ph ^ 1, limit, abort_flag)) {
             give_up(p, abort_flag);
             stop = true;
@@ -340,8 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (threadIdx.x == 0) {
             mbar_arrive_expect_tx(&bars->full[s], kBBytes);
             uint8_t *b = sB + s * kBBytes;
-            tma_load_2d(b, &tm_b, &bars->full[s], kb * BK, b_row);                       // gate
-            tma_load_2d(b + kBBytes / 2, &tm_b, &bars->full[s], kb * BK, b_row + p.I);  // up
+            tma_load_2d(b, &tm_b1, &bars->full[s], kb * BK, b_row);                       // gate
+            tma_load_2d(b + kBBytes / 2, &tm_b1, &bars->full[s], kb * BK, b_row + p.I);  // up
           }
           const uint32_t a_base = smem_addr(sA + s * kABytes);
 #pragma unroll
@@ -361,30 +427,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     } else if (threadIdx.x == 0) {
-      int it = 0;
+      int s = 0;  // ring slot and its phase parity, advanced per k-block
+      uint32_t ph = 0;
       bool stop = false;
       for (int t = unit; t < total && !stop; t += nunits) {
-        const Tile tl = decode_tile<TM>(t, NT, p.E, s_tile_off, s_exp_off);
-        const int a_row = tl.row0 + static_cast<int>(rank) * BM;
+        const Work w = get_work<MODE>(t, total1, p, s_tile_off, s_exp_off);
+        if (MODE == kModeFused && w.phase == 2) {
+          // the act rows of this m-tile come from other CTAs' GEMM1 epilogues
+          if (!wait_geq(p.ready + w.mi, kReadyPerTile * p.nt1, limit, abort_flag)) {
+            give_up(p, abort_flag);
+            break;
+          }
+          fence_proxy_async_global();
+        }
+        const bool g1 = w.phase == 1;
+        const CUtensorMap *am = g1 ? &tm_a1 : &tm_a2;
+        const CUtensorMap *bm = g1 ? &tm_b1 : &tm_b2;
+        const int KB = (g1 ? p.H : p.I) / BK;
+        const int a_row = w.tl.row0 + static_cast<int>(rank) * BM;
         // GEMM1: rank 0 the n-tile's gate rows, rank 1 its up rows;
         // GEMM2: rank r rows 128r.. of the n-tile's 256 rows of w2
-        const int b_row = tl.e * p.b_rows_per_expert +
-                          (kSwiglu ? static_cast<int>(rank) * p.I + tl.nt * (kAccN / 2)
-                                   : tl.nt * kAccN + static_cast<int>(rank) * C::kBRows);
-        for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
+        const int b_row = g1 ? w.tl.e * 2 * p.I + static_cast<int>(rank) * p.I +
+                                   w.tl.nt * (kAccN / 2)
+                             : w.tl.e * p.H + w.tl.nt * kAccN + static_cast<int>(rank) * C::kBRows;
+        for (int kb = 0; kb < KB; ++kb, s = s + 1 == kStages ? 0 : s + 1, ph ^= s == 0) {
           if (!mbar_wait(&bars->empty[s], ph ^ 1, limit, abort_flag)) {
             give_up(p, abort_flag);
             stop = true;
             break;
           }
           if (leader) mbar_arrive_expect_tx(&bars->full[s], CG * (kABytes + kBBytes));
-          tma_load_2d_pair(sA + s * kABytes, &tm_a, full0 + 8u * s, kb * BK, a_row);
-          tma_load_2d_pair(sB + s * kBBytes, &tm_b, full0 + 8u * s, kb * BK, b_row);
+          tma_load_2d_pair(sA + s * kABytes, am, full0 + 8u * s, kb * BK, a_row);
+          tma_load_2d_pair(sB + s * kBBytes, bm, full0 + 8u * s, kb * BK, b_row);
         }
       }
-      if (stop) {
+      if (*abort_flag) {
         const uint64_t t0 = global_timer_ns();
         while (global_timer_ns() - t0 < 200000) {
         }
@@ -394,9 +471,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && leader) {
       // ---------------------------------------------------------- MMA issuer
       const uint32_t idesc = idesc_bf16_f32(TM, kAccN);
-      int it = 0, acc_it = 0;
+      int s = 0, acc_it = 0;  // ring slot and its phase parity, advanced per k-block
+      uint32_t ph = 0;
       bool stop = false;
       for (int t = unit; t < total && !stop; t += nunits, ++acc_it) {
+        const int KB = (get_work<MODE>(t, total1, p, s_tile_off, s_exp_off).phase == 1 ? p.H : p.I) / BK;
         const int a = acc_it & 1;
         const uint32_t aph = (acc_it >> 1) & 1;
         if (!mbar_wait(&bars->acc_empty[a], aph ^ 1, limit, abort_flag)) {
@@ -405,9 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + a * kAccN;
-        for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
+        for (int kb = 0; kb < KB; ++kb, s = s + 1 == kStages ? 0 : s + 1, ph ^= s == 0) {
           if (!mbar_wait(&bars->full[s], ph, limit, abort_flag)) {
             give_up(p, abort_flag);
             stop = true;
@@ -457,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = ew >> 2;               // which half of the tile's columns
     const int row = q * 32 + lane;
     uint8_t *ebuf = sEpi + ew * kEpiWarpBytes;  // GEMM2: this warp's staging buffer
-    if (kSwiglu && p.zero_n4 > 0) {
+    if (MODE != kModeGemm2 && p.zero_n4 > 0) {
       // out must read zero before GEMM2 adds into it; this runs while the
       // first tiles' MMAs are in flight
       const int64_t nw = static_cast<int64_t>(gridDim.x) * kEpiWarps;
@@ -465,9 +542,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t i = (static_cast<int64_t>(blockIdx.x) * kEpiWarps + ew) * 32 + lane;
            i < p.zero_n4; i += nw * 32)
         p.zero_out[i] = z;
+      if (MODE == kModeFused && p.run_gemm2) {
+        // publish: GEMM2 tiles of any CTA add into out only after every
+        // epilogue warp of the grid has zeroed its part
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(p.zero_done, 1);
+      }
     }
+    bool zero_seen = MODE != kModeFused || p.zero_n4 == 0 || !p.run_gemm2;
     int acc_it = 0;
     for (int t = unit; t < total; t += nunits, ++acc_it) {
+      const Work w = get_work<MODE>(t, total1, p, s_tile_off, s_exp_off);
+      const Tile &tl = w.tl;
       const int a = acc_it & 1;
       const uint32_t aph = (acc_it >> 1) & 1;
       if (!mbar_wait(&bars->acc_full[a], aph, limit, abort_flag)) {
@@ -475,12 +562,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after_sync();
-      const Tile tl = decode_tile<TM>(t, NT, p.E, s_tile_off, s_exp_off);
       const int my_row0 = tl.row0 + static_cast<int>(rank) * BM;
       const int my_rows = min(BM, max(0, tl.rows - static_cast<int>(rank) * BM));
       const bool valid = row < my_rows;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kAccN;
-      if (kSwiglu) {
+      if (w.phase == 1) {
         __nv_bfloat16 *dst =
             p.act + static_cast<size_t>(my_row0 + (valid ? row : 0)) * p.I + tl.nt * (kAccN / 2);
 #pragma unroll 1
@@ -505,6 +591,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
         }
       } else if (p.fuse_combine) {
+        if (!zero_seen) {
+          if (!wait_geq(p.zero_done, static_cast<int>(gridDim.x) * kEpiWarps, limit, abort_flag))
+            give_up(p, abort_flag);
+          fence_proxy_async_global();
+          zero_seen = true;
+        }
         // row -> (token, weight); each lane stages and reduces its own row,
         // so the lanes need no synchronisation with one another
         float wgt = 0.f;
@@ -521,8 +613,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_32cols(tbase + c0, v);
           tmem_ld_wait();
           const int col = tl.nt * kAccN + c0;
-          if (col < p.H && valid) {
-            // the previous reduction from this row buffer must have read it
+          if (col < p.H && valid && !*abort_flag) {
+            // the previous reduction from this row must have read it
             bulk_wait_group_read<0>();
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -544,24 +636,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_32cols(tbase + c0, v);
           tmem_ld_wait();
           const int col = tl.nt * kAccN + c0;
-          if (col >= p.H) continue;  // masked half of a last n-tile (H % 256 == 128)
-          if (whole) {
-            uint8_t *blk = ebuf;
+          if (col < p.H && whole) {
             // the previous store from this buffer must have read it
             if (lane == 0) bulk_wait_group_read<0>();
             __syncwarp();
             // row `lane` as 8 chunks of 16 bytes, 128-byte swizzle
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<uint4 *>(blk + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+              *reinterpret_cast<uint4 *>(ebuf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
                   make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tm_out, blk, col, my_row0 + q * 32);
+              tma_store_2d(&tm_out, ebuf, col, my_row0 + q * 32);
               bulk_commit_group();
             }
-          } else if (valid) {
+          } else if (col < p.H && valid) {
             // the block crosses the end of the expert's rows: plain stores
             float4 *d4 = reinterpret_cast<float4 *>(
                 p.P + static_cast<size_t>(my_row0 + row) * p.H + col);
@@ -581,8 +671,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         else
           mbar_arrive(&bars->acc_empty[a]);
       }
+      if (MODE == kModeFused && w.phase == 1 && p.run_gemm2) {
+        // publish this warp's act rows of the m-tile to GEMM2 tiles (after
+        // the accumulator is released, so the fence does not hold up MMAs)
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(p.ready + w.mi, 1);
+      }
     }
-    if (MODE == kModeGemm2) bulk_wait_group_all();
+    if (MODE != kModeGemm1) bulk_wait_group_all();
   }
 
   tc_fence_before_sync();
@@ -650,15 +747,18 @@ bool make_bf16_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t ou
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, inner, outer, BK, box_rows);
 }
 
-int g_max_pairs[64] = {};  // 2-CTA clusters of GEMM2 resident at once, per device
+int g_max_pairs[64] = {};  // 2-CTA clusters resident at once, per device
 
 template <int MODE>
 int grid_for(const GroupedGemmArgs &a, int n_tiles_n, int device) {
   constexpr int CG = Cfg<MODE>::CG;
   const int64_t rows = a.T * a.k;
   const int64_t max_tiles = ((rows + tile_m<MODE>() - 1) / tile_m<MODE>() + a.E) * n_tiles_n;
+  // never more units than can be resident together: the fused kernel's
+  // GEMM2 tiles wait for other CTAs' GEMM1 tiles
   int units = a.num_sms / CG;
-  if (CG == 2 && device >= 0 && device < 64 && g_max_pairs[device] > 0) units = g_max_pairs[device];
+  if (CG == 2 && device >= 0 && device < 64 && g_max_pairs[device] > 0)
+    units = std::min(units, g_max_pairs[device]);
   if (max_tiles < units) units = static_cast<int>(max_tiles);
   return CG * (units > 0 ? units : 1);
 }
@@ -674,21 +774,29 @@ Params base_params(const GroupedGemmArgs &a) {
   p.I = a.I;
   p.E = a.E;
   p.k = a.k;
+  p.nt1 = a.I / (kAccN / 2);
+  p.nt2 = (a.H + kAccN - 1) / kAccN;  // H % 128 == 0: a last half tile is masked
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
+  p.fuse_combine = a.fuse_combine;
   if (a.fuse_combine) {
     p.out = a.out;
     p.topk_weights = a.topk_weights;
+    p.zero_out = reinterpret_cast<float4 *>(a.out);
+    p.zero_n4 = a.T * a.H / 4;
   }
+  p.ready = a.ready;
+  p.zero_done = a.zero_done;
   return p;
 }
 
 template <int MODE>
-cudaLaunchConfig_t launch_config(int grid, cudaStream_t s, bool pdl, cudaLaunchAttribute (&attr)[2]) {
+cudaLaunchConfig_t launch_config(int grid, size_t smem, cudaStream_t s, bool pdl,
+                                 cudaLaunchAttribute (&attr)[2]) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem_bytes<MODE>();
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   int n = 0;
   if (Cfg<MODE>::CG == 2) {
@@ -708,6 +816,44 @@ cudaLaunchConfig_t launch_config(int grid, cudaStream_t s, bool pdl, cudaLaunchA
   return cfg;
 }
 
+template <int MODE>
+cudaError_t set_smem_attr() {
+  return cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(kSmemMax));
+}
+
+template <int MODE>
+cudaError_t max_pairs(int *clusters) {
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = launch_config<MODE>(2, kSmemMax, nullptr, false, attr);
+  return cudaOccupancyMaxActiveClusters(clusters, grouped_gemm_kernel<MODE>, &cfg);
+}
+
+// The maps GEMM2 uses: act [T*k, I] and w2 [E*H, I] with 64 x 128-row boxes,
+// and P [T*k, H] fp32 in 32 x 32 blocks (a stand-in map over act when P is
+// not written).
+bool gemm2_maps(const GroupedGemmArgs &a, CUtensorMap *tm_act, CUtensorMap *tm_w2,
+                CUtensorMap *tm_p) {
+  const uint64_t rows = static_cast<uint64_t>(a.T) * a.k;
+  if (!make_bf16_map(tm_act, a.act, static_cast<uint64_t>(a.I), rows, BM) ||
+      !make_bf16_map(tm_w2, a.w2, static_cast<uint64_t>(a.I), static_cast<uint64_t>(a.E) * a.H,
+                     Cfg<kModeGemm2>::kBRows))
+    return false;
+  if (a.P == nullptr) {
+    *tm_p = *tm_act;
+    return true;
+  }
+  return make_map(tm_p, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.P, static_cast<uint64_t>(a.H), rows,
+                  32, 32);
+}
+
+// w1 [E*2I, H], box 64 x 128 rows (128 gate or 128 up rows of an n-tile)
+bool w1_map(const GroupedGemmArgs &a, CUtensorMap *tm_w1) {
+  return make_bf16_map(tm_w1, a.w1, static_cast<uint64_t>(a.H),
+                       static_cast<uint64_t>(a.E) * 2 * a.I, kAccN / 2);
+}
+
 }  // namespace
 
 cudaError_t grouped_gemm_setup(int device) {
@@ -715,30 +861,17 @@ cudaError_t grouped_gemm_setup(int device) {
   static uint64_t done_mask = 0;
   std::lock_guard<std::mutex> lock(mu);
   if (device >= 0 && device < 64 && (done_mask >> device) & 1) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<kModeGemm1>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem_bytes<kModeGemm1>()));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(grouped_gemm_kernel<kModeGemm2>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem_bytes<kModeGemm2>()));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(grouped_gemm_kernel<kModeGemm1Pair>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem_bytes<kModeGemm1Pair>()));
+  cudaError_t e = set_smem_attr<kModeGemm1>();
+  if (e == cudaSuccess) e = set_smem_attr<kModeGemm2>();
+  if (e == cudaSuccess) e = set_smem_attr<kModeFused>();
   if (e != cudaSuccess) return e;
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
   // how many 2-CTA clusters can be resident at once (both pair kernels take
-  // one CTA per SM; the smaller count of the two is used for both)
-  cudaLaunchAttribute attr[2];
-  cudaLaunchConfig_t cfg = launch_config<kModeGemm2>(2, nullptr, false, attr);
-  int clusters = 0, clusters1 = 0;
-  e = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<kModeGemm2>, &cfg);
-  if (e == cudaSuccess) {
-    cfg = launch_config<kModeGemm1Pair>(2, nullptr, false, attr);
-    e = cudaOccupancyMaxActiveClusters(&clusters1, grouped_gemm_kernel<kModeGemm1Pair>, &cfg);
-    clusters = std::min(clusters, clusters1);
-  }
+  // one CTA per SM; the smaller count is used for both)
+  int c2 = 0, cf = 0;
+  e = max_pairs<kModeGemm2>(&c2);
+  if (e == cudaSuccess) e = max_pairs<kModeFused>(&cf);
+  const int clusters = std::min(c2, cf);
   if (e != cudaSuccess || clusters < 1) {
     cudaGetLastError();
     return e != cudaSuccess ? e : cudaErrorNotSupported;
@@ -751,59 +884,62 @@ cudaError_t grouped_gemm_setup(int device) {
 }
 
 cudaError_t launch_gemm1_swiglu(const GroupedGemmArgs &a, cudaStream_t s, const StageHook &hook) {
-  CUtensorMap tm_w1, tm_xs;
-  if (!make_bf16_map(&tm_w1, a.w1, static_cast<uint64_t>(a.H),
-                     static_cast<uint64_t>(a.E) * 2 * a.I, kAccN / 2))
-    return cudaErrorInvalidValue;
-  if (a.xs != nullptr && !make_bf16_map(&tm_xs, a.xs, static_cast<uint64_t>(a.H),
-                                        static_cast<uint64_t>(a.T) * a.k, BM))
-    return cudaErrorInvalidValue;
+  CUtensorMap tm_w1;
+  if (!w1_map(a, &tm_w1)) return cudaErrorInvalidValue;
   int dev = 0;
   cudaGetDevice(&dev);
   Params p = base_params(a);
-  if (a.fuse_combine) {
-    p.zero_out = reinterpret_cast<float4 *>(a.out);
-    p.zero_n4 = a.T * a.H / 4;
-  }
-  p.K = a.H;
-  p.n_tiles_n = a.I / (kAccN / 2);
-  p.b_rows_per_expert = 2 * a.I;
+  p.stages = stages_for<kModeGemm1>(a.E);
   cudaLaunchAttribute attr[2];
+  const cudaLaunchConfig_t cfg =
+      launch_config<kModeGemm1>(grid_for<kModeGemm1>(a, p.nt1, dev),
+                                smem_bytes<kModeGemm1>(a.E, p.stages), s, hook.pdl, attr);
   hook.begin("gemm1_swiglu");
-  cudaError_t e;
-  if (a.xs != nullptr) {
-    const cudaLaunchConfig_t cfg = launch_config<kModeGemm1Pair>(
-        grid_for<kModeGemm1Pair>(a, p.n_tiles_n, dev), s, hook.pdl, attr);
-    e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm1Pair>, tm_xs, tm_w1, tm_xs, p);
-  } else {
-    const cudaLaunchConfig_t cfg =
-        launch_config<kModeGemm1>(grid_for<kModeGemm1>(a, p.n_tiles_n, dev), s, hook.pdl, attr);
-    e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm1>, tm_w1, tm_w1, tm_w1, p);
-  }
+  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm1>, tm_w1, tm_w1, tm_w1,
+                                     tm_w1, tm_w1, p);
   return hook.end(e);
 }
 
 cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s, const StageHook &hook) {
   CUtensorMap tm_act, tm_w2, tm_p;
-  const uint64_t rows = static_cast<uint64_t>(a.T) * a.k;
-  if (!make_bf16_map(&tm_act, a.act, static_cast<uint64_t>(a.I), rows, BM) ||
-      !make_bf16_map(&tm_w2, a.w2, static_cast<uint64_t>(a.I), static_cast<uint64_t>(a.E) * a.H,
-                     Cfg<kModeGemm2>::kBRows) ||
-      !make_map(&tm_p, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.P, static_cast<uint64_t>(a.H), rows,
-                32, 32))
+  if (!gemm2_maps(a, &tm_act, &tm_w2, &tm_p)) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  Params p = base_params(a);
+  p.zero_out = nullptr;  // zeroed by GEMM1
+  p.zero_n4 = 0;
+  p.stages = stages_for<kModeGemm2>(a.E);
+  cudaLaunchAttribute attr[2];
+  const cudaLaunchConfig_t cfg =
+      launch_config<kModeGemm2>(grid_for<kModeGemm2>(a, p.nt2, dev),
+                                smem_bytes<kModeGemm2>(a.E, p.stages), s, hook.pdl, attr);
+  hook.begin("gemm2");
+  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm2>, tm_act, tm_w2, tm_act,
+                                     tm_w2, tm_p, p);
+  return hook.end(e);
+}
+
+cudaError_t launch_fused_gemm(const GroupedGemmArgs &a, bool with_gemm2, cudaStream_t s,
+                              const StageHook &hook) {
+  if (a.xs == nullptr || (with_gemm2 && (a.ready == nullptr || a.zero_done == nullptr)))
+    return cudaErrorInvalidValue;
+  CUtensorMap tm_xs, tm_w1, tm_act, tm_w2, tm_p;
+  if (!make_bf16_map(&tm_xs, a.xs, static_cast<uint64_t>(a.H), static_cast<uint64_t>(a.T) * a.k,
+                     BM) ||
+      !w1_map(a, &tm_w1) || !gemm2_maps(a, &tm_act, &tm_w2, &tm_p))
     return cudaErrorInvalidValue;
   int dev = 0;
   cudaGetDevice(&dev);
   Params p = base_params(a);
-  p.fuse_combine = a.fuse_combine;
-  p.K = a.I;
-  p.n_tiles_n = (a.H + kAccN - 1) / kAccN;  // H % 128 == 0: a last half tile is masked
-  p.b_rows_per_expert = a.H;
+  p.run_gemm2 = with_gemm2 ? 1 : 0;
+  p.stages = stages_for<kModeFused>(a.E, with_gemm2);
   cudaLaunchAttribute attr[2];
-  const cudaLaunchConfig_t cfg =
-      launch_config<kModeGemm2>(grid_for<kModeGemm2>(a, p.n_tiles_n, dev), s, hook.pdl, attr);
-  hook.begin("gemm2");
-  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm2>, tm_act, tm_w2, tm_p, p);
+  const cudaLaunchConfig_t cfg = launch_config<kModeFused>(
+      grid_for<kModeFused>(a, with_gemm2 ? p.nt1 + p.nt2 : p.nt1, dev),
+      smem_bytes<kModeFused>(a.E, p.stages, with_gemm2), s, hook.pdl, attr);
+  hook.begin(with_gemm2 ? "gemm_fused" : "gemm1_swiglu");
+  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeFused>, tm_xs, tm_w1, tm_act,
+                                     tm_w2, tm_p, p);
   return hook.end(e);
 }
 

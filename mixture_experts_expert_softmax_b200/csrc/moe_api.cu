@@ -17,6 +17,9 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 16;
+// above this many waves of GEMM tiles (per resident CTA pair) the two GEMMs
+// run as separate launches
+constexpr int64_t kFusedMaxWaves = 12;
 
 std::mutex g_mu;  // guards the per-device state and the profiler
 
@@ -288,9 +291,12 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
   // token and lets GEMM1 run on CTA pairs with TMA operands; with few slots
   // per token that pays off.
   const bool gather_rows = k <= 2;
+  const int64_t n_ready = moe::fused_gemm_ready_count(n, E);
   const size_t need = permute_ws_bytes(n, E) + align256(static_cast<size_t>(n) * 4) +
                       align256(static_cast<size_t>(n) * I * 2) +
-                      (gather_rows ? align256(static_cast<size_t>(n) * H * 2) : 0) +
+                      (gather_rows ? align256(static_cast<size_t>(n) * H * 2) +
+                                         align256(static_cast<size_t>(n_ready + 1) * 4)
+                                   : 0) +
                       (fuse_combine ? 0 : align256(static_cast<size_t>(n) * H * sizeof(float)));
   if ((rc = ensure_workspace(*d, need)) != MOE_OK) return rc;
   Carver cv{static_cast<char *>(d->ws)};
@@ -302,6 +308,7 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
   uint16_t *act = cv.take<uint16_t>(static_cast<size_t>(n) * I);
   float *P = fuse_combine ? nullptr : cv.take<float>(static_cast<size_t>(n) * H);
   uint16_t *xs = gather_rows ? cv.take<uint16_t>(static_cast<size_t>(n) * H) : nullptr;
+  int *ready = gather_rows ? cv.take<int>(static_cast<size_t>(n_ready) + 1) : nullptr;
 
   // the forward's result does not depend on the order of rows inside an
   // expert, so a single-CTA grouping replaces the stable three-kernel one
@@ -311,9 +318,10 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
                       : moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets,
                                             sorted_rows, inv, d->status, ctx.stream, hook);
   if (e != cudaSuccess) return to_code(e);
-  if (gather_rows && (e = moe::launch_gather_rows(hidden, H, k, sorted_rows, expert_offsets, E, n,
-                                                  d->num_sms, xs, ctx.stream, hook)) !=
-                         cudaSuccess)
+  if (gather_rows &&
+      (e = moe::launch_gather_rows(hidden, H, k, sorted_rows, expert_offsets, E, n, d->num_sms, xs,
+                                   ready, static_cast<int>(n_ready), ready + n_ready, ctx.stream,
+                                   hook)) != cudaSuccess)
     return to_code(e);
   moe::GroupedGemmArgs ga = {};
   ga.hidden = hidden;
@@ -335,8 +343,22 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
   ga.out = out;
   ga.topk_weights = topk_weights;
   ga.fuse_combine = fuse_combine ? 1 : 0;
-  if ((e = moe::launch_gemm1_swiglu(ga, ctx.stream, hook)) != cudaSuccess) return to_code(e);
-  if ((e = moe::launch_gemm2(ga, ctx.stream, hook)) != cudaSuccess) return to_code(e);
+  if (gather_rows) {
+    ga.ready = ready;
+    ga.zero_done = ready + n_ready;
+    // One launch for both GEMMs fills GEMM1's last partial wave with GEMM2
+    // tiles; with many waves that gain is small and two launches, each with
+    // the deepest operand ring its shared memory allows, run faster.
+    const int64_t tiles = ((n + 255) / 256) * (I / 128 + (H + 255) / 256);
+    const bool one_launch = tiles <= kFusedMaxWaves * std::max(1, d->num_sms / 2);
+    if ((e = moe::launch_fused_gemm(ga, one_launch, ctx.stream, hook)) != cudaSuccess)
+      return to_code(e);
+    if (!one_launch && (e = moe::launch_gemm2(ga, ctx.stream, hook)) != cudaSuccess)
+      return to_code(e);
+  } else {
+    if ((e = moe::launch_gemm1_swiglu(ga, ctx.stream, hook)) != cudaSuccess) return to_code(e);
+    if ((e = moe::launch_gemm2(ga, ctx.stream, hook)) != cudaSuccess) return to_code(e);
+  }
   if (fuse_combine) return MOE_OK;
   e = moe::launch_combine(P, inv, topk_weights, out, T, H, k, d->status, ctx.stream, hook);
   return to_code(e);

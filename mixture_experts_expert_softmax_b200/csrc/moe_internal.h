@@ -54,10 +54,12 @@ cudaError_t launch_permute_fused(const int32_t *ids, int64_t n, int E, int32_t *
                                  cudaStream_t s, const StageHook &hook);
 
 // Expert-sorted copy of the hidden rows, xs[r] = hidden[sorted_rows[r] / k]
-// for r < expert_offsets[E] (device value); n = T*k bounds the grid.
+// for r < expert_offsets[E] (device value); n = T*k bounds the grid.  Also
+// zeroes the fused GEMM's counters: ready[0..n_ready) and *zero_done.
 cudaError_t launch_gather_rows(const uint16_t *hidden, int H, int k, const int32_t *sorted_rows,
                                const int32_t *expert_offsets, int E, int64_t n, int num_sms,
-                               uint16_t *xs, cudaStream_t s, const StageHook &hook);
+                               uint16_t *xs, int *ready, int n_ready, int *zero_done,
+                               cudaStream_t s, const StageHook &hook);
 
 // grouped_gemm.cu
 struct GroupedGemmArgs {
@@ -76,6 +78,10 @@ struct GroupedGemmArgs {
   float *out;                 // [T, H] fp32
   const float *topk_weights;  // [T, k] fp32
   int fuse_combine;
+  // launch_fused_gemm: one counter per 256-row m-tile (at most
+  // fused_gemm_ready_count(T*k, E)) and one more, all zero at launch
+  int *ready;
+  int *zero_done;
   int64_t T;
   int H, I, E, k;
   int num_sms;
@@ -85,6 +91,12 @@ struct GroupedGemmArgs {
 cudaError_t grouped_gemm_setup(int device);
 cudaError_t launch_gemm1_swiglu(const GroupedGemmArgs &a, cudaStream_t s, const StageHook &hook);
 cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s, const StageHook &hook);
+// GEMM1 + SwiGLU on CTA pairs from the expert-sorted rows xs, and (with_gemm2)
+// GEMM2 in the same launch, which needs ready and zero_done.  Without it,
+// launch_gemm2 follows.
+cudaError_t launch_fused_gemm(const GroupedGemmArgs &a, bool with_gemm2, cudaStream_t s,
+                              const StageHook &hook);
+inline int64_t fused_gemm_ready_count(int64_t n, int E) { return (n + 255) / 256 + E; }
 cudaError_t launch_wait_probe(uint32_t *status, uint64_t limit_ns, cudaStream_t s);
 
 // combine.cu

@@ -226,14 +226,19 @@ __global__ void __launch_bounds__(kFusedThreads)
 // Copies the hidden row of every grouped (token, slot) entry into expert-
 // sorted order, xs[r] = hidden[sorted_rows[r] / k], so that GEMM1 can load
 // its A tiles with TMA.  One warp per row, 16-byte chunks; rows past
-// expert_offsets[E] (entries with invalid ids) are not written.
+// expert_offsets[E] (entries with invalid ids) are not written.  Block 0
+// also zeroes the fused GEMM's counters.
 __global__ void __launch_bounds__(256)
     gather_rows_kernel(const uint4 *__restrict__ hidden, int H8, int k,
                        const int32_t *__restrict__ sorted_rows,
                        const int32_t *__restrict__ expert_offsets, int E,
-                       uint4 *__restrict__ xs) {
+                       uint4 *__restrict__ xs, int *ready, int n_ready, int *zero_done) {
   grid_dep_wait();
   grid_dep_launch();
+  if (blockIdx.x == 0) {
+    for (int i = threadIdx.x; i < n_ready; i += blockDim.x) ready[i] = 0;
+    if (threadIdx.x == 0) *zero_done = 0;
+  }
   const int64_t n_valid = expert_offsets[E];
   const int lane = threadIdx.x & 31;
   const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -251,14 +256,16 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_gather_rows(const uint16_t *hidden, int H, int k, const int32_t *sorted_rows,
                                const int32_t *expert_offsets, int E, int64_t n, int num_sms,
-                               uint16_t *xs, cudaStream_t s, const StageHook &hook) {
+                               uint16_t *xs, int *ready, int n_ready, int *zero_done,
+                               cudaStream_t s, const StageHook &hook) {
   const int64_t want = (n + 7) / 8;  // 8 warps per CTA, one row each per pass
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   const int blocks = static_cast<int>(want < cap ? want : cap);
   hook.begin("gather_rows");
   cudaError_t e = launch_pdl(gather_rows_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, s,
                              hook.pdl, reinterpret_cast<const uint4 *>(hidden), H / 8, k,
-                             sorted_rows, expert_offsets, E, reinterpret_cast<uint4 *>(xs));
+                             sorted_rows, expert_offsets, E, reinterpret_cast<uint4 *>(xs), ready,
+                             n_ready, zero_done);
   return hook.end(e);
 }
 
