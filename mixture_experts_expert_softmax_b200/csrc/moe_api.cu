@@ -138,7 +138,7 @@ int current_device(DeviceState **out) {
     if (prop.major != 10 || prop.minor != 0) return MOE_ERR_NO_DEVICE;
     d.num_sms = prop.multiProcessorCount;
     if (cudaMalloc(&d.status, 256) != cudaSuccess || cudaMemset(d.status, 0, 256) != cudaSuccess ||
-        moe::grouped_gemm_setup(dev) != cudaSuccess) {
+        moe::grouped_gemm_setup(dev) != cudaSuccess || moe::group_setup() != cudaSuccess) {
       cudaGetLastError();
       return MOE_ERR_CUDA;
     }
@@ -310,19 +310,24 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
   uint16_t *xs = gather_rows ? cv.take<uint16_t>(static_cast<size_t>(n) * H) : nullptr;
   int *ready = gather_rows ? cv.take<int>(static_cast<size_t>(n_ready) + 1) : nullptr;
 
-  // the forward's result does not depend on the order of rows inside an
-  // expert, so a single-CTA grouping replaces the stable three-kernel one
-  cudaError_t e = moe::permute_fused_supported(n)
-                      ? moe::launch_permute_fused(topk_ids, n, E, expert_offsets, sorted_rows,
-                                                  inv, d->status, ctx.stream, hook)
-                      : moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets,
-                                            sorted_rows, inv, d->status, ctx.stream, hook);
-  if (e != cudaSuccess) return to_code(e);
-  if (gather_rows &&
-      (e = moe::launch_gather_rows(hidden, H, k, sorted_rows, expert_offsets, E, n, d->num_sms, xs,
-                                   ready, static_cast<int>(n_ready), ready + n_ready, ctx.stream,
-                                   hook)) != cudaSuccess)
-    return to_code(e);
+  // grouping (and the sorted row copy): one kernel up to 8192 entries, the
+  // three-kernel grouping and a separate copy above
+  cudaError_t e;
+  if (moe::group_supported(n)) {
+    e = moe::launch_group(topk_ids, n, E, k, expert_offsets, sorted_rows, inv, d->status, hidden,
+                          H, xs, ready, static_cast<int>(n_ready), ready + n_ready, d->num_sms,
+                          ctx.stream, hook);
+    if (e != cudaSuccess) return to_code(e);
+  } else {
+    e = moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets, sorted_rows, inv,
+                            d->status, ctx.stream, hook);
+    if (e != cudaSuccess) return to_code(e);
+    if (gather_rows &&
+        (e = moe::launch_gather_rows(hidden, H, k, sorted_rows, expert_offsets, E, n, d->num_sms,
+                                     xs, ready, static_cast<int>(n_ready), ready + n_ready,
+                                     ctx.stream, hook)) != cudaSuccess)
+      return to_code(e);
+  }
   moe::GroupedGemmArgs ga = {};
   ga.hidden = hidden;
   ga.w1 = w1;

@@ -48,10 +48,17 @@ cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int32_t *chunk_
                            int32_t *expert_offsets, int32_t *sorted_rows, int32_t *inv,
                            uint32_t *status, cudaStream_t s, const StageHook &hook);
 
-bool permute_fused_supported(int64_t n);
-cudaError_t launch_permute_fused(const int32_t *ids, int64_t n, int E, int32_t *expert_offsets,
-                                 int32_t *sorted_rows, int32_t *inv, uint32_t *status,
-                                 cudaStream_t s, const StageHook &hook);
+// Stable grouping of n <= 8192 entries in one kernel (the same result as
+// launch_permute), with the expert-sorted copy of the hidden rows when xs
+// is given (then also zeroing the fused GEMM's counters, as
+// launch_gather_rows does).  group_setup raises the kernel's shared-memory
+// limit once per device.
+bool group_supported(int64_t n);
+cudaError_t group_setup();
+cudaError_t launch_group(const int32_t *ids, int64_t n, int E, int k, int32_t *expert_offsets,
+                         int32_t *sorted_rows, int32_t *inv, uint32_t *status,
+                         const uint16_t *hidden, int H, uint16_t *xs, int *ready, int n_ready,
+                         int *zero_done, int num_sms, cudaStream_t s, const StageHook &hook);
 
 // Expert-sorted copy of the hidden rows, xs[r] = hidden[sorted_rows[r] / k]
 // for r < expert_offsets[E] (device value); n = T*k bounds the grid.  Also

@@ -146,80 +146,139 @@ __global__ void __launch_bounds__(kPermThreads)
   }
 }
 
-// One CTA groups the whole (token, slot) index range by expert: per-expert
-// counts (warp-aggregated shared-memory atomics), an exclusive scan into
-// expert_offsets, then placement with a shared-memory cursor per expert.
-// Positions inside an expert follow atomic order, so the grouping is not
-// stable; the fused forward does not need it to be (each row's products and
-// the fixed-order combine do not depend on where a row sits), and the
-// exported stable grouping uses the three kernels above.
-constexpr int kFusedThreads = 1024;
-constexpr int64_t kFusedMaxN = 8192;  // above this the multi-CTA kernels are faster
+// Grouping of up to kGroupMaxN entries inside one kernel, optionally with
+// the copy of each grouped row's hidden vector into expert-sorted order
+// (xs[r] = hidden[sorted_rows[r] / k]).  Every CTA computes the same stable
+// counting sort in shared memory -- warp w owns a contiguous chunk of the
+// entries and counts it into its own 16-bit histogram row, a scan over
+// (expert, warp) turns the counts into bases, and a second pass ranks each
+// warp step with __match_any_sync -- so the result equals the three-kernel
+// grouping above.  CTA 0 publishes it (expert_offsets, sorted_rows, inv);
+// all CTAs then copy their share of rows from their own copy of the
+// permutation, with no grid-wide synchronisation.  Only CTA 0 runs when
+// nothing is copied.
+constexpr int kGroupThreads = 1024;
+constexpr int kGroupWarps = kGroupThreads / 32;
+constexpr int64_t kGroupMaxN = 8192;  // above this the multi-CTA kernels are faster
+constexpr int kGroupSteps = kGroupMaxN / kGroupThreads;  // 32-entry steps per warp, at most
 
-__global__ void __launch_bounds__(kFusedThreads)
-    permute_fused_kernel(const int32_t *__restrict__ ids, int n, int E,
-                         int32_t *__restrict__ expert_offsets, int32_t *__restrict__ sorted_rows,
-                         int32_t *__restrict__ inv, uint32_t *status) {
-  __shared__ int32_t cnt[1024];
-  __shared__ int32_t warp_tot[32];
+size_t group_smem_bytes(int n, int E) {
+  return static_cast<size_t>((n + 3) & ~3) * sizeof(int32_t) +
+         static_cast<size_t>(kGroupWarps) * E * sizeof(uint16_t);
+}
+
+__global__ void __launch_bounds__(kGroupThreads)
+    group_kernel(const int32_t *__restrict__ ids, int n, int E, int k,
+                 int32_t *__restrict__ expert_offsets, int32_t *__restrict__ sorted_rows,
+                 int32_t *__restrict__ inv, uint32_t *status, const uint4 *__restrict__ hidden,
+                 int H8, uint4 *__restrict__ xs, int *ready, int n_ready, int *zero_done) {
+  extern __shared__ __align__(16) unsigned char group_smem[];
+  int32_t *s_sorted = reinterpret_cast<int32_t *>(group_smem);      // [n]
+  uint16_t *s_hist = reinterpret_cast<uint16_t *>(s_sorted + ((n + 3) & ~3));  // [warps][E]
+  __shared__ int32_t s_warp_tot[kGroupWarps];
+  __shared__ int32_t s_nvalid;
   grid_dep_wait();
   grid_dep_launch();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int e = tid; e < E; e += kFusedThreads) cnt[e] = 0;
-  __syncthreads();
+  const bool publish = blockIdx.x == 0;
+  // entries of warp w: [w * per_warp, (w + 1) * per_warp), a multiple of 32
+  const int per_warp = (n + kGroupThreads - 1) / kGroupThreads * 32;
+  const int i0 = warp * per_warp;
   const uint32_t lt = (1u << lane) - 1u;
-  for (int base = 0; base < n; base += kFusedThreads) {
-    const int i = base + tid;
-    int e = i < n ? __ldg(ids + i) : -1;
-    if (e >= E) e = -1;
+  for (int x = tid; x < kGroupWarps * E; x += kGroupThreads) s_hist[x] = 0;
+  __syncthreads();
+  uint16_t *my_hist = s_hist + warp * E;
+  // the warp's ids, loaded once (per_warp <= 32 * kGroupSteps)
+  int ev[kGroupSteps];
+#pragma unroll
+  for (int q = 0; q < kGroupSteps; ++q) {
+    const int i = i0 + 32 * q + lane;
+    int e = -1;
+    if (32 * q < per_warp && i < n) {
+      e = __ldg(ids + i);
+      if (e < 0 || e >= E) e = -1;
+    }
+    ev[q] = e;
+  }
+#pragma unroll
+  for (int q = 0; q < kGroupSteps; ++q) {
+    if (32 * q >= per_warp) break;
+    const int i = i0 + 32 * q + lane;
+    const int e = ev[q];
     const uint32_t peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && (peers & lt) == 0) atomicAdd(&cnt[e], __popc(peers));
+    if (e >= 0 && (peers & lt) == 0) my_hist[e] += static_cast<uint16_t>(__popc(peers));
+    if (publish && status != nullptr && __any_sync(0xffffffffu, i < n && e < 0) && lane == 0)
+      atomicOr(status, kStatusBadId);
+    __syncwarp();
   }
   __syncthreads();
-  // exclusive scan of cnt[0..E) (E <= 1024 = one entry per thread)
-  const int c = tid < E ? cnt[tid] : 0;
-  int incl = c;
+  // per-expert totals, exclusive scan over experts (E <= 1024: one per thread)
+  int tot = 0;
+  if (tid < E)
+    for (int w = 0; w < kGroupWarps; ++w) tot += s_hist[w * E + tid];
+  int incl = tot;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int x = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += x;
   }
-  if (lane == 31) warp_tot[warp] = incl;
+  if (lane == 31) s_warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int w = warp_tot[lane];
+    int w = s_warp_tot[lane];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int x = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += x;
     }
-    warp_tot[lane] = w;
+    s_warp_tot[lane] = w;
   }
   __syncthreads();
-  const int excl = incl - c + (warp > 0 ? warp_tot[warp - 1] : 0);
-  __syncthreads();
+  const int excl = incl - tot + (warp > 0 ? s_warp_tot[warp - 1] : 0);
   if (tid < E) {
-    cnt[tid] = excl;  // becomes the placement cursor
-    expert_offsets[tid] = excl;
-  }
-  if (tid == E - 1) expert_offsets[E] = excl + c;
-  __syncthreads();
-  for (int base = 0; base < n; base += kFusedThreads) {
-    const int i = base + tid;
-    int e = i < n ? __ldg(ids + i) : -1;
-    if (e >= E) e = -1;
-    const uint32_t peers = __match_any_sync(0xffffffffu, e);
-    if (status != nullptr && __any_sync(0xffffffffu, i < n && e < 0) && lane == 0)
-      atomicOr(status, kStatusBadId);
-    const int leader = __ffs(static_cast<int>(peers)) - 1;
-    int pos0 = 0;
-    if (e >= 0 && lane == leader) pos0 = atomicAdd(&cnt[e], __popc(peers));
-    pos0 = __shfl_sync(0xffffffffu, pos0, leader);
-    if (i < n) {
-      const int pos = e >= 0 ? pos0 + __popc(peers & lt) : -1;
-      if (e >= 0) sorted_rows[pos] = i;
-      inv[i] = pos;
+    if (publish) expert_offsets[tid] = excl;
+    if (tid == E - 1) {
+      s_nvalid = excl + tot;
+      if (publish) expert_offsets[E] = excl + tot;
     }
+    // counts -> running bases, warps in order (positions < n fit 16 bits)
+    int run = excl;
+    for (int w = 0; w < kGroupWarps; ++w) {
+      const int c = s_hist[w * E + tid];
+      s_hist[w * E + tid] = static_cast<uint16_t>(run);
+      run += c;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < kGroupSteps; ++q) {
+    if (32 * q >= per_warp) break;
+    const int i = i0 + 32 * q + lane;
+    const int e = ev[q];
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int pos = e >= 0 ? my_hist[e] + __popc(peers & lt) : -1;
+    __syncwarp();
+    if (e >= 0 && (peers & lt) == 0) my_hist[e] += static_cast<uint16_t>(__popc(peers));
+    if (pos >= 0) s_sorted[pos] = i;
+    if (publish && i < n) {
+      inv[i] = pos;
+      if (pos >= 0) sorted_rows[pos] = i;
+    }
+    __syncwarp();
+  }
+  if (publish && ready != nullptr) {
+    for (int x = tid; x < n_ready; x += kGroupThreads) ready[x] = 0;
+    if (tid == 0) *zero_done = 0;
+  }
+  if (xs == nullptr) return;
+  __syncthreads();
+  const int nv = s_nvalid;
+  for (int r = blockIdx.x * kGroupWarps + warp; r < nv; r += gridDim.x * kGroupWarps) {
+    const int64_t tok = s_sorted[r] / k;
+    const uint4 *src = hidden + tok * H8;
+    uint4 *dst = xs + static_cast<int64_t>(r) * H8;
+#pragma unroll 8
+    for (int c = lane; c < H8; c += 32) dst[c] = __ldg(src + c);
   }
 }
 
@@ -271,16 +330,30 @@ cudaError_t launch_gather_rows(const uint16_t *hidden, int H, int k, const int32
 
 int permute_num_chunks(int64_t n) { return static_cast<int>((n + kChunk - 1) / kChunk); }
 
-bool permute_fused_supported(int64_t n) { return n <= kFusedMaxN; }
+bool group_supported(int64_t n) { return n <= kGroupMaxN; }
 
-cudaError_t launch_permute_fused(const int32_t *ids, int64_t n, int E, int32_t *expert_offsets,
-                                 int32_t *sorted_rows, int32_t *inv, uint32_t *status,
-                                 cudaStream_t s, const StageHook &hook) {
-  hook.begin("permute");
-  // first kernel of the call: ordinary stream order after earlier work
-  cudaError_t err = launch_pdl(permute_fused_kernel, dim3(1), dim3(kFusedThreads), 0, s, false,
-                               ids, static_cast<int>(n), E, expert_offsets, sorted_rows, inv,
-                               status);
+cudaError_t group_setup() {
+  return cudaFuncSetAttribute(group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(group_smem_bytes(kGroupMaxN, 1024)));
+}
+
+cudaError_t launch_group(const int32_t *ids, int64_t n, int E, int k, int32_t *expert_offsets,
+                         int32_t *sorted_rows, int32_t *inv, uint32_t *status,
+                         const uint16_t *hidden, int H, uint16_t *xs, int *ready, int n_ready,
+                         int *zero_done, int num_sms, cudaStream_t s, const StageHook &hook) {
+  int grid = 1;
+  if (xs != nullptr) {
+    const int64_t want = (n + kGroupWarps - 1) / kGroupWarps;  // one row per warp
+    grid = static_cast<int>(want < num_sms ? want : num_sms);
+    if (grid < 1) grid = 1;
+  }
+  hook.begin(xs != nullptr ? "group_gather" : "permute");
+  // may start under the previous kernel (it waits for it before reading ids)
+  cudaError_t err = launch_pdl(group_kernel, dim3(grid), dim3(kGroupThreads),
+                               group_smem_bytes(static_cast<int>(n), E), s, hook.pdl, ids,
+                               static_cast<int>(n), E, k, expert_offsets, sorted_rows, inv, status,
+                               reinterpret_cast<const uint4 *>(hidden), H / 8,
+                               reinterpret_cast<uint4 *>(xs), ready, n_ready, zero_done);
   return hook.end(err);
 }
 
@@ -291,9 +364,9 @@ cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int32_t *chunk_
   cudaError_t err;
   if (n_chunks > 0) {
     hook.begin("permute_count");
-    // first kernel of the call: ordinary stream order after earlier work
+    // may start under the previous kernel (it waits for it before reading ids)
     err = launch_pdl(permute_count_kernel, dim3(n_chunks), dim3(kPermThreads),
-                     static_cast<size_t>(E) * sizeof(int32_t), s, false, ids, n, E,
+                     static_cast<size_t>(E) * sizeof(int32_t), s, hook.pdl, ids, n, E,
                      chunk_counts);
     if ((err = hook.end(err)) != cudaSuccess) return err;
   }

@@ -21,7 +21,9 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
                  int32_t *__restrict__ ids, float *__restrict__ weights) {
   const int lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kRouteWarps + (threadIdx.x >> 5);
+  // may start under the previous kernel: wait for it before reading logits
   grid_dep_wait();
+  grid_dep_launch();
   if (t >= T) return;
   const float *row = logits + t * E;
 
@@ -95,9 +97,8 @@ template <int VPT>
 cudaError_t launch_route_vpt(const float *logits, int64_t T, int E, int k, int renorm,
                              int32_t *ids, float *weights, cudaStream_t s) {
   const int64_t blocks = (T + kRouteWarps - 1) / kRouteWarps;
-  route_kernel<VPT><<<static_cast<unsigned>(blocks), kRouteWarps * 32, 0, s>>>(
-      logits, T, E, k, renorm, ids, weights);
-  return cudaGetLastError();
+  return launch_pdl(route_kernel<VPT>, dim3(static_cast<unsigned>(blocks)), dim3(kRouteWarps * 32),
+                    0, s, true, logits, T, E, k, renorm, ids, weights);
 }
 
 }  // namespace

@@ -327,7 +327,7 @@ def test_sync_each_stage_mode_and_profiler():
     prof = moe.profile_read()
     # top-2: hidden rows copied into expert order, both GEMMs in one launch
     # that also adds into out, no separate combine
-    for kname in ("permute", "gather_rows", "gemm_fused"):
+    for kname in ("group_gather", "gemm_fused"):
         assert prof[kname][0] == 1 and prof[kname][1] > 0
     assert "combine" not in prof and "gemm2" not in prof
     ref = oracle.moe_token_loop(hidden, w1, w2, w, ids)
