@@ -28,7 +28,7 @@ struct DeviceState {
   bool usable = false;
   int num_sms = 0;
   uint32_t *status = nullptr;  // 256 B: status word at 0, small-T grid counter at 64
-  unsigned long long small_t_launches = 0;
+  unsigned long long small_t_arrivals = 0;  // small-T grid-barrier counter target
   void *ws = nullptr;          // grow-only workspace
   size_t ws_bytes = 0;
 };
@@ -282,7 +282,7 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
     return to_code(moe::launch_small_t(
         hidden, w1, w2, topk_weights, topk_ids, act, out, T, H, I, E, k, d->status,
         reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(d->status) + 64),
-        &d->small_t_launches, static_cast<uint64_t>(g_wait_limit_ns), ctx.stream, hook));
+        &d->small_t_arrivals, static_cast<uint64_t>(g_wait_limit_ns), ctx.stream, hook));
   }
 
   // top-k <= 2: GEMM2 adds its rows straight into out and no P is needed

@@ -114,12 +114,13 @@ cudaError_t launch_combine(const float *P, const int32_t *inv, const float *topk
 // small_t.cu
 bool small_t_supported(int H, int I);
 // grid_sync: a 64-bit device counter that only this launcher's kernels
-// touch, 0 before the first launch; launches: host count of launches made
-// with it (advanced by the call).
+// touch, 0 before the first launch; arrivals: the host's copy of the value
+// it reaches once every launch made so far has finished (advanced by the
+// call).  act: T*k*I fp32 scratch.
 cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
                            const float *topk_weights, const int32_t *topk_ids, float *act,
                            float *out, int64_t T, int H, int I, int E, int k, uint32_t *status,
-                           unsigned long long *grid_sync, unsigned long long *launches,
+                           unsigned long long *grid_sync, unsigned long long *arrivals,
                            uint64_t wait_limit_ns, cudaStream_t s, const StageHook &hook);
 
 }  // namespace moe

@@ -35,7 +35,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 std::mutex g_noalloc_mu;
 void *g_noalloc_addr[kNoAllocMaxDevices] = {};
-unsigned long long g_noalloc_launches[kNoAllocMaxDevices] = {};
+unsigned long long g_noalloc_arrivals[kNoAllocMaxDevices] = {};
 
 }  // namespace
 
@@ -92,7 +92,7 @@ extern "C" int moe_forward_small_noalloc(const uint16_t *hidden, const uint16_t 
   hook.pdl = true;
   const cudaError_t e =
       moe::launch_small_t(hidden, w1, w2, topk_weights, topk_ids, act, out, T, H, I, E, k, status,
-                          grid_sync, &g_noalloc_launches[dev], 2000000000ull,
+                          grid_sync, &g_noalloc_arrivals[dev], 2000000000ull,
                           static_cast<cudaStream_t>(stream), hook);
   if (e != cudaSuccess) {
     cudaGetLastError();

@@ -1,24 +1,27 @@
 // small_t.cu -- the fused MoE forward for a handful of tokens (decode).
-// With T <= 16 the work is a stream over the chosen experts' weights, so it
-// runs as one persistent, HBM-bound streaming kernel instead of tensor-core
-// tiles: one CTA per SM (a cooperative launch, so all CTAs are resident),
-// one producer thread that moves weights with bulk async copies (the TMA
-// engine) through a ring of shared-memory stages, and eight consumer warps.
+// With T <= 16 the work is a stream over the chosen experts' weights (tens
+// of MB; the arithmetic is negligible), so it runs as one HBM-bound GEMV
+// kernel on the CUDA cores: every warp streams whole weight rows with
+// 128-bit loads, many rows in flight per SM, so that the loads alone keep
+// HBM busy.  One cooperative launch (all CTAs resident, one per SM, 16
+// compute warps and one copy warp):
 //
-//   phase 1 (gate/up + SwiGLU): the work is (distinct chosen expert, row
-//     pair), row pair i = (w1[e, i, :] gate, w1[e, I+i, :] up); chunks of
-//     consecutive row pairs of one expert are dealt round-robin to the CTAs.
-//     Consumers dot each row with every token routed to e and store
+//   phase 1 (gate/up + SwiGLU): the work items are (distinct chosen expert,
+//     row i) row pairs -- gate row w1[e, i, :] and up row w1[e, I+i, :] --
+//     dealt round-robin to every warp of the grid.  A warp dots both rows
+//     with the hidden vector of each token routed to e and stores
 //     act[t*k + j, i] = silu(g) * u in fp32 (global memory).
+//     Meanwhile the copy warp moves the w2 rows this CTA needs in phase 2
+//     into shared memory with bulk copies (or, when they do not fit, asks L2
+//     to prefetch them), so w2 streams from HBM alongside w1.  Bulk copies
+//     can stall the issuing warp for microseconds while the copy engine is
+//     busy, which is why a warp of its own issues them.
 //   grid barrier: every CTA has written its act values (bounded wait).
 //   phase 2 (down + weighted combine): each CTA owns a slice of output rows
-//     h and dots w2[e][h, :] with act[t*k + j, :] for every pair of every
-//     chosen expert, then forms out[t, h] = sum_{j=0..k-1} w[t, j] * dot_j in
-//     fixed j order -- deterministic, no extra buffer.
-// The producer does not wait for the barrier: it keeps issuing the phase-2
-// w2 rows (which depend on nothing from phase 1) as ring stages free up, so
-// HBM keeps streaming while the consumers finish phase 1 and cross the
-// barrier.
+//     h; a warp dots w2[e][h, :] (now on chip) with act of every pair of e,
+//     one pair and four rows h at a time (four independent sums), and
+//     out[t, h] = sum_{j=0..k-1} w[t, j] * dot_j is summed in fixed j order
+//     -- deterministic, no extra buffer.
 //
 // Same function as ref_moe on the page "tpu_inference/kernels/fused_moe/v1/
 // kernel.py" (per token: x.[W_gate|W_up] -> silu(gate)*up -> .W2, weighted
@@ -26,6 +29,7 @@
 // the decode dispatch of "metrale_model_layers/layers/moe/forward_k2.rs"
 // (gate-up, silu-down, weighted blend) with the activation fused into the
 // first phase and the blend into the second.
+#include <algorithm>
 #include <mutex>
 
 #include "moe_internal.h"
@@ -33,18 +37,18 @@
 namespace moe {
 namespace {
 
-constexpr int kThreads = 288;  // warp 0: producer; warps 1..8: compute
-constexpr int kComputeWarps = 8;
+constexpr int kWarps = 15;  // compute warps (with the copy warp, 4 warps per SM sub-partition)
+constexpr int kCopyWarp = kWarps;         // issues the w2 bulk copies
+constexpr int kThreads = (kWarps + 1) * 32;
+constexpr int kBlocksPerSm = 1;
 constexpr int kMaxPairs = 256;  // T*k <= 16*16
-constexpr int kMaxStages = 8;
-constexpr int kMaxRp = 4;     // phase 1: row pairs per chunk at most
-constexpr int kRowSlots = 4;  // phase 2: rows per warp (rows per CTA <= 32)
-constexpr int kMaxT = 16;     // tokens of the small-T path
-constexpr int kU1 = 8;        // phase 1: 16-byte column chunks per lane per block
-constexpr int kU2 = 4;        // phase 2: 16-byte column chunks per lane per block
-constexpr uint32_t kStageBytes = 24576;
-constexpr size_t kActCacheMax = 32768;
-constexpr size_t kSmemBudgetMax = 216 * 1024;  // dynamic shared memory of the kernel, at most
+constexpr int kMaxT = 16;       // tokens of the small-T path
+constexpr int kU2 = 4;          // phase 2: 16-byte chunks per lane per block of loads
+constexpr int kR2 = 4;          // phase 2: output rows per item (independent dot products)
+constexpr size_t kActCacheMax = 48 * 1024;
+constexpr uint64_t kW2WaitNs = 2000000000ull;
+constexpr int kMaxH = 4096;
+constexpr int kMaxI = 12288;
 
 struct Lists {
   uint32_t bitmap[32];
@@ -56,12 +60,6 @@ struct Lists {
   int dcur[kMaxPairs];
   int plist[kMaxPairs];   // pairs grouped by distinct expert, ascending
   int n_distinct;
-};
-
-struct Pipe {
-  uint64_t full[kMaxStages];
-  uint64_t empty[kMaxStages];
-  int abort_flag;
 };
 
 // Warp 0 builds the distinct-expert list and the pairs of each expert.
@@ -134,6 +132,16 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
   }
 }
 
+// sum over q of w[q] * x[q] for 8 bf16 weights and 8 fp32 values
+__device__ __forceinline__ float dot8(const uint4 &w, const float (&x)[8]) {
+  float f[8];
+  bf16x8_to_f32(w, f);
+  float v = f[0] * x[0];
+#pragma unroll
+  for (int q = 1; q < 8; ++q) v = fmaf(f[q], x[q], v);
+  return v;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -146,376 +154,375 @@ __device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long
   return v;
 }
 
-// Barrier among the 256 consumer threads (warps 1..8).
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kComputeWarps * 32) : "memory");
+// Dynamic shared memory of a CTA: the single token's vector in fp32 [H]
+// (one-token kernel only); the CTA's w2 rows of every chosen expert in bf16
+// [nd_max][rows_per_cta][I] when they fit (w2_smem); act in fp32 [T*k][I]
+// when it fits (phase 2); the dot products [rows_per_cta][T*k].
+struct SmemLayout {
+  size_t w2_off, act_off, dots_off, total;
+};
+
+__host__ __device__ inline SmemLayout smem_layout(bool one_token, int TK, int H, int I,
+                                                  int rows_per_cta, int nd_max, int w2_smem,
+                                                  int cache_act) {
+  SmemLayout s;
+  s.w2_off = one_token ? static_cast<size_t>(H) * sizeof(float) : 0;
+  s.act_off =
+      s.w2_off + (w2_smem ? static_cast<size_t>(nd_max) * rows_per_cta * I * 2 : 0);
+  s.dots_off = s.act_off + (cache_act ? static_cast<size_t>(TK) * I * sizeof(float) : 0);
+  s.total = s.dots_off + static_cast<size_t>(rows_per_cta) * TK * sizeof(float);
+  return s;
 }
 
-__device__ __forceinline__ void fail(uint32_t *status, int *abort_flag) {
-  *reinterpret_cast<volatile int *>(abort_flag) = 1;
-  atomicOr(status, kStatusTimeout);
-}
-
-// kTokens: the number of tokens, when it is 1 (decode), else kMaxT.
+// kTokens: 1 (decode: the token vector lives in shared memory as fp32 and 8
+// chunks per lane and row are in flight) or kMaxT (up to 16 tokens per
+// expert, token vectors read through L1, 4 chunks in flight).
 template <int kTokens>
-__global__ void __launch_bounds__(kThreads, 1)
-    small_t_kernel(const uint4 *__restrict__ hidden, const char *__restrict__ w1,
-                   const char *__restrict__ w2, const float *__restrict__ topk_w,
+__global__ void __launch_bounds__(kThreads, kBlocksPerSm)
+    small_t_kernel(const uint4 *__restrict__ hidden, const uint4 *__restrict__ w1,
+                   const uint4 *__restrict__ w2, const float *__restrict__ topk_w,
                    const int32_t *__restrict__ ids, float *__restrict__ act,
-                   float *__restrict__ out, int T, int k, int H, int I, int E, int stages, int rp,
-                   int rows_per_cta, int hr, int cache_act, uint32_t *status,
-                   unsigned long long *grid_sync, unsigned long long sync_target, uint64_t limit) {
-  extern __shared__ __align__(128) uint8_t ring[];
+                   float *__restrict__ out, int T, int k, int H, int I, int E, int rows_per_cta,
+                   int nd_max, int w2_smem, int cache_act, uint32_t *status,
+                   unsigned long long *grid_sync,
+                   unsigned long long sync_target, uint64_t limit) {
+  constexpr int kU1 = kTokens == 1 ? 8 : 4;  // phase 1: chunks per lane and row in flight
+  extern __shared__ __align__(16) uint8_t smem[];
   __shared__ Lists L;
-  __shared__ Pipe pipe;
+  __shared__ int s_abort;
+  __shared__ uint64_t w2_full;  // the CTA's w2 rows have landed (w2_smem)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int TK = T * k;
+  const int H8 = H / 8, I8 = I / 8;
+  const SmemLayout lay =
+      smem_layout(kTokens == 1, TK, H, I, rows_per_cta, nd_max, w2_smem, cache_act);
+  float *sx = reinterpret_cast<float *>(smem);
+  uint8_t *sw2 = smem + lay.w2_off;
+  float *sact = reinterpret_cast<float *>(smem + lay.act_off);
+  float *sdots = reinterpret_cast<float *>(smem + lay.dots_off);
+  const int h0 = blockIdx.x * rows_per_cta;
+  const int nrows = max(0, min(H, h0 + rows_per_cta) - h0);
+
   if (warp == 0) build_lists(L, ids, TK, E);
   if (threadIdx.x == 32) {
-    for (int s = 0; s < stages; ++s) {
-      mbar_init(&pipe.full[s], 1);
-      mbar_init(&pipe.empty[s], kComputeWarps);
-    }
-    pipe.abort_flag = 0;
+    s_abort = 0;
+    mbar_init(&w2_full, 1);
     fence_mbar_init();
+  }
+  if (kTokens == 1) {
+    for (int c = threadIdx.x; c < H8; c += kThreads) {
+      float f[8];
+      bf16x8_to_f32(__ldg(hidden + c), f);
+      float4 *d = reinterpret_cast<float4 *>(sx + static_cast<size_t>(c) * 8);
+      d[0] = make_float4(f[0], f[1], f[2], f[3]);
+      d[1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
   }
   __syncthreads();
   const int nd = L.n_distinct;
-  const size_t row1 = static_cast<size_t>(H) * 2;  // bytes of a w1 row
-  const size_t row2 = static_cast<size_t>(I) * 2;  // bytes of a w2 row
-  // phase 1: chunks of rp row pairs, dealt round-robin over the grid
-  const int cpe1 = (I + rp - 1) / rp;
-  const int NC1 = nd * cpe1;
-  const int n1 = blockIdx.x < NC1 ? (NC1 - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
-  // phase 2: this CTA's output rows, hr rows per chunk, for every expert
-  const int h0 = blockIdx.x * rows_per_cta;
-  const int nrows = max(0, min(H, h0 + rows_per_cta) - h0);
-  const int cpe2 = (nrows + hr - 1) / hr;
-  const int n2 = nd * cpe2;
-  // act of every pair, when it is small enough to keep in shared memory
-  float4 *sact = reinterpret_cast<float4 *>(ring + static_cast<size_t>(stages) * kStageBytes);
-
-  if (warp == 0) {
+  const int nw = gridDim.x * kWarps;
+  const int n1 = nd * I;
+  if (warp == kCopyWarp) {
+    // this CTA's w2 rows of every chosen expert, for phase 2
     if (lane == 0) {
-      for (int it = 0; it < n1 + n2; ++it) {
-        const int s = it % stages;
-        const uint32_t ph = (it / stages) & 1;
-        if (!mbar_wait(&pipe.empty[s], ph ^ 1, limit, &pipe.abort_flag)) {
-          fail(status, &pipe.abort_flag);
-          break;
-        }
-        uint8_t *stage = ring + static_cast<size_t>(s) * kStageBytes;
-        if (it < n1) {
-          const int c = blockIdx.x + it * gridDim.x;
-          const int d = c / cpe1, i0 = (c - d * cpe1) * rp;
-          const int nr = min(rp, I - i0);
-          const int e = L.dexp[d];
-          const uint32_t bytes = static_cast<uint32_t>(nr * row1);
-          mbar_arrive_expect_tx(&pipe.full[s], 2 * bytes);
-          bulk_load(stage, w1 + (static_cast<size_t>(e) * 2 * I + i0) * row1, bytes,
-                    &pipe.full[s]);
-          bulk_load(stage + rp * row1, w1 + (static_cast<size_t>(e) * 2 * I + I + i0) * row1,
-                    bytes, &pipe.full[s]);
-        } else {
-          const int c = it - n1;
-          const int d = c / cpe2, hs = h0 + (c - d * cpe2) * hr;
-          const int nr = min(hr, h0 + nrows - hs);
-          const uint32_t bytes = static_cast<uint32_t>(nr * row2);
-          mbar_arrive_expect_tx(&pipe.full[s], bytes);
-          bulk_load(stage, w2 + (static_cast<size_t>(L.dexp[d]) * H + hs) * row2, bytes,
-                    &pipe.full[s]);
-        }
+      const uint32_t bytes = static_cast<uint32_t>(nrows) * I * 2;
+      if (w2_smem) {
+        // nd <= nd_max: the host sized the slots for the distinct experts a
+        // call can have
+        mbar_arrive_expect_tx(&w2_full, bytes * static_cast<uint32_t>(nd));
+        for (int d = 0; d < nd && nrows > 0; ++d)
+          bulk_load(sw2 + static_cast<size_t>(d) * rows_per_cta * I * 2,
+                    w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * I8, bytes, &w2_full);
+      } else {
+        for (int d = 0; d < nd && nrows > 0; ++d)
+          bulk_prefetch_l2(w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * I8, bytes);
       }
     }
-    __syncthreads();  // pairs with the consumers' final barrier
-    return;
   }
 
-  // ---------------------------------------------------------------- consumers
-  // Phase 1: one warp per (row pair, token) task; the tasks of successive
-  // chunks are dealt to the warps round-robin so that every warp stays busy
-  // while chunks stream in.
-  const int cw = warp - 1;
-  const int H8 = H / 8, I8 = I / 8;
-  int task_base = 0;
-  int it = 0;
-  bool stop = false;
-  for (; it < n1 && !stop; ++it) {
-    const int s = it % stages;
-    const uint32_t ph = (it / stages) & 1;
-    if (!mbar_wait(&pipe.full[s], ph, limit, &pipe.abort_flag)) {
-      if (lane == 0) fail(status, &pipe.abort_flag);
-      stop = true;
-      break;
-    }
-    const int c = blockIdx.x + it * gridDim.x;
-    const int d = c / cpe1, i0 = (c - d * cpe1) * rp;
-    const int nr = min(rp, I - i0);
+  // ------------------------------------------------------------ phase 1
+  for (int task = blockIdx.x * kWarps + warp; task < n1 && warp < kWarps; task += nw) {
+    const int d = task / I, i = task - d * I;
     const int p0 = L.dstart[d], np = L.dstart[d + 1] - p0;
-    const uint8_t *stage = ring + static_cast<size_t>(s) * kStageBytes;
-    const int ntask = nr * np;
-    for (int task = (cw - task_base % kComputeWarps + kComputeWarps) % kComputeWarps;
-         task < ntask; task += kComputeWarps) {
-      const int r = task / np;
-      const int pair = L.plist[p0 + task - r * np];
-      const uint4 *g = reinterpret_cast<const uint4 *>(stage + r * row1);
-      const uint4 *u = reinterpret_cast<const uint4 *>(stage + (rp + r) * row1);
-      const uint4 *x = hidden + static_cast<size_t>(pair / k) * H8;
-      // blocks of kU column chunks per lane: all loads of a block are in
-      // flight together, each chunk has its own accumulators
+    const uint4 *g = w1 + (static_cast<size_t>(L.dexp[d]) * 2 * I + i) * H8;
+    const uint4 *u = g + static_cast<size_t>(I) * H8;
+    if (kTokens == 1) {
+      // one token: its pairs on e (more than one only for repeated ids) share
+      // the same dot products
       float ag = 0.f, au = 0.f;
       for (int base = 0; base < H8; base += 32 * kU1) {
-        uint4 xv[kU1], gv[kU1], uv[kU1];
+        uint4 gv[kU1], uv[kU1];
 #pragma unroll
         for (int j = 0; j < kU1; ++j) {
-          const int c8 = base + lane + 32 * j;
-          if (c8 < H8) {
-            xv[j] = __ldg(x + c8);
-            gv[j] = g[c8];
-            uv[j] = u[c8];
+          const int c = base + lane + 32 * j;
+          if (c < H8) {
+            gv[j] = __ldcs(g + c);
+            uv[j] = __ldcs(u + c);
           }
         }
 #pragma unroll
         for (int j = 0; j < kU1; ++j) {
-          if (base + lane + 32 * j < H8) {
-            float xf[8], gf[8], uf[8];
-            bf16x8_to_f32(xv[j], xf);
-            bf16x8_to_f32(gv[j], gf);
-            bf16x8_to_f32(uv[j], uf);
-            float pg = 0.f, pu = 0.f;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              pg = fmaf(gf[q], xf[q], pg);
-              pu = fmaf(uf[q], xf[q], pu);
-            }
-            ag += pg;
-            au += pu;
+          const int c = base + lane + 32 * j;
+          if (c < H8) {
+            const float4 x0 = reinterpret_cast<const float4 *>(sx)[2 * c];
+            const float4 x1 = reinterpret_cast<const float4 *>(sx)[2 * c + 1];
+            const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            ag += dot8(gv[j], x);
+            au += dot8(uv[j], x);
           }
         }
       }
       ag = warp_sum(ag);
       au = warp_sum(au);
-      if (lane == 0) act[static_cast<size_t>(pair) * I + i0 + r] = silu_f(ag) * au;
+      if (lane == 0) {
+        const float a = silu_f(ag) * au;
+        for (int q = 0; q < np; ++q) act[static_cast<size_t>(L.plist[p0 + q]) * I + i] = a;
+      }
+    } else {
+      // the tokens routed to e, kMaxT accumulator pairs at a time
+      for (int q0 = 0; q0 < np; q0 += kMaxT) {
+        const int nq = min(kMaxT, np - q0);
+        float ag[kMaxT], au[kMaxT];
+#pragma unroll
+        for (int q = 0; q < kMaxT; ++q) ag[q] = au[q] = 0.f;
+        for (int base = 0; base < H8; base += 32 * kU1) {
+          uint4 gv[kU1], uv[kU1];
+#pragma unroll
+          for (int j = 0; j < kU1; ++j) {
+            const int c = base + lane + 32 * j;
+            if (c < H8) {
+              gv[j] = __ldcs(g + c);
+              uv[j] = __ldcs(u + c);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < kU1; ++j) {
+            const int c = base + lane + 32 * j;
+            if (c < H8) {
+              float gf[8], uf[8];
+              bf16x8_to_f32(gv[j], gf);
+              bf16x8_to_f32(uv[j], uf);
+#pragma unroll
+              for (int q = 0; q < kMaxT; ++q) {
+                if (q < nq) {
+                  const int t = L.plist[p0 + q0 + q] / k;
+                  float x[8];
+                  bf16x8_to_f32(__ldg(hidden + static_cast<size_t>(t) * H8 + c), x);
+                  float pg = gf[0] * x[0], pu = uf[0] * x[0];
+#pragma unroll
+                  for (int z = 1; z < 8; ++z) {
+                    pg = fmaf(gf[z], x[z], pg);
+                    pu = fmaf(uf[z], x[z], pu);
+                  }
+                  ag[q] += pg;
+                  au[q] += pu;
+                }
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < kMaxT; ++q) {
+          if (q < nq) {
+            const float gs = warp_sum(ag[q]);
+            const float us = warp_sum(au[q]);
+            if (lane == 0)
+              act[static_cast<size_t>(L.plist[p0 + q0 + q]) * I + i] = silu_f(gs) * us;
+          }
+        }
+      }
     }
-    task_base += ntask;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&pipe.empty[s]);
   }
 
   // ------------------------------------------------------------ grid barrier
-  // Every CTA arrives exactly once per launch, so the counter reaches
-  // sync_target = (launches so far) * gridDim when all act values are written.
+  // Every CTA adds one per launch; the host passes the counter value that
+  // means every CTA of this launch has written its act values.
   __threadfence();
-  asm volatile("bar.sync 1, %0;" ::"n"(kComputeWarps * 32) : "memory");
-  if (threadIdx.x == 32) {
-    __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
     atomicAdd(grid_sync, 1ull);
     const uint64_t t0 = global_timer_ns();
     while (ld_acquire_gpu(grid_sync) < sync_target) {
       if (global_timer_ns() - t0 > limit) {
-        fail(status, &pipe.abort_flag);
+        s_abort = 1;
+        atomicOr(status, kStatusTimeout);
         break;
       }
+      __nanosleep(32);
     }
     __threadfence();
   }
-  asm volatile("bar.sync 1, %0;" ::"n"(kComputeWarps * 32) : "memory");
-  stop = stop || *reinterpret_cast<volatile int *>(&pipe.abort_flag) != 0;
+  // the CTA's w2 rows: one thread waits (bounded) so that the decision to
+  // go on is the same for every thread; then each thread observes the
+  // completed phase itself, which orders the copied data before its reads
+  if (w2_smem && threadIdx.x == 0 && !s_abort && !mbar_wait(&w2_full, 0, kW2WaitNs)) {
+    s_abort = 1;
+    atomicOr(status, kStatusTimeout);
+  }
+  __syncthreads();
+  if (s_abort) return;
+  if (w2_smem) mbar_wait(&w2_full, 0, kW2WaitNs);
 
+  // ------------------------------------------------------------ phase 2
   const float4 *act4 = reinterpret_cast<const float4 *>(act);
-  if (cache_act && !stop) {
+  if (cache_act) {
     // act was written by other CTAs in this launch: read it from L2
     const int n4 = TK * I / 4;
-    constexpr int kU = 8;  // loads in flight per thread
-    for (int x0 = threadIdx.x - 32; x0 < n4; x0 += kU * kComputeWarps * 32) {
-      float4 v[kU];
-#pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int x = x0 + u * kComputeWarps * 32;
-        if (x < n4) v[u] = __ldcg(act4 + x);
-      }
-#pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int x = x0 + u * kComputeWarps * 32;
-        if (x < n4) sact[x] = v[u];
-      }
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(kComputeWarps * 32) : "memory");
-    act4 = sact;
+    float4 *d4 = reinterpret_cast<float4 *>(sact);
+    for (int x = threadIdx.x; x < n4; x += kThreads) d4[x] = __ldcg(act4 + x);
+    __syncthreads();
+    act4 = d4;
   }
-  // Phase 2: warp cw owns local output rows cw + 8*rs.  For every pair of
-  // each chunk's expert, each lane adds w_pair * (its slice of the dot) to a
-  // per-(row, token) accumulator; one warp reduction per (row, token) at the
-  // end gives out[t, h].  Terms are added in a fixed order (chunks by
-  // ascending expert, then lanes by a fixed tree), so the result is
-  // bit-reproducible.
-  float acc[kRowSlots][kTokens];
+  // items (distinct expert d, its pair q, group of kR2 local rows): the act
+  // chunks of the pair are loaded once and shared by kR2 independent dot
+  // products with w2[e][h0 + r, :] (on chip), one per row of the group
+  const int rgroups = (nrows + kR2 - 1) / kR2;
+  const int n2 = L.dstart[nd] * rgroups;
+  for (int item = warp; item < n2 && warp < kWarps; item += kWarps) {
+    const int pq = item / rgroups, rg = item - pq * rgroups;  // pq: position in plist
+    const int pair = L.plist[pq];
+    const int d = L.pd[pair];
+    const int r0 = rg * kR2;
+    const float4 *a = act4 + static_cast<size_t>(pair) * (I / 4);
+    float v[kR2];
 #pragma unroll
-  for (int rs = 0; rs < kRowSlots; ++rs)
+    for (int rr = 0; rr < kR2; ++rr) v[rr] = 0.f;
+    for (int base = 0; base < I8; base += 32 * kU2) {
 #pragma unroll
-    for (int tt = 0; tt < kTokens; ++tt) acc[rs][tt] = 0.f;
-  for (int c = 0; c < n2 && !stop; ++c, ++it) {
-    const int s = it % stages;
-    const uint32_t ph = (it / stages) & 1;
-    if (!mbar_wait(&pipe.full[s], ph, limit, &pipe.abort_flag)) {
-      if (lane == 0) fail(status, &pipe.abort_flag);
-      stop = true;
-      break;
-    }
-    const int d = c / cpe2, hs = h0 + (c - d * cpe2) * hr;
-    const int nr = min(hr, h0 + nrows - hs);
-    const int p0 = L.dstart[d], np = L.dstart[d + 1] - p0;
-    const uint8_t *stage = ring + static_cast<size_t>(s) * kStageBytes;
+      for (int j = 0; j < kU2; ++j) {
+        const int c = base + lane + 32 * j;
+        if (c < I8) {
+          const float4 a0 = cache_act ? a[2 * c] : __ldcg(a + 2 * c);
+          const float4 a1 = cache_act ? a[2 * c + 1] : __ldcg(a + 2 * c + 1);
+          const float x[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-    for (int rs = 0; rs < kRowSlots; ++rs) {
-      // this warp's row of the chunk, in CTA-local row numbering
-      const int r = (cw + rs * kComputeWarps) - (hs - h0);
-      if (r < 0 || r >= nr) continue;
-      const uint4 *wrow = reinterpret_cast<const uint4 *>(stage + r * row2);
-      for (int base = 0; base < I8; base += 32 * kU2) {
-        uint4 wv[kU2];
-#pragma unroll
-        for (int j = 0; j < kU2; ++j)
-          if (base + lane + 32 * j < I8) wv[j] = wrow[base + lane + 32 * j];
-        for (int q = 0; q < np; ++q) {
-          const int pair = L.plist[p0 + q];
-          const float4 *a = act4 + static_cast<size_t>(pair) * (I / 4);
-          float v = 0.f;
-#pragma unroll
-          for (int j = 0; j < kU2; ++j) {
-            const int c8 = base + lane + 32 * j;
-            if (c8 < I8) {
-              const float4 a0 = cache_act ? a[2 * c8] : __ldcg(a + 2 * c8);
-              const float4 a1 = cache_act ? a[2 * c8 + 1] : __ldcg(a + 2 * c8 + 1);
-              float wf[8];
-              bf16x8_to_f32(wv[j], wf);
-              float pv = 0.f;
-              pv = fmaf(wf[0], a0.x, pv);
-              pv = fmaf(wf[1], a0.y, pv);
-              pv = fmaf(wf[2], a0.z, pv);
-              pv = fmaf(wf[3], a0.w, pv);
-              pv = fmaf(wf[4], a1.x, pv);
-              pv = fmaf(wf[5], a1.y, pv);
-              pv = fmaf(wf[6], a1.z, pv);
-              pv = fmaf(wf[7], a1.w, pv);
-              v += pv;
+          for (int rr = 0; rr < kR2; ++rr) {
+            const int r = r0 + rr;
+            if (r < nrows) {
+              const uint4 wv =
+                  w2_smem ? reinterpret_cast<const uint4 *>(sw2)[(d * rows_per_cta + r) * I8 + c]
+                          : __ldg(w2 + (static_cast<size_t>(L.dexp[d]) * H + h0 + r) * I8 + c);
+              v[rr] += dot8(wv, x);
             }
           }
-          const float wp = __ldg(topk_w + pair);
-          if (kTokens == 1) {
-            acc[rs][0] = fmaf(wp, v, acc[rs][0]);
-          } else {
-            const int t = pair / k;
-#pragma unroll
-            for (int tt = 0; tt < kTokens; ++tt)
-              if (tt == t) acc[rs][tt] = fmaf(wp, v, acc[rs][tt]);
-          }
         }
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&pipe.empty[s]);
-  }
-  // out[t, h]: one warp reduction per (row, token); rows of this CTA only
-  if (!stop) {
 #pragma unroll
-    for (int rs = 0; rs < kRowSlots; ++rs) {
-      const int r = cw + rs * kComputeWarps;
-#pragma unroll
-      for (int tt = 0; tt < kTokens; ++tt) {
-        if (tt < T && r < nrows) {
-          const float v = warp_sum(acc[rs][tt]);
-          if (lane == 0) out[static_cast<size_t>(tt) * H + h0 + r] = v;
-        }
-      }
+    for (int rr = 0; rr < kR2; ++rr) {
+      const float sv = warp_sum(v[rr]);
+      if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
     }
   }
-  bool bad = false;
-  if (threadIdx.x == 32)
-    for (int i = 0; i < TK; ++i) bad = bad || L.pd[i] < 0;
-  if (bad && blockIdx.x == 0) atomicOr(status, kStatusBadId);
   __syncthreads();
+  // out[t, h] = sum over j in ascending order of w[t, j] * dot(t*k + j)
+  for (int x = threadIdx.x; x < T * nrows; x += kThreads) {
+    const int t = x / nrows, r = x - t * nrows;
+    float acc = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int pair = t * k + j;
+      if (L.pd[pair] >= 0) acc = fmaf(__ldg(topk_w + pair), sdots[r * TK + pair], acc);
+    }
+    out[static_cast<size_t>(t) * H + h0 + r] = acc;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    bool bad = false;
+    for (int i = 0; i < TK; ++i) bad = bad || L.pd[i] < 0;
+    if (bad) atomicOr(status, kStatusBadId);
+  }
 }
 
 struct SmallTConfig {
-  int stages, rp, hr, rows_per_cta, grid, cache_act;
+  int rows_per_cta, nd_max, w2_smem, cache_act;
   size_t smem;
 };
 
-SmallTConfig small_t_config(int TK, int H, int I, int num_sms, size_t kSmemBudget) {
+// What goes into `budget` bytes of dynamic shared memory, in order of gain:
+// the CTA's w2 rows, then the act cache.
+SmallTConfig small_t_config(int T, int TK, int H, int I, int E, int grid, size_t budget) {
   SmallTConfig c;
-  c.rp = static_cast<int>(kStageBytes / (4u * H));
-  if (c.rp > kMaxRp) c.rp = kMaxRp;
-  c.hr = static_cast<int>(kStageBytes / (2u * I));
-  if (c.hr > kRowSlots * kComputeWarps) c.hr = kRowSlots * kComputeWarps;
-  c.grid = num_sms;
-  c.rows_per_cta = (H + num_sms - 1) / num_sms;
-  const size_t act_bytes = static_cast<size_t>(TK) * I * sizeof(float);
-  c.cache_act = act_bytes + 2 * kStageBytes <= kSmemBudget && act_bytes <= kActCacheMax;
-  const size_t extra = c.cache_act ? act_bytes : 0;
-  const size_t fit = extra < kSmemBudget ? (kSmemBudget - extra) / kStageBytes : 0;
-  c.stages = static_cast<int>(fit < static_cast<size_t>(kMaxStages) ? fit : kMaxStages);
-  c.smem = static_cast<size_t>(c.stages) * kStageBytes + extra;
+  c.rows_per_cta = (H + grid - 1) / grid;
+  c.nd_max = std::min(TK, E);
+  c.w2_smem = 1;
+  c.cache_act = 1;
+  auto size = [&] {
+    return smem_layout(T == 1, TK, H, I, c.rows_per_cta, c.nd_max, c.w2_smem, c.cache_act).total;
+  };
+  if (static_cast<size_t>(TK) * I * sizeof(float) > kActCacheMax || size() > budget)
+    c.cache_act = 0;
+  if (size() > budget) c.w2_smem = 0;
+  c.smem = size();
   return c;
+}
+
+// The dynamic shared memory the kernel may use next to its static shared
+// memory, with kBlocksPerSm CTAs on an SM.
+size_t smem_budget(int dev, const void *kern) {
+  int per_sm = 0, reserved = 0;
+  cudaFuncAttributes fa;
+  if (cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) !=
+          cudaSuccess ||
+      cudaFuncGetAttributes(&fa, kern) != cudaSuccess)
+    return 0;
+  const size_t per_block = static_cast<size_t>(per_sm) / kBlocksPerSm;
+  const size_t fixed = fa.sharedSizeBytes + static_cast<size_t>(reserved);
+  return per_block > fixed ? (per_block - fixed) & ~static_cast<size_t>(127) : 0;
 }
 
 }  // namespace
 
-bool small_t_supported(int H, int I) {
-  // a stage holds a w1 row pair and a w2 row; a CTA owns <= 32 output rows
-  return H <= 4096 && 4u * static_cast<uint32_t>(H) <= kStageBytes &&
-         2u * static_cast<uint32_t>(I) <= kStageBytes;
-}
+bool small_t_supported(int H, int I) { return H <= kMaxH && I <= kMaxI; }
 
 cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
                            const float *topk_weights, const int32_t *topk_ids, float *act,
                            float *out, int64_t T, int H, int I, int E, int k, uint32_t *status,
-                           unsigned long long *grid_sync, unsigned long long *launches,
+                           unsigned long long *grid_sync, unsigned long long *arrivals,
                            uint64_t wait_limit_ns, cudaStream_t s, const StageHook &hook) {
   static std::mutex mu;
   static uint64_t ready_mask = 0;
-  static size_t budget[64] = {};
+  static int grid_of[64] = {};
+  static size_t budget_of[64] = {};
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  if (!small_t_supported(H, I) || dev >= 64) return cudaErrorInvalidValue;
+  if (!small_t_supported(H, I) || dev >= 64 || T < 1 || T > kMaxT || T * k > kMaxPairs)
+    return cudaErrorInvalidValue;
   {
     std::lock_guard<std::mutex> lock(mu);
     if (!((ready_mask >> dev) & 1)) {
-      // dynamic shared memory left next to the kernel's static shared memory
-      int optin = 0;
-      cudaFuncAttributes fa;
-      e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-      if (e != cudaSuccess) return e;
-      size_t b = kSmemBudgetMax;
-      for (auto kern : {small_t_kernel<1>, small_t_kernel<kMaxT>}) {
-        e = cudaFuncGetAttributes(&fa, kern);
-        if (e != cudaSuccess) return e;
-        const size_t left = static_cast<size_t>(optin) - fa.sharedSizeBytes;
-        if (left < b) b = left;
-      }
+      // every CTA must be resident at once (the grid barrier): the grid is
+      // the number of CTAs both kernels can keep on every SM
+      const size_t smem = std::min(smem_budget(dev, reinterpret_cast<const void *>(small_t_kernel<1>)),
+                                   smem_budget(dev, reinterpret_cast<const void *>(small_t_kernel<kMaxT>)));
+      if (smem < 16384) return cudaErrorInvalidValue;
+      budget_of[dev] = smem;
+      int per_sm = kBlocksPerSm;
       for (auto kern : {small_t_kernel<1>, small_t_kernel<kMaxT>}) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(b));
+                                 static_cast<int>(smem));
         if (e != cudaSuccess) return e;
-        int per_sm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, b);
+        int n = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, smem);
         if (e != cudaSuccess) return e;
-        if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+        per_sm = std::min(per_sm, n);
       }
-      budget[dev] = b;
+      if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+      grid_of[dev] = per_sm * sms;
       ready_mask |= 1ull << dev;
     }
   }
-  const SmallTConfig cfg = small_t_config(static_cast<int>(T) * k, H, I, sms, budget[dev]);
-  // each consumer warp owns at most kRowSlots of the CTA's output rows
-  if (cfg.stages < 2 || cfg.rows_per_cta > kRowSlots * kComputeWarps || T > kMaxT)
-    return cudaErrorInvalidValue;
-  // every CTA adds one to the grid-sync counter per launch
-  const unsigned long long target = (*launches + 1) * static_cast<unsigned long long>(cfg.grid);
+  const int grid = grid_of[dev];
+  const SmallTConfig cfg = small_t_config(static_cast<int>(T), static_cast<int>(T) * k, H, I, E,
+                                          grid, budget_of[dev]);
+  if (cfg.smem > budget_of[dev]) return cudaErrorInvalidValue;
+  // each CTA adds one to the grid-sync counter per launch: the target is the
+  // arrivals of all earlier launches plus this grid
+  const unsigned long long target = *arrivals + static_cast<unsigned long long>(grid);
   cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3(cfg.grid);
+  lc.gridDim = dim3(grid);
   lc.blockDim = dim3(kThreads);
   lc.dynamicSmemBytes = cfg.smem;
   lc.stream = s;
@@ -527,11 +534,12 @@ cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uin
   hook.begin("small_t");
   e = cudaLaunchKernelEx(&lc, T == 1 ? small_t_kernel<1> : small_t_kernel<kMaxT>,
                          reinterpret_cast<const uint4 *>(hidden),
-                         reinterpret_cast<const char *>(w1), reinterpret_cast<const char *>(w2),
+                         reinterpret_cast<const uint4 *>(w1), reinterpret_cast<const uint4 *>(w2),
                          topk_weights, topk_ids, act, out, static_cast<int>(T), k, H, I, E,
-                         cfg.stages, cfg.rp, cfg.rows_per_cta, cfg.hr, cfg.cache_act, status,
-                         grid_sync, target, wait_limit_ns);
-  if (e == cudaSuccess) *launches += 1;
+                         cfg.rows_per_cta, cfg.nd_max, cfg.w2_smem, cfg.cache_act, status,
+                         grid_sync, target,
+                         wait_limit_ns);
+  if (e == cudaSuccess) *arrivals = target;
   return hook.end(e);
 }
 
