@@ -3,7 +3,7 @@
 // of MB; the arithmetic is negligible), so it runs as one HBM-bound GEMV
 // kernel on the CUDA cores: every warp streams whole weight rows with
 // 128-bit loads, many rows in flight per SM, so that the loads alone keep
-// HBM busy.  One cooperative launch (all CTAs resident, one per SM, 16
+// HBM busy.  One cooperative launch (all CTAs resident, one per SM, 15
 // compute warps and one copy warp):
 //
 //   phase 1 (gate/up + SwiGLU): the work items are (distinct chosen expert,
