@@ -123,23 +123,72 @@ __device__ void build_lists(Lists &L, const int32_t *ids, int TK, int E) {
   }
 }
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
+// acc + sum over q = 0..7 of w[q] * x[q] for 8 bf16 weights and 8 bf16
+// values, one fp32 FMA per term with bf16 operands (fma.rn.f32.bf16: the
+// products are exact, the sum rounds once per term, as fmaf on the
+// widened values would) -- no separate conversions.
+__device__ __forceinline__ float fma8_bf16(const uint4 &w, const uint4 &x, float acc) {
+  asm("{\n\t"
+      ".reg .b16 w0, w1, w2, w3, w4, w5, w6, w7, x0, x1, x2, x3, x4, x5, x6, x7;\n\t"
+      "mov.b32 {w0, w1}, %1;\n\t"
+      "mov.b32 {w2, w3}, %2;\n\t"
+      "mov.b32 {w4, w5}, %3;\n\t"
+      "mov.b32 {w6, w7}, %4;\n\t"
+      "mov.b32 {x0, x1}, %5;\n\t"
+      "mov.b32 {x2, x3}, %6;\n\t"
+      "mov.b32 {x4, x5}, %7;\n\t"
+      "mov.b32 {x6, x7}, %8;\n\t"
+      "fma.rn.f32.bf16 %0, w0, x0, %0;\n\t"
+      "fma.rn.f32.bf16 %0, w1, x1, %0;\n\t"
+      "fma.rn.f32.bf16 %0, w2, x2, %0;\n\t"
+      "fma.rn.f32.bf16 %0, w3, x3, %0;\n\t"
+      "fma.rn.f32.bf16 %0, w4, x4, %0;\n\t"
+      "fma.rn.f32.bf16 %0, w5, x5, %0;\n\t"
+      "fma.rn.f32.bf16 %0, w6, x6, %0;\n\t"
+      "fma.rn.f32.bf16 %0, w7, x7, %0;\n\t"
+      "}"
+      : "+f"(acc)
+      : "r"(w.x), "r"(w.y), "r"(w.z), "r"(w.w), "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w));
+  return acc;
 }
 
-// sum over q of w[q] * x[q] for 8 bf16 weights and 8 fp32 values
-__device__ __forceinline__ float dot8(const uint4 &w, const float (&x)[8]) {
-  float f[8];
-  bf16x8_to_f32(w, f);
-  float v = f[0] * x[0];
-#pragma unroll
-  for (int q = 1; q < 8; ++q) v = fmaf(f[q], x[q], v);
-  return v;
+// Two fp32 sums in one 64-bit register (even and odd terms), advanced with
+// the packed fma.rn.f32x2: acc += w[q] * x[q] for 8 bf16 weights and 8 fp32
+// values (x0 = terms 0..3, x1 = terms 4..7).
+__device__ __forceinline__ void fma8_f32x2(const uint4 &w, const float4 &x0, const float4 &x1,
+                                           unsigned long long &acc) {
+  asm("{\n\t"
+      ".reg .b32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
+      ".reg .b64 p0, p1, p2, p3, q0, q1, q2, q3;\n\t"
+      "shl.b32 l0, %1, 16;\n\t"
+      "and.b32 h0, %1, 0xffff0000;\n\t"
+      "shl.b32 l1, %2, 16;\n\t"
+      "and.b32 h1, %2, 0xffff0000;\n\t"
+      "shl.b32 l2, %3, 16;\n\t"
+      "and.b32 h2, %3, 0xffff0000;\n\t"
+      "shl.b32 l3, %4, 16;\n\t"
+      "and.b32 h3, %4, 0xffff0000;\n\t"
+      "mov.b64 p0, {l0, h0};\n\t"
+      "mov.b64 p1, {l1, h1};\n\t"
+      "mov.b64 p2, {l2, h2};\n\t"
+      "mov.b64 p3, {l3, h3};\n\t"
+      "mov.b64 q0, {%5, %6};\n\t"
+      "mov.b64 q1, {%7, %8};\n\t"
+      "mov.b64 q2, {%9, %10};\n\t"
+      "mov.b64 q3, {%11, %12};\n\t"
+      "fma.rn.f32x2 %0, p0, q0, %0;\n\t"
+      "fma.rn.f32x2 %0, p1, q1, %0;\n\t"
+      "fma.rn.f32x2 %0, p2, q2, %0;\n\t"
+      "fma.rn.f32x2 %0, p3, q3, %0;\n\t"
+      "}"
+      : "+l"(acc)
+      : "r"(w.x), "r"(w.y), "r"(w.z), "r"(w.w), "f"(x0.x), "f"(x0.y), "f"(x0.z), "f"(x0.w),
+        "f"(x1.x), "f"(x1.y), "f"(x1.z), "f"(x1.w));
+}
+
+__device__ __forceinline__ float sum_f32x2(unsigned long long acc) {
+  return __uint_as_float(static_cast<uint32_t>(acc)) +
+         __uint_as_float(static_cast<uint32_t>(acc >> 32));
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -154,7 +203,7 @@ __device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long
   return v;
 }
 
-// Dynamic shared memory of a CTA: the single token's vector in fp32 [H]
+// Dynamic shared memory of a CTA: the single token's vector in bf16 [H]
 // (one-token kernel only); the CTA's w2 rows of every chosen expert in bf16
 // [nd_max][rows_per_cta][I] when they fit (w2_smem); act in fp32 [T*k][I]
 // when it fits (phase 2); the dot products [rows_per_cta][T*k].
@@ -166,7 +215,7 @@ __host__ __device__ inline SmemLayout smem_layout(bool one_token, int TK, int H,
                                                   int rows_per_cta, int nd_max, int w2_smem,
                                                   int cache_act) {
   SmemLayout s;
-  s.w2_off = one_token ? static_cast<size_t>(H) * sizeof(float) : 0;
+  s.w2_off = one_token ? static_cast<size_t>(H) * 2 : 0;
   s.act_off =
       s.w2_off + (w2_smem ? static_cast<size_t>(nd_max) * rows_per_cta * I * 2 : 0);
   s.dots_off = s.act_off + (cache_act ? static_cast<size_t>(TK) * I * sizeof(float) : 0);
@@ -174,7 +223,7 @@ __host__ __device__ inline SmemLayout smem_layout(bool one_token, int TK, int H,
   return s;
 }
 
-// kTokens: 1 (decode: the token vector lives in shared memory as fp32 and 8
+// kTokens: 1 (decode: the token vector lives in shared memory as bf16 and 8
 // chunks per lane and row are in flight) or kMaxT (up to 16 tokens per
 // expert, token vectors read through L1, 4 chunks in flight).
 template <int kTokens>
@@ -196,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   const int H8 = H / 8, I8 = I / 8;
   const SmemLayout lay =
       smem_layout(kTokens == 1, TK, H, I, rows_per_cta, nd_max, w2_smem, cache_act);
-  float *sx = reinterpret_cast<float *>(smem);
+  uint8_t *sx = smem;  // the token's vector (one-token kernel)
   uint8_t *sw2 = smem + lay.w2_off;
   float *sact = reinterpret_cast<float *>(smem + lay.act_off);
   float *sdots = reinterpret_cast<float *>(smem + lay.dots_off);
@@ -209,15 +258,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     mbar_init(&w2_full, 1);
     fence_mbar_init();
   }
-  if (kTokens == 1) {
-    for (int c = threadIdx.x; c < H8; c += kThreads) {
-      float f[8];
-      bf16x8_to_f32(__ldg(hidden + c), f);
-      float4 *d = reinterpret_cast<float4 *>(sx + static_cast<size_t>(c) * 8);
-      d[0] = make_float4(f[0], f[1], f[2], f[3]);
-      d[1] = make_float4(f[4], f[5], f[6], f[7]);
-    }
-  }
+  if (kTokens == 1)
+    for (int c = threadIdx.x; c < H8; c += kThreads)
+      reinterpret_cast<uint4 *>(sx)[c] = __ldg(hidden + c);
   __syncthreads();
   const int nd = L.n_distinct;
   const int nw = gridDim.x * kWarps;
@@ -264,11 +307,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
         for (int j = 0; j < kU1; ++j) {
           const int c = base + lane + 32 * j;
           if (c < H8) {
-            const float4 x0 = reinterpret_cast<const float4 *>(sx)[2 * c];
-            const float4 x1 = reinterpret_cast<const float4 *>(sx)[2 * c + 1];
-            const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-            ag += dot8(gv[j], x);
-            au += dot8(uv[j], x);
+            const uint4 xv = reinterpret_cast<const uint4 *>(sx)[c];
+            ag = fma8_bf16(gv[j], xv, ag);
+            au = fma8_bf16(uv[j], xv, au);
           }
         }
       }
@@ -299,23 +340,13 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
           for (int j = 0; j < kU1; ++j) {
             const int c = base + lane + 32 * j;
             if (c < H8) {
-              float gf[8], uf[8];
-              bf16x8_to_f32(gv[j], gf);
-              bf16x8_to_f32(uv[j], uf);
 #pragma unroll
               for (int q = 0; q < kMaxT; ++q) {
                 if (q < nq) {
                   const int t = L.plist[p0 + q0 + q] / k;
-                  float x[8];
-                  bf16x8_to_f32(__ldg(hidden + static_cast<size_t>(t) * H8 + c), x);
-                  float pg = gf[0] * x[0], pu = uf[0] * x[0];
-#pragma unroll
-                  for (int z = 1; z < 8; ++z) {
-                    pg = fmaf(gf[z], x[z], pg);
-                    pu = fmaf(uf[z], x[z], pu);
-                  }
-                  ag[q] += pg;
-                  au[q] += pu;
+                  const uint4 xv = __ldg(hidden + static_cast<size_t>(t) * H8 + c);
+                  ag[q] = fma8_bf16(gv[j], xv, ag[q]);
+                  au[q] = fma8_bf16(uv[j], xv, au[q]);
                 }
               }
             }
@@ -384,9 +415,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     const int d = L.pd[pair];
     const int r0 = rg * kR2;
     const float4 *a = act4 + static_cast<size_t>(pair) * (I / 4);
-    float v[kR2];
+    unsigned long long v[kR2];  // two fp32 partial sums each
 #pragma unroll
-    for (int rr = 0; rr < kR2; ++rr) v[rr] = 0.f;
+    for (int rr = 0; rr < kR2; ++rr) v[rr] = 0ull;
     for (int base = 0; base < I8; base += 32 * kU2) {
 #pragma unroll
       for (int j = 0; j < kU2; ++j) {
@@ -394,7 +425,6 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
         if (c < I8) {
           const float4 a0 = cache_act ? a[2 * c] : __ldcg(a + 2 * c);
           const float4 a1 = cache_act ? a[2 * c + 1] : __ldcg(a + 2 * c + 1);
-          const float x[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
           for (int rr = 0; rr < kR2; ++rr) {
             const int r = r0 + rr;
@@ -402,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
               const uint4 wv =
                   w2_smem ? reinterpret_cast<const uint4 *>(sw2)[(d * rows_per_cta + r) * I8 + c]
                           : __ldg(w2 + (static_cast<size_t>(L.dexp[d]) * H + h0 + r) * I8 + c);
-              v[rr] += dot8(wv, x);
+              fma8_f32x2(wv, a0, a1, v[rr]);
             }
           }
         }
@@ -410,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     }
 #pragma unroll
     for (int rr = 0; rr < kR2; ++rr) {
-      const float sv = warp_sum(v[rr]);
+      const float sv = warp_sum(sum_f32x2(v[rr]));
       if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
     }
   }
