@@ -164,6 +164,7 @@ constexpr int kGroupSteps = kGroupMaxN / kGroupThreads;  // 32-entry steps per w
 
 size_t group_smem_bytes(int n, int E) {
   return static_cast<size_t>((n + 3) & ~3) * sizeof(int32_t) +
+         static_cast<size_t>(E) * sizeof(int32_t) +
          static_cast<size_t>(kGroupWarps) * E * sizeof(uint16_t);
 }
 
@@ -174,7 +175,8 @@ __global__ void __launch_bounds__(kGroupThreads)
                  int H8, uint4 *__restrict__ xs, int *ready, int n_ready, int *zero_done) {
   extern __shared__ __align__(16) unsigned char group_smem[];
   int32_t *s_sorted = reinterpret_cast<int32_t *>(group_smem);      // [n]
-  uint16_t *s_hist = reinterpret_cast<uint16_t *>(s_sorted + ((n + 3) & ~3));  // [warps][E]
+  int32_t *s_tot = s_sorted + ((n + 3) & ~3);                         // [E]
+  uint16_t *s_hist = reinterpret_cast<uint16_t *>(s_tot + E);         // [warps][E]
   __shared__ int32_t s_warp_tot[kGroupWarps];
   __shared__ int32_t s_nvalid;
   grid_dep_wait();
@@ -188,8 +190,10 @@ __global__ void __launch_bounds__(kGroupThreads)
   for (int x = tid; x < kGroupWarps * E; x += kGroupThreads) s_hist[x] = 0;
   __syncthreads();
   uint16_t *my_hist = s_hist + warp * E;
-  // the warp's ids, loaded once (per_warp <= 32 * kGroupSteps)
+  // the warp's ids, loaded once (per_warp <= 32 * kGroupSteps), and the
+  // __match_any_sync masks of the counting pass, reused by the ranking pass
   int ev[kGroupSteps];
+  uint32_t pm[kGroupSteps];
 #pragma unroll
   for (int q = 0; q < kGroupSteps; ++q) {
     const int i = i0 + 32 * q + lane;
@@ -206,16 +210,29 @@ __global__ void __launch_bounds__(kGroupThreads)
     const int i = i0 + 32 * q + lane;
     const int e = ev[q];
     const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    pm[q] = peers;
     if (e >= 0 && (peers & lt) == 0) my_hist[e] += static_cast<uint16_t>(__popc(peers));
     if (publish && status != nullptr && __any_sync(0xffffffffu, i < n && e < 0) && lane == 0)
       atomicOr(status, kStatusBadId);
     __syncwarp();
   }
   __syncthreads();
-  // per-expert totals, exclusive scan over experts (E <= 1024: one per thread)
-  int tot = 0;
-  if (tid < E)
-    for (int w = 0; w < kGroupWarps; ++w) tot += s_hist[w * E + tid];
+  // per expert: a warp scans the 32 warps' counts (lane w holds warp w's),
+  // leaving each warp's exclusive prefix in place and the total in s_tot
+  for (int e = warp; e < E; e += kGroupWarps) {
+    const int c = s_hist[lane * E + e];
+    int wi = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += x;
+    }
+    s_hist[lane * E + e] = static_cast<uint16_t>(wi - c);
+    if (lane == 31) s_tot[e] = wi;
+  }
+  __syncthreads();
+  // exclusive scan over experts (E <= 1024: one per thread)
+  const int tot = tid < E ? s_tot[tid] : 0;
   int incl = tot;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -236,18 +253,18 @@ __global__ void __launch_bounds__(kGroupThreads)
   __syncthreads();
   const int excl = incl - tot + (warp > 0 ? s_warp_tot[warp - 1] : 0);
   if (tid < E) {
+    s_tot[tid] = excl;  // becomes the expert's offset
     if (publish) expert_offsets[tid] = excl;
     if (tid == E - 1) {
       s_nvalid = excl + tot;
       if (publish) expert_offsets[E] = excl + tot;
     }
-    // counts -> running bases, warps in order (positions < n fit 16 bits)
-    int run = excl;
-    for (int w = 0; w < kGroupWarps; ++w) {
-      const int c = s_hist[w * E + tid];
-      s_hist[w * E + tid] = static_cast<uint16_t>(run);
-      run += c;
-    }
+  }
+  __syncthreads();
+  // warp prefixes -> running bases (positions < n fit 16 bits)
+  for (int x = tid; x < kGroupWarps * E; x += kGroupThreads) {
+    const int e = x - (x / E) * E;
+    s_hist[x] = static_cast<uint16_t>(s_hist[x] + s_tot[e]);
   }
   __syncthreads();
 #pragma unroll
@@ -255,7 +272,7 @@ __global__ void __launch_bounds__(kGroupThreads)
     if (32 * q >= per_warp) break;
     const int i = i0 + 32 * q + lane;
     const int e = ev[q];
-    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const uint32_t peers = pm[q];
     const int pos = e >= 0 ? my_hist[e] + __popc(peers & lt) : -1;
     __syncwarp();
     if (e >= 0 && (peers & lt) == 0) my_hist[e] += static_cast<uint16_t>(__popc(peers));
