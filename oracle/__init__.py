@@ -54,8 +54,13 @@ def _load(mutation: int = 0) -> ctypes.CDLL:
     lib.oracle_permute.argtypes = [P, i64, i32, P, P]
     lib.oracle_moe_token_loop.argtypes = [P, P, P, P, P, i64, i64, i64, i32, i32, P, i64, P]
     lib.oracle_moe_expert_loop.argtypes = [P, P, P, P, P, i64, i64, i64, i32, i32, P]
+    lib.oracle_moe_token_loop_ex.argtypes = [P, P, P, P, P, i32, P, P, i64, i64, i64, i32, i32,
+                                             P, i64, P]
+    lib.oracle_moe_expert_loop_ex.argtypes = [P, P, P, P, P, i32, P, P, i64, i64, i64, i32, i32,
+                                              P]
     for f in ("oracle_route", "oracle_permute", "oracle_moe_token_loop",
-              "oracle_moe_expert_loop", "oracle_max_threads", "oracle_mutation"):
+              "oracle_moe_expert_loop", "oracle_moe_token_loop_ex", "oracle_moe_expert_loop_ex",
+              "oracle_max_threads", "oracle_mutation"):
         getattr(lib, f).restype = ctypes.c_int
     lib.oracle_set_threads.argtypes = [i32]
     lib.oracle_set_threads.restype = None
@@ -129,30 +134,52 @@ def _forward_args(hidden, w1, w2, topk_w, ids):
     return hb, w1b, w2b, tw, ti, T, H, I, E, k
 
 
-def moe_token_loop(hidden, w1, w2, topk_w, ids, rows=None, mutation: int = 0):
+# activations of the 0.13.2 page's activation_fn
+ACTS = {"silu": 0, "gelu": 1, "swigluoai": 2}
+
+
+def _variant_args(act, b1, b2, E, H, I):
+    if act not in ACTS:
+        raise ValueError(f"unknown activation {act!r}")
+    b1a = b2a = None
+    if b1 is not None:
+        b1a = np.ascontiguousarray(np.asarray(b1, dtype=np.float32).reshape(E, 2 * I))
+    if b2 is not None:
+        b2a = np.ascontiguousarray(np.asarray(b2, dtype=np.float32).reshape(E, H))
+    return ACTS[act], b1a, b2a
+
+
+def moe_token_loop(hidden, w1, w2, topk_w, ids, rows=None, mutation: int = 0,
+                   act: str = "silu", b1=None, b2=None):
     """Formulation A (per-token loop).  Returns float64 [T, H], or
-    [len(rows), H] for the listed tokens only."""
+    [len(rows), H] for the listed tokens only.  act: "silu", "gelu" (tanh
+    form) or "swigluoai"; b1 fp32 [E, 2I] (gate then up), b2 fp32 [E, H]."""
     hb, w1b, w2b, tw, ti, T, H, I, E, k = _forward_args(hidden, w1, w2, topk_w, ids)
+    a, b1a, b2a = _variant_args(act, b1, b2, E, H, I)
     if rows is None:
         rr, nrows, n = None, -1, T
     else:
         rr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
         nrows = n = rr.shape[0]
     out = np.empty((max(n, 1), H), np.float64)
-    rc = _load(mutation).oracle_moe_token_loop(
-        _ptr(hb), _ptr(w1b), _ptr(w2b), _ptr(tw), _ptr(ti), T, H, I, E, k,
+    rc = _load(mutation).oracle_moe_token_loop_ex(
+        _ptr(hb), _ptr(w1b), _ptr(w2b), None if b1a is None else _ptr(b1a),
+        None if b2a is None else _ptr(b2a), a, _ptr(tw), _ptr(ti), T, H, I, E, k,
         None if rr is None else _ptr(rr), nrows, _ptr(out))
     if rc != 0:
         raise RuntimeError("oracle_moe_token_loop failed")
     return out[:n]
 
 
-def moe_expert_loop(hidden, w1, w2, topk_w, ids, mutation: int = 0):
+def moe_expert_loop(hidden, w1, w2, topk_w, ids, mutation: int = 0,
+                    act: str = "silu", b1=None, b2=None):
     """Formulation B (per-expert mask loop).  Returns float64 [T, H]."""
     hb, w1b, w2b, tw, ti, T, H, I, E, k = _forward_args(hidden, w1, w2, topk_w, ids)
+    a, b1a, b2a = _variant_args(act, b1, b2, E, H, I)
     out = np.empty((max(T, 1), H), np.float64)
-    rc = _load(mutation).oracle_moe_expert_loop(
-        _ptr(hb), _ptr(w1b), _ptr(w2b), _ptr(tw), _ptr(ti), T, H, I, E, k, _ptr(out))
+    rc = _load(mutation).oracle_moe_expert_loop_ex(
+        _ptr(hb), _ptr(w1b), _ptr(w2b), None if b1a is None else _ptr(b1a),
+        None if b2a is None else _ptr(b2a), a, _ptr(tw), _ptr(ti), T, H, I, E, k, _ptr(out))
     if rc != 0:
         raise RuntimeError("oracle_moe_expert_loop failed")
     return out[:T]

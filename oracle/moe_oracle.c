@@ -32,6 +32,13 @@
  *   - expert ids outside [0, E) in the forward input are skipped (the
  *     per-expert loop of Model.forward only visits 0..E-1).
  *   - silu(z) = z / (1 + exp(-z)).
+ *   - the variants of the 0.13.2 page (activation_fn, swigluoai, b1/b2 in
+ *     ref_moe): gelu is the tanh form, which is what jax.nn.gelu computes
+ *     when called as activation_fn calls it (approximate defaults to true);
+ *     swigluoai(g, u) = (clip(u, -7, 7) + 1) * g' * sigmoid(1.702 g') with
+ *     g' = min(g, 7); b1 (fp32 [E, 2I]: gate bias, then up bias) is added to
+ *     the two projections before the activation, b2 (fp32 [E, H]) to the
+ *     expert output before the top-k weighting.
  */
 #include <math.h>
 #include <stdint.h>
@@ -58,6 +65,29 @@ static double bf16_to_double(uint16_t b)
 }
 
 static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+enum { ACT_SILU = 0, ACT_GELU_TANH = 1, ACT_SWIGLUOAI = 2 };
+
+/* 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))) */
+static double gelu_tanh(double z)
+{
+    const double c = sqrt(2.0 / 3.14159265358979323846);
+    if (MUTATED(8)) return 0.5 * z * (1.0 + erf(z / sqrt(2.0)));  /* the erf form */
+    return 0.5 * z * (1.0 + tanh(c * (z + 0.044715 * z * z * z)));
+}
+
+/* the gated activation of activation_fn: act(gate) * up, or swigluoai */
+static double gated(int act, double g, double u)
+{
+    if (act == ACT_GELU_TANH) return gelu_tanh(g) * u;
+    if (act == ACT_SWIGLUOAI) {
+        const double alpha = 1.702, limit = 7.0;
+        double gc = g < limit ? g : limit;
+        double uc = u < -limit ? -limit : (u > limit ? limit : u);
+        return (uc + 1.0) * gc / (1.0 + exp(-alpha * gc));
+    }
+    return silu(g) * u;
+}
 
 int oracle_mutation(void) { return ORACLE_MUTATION; }
 
@@ -165,16 +195,17 @@ int oracle_permute(const int32_t *ids, int64_t n, int E,
 }
 
 /*
- * One expert's SwiGLU FFN on one token, in double:
- *   g_i = W1[e][i,:] . x, u_i = W1[e][I+i,:] . x, a_i = silu(g_i) * u_i,
- *   y_h = W2[e][h,:] . a.
+ * One expert's gated FFN on one token, in double:
+ *   g_i = W1[e][i,:] . x + b1[e][i], u_i = W1[e][I+i,:] . x + b1[e][I+i],
+ *   a_i = act(g_i, u_i), y_h = W2[e][h,:] . a + b2[e][h]
+ * (absent biases count as zero; act is silu(g)*u unless a variant is asked).
  * Layout of atrex-bench #009: F.linear(x, w1_e) is x . w1_e^T with w1_e of
  * shape [2I, H]; the first I outputs are gate, the next I are up;
  * F.linear(act, w2_e) with w2_e of shape [H, I].
  */
-static void expert_ffn(const uint16_t *w1, const uint16_t *w2, int e,
-                       int64_t H, int64_t I, const double *x, double *a,
-                       double *y)
+static void expert_ffn(const uint16_t *w1, const uint16_t *w2, const float *b1,
+                       const float *b2, int act, int e, int64_t H, int64_t I,
+                       const double *x, double *a, double *y)
 {
     const uint16_t *W1 = w1 + (size_t)e * 2 * I * H;
     const uint16_t *W2 = w2 + (size_t)e * H * I;
@@ -187,7 +218,14 @@ static void expert_ffn(const uint16_t *w1, const uint16_t *w2, int e,
             g += bf16_to_double(rg[h]) * x[h];
             u += bf16_to_double(ru[h]) * x[h];
         }
-        a[i] = silu(g) * u;
+        if (b1) {
+            double bg = (double)b1[(size_t)e * 2 * I + i];
+            double bu = (double)b1[(size_t)e * 2 * I + I + i];
+            if (MUTATED(6)) { double tmp = bg; bg = bu; bu = tmp; }
+            g += bg;
+            u += bu;
+        }
+        a[i] = gated(act, g, u);
     }
     for (int64_t h = 0; h < H; ++h) {
         double acc = 0.0;
@@ -198,8 +236,15 @@ static void expert_ffn(const uint16_t *w1, const uint16_t *w2, int e,
                                    : bf16_to_double(W2[(size_t)h * I + i]);
             acc += wv * a[i];
         }
-        y[h] = acc;
+        y[h] = acc + (b2 && !MUTATED(7) ? (double)b2[(size_t)e * H + h] : 0.0);
     }
+}
+
+/* planted mistake 7: b2 added once per chosen expert after the weighting */
+static void add_b2_unweighted(const float *b2, int e, int64_t H, double *o)
+{
+    if (MUTATED(7) && b2)
+        for (int64_t h = 0; h < H; ++h) o[h] += (double)b2[(size_t)e * H + h];
 }
 
 /*
@@ -209,12 +254,13 @@ static void expert_ffn(const uint16_t *w1, const uint16_t *w2, int e,
  * skipped.  hidden [T,H], w1 [E,2I,H], w2 [E,H,I] are bf16 bit patterns;
  * topk_w [T,k] double; out is [nrows or T, H] double, overwritten.
  */
-int oracle_moe_token_loop(const uint16_t *hidden, const uint16_t *w1,
-                          const uint16_t *w2, const double *topk_w,
-                          const int32_t *ids, int64_t T, int64_t H, int64_t I,
-                          int E, int k, const int64_t *rows, int64_t nrows,
-                          double *out)
+int oracle_moe_token_loop_ex(const uint16_t *hidden, const uint16_t *w1,
+                             const uint16_t *w2, const float *b1, const float *b2,
+                             int act, const double *topk_w, const int32_t *ids,
+                             int64_t T, int64_t H, int64_t I, int E, int k,
+                             const int64_t *rows, int64_t nrows, double *out)
 {
+    if (act < ACT_SILU || act > ACT_SWIGLUOAI) return -1;
     if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1) return -1;
     int64_t n = nrows >= 0 ? nrows : T;
     int err = 0;
@@ -237,15 +283,26 @@ int oracle_moe_token_loop(const uint16_t *hidden, const uint16_t *w1,
                 for (int j = 0; j < k; ++j) {
                     int e = ids[t * k + j];
                     if (e < 0 || e >= E) continue;
-                    expert_ffn(w1, w2, e, H, I, x, a, y);
+                    expert_ffn(w1, w2, b1, b2, act, e, H, I, x, a, y);
                     double wj = topk_w[t * k + j];
                     for (int64_t h = 0; h < H; ++h) o[h] += wj * y[h];
+                    add_b2_unweighted(b2, e, H, o);
                 }
             }
         }
         free(x); free(a); free(y);
     }
     return err ? -1 : 0;
+}
+
+int oracle_moe_token_loop(const uint16_t *hidden, const uint16_t *w1,
+                          const uint16_t *w2, const double *topk_w,
+                          const int32_t *ids, int64_t T, int64_t H, int64_t I,
+                          int E, int k, const int64_t *rows, int64_t nrows,
+                          double *out)
+{
+    return oracle_moe_token_loop_ex(hidden, w1, w2, NULL, NULL, ACT_SILU, topk_w, ids,
+                                    T, H, I, E, k, rows, nrows, out);
 }
 
 /*
@@ -255,12 +312,13 @@ int oracle_moe_token_loop(const uint16_t *hidden, const uint16_t *w1,
  * A token routed twice to e thus gets the summed weight.  Same argument
  * layout as formulation A (all T rows).
  */
-int oracle_moe_expert_loop(const uint16_t *hidden, const uint16_t *w1,
-                           const uint16_t *w2, const double *topk_w,
-                           const int32_t *ids, int64_t T, int64_t H, int64_t I,
-                           int E, int k, double *out)
+int oracle_moe_expert_loop_ex(const uint16_t *hidden, const uint16_t *w1,
+                              const uint16_t *w2, const float *b1, const float *b2,
+                              int act, const double *topk_w, const int32_t *ids,
+                              int64_t T, int64_t H, int64_t I, int E, int k, double *out)
 {
     if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1) return -1;
+    if (act < ACT_SILU || act > ACT_SWIGLUOAI) return -1;
     double *what = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
     if (!what) return -1;
     for (int64_t i = 0; i < T * H; ++i) out[i] = 0.0;
@@ -285,7 +343,7 @@ int oracle_moe_expert_loop(const uint16_t *hidden, const uint16_t *w1,
                 for (int64_t t = 0; t < T; ++t) {
                     if (what[t] == 0.0) continue;
                     for (int64_t h = 0; h < H; ++h) x[h] = bf16_to_double(hidden[(size_t)t * H + h]);
-                    expert_ffn(w1, w2, e, H, I, x, a, y);
+                    expert_ffn(w1, w2, b1, b2, act, e, H, I, x, a, y);
                     double *o = out + (size_t)t * H;
                     for (int64_t h = 0; h < H; ++h) o[h] += what[t] * y[h];
                 }
@@ -295,4 +353,13 @@ int oracle_moe_expert_loop(const uint16_t *hidden, const uint16_t *w1,
     }
     free(what);
     return err ? -1 : 0;
+}
+
+int oracle_moe_expert_loop(const uint16_t *hidden, const uint16_t *w1,
+                           const uint16_t *w2, const double *topk_w,
+                           const int32_t *ids, int64_t T, int64_t H, int64_t I,
+                           int E, int k, double *out)
+{
+    return oracle_moe_expert_loop_ex(hidden, w1, w2, NULL, NULL, ACT_SILU, topk_w, ids, T, H,
+                                     I, E, k, out);
 }

@@ -159,6 +159,116 @@ def pin_forward_dense(mutation=0, seed=4, H=64, I=32):
     return bool(ok)
 
 
+# ------------------------------------------- pins of the epilogue variants
+# (activation_fn, swigluoai and the b1/b2 biases of the 0.13.2 TPU page)
+
+
+def _dense_mlp(act, hidden, w1e, w2e):
+    """One expert on every token with torch fp64 library routines."""
+    X = torch.tensor(to64(hidden))
+    W1, W2 = torch.tensor(to64(w1e)), torch.tensor(to64(w2e))
+    I = W1.shape[0] // 2
+    G = X @ W1[:I].T
+    U = X @ W1[I:].T
+    if act == "gelu":
+        A = torch.nn.functional.gelu(G, approximate="tanh") * U
+    elif act == "swigluoai":
+        # unclamped range only: g * sigmoid(1.702 g) = silu(1.702 g) / 1.702
+        assert G.max() < 7 and U.abs().max() < 7
+        A = (U + 1.0) * torch.nn.functional.silu(1.702 * G) / 1.702
+    else:
+        A = torch.nn.functional.silu(G) * U
+    return (A @ W2.T).numpy()
+
+
+def pin_activation_library(mutation=0, seed=21):
+    """E = k = 1 with weight 1 is one expert's MLP: gelu (tanh form) and
+    swigluoai (in its unclamped range) against torch fp64."""
+    ok = True
+    for act in ("gelu", "swigluoai", "silu"):
+        hidden, w1, w2, _ = make_inputs(11, 64, 32, 1, seed=seed)
+        ids = np.zeros((11, 1), np.int32)
+        w = np.ones((11, 1))
+        ref = _dense_mlp(act, hidden, w1[0], w2[0])
+        a = oracle.moe_token_loop(hidden, w1, w2, w, ids, mutation=mutation, act=act)
+        b = oracle.moe_expert_loop(hidden, w1, w2, w, ids, mutation=mutation, act=act)
+        ok &= close(a, ref) and close(b, ref)
+    return bool(ok)
+
+
+def pin_swigluoai_clamped(mutation=0):
+    """All gate values 8 and up values -8 or 9: both clip, so every
+    activation is (clip(u) + 1) * 7 * sigmoid(11.914), and doubling w1
+    changes nothing."""
+    H, I, E = 64, 32, 2
+    hidden = bf16(np.ones((3, H)))
+    w1 = np.zeros((E, 2 * I, H), np.float32)
+    w1[:, :I, :] = 0.125                       # g = 8
+    w1[0, I:, :] = -0.125                      # u = -8 -> -7
+    w1[1, I:, :] = 9.0 / 64                    # u = 9 -> 7
+    w2 = np.random.default_rng(3).standard_normal((E, H, I)).astype(np.float32) * 0.1
+    ids = np.array([[0, 1], [1, 0], [1, 1]], np.int32)
+    w = np.array([[0.25, 0.75], [0.5, 0.5], [0.1, 0.9]])
+    sig = scipy.special.expit(1.702 * 7.0)
+    acts = np.stack([np.full(I, (-7.0 + 1.0) * 7.0 * sig), np.full(I, (7.0 + 1.0) * 7.0 * sig)])
+    W2 = to64(bf16(w2.reshape(-1)).reshape(E, H, I))
+    y = np.einsum("ehi,ei->eh", W2, acts)
+    ref = np.stack([sum(w[t, j] * y[ids[t, j]] for j in range(2)) for t in range(3)])
+    ok = True
+    for scale in (1.0, 2.0):
+        a = oracle.moe_token_loop(hidden, bf16(w1 * scale), bf16(w2), w, ids,
+                                  mutation=mutation, act="swigluoai")
+        ok &= close(a, ref, 1e-12)
+    return bool(ok)
+
+
+def pin_b1_with_zero_w1(mutation=0):
+    """w1 = 0: the projections are the biases alone, so
+    act = silu(b1_gate) * b1_up per expert, the same for every token."""
+    T, H, I, E, k = 5, 48, 16, 3, 2
+    hidden, _, w2, logits = make_inputs(T, H, I, E, seed=22)
+    w1 = bf16(np.zeros((E, 2 * I, H)))
+    b1 = np.random.default_rng(5).standard_normal((E, 2 * I)).astype(np.float32)
+    ids, w = oracle.route(logits.numpy(), k, True)
+    G, U = b1[:, :I].astype(np.float64), b1[:, I:].astype(np.float64)
+    A = G * scipy.special.expit(G) * U
+    y = np.einsum("ehi,ei->eh", to64(w2), A)
+    ref = np.stack([sum(w[t, j] * y[ids[t, j]] for j in range(k)) for t in range(T)])
+    a = oracle.moe_token_loop(hidden, w1, w2, w, ids, mutation=mutation, b1=b1)
+    b = oracle.moe_expert_loop(hidden, w1, w2, w, ids, mutation=mutation, b1=b1)
+    return bool(close(a, ref) and close(b, ref))
+
+
+def pin_b2_with_zero_w2(mutation=0):
+    """w2 = 0: each expert's output is its bias b2[e], so
+    out[t] = sum_j w[t, j] * b2[ids[t, j]] exactly."""
+    T, H, I, E, k = 6, 32, 16, 4, 3
+    hidden, w1, _, logits = make_inputs(T, H, I, E, seed=23)
+    w2 = bf16(np.zeros((E, H, I)))
+    b2 = np.random.default_rng(6).standard_normal((E, H)).astype(np.float32)
+    ids, w = oracle.route(logits.numpy(), k, False)
+    ref = np.stack([sum(w[t, j] * b2[ids[t, j]].astype(np.float64) for j in range(k))
+                    for t in range(T)])
+    a = oracle.moe_token_loop(hidden, w1, w2, w, ids, mutation=mutation, b2=b2)
+    b = oracle.moe_expert_loop(hidden, w1, w2, w, ids, mutation=mutation, b2=b2)
+    return bool(close(a, ref) and close(b, ref))
+
+
+def pin_variants_formulations_agree(mutation=0):
+    ok = True
+    for act in ("silu", "gelu", "swigluoai"):
+        hidden, w1, w2, logits = make_inputs(13, 64, 32, 5, seed=24)
+        rng = np.random.default_rng(7)
+        b1 = rng.standard_normal((5, 64)).astype(np.float32) * 0.1
+        b2 = rng.standard_normal((5, 64)).astype(np.float32) * 0.1
+        ids, w = oracle.route(logits.numpy(), 2, True)
+        a = oracle.moe_token_loop(hidden, w1, w2, w, ids, mutation=mutation, act=act, b1=b1, b2=b2)
+        b = oracle.moe_expert_loop(hidden, w1, w2, w, ids, mutation=mutation, act=act, b1=b1,
+                                   b2=b2)
+        ok &= close(a, b)
+    return bool(ok)
+
+
 # ---------------------------------------------------------------- tests
 
 def test_golden_route(golden_dir):
@@ -298,6 +408,33 @@ def test_forward_duplicate_ids_sum_weights():
     assert close(a[rows], c[rows]) and close(b[rows], c[rows])
 
 
+def test_activation_variants_against_torch():
+    assert pin_activation_library()
+
+
+def test_swigluoai_clamps():
+    assert pin_swigluoai_clamped()
+
+
+def test_b1_with_zero_w1_is_closed_form():
+    assert pin_b1_with_zero_w1()
+
+
+def test_b2_with_zero_w2_is_weighted_bias_sum():
+    assert pin_b2_with_zero_w2()
+
+
+def test_variant_formulations_agree():
+    assert pin_variants_formulations_agree()
+
+
+def test_unknown_activation_rejected():
+    hidden, w1, w2, logits = make_inputs(2, 64, 32, 2, seed=25)
+    ids, w = oracle.route(logits.numpy(), 1, True)
+    with pytest.raises(ValueError):
+        oracle.moe_token_loop(hidden, w1, w2, w, ids, act="relu")
+
+
 def test_forward_invalid_ids_skipped():
     hidden, w1, w2, _ = make_inputs(3, 64, 32, 4, seed=13)
     ids = np.array([[1, 9], [-1, 2], [-5, 4]], np.int32)
@@ -336,6 +473,9 @@ MUTATIONS = {
     3: "renormalisation dropped",
     4: "ties broken towards the highest index",
     5: "permutation visits indices from the back (unstable)",
+    6: "gate and up biases of b1 swapped",
+    7: "b2 added once per expert after the top-k weighting",
+    8: "gelu in its erf form instead of the tanh form",
 }
 
 
@@ -350,6 +490,11 @@ def test_planted_mistakes_are_caught(mutation, golden_dir):
         "route_library": pin_route_library(mutation),
         "permute_library": pin_permute_library(mutation),
         "forward_dense": pin_forward_dense(mutation) and pin_forward_dense(mutation, H=48, I=48),
+        "activation_library": pin_activation_library(mutation),
+        "swigluoai_clamped": pin_swigluoai_clamped(mutation),
+        "b1_zero_w1": pin_b1_with_zero_w1(mutation),
+        "b2_zero_w2": pin_b2_with_zero_w2(mutation),
+        "variants_agree": pin_variants_formulations_agree(mutation),
     }
     assert oracle._load(mutation).oracle_mutation() == mutation
     caught = [k for k, v in results.items() if not v]
