@@ -111,6 +111,35 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
                 int64_t T, int H, int I, int E, int k, void *stream);
 
 /*
+ * moe_forward_ex -- moe_forward with the expert-FFN variants of the 0.13.2
+ * version of the TPU page: its activation_fn choice and the optional
+ * per-expert biases that ref_moe adds to both projections.
+ *
+ *   b1    [E, 2I] fp32 or NULL; b1[e, 0..I-1] is added to the gate
+ *         projection and b1[e, I..2I-1] to the up projection, before the
+ *         activation
+ *   b2    [E, H] fp32 or NULL; added to the expert's output, so it is
+ *         scaled by the top-k weight like the rest of that output
+ *   act   MOE_ACT_SILU:      silu(gate) * up (what moe_forward computes)
+ *         MOE_ACT_GELU_TANH: gelu(gate) * up, gelu in its tanh form
+ *                            0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3)))
+ *         MOE_ACT_SWIGLUOAI: (clip(up, -7, 7) + 1) * g * sigmoid(1.702 g)
+ *                            with g = min(gate, 7)
+ * Everything else (arguments, layouts, numerics, paths, determinism) is as
+ * in moe_forward, which equals moe_forward_ex(..., NULL, NULL,
+ * MOE_ACT_SILU, ...).  b1 and b2 must start on a 16-byte boundary.
+ * Errors: those of moe_forward, plus INVALID_ARG for an unknown act or an
+ *         unaligned b1/b2.
+ */
+#define MOE_ACT_SILU 0
+#define MOE_ACT_GELU_TANH 1
+#define MOE_ACT_SWIGLUOAI 2
+int moe_forward_ex(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
+                   const float *b1, const float *b2, int act,
+                   const float *topk_weights, const int32_t *topk_ids, float *out,
+                   int64_t T, int H, int I, int E, int k, void *stream);
+
+/*
  * moe_forward_small_noalloc -- the small-batch path of moe_forward (the two
  * GEMV kernels) in a form that never allocates device memory.  The pages
  * have no counterpart: it exists for callers that cannot allocate once they

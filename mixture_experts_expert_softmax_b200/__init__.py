@@ -32,6 +32,10 @@ MOE_NOALLOC_MAX_T = 16
 MOE_NOALLOC_MAX_ACT = 262144
 MOE_STATUS_TIMEOUT = 0x1
 MOE_STATUS_BAD_ID = 0x2
+MOE_ACT_SILU = 0
+MOE_ACT_GELU_TANH = 1
+MOE_ACT_SWIGLUOAI = 2
+ACTS = {"silu": MOE_ACT_SILU, "gelu": MOE_ACT_GELU_TANH, "swigluoai": MOE_ACT_SWIGLUOAI}
 
 # every symbol declared in include/moe.h
 EXPORTED = (
@@ -39,7 +43,7 @@ EXPORTED = (
     "moe_get_device_status", "moe_set_small_t_max", "moe_set_sync_each_stage",
     "moe_set_wait_limit_ns", "moe_last_failed_stage", "moe_debug_wait_timeout",
     "moe_profile_enable", "moe_profile_reset", "moe_profile_read",
-    "moe_forward_small_noalloc",
+    "moe_forward_small_noalloc", "moe_forward_ex",
 )
 
 
@@ -71,6 +75,7 @@ def _load() -> ctypes.CDLL:
         "moe_profile_reset": ([], I32),
         "moe_profile_read": ([I32, P, P, P], I32),
         "moe_forward_small_noalloc": ([P, P, P, P, P, P, I64, I32, I32, I32, I32, P], I32),
+        "moe_forward_ex": ([P, P, P, P, P, I32, P, P, P, I64, I32, I32, I32, I32, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -133,9 +138,16 @@ def moe_route(logits: torch.Tensor, k: int, renorm: bool = True,
 
 def moe_forward(hidden: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
                 topk_weights: torch.Tensor, topk_ids: torch.Tensor,
-                out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                out: torch.Tensor | None = None, stream=None, *, act: str = "silu",
+                b1: torch.Tensor | None = None, b2: torch.Tensor | None = None) -> torch.Tensor:
     """Fused MoE forward: hidden [T,H] bf16, w1 [E,2I,H] bf16, w2 [E,H,I] bf16,
-    topk_weights [T,k] fp32, topk_ids [T,k] int32 -> out [T,H] fp32."""
+    topk_weights [T,k] fp32, topk_ids [T,k] int32 -> out [T,H] fp32.
+
+    act ("silu", "gelu" (tanh form) or "swigluoai") and the optional fp32
+    biases b1 [E,2I] and b2 [E,H] select the expert-FFN variant; anything
+    but the default goes through moe_forward_ex."""
+    if act not in ACTS:
+        raise ValueError(f"act must be one of {sorted(ACTS)}, got {act!r}")
     _need(hidden, "hidden", torch.bfloat16)
     T, H = hidden.shape
     _need(w1, "w1", torch.bfloat16)
@@ -149,9 +161,20 @@ def moe_forward(hidden: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
     if out is None:
         out = torch.empty((T, H), dtype=torch.float32, device=hidden.device)
     _need(out, "out", torch.float32, (T, H))
-    _check(_lib.moe_forward(hidden.data_ptr(), w1.data_ptr(), w2.data_ptr(),
-                            topk_weights.data_ptr(), topk_ids.data_ptr(), out.data_ptr(),
-                            T, H, I, E, k, _stream(stream)), "moe_forward")
+    if act == "silu" and b1 is None and b2 is None:
+        _check(_lib.moe_forward(hidden.data_ptr(), w1.data_ptr(), w2.data_ptr(),
+                                topk_weights.data_ptr(), topk_ids.data_ptr(), out.data_ptr(),
+                                T, H, I, E, k, _stream(stream)), "moe_forward")
+        return out
+    if b1 is not None:
+        _need(b1, "b1", torch.float32, (E, 2 * I))
+    if b2 is not None:
+        _need(b2, "b2", torch.float32, (E, H))
+    _check(_lib.moe_forward_ex(hidden.data_ptr(), w1.data_ptr(), w2.data_ptr(),
+                               None if b1 is None else b1.data_ptr(),
+                               None if b2 is None else b2.data_ptr(), ACTS[act],
+                               topk_weights.data_ptr(), topk_ids.data_ptr(), out.data_ptr(),
+                               T, H, I, E, k, _stream(stream)), "moe_forward_ex")
     return out
 
 
@@ -248,5 +271,5 @@ __all__ = [
     "moe_route", "moe_forward", "moe_forward_small_noalloc", "moe_permute", "get_device_status", "set_small_t_max",
     "set_sync_each_stage", "set_wait_limit_ns", "last_failed_stage", "debug_wait_timeout",
     "profile_enable", "profile_reset", "profile_read", "error_string", "MoEError",
-    "LIB_PATH", "EXPORTED",
+    "LIB_PATH", "EXPORTED", "ACTS",
 ]

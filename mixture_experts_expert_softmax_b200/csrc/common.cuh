@@ -384,6 +384,34 @@ __device__ __forceinline__ void grid_dep_launch() {
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
 
+// The gated activations of activation_fn on the 0.13.2 page
+// "tpu_inference/kernels/fused_moe/v1/kernel.py": act(gate) * up for silu
+// and gelu (tanh approximation), and swigluoai, which clips gate from above
+// and up on both sides at 7 and weighs gate by sigmoid(1.702 gate).
+enum : int { kActSilu = 0, kActGeluTanh = 1, kActSwigluOai = 2 };
+
+__device__ __forceinline__ float gelu_tanh_f(float z) {
+  // 0.5 z (1 + tanh(sqrt(2 / pi) (z + 0.044715 z^3)))
+  const float kS = 0.7978845608028654f;
+  return 0.5f * z * (1.0f + tanhf(kS * fmaf(0.044715f * z, z * z, z)));
+}
+
+template <int ACT>
+__device__ __forceinline__ float gated_f(float g, float u) {
+  if (ACT == kActGeluTanh) return gelu_tanh_f(g) * u;
+  if (ACT == kActSwigluOai) {
+    const float gc = fminf(g, 7.0f), uc = fminf(fmaxf(u, -7.0f), 7.0f);
+    return (uc + 1.0f) * (gc / (1.0f + __expf(-1.702f * gc)));
+  }
+  return silu_f(g) * u;
+}
+
+__device__ __forceinline__ float gated_rt(int act, float g, float u) {
+  return act == kActGeluTanh    ? gated_f<kActGeluTanh>(g, u)
+         : act == kActSwigluOai ? gated_f<kActSwigluOai>(g, u)
+                                : gated_f<kActSilu>(g, u);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);

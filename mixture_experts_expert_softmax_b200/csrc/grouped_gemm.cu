@@ -3,8 +3,11 @@
 //
 //   GEMM1 (+SwiGLU): for the rows of expert e in expert-sorted order,
 //     g = x . w1[e, 0:I, :]^T, u = x . w1[e, I:2I, :]^T  (fp32 in TMEM),
-//     act = silu(g) * u, stored as bf16 [rows, I].
-//   GEMM2: y = act . w2[e]^T (fp32 in TMEM).  For top-k <= 2 the epilogue
+//     act = silu(g) * u, stored as bf16 [rows, I].  Variants (the 0.13.2
+//     version of the page below): gelu (tanh form) or swigluoai in place of
+//     silu, and a bias b1[e] added to g and u before the activation.
+//   GEMM2: y = act . w2[e]^T (fp32 in TMEM), plus the bias b2[e] when given
+//     (before the top-k weight).  For top-k <= 2 the epilogue
 //     adds w_j * y_j of each row straight into out[token] with bulk
 //     reductions at L2 (out was zeroed first); out[t] = 0 + a + b is the
 //     same in either arrival order, so the result is still deterministic.
@@ -192,6 +195,11 @@ struct Params {
   // that finished zeroing out (both zero at launch)
   int *ready;
   int *zero_done;
+  // epilogue variant: activation (kAct*) and optional fp32 biases
+  // b1 [E, 2I] (gate, then up) and b2 [E, H]
+  const float *b1;
+  const float *b2;
+  int act_kind;
 };
 
 struct Tile {
@@ -263,6 +271,29 @@ __device__ __forceinline__ void give_up(const Params &p, volatile int *abort_fla
 }
 
 __device__ __forceinline__ float as_f32(uint32_t u) { return __uint_as_float(u); }
+
+// v[c] += b[c] for 32 fp32 values held as bits; b is 16-byte aligned and
+// the same for every lane (a broadcast load)
+__device__ __forceinline__ void add_bias32(uint32_t (&v)[32], const float *b) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float4 bb = __ldg(reinterpret_cast<const float4 *>(b) + j);
+    v[4 * j] = __float_as_uint(as_f32(v[4 * j]) + bb.x);
+    v[4 * j + 1] = __float_as_uint(as_f32(v[4 * j + 1]) + bb.y);
+    v[4 * j + 2] = __float_as_uint(as_f32(v[4 * j + 2]) + bb.z);
+    v[4 * j + 3] = __float_as_uint(as_f32(v[4 * j + 3]) + bb.w);
+  }
+}
+
+// act = ACT(g, u) for 32 columns, packed to bf16 pairs
+template <int ACT>
+__device__ __forceinline__ void gated_pack32(const uint32_t (&g)[32], const uint32_t (&u)[32],
+                                             uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int v = 0; v < 16; ++v)
+    pk[v] = pack_bf16x2(gated_f<ACT>(as_f32(g[2 * v]), as_f32(u[2 * v])),
+                        gated_f<ACT>(as_f32(g[2 * v + 1]), as_f32(u[2 * v + 1])));
+}
 
 // What one tile of the static schedule is: GEMM1 or GEMM2 (phase 1 or 2),
 // its place, and its global m-tile index.
@@ -569,6 +600,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (w.phase == 1) {
         __nv_bfloat16 *dst =
             p.act + static_cast<size_t>(my_row0 + (valid ? row : 0)) * p.I + tl.nt * (kAccN / 2);
+        const float *bg =
+            p.b1 ? p.b1 + static_cast<size_t>(tl.e) * 2 * p.I + tl.nt * (kAccN / 2) : nullptr;
 #pragma unroll 1
         for (int c0 = half * (kAccN / 4); c0 < (half + 1) * (kAccN / 4); c0 += 32) {
           uint32_t g[32], u[32];
@@ -576,13 +609,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_32cols(tbase + kAccN / 2 + c0, u);
           tmem_ld_wait();
           if (valid) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int v = 0; v < 16; ++v) {
-              const float a0 = silu_f(as_f32(g[2 * v])) * as_f32(u[2 * v]);
-              const float a1 = silu_f(as_f32(g[2 * v + 1])) * as_f32(u[2 * v + 1]);
-              pk[v] = pack_bf16x2(a0, a1);
+            if (bg) {
+              add_bias32(g, bg + c0);
+              add_bias32(u, bg + p.I + c0);
             }
+            uint32_t pk[16];
+            if (p.act_kind == kActGeluTanh)
+              gated_pack32<kActGeluTanh>(g, u, pk);
+            else if (p.act_kind == kActSwigluOai)
+              gated_pack32<kActSwigluOai>(g, u, pk);
+            else
+              gated_pack32<kActSilu>(g, u, pk);
             uint4 *d4 = reinterpret_cast<uint4 *>(dst + c0);
 #pragma unroll
             for (int v = 0; v < 4; ++v)
@@ -607,12 +644,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           orow = p.out + static_cast<size_t>(slot / p.k) * p.H;
         }
         uint8_t *srow = ebuf + lane * kRedPitch;
+        const float *b2row = p.b2 ? p.b2 + static_cast<size_t>(tl.e) * p.H : nullptr;
 #pragma unroll 1
         for (int c0 = half * (kAccN / 2); c0 < (half + 1) * (kAccN / 2); c0 += 32) {
           uint32_t v[32];
           tmem_ld_32cols(tbase + c0, v);
           tmem_ld_wait();
           const int col = tl.nt * kAccN + c0;
+          if (b2row && col < p.H) add_bias32(v, b2row + col);
           if (col < p.H && valid && !*abort_flag) {
             // the previous reduction from this row must have read it
             bulk_wait_group_read<0>();
@@ -630,12 +669,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         // this warp's 32 rows: whole blocks go out through TMA stores
         const bool whole = q * 32 + 32 <= my_rows;
+        const float *b2row = p.b2 ? p.b2 + static_cast<size_t>(tl.e) * p.H : nullptr;
 #pragma unroll 1
         for (int c0 = half * (kAccN / 2); c0 < (half + 1) * (kAccN / 2); c0 += 32) {
           uint32_t v[32];
           tmem_ld_32cols(tbase + c0, v);
           tmem_ld_wait();
           const int col = tl.nt * kAccN + c0;
+          if (b2row && col < p.H) add_bias32(v, b2row + col);
           if (col < p.H && whole) {
             // the previous store from this buffer must have read it
             if (lane == 0) bulk_wait_group_read<0>();
@@ -787,6 +828,9 @@ Params base_params(const GroupedGemmArgs &a) {
   }
   p.ready = a.ready;
   p.zero_done = a.zero_done;
+  p.b1 = a.b1;
+  p.b2 = a.b2;
+  p.act_kind = a.act_kind;
   return p;
 }
 

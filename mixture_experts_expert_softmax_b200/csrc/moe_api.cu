@@ -254,14 +254,28 @@ int moe_permute(const int32_t *topk_ids, int64_t T, int k, int E, int32_t *sorte
   return to_code(e);
 }
 
-int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
-                const float *topk_weights, const int32_t *topk_ids, float *out, int64_t T, int H,
-                int I, int E, int k, void *stream) {
+}  // extern "C"
+
+namespace {
+
+static_assert(MOE_ACT_SILU == moe::kActSilu && MOE_ACT_GELU_TANH == moe::kActGeluTanh &&
+                  MOE_ACT_SWIGLUOAI == moe::kActSwigluOai,
+              "activation codes of the ABI and the kernels agree");
+
+// moe_forward and moe_forward_ex: the variant is (b1, b2, act); b1 and b2
+// may be null.
+int forward_impl(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2, const float *b1,
+                 const float *b2, int act_kind, const float *topk_weights,
+                 const int32_t *topk_ids, float *out, int64_t T, int H, int I, int E, int k,
+                 void *stream) {
   if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (act_kind != MOE_ACT_SILU && act_kind != MOE_ACT_GELU_TANH && act_kind != MOE_ACT_SWIGLUOAI)
+    return MOE_ERR_INVALID_ARG;
   if (T > 0 && (hidden == nullptr || w1 == nullptr || w2 == nullptr || topk_weights == nullptr ||
                 topk_ids == nullptr || out == nullptr))
     return MOE_ERR_INVALID_ARG;
-  if (!aligned16(hidden) || !aligned16(w1) || !aligned16(w2) || !aligned16(out))
+  if (!aligned16(hidden) || !aligned16(w1) || !aligned16(w2) || !aligned16(out) ||
+      !aligned16(b1) || !aligned16(b2))
     return MOE_ERR_INVALID_ARG;
   if (H % 128 != 0 || I % 128 != 0 || E > kMaxExperts || k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
   const int64_t n = T * k;
@@ -280,7 +294,8 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
     Carver cv{static_cast<char *>(d->ws)};
     float *act = cv.take<float>(static_cast<size_t>(n) * I);
     return to_code(moe::launch_small_t(
-        hidden, w1, w2, topk_weights, topk_ids, act, out, T, H, I, E, k, d->status,
+        hidden, w1, w2, b1, b2, act_kind, topk_weights, topk_ids, act, out, T, H, I, E, k,
+        d->status,
         reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(d->status) + 64),
         &d->small_t_arrivals, static_cast<uint64_t>(g_wait_limit_ns), ctx.stream, hook));
   }
@@ -348,6 +363,9 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
   ga.out = out;
   ga.topk_weights = topk_weights;
   ga.fuse_combine = fuse_combine ? 1 : 0;
+  ga.b1 = b1;
+  ga.b2 = b2;
+  ga.act_kind = act_kind;
   if (gather_rows) {
     ga.ready = ready;
     ga.zero_done = ready + n_ready;
@@ -367,6 +385,25 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
   if (fuse_combine) return MOE_OK;
   e = moe::launch_combine(P, inv, topk_weights, out, T, H, k, d->status, ctx.stream, hook);
   return to_code(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
+                const float *topk_weights, const int32_t *topk_ids, float *out, int64_t T, int H,
+                int I, int E, int k, void *stream) {
+  return forward_impl(hidden, w1, w2, nullptr, nullptr, MOE_ACT_SILU, topk_weights, topk_ids,
+                      out, T, H, I, E, k, stream);
+}
+
+int moe_forward_ex(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
+                   const float *b1, const float *b2, int act, const float *topk_weights,
+                   const int32_t *topk_ids, float *out, int64_t T, int H, int I, int E, int k,
+                   void *stream) {
+  return forward_impl(hidden, w1, w2, b1, b2, act, topk_weights, topk_ids, out, T, H, I, E, k,
+                      stream);
 }
 
 int moe_get_device_status(void *stream, uint32_t *status) {

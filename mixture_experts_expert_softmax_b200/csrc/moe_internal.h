@@ -89,6 +89,11 @@ struct GroupedGemmArgs {
   // fused_gemm_ready_count(T*k, E)) and one more, all zero at launch
   int *ready;
   int *zero_done;
+  // epilogue variant: activation (kAct* of common.cuh) and optional fp32
+  // biases b1 [E, 2I] (gate, then up) and b2 [E, H], 16-byte aligned
+  const float *b1;
+  const float *b2;
+  int act_kind;
   int64_t T;
   int H, I, E, k;
   int num_sms;
@@ -117,7 +122,9 @@ bool small_t_supported(int H, int I);
 // touch, 0 before the first launch; arrivals: the host's copy of the value
 // it reaches once every launch made so far has finished (advanced by the
 // call).  act: T*k*I fp32 scratch.
+// b1, b2, act_kind: the epilogue variant, as in GroupedGemmArgs.
 cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
+                           const float *b1, const float *b2, int act_kind,
                            const float *topk_weights, const int32_t *topk_ids, float *act,
                            float *out, int64_t T, int H, int I, int E, int k, uint32_t *status,
                            unsigned long long *grid_sync, unsigned long long *arrivals,

@@ -10,7 +10,8 @@
 //     row i) row pairs -- gate row w1[e, i, :] and up row w1[e, I+i, :] --
 //     dealt round-robin to every warp of the grid.  A warp dots both rows
 //     with the hidden vector of each token routed to e and stores
-//     act[t*k + j, i] = silu(g) * u in fp32 (global memory).
+//     act[t*k + j, i] = silu(g) * u in fp32 (global memory) -- or the
+//     variant's activation of g + b1[e, i] and u + b1[e, I + i].
 //     Meanwhile the copy warp moves the w2 rows this CTA needs in phase 2
 //     into shared memory with bulk copies (or, when they do not fit, asks L2
 //     to prefetch them), so w2 streams from HBM alongside w1.  Bulk copies
@@ -20,8 +21,8 @@
 //   phase 2 (down + weighted combine): each CTA owns a slice of output rows
 //     h; a warp dots w2[e][h, :] (now on chip) with act of every pair of e,
 //     one pair and four rows h at a time (four independent sums), and
-//     out[t, h] = sum_{j=0..k-1} w[t, j] * dot_j is summed in fixed j order
-//     -- deterministic, no extra buffer.
+//     out[t, h] = sum_{j=0..k-1} w[t, j] * (dot_j + b2[e_j, h]) is summed in
+//     fixed j order (b2 only when given) -- deterministic, no extra buffer.
 //
 // Same function as ref_moe on the page "tpu_inference/kernels/fused_moe/v1/
 // kernel.py" (per token: x.[W_gate|W_up] -> silu(gate)*up -> .W2, weighted
@@ -229,7 +230,8 @@ __host__ __device__ inline SmemLayout smem_layout(bool one_token, int TK, int H,
 template <int kTokens>
 __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     small_t_kernel(const uint4 *__restrict__ hidden, const uint4 *__restrict__ w1,
-                   const uint4 *__restrict__ w2, const float *__restrict__ topk_w,
+                   const uint4 *__restrict__ w2, const float *__restrict__ b1,
+                   const float *__restrict__ b2, int act_kind, const float *__restrict__ topk_w,
                    const int32_t *__restrict__ ids, float *__restrict__ act,
                    float *__restrict__ out, int T, int k, int H, int I, int E, int rows_per_cta,
                    int nd_max, int w2_smem, int cache_act, uint32_t *status,
@@ -289,6 +291,12 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     const int p0 = L.dstart[d], np = L.dstart[d + 1] - p0;
     const uint4 *g = w1 + (static_cast<size_t>(L.dexp[d]) * 2 * I + i) * H8;
     const uint4 *u = g + static_cast<size_t>(I) * H8;
+    // the variant's bias of this row pair (0 without b1)
+    float bg = 0.f, bu = 0.f;
+    if (b1 != nullptr) {
+      bg = __ldg(b1 + static_cast<size_t>(L.dexp[d]) * 2 * I + i);
+      bu = __ldg(b1 + static_cast<size_t>(L.dexp[d]) * 2 * I + I + i);
+    }
     if (kTokens == 1) {
       // one token: its pairs on e (more than one only for repeated ids) share
       // the same dot products
@@ -316,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       ag = warp_sum(ag);
       au = warp_sum(au);
       if (lane == 0) {
-        const float a = silu_f(ag) * au;
+        const float a = b1 != nullptr ? gated_rt(act_kind, ag + bg, au + bu)
+                                      : gated_rt(act_kind, ag, au);
         for (int q = 0; q < np; ++q) act[static_cast<size_t>(L.plist[p0 + q]) * I + i] = a;
       }
     } else {
@@ -358,7 +367,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
             const float gs = warp_sum(ag[q]);
             const float us = warp_sum(au[q]);
             if (lane == 0)
-              act[static_cast<size_t>(L.plist[p0 + q0 + q]) * I + i] = silu_f(gs) * us;
+              act[static_cast<size_t>(L.plist[p0 + q0 + q]) * I + i] =
+                  b1 != nullptr ? gated_rt(act_kind, gs + bg, us + bu)
+                                : gated_rt(act_kind, gs, us);
           }
         }
       }
@@ -451,7 +462,11 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     float acc = 0.f;
     for (int j = 0; j < k; ++j) {
       const int pair = t * k + j;
-      if (L.pd[pair] >= 0) acc = fmaf(__ldg(topk_w + pair), sdots[r * TK + pair], acc);
+      if (L.pd[pair] >= 0) {
+        float y = sdots[r * TK + pair];
+        if (b2 != nullptr) y += __ldg(b2 + static_cast<size_t>(L.ids[pair]) * H + h0 + r);
+        acc = fmaf(__ldg(topk_w + pair), y, acc);
+      }
     }
     out[static_cast<size_t>(t) * H + h0 + r] = acc;
   }
@@ -506,6 +521,7 @@ size_t smem_budget(int dev, const void *kern) {
 bool small_t_supported(int H, int I) { return H <= kMaxH && I <= kMaxI; }
 
 cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
+                           const float *b1, const float *b2, int act_kind,
                            const float *topk_weights, const int32_t *topk_ids, float *act,
                            float *out, int64_t T, int H, int I, int E, int k, uint32_t *status,
                            unsigned long long *grid_sync, unsigned long long *arrivals,
@@ -565,7 +581,7 @@ cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uin
   e = cudaLaunchKernelEx(&lc, T == 1 ? small_t_kernel<1> : small_t_kernel<kMaxT>,
                          reinterpret_cast<const uint4 *>(hidden),
                          reinterpret_cast<const uint4 *>(w1), reinterpret_cast<const uint4 *>(w2),
-                         topk_weights, topk_ids, act, out, static_cast<int>(T), k, H, I, E,
+                         b1, b2, act_kind, topk_weights, topk_ids, act, out, static_cast<int>(T), k, H, I, E,
                          cfg.rows_per_cta, cfg.nd_max, cfg.w2_smem, cfg.cache_act, status,
                          grid_sync, target,
                          wait_limit_ns);

@@ -69,5 +69,18 @@ def make_inputs(T: int, H: int, I: int, E: int, seed: int = 0,
     return hidden, w1, w2, logits
 
 
+def make_biases(E: int, H: int, I: int, seed: int = 0, b1_scale: float = 0.1,
+                b2_scale: float = 0.005, device: str = "cpu"):
+    """Draw fp32 expert biases (b1 [E,2I], b2 [E,H]) for the variant forward
+    of the 0.13.2 TPU page, ``randn`` times a scale comparable to the
+    projections (b1) and to an expert's output (b2) of make_inputs."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    kw = dict(generator=g, device=device)
+    b1 = torch.randn(E, 2 * I, dtype=torch.float32, **kw) * b1_scale
+    b2 = torch.randn(E, H, dtype=torch.float32, **kw) * b2_scale
+    return b1, b2
+
+
 def make_shape_inputs(shape: MoEShape, seed: int = 0, device: str = "cpu"):
     return make_inputs(shape.T, shape.H, shape.I, shape.E, seed=seed, device=device)

@@ -84,6 +84,32 @@ def test_forward_argument_checks(kw, code):
     assert fwd(**kw) == code
 
 
+def fwd_ex(b1=NULL, b2=NULL, act=0, **kw):
+    a = dict(FWD_OK, **kw)
+    return L.moe_forward_ex(a["h"], a["w1"], a["w2"], b1, b2, act, a["w"], a["ids"], a["out"],
+                            a["T"], a["H"], a["I"], a["E"], a["k"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(act=3), moe.MOE_ERR_INVALID_ARG),         # unknown activation
+    (dict(act=-1), moe.MOE_ERR_INVALID_ARG),
+    (dict(b1=260), moe.MOE_ERR_INVALID_ARG),        # b1 not 16-byte aligned
+    (dict(b2=264, act=2), moe.MOE_ERR_INVALID_ARG),  # b2 not 16-byte aligned
+    (dict(act=1, H=200), moe.MOE_ERR_UNSUPPORTED),
+    (dict(act=2, h=NULL), moe.MOE_ERR_INVALID_ARG),
+    (dict(act=1, T=0, h=NULL, out=NULL), moe.MOE_OK),
+])
+def test_forward_ex_argument_checks(kw, code):
+    assert fwd_ex(**kw) == code
+
+
+def test_binding_rejects_unknown_activation():
+    import torch
+    t = torch.empty(0)
+    with pytest.raises(ValueError, match="act must be one of"):
+        moe.moe_forward(t, t, t, t, t, act="relu")
+
+
 def test_permute_argument_checks():
     assert L.moe_permute(NULL, 4, 2, 8, NULL, NULL, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_permute(1, 4, 0, 8, 1, 1, None) == moe.MOE_ERR_INVALID_ARG
@@ -107,3 +133,4 @@ def test_no_gpu_fails_loudly():
         pytest.skip("a GPU is present")
     assert L.moe_route(1, 4, 8, 2, 1, 1, 1, None) == moe.MOE_ERR_NO_DEVICE
     assert fwd() == moe.MOE_ERR_NO_DEVICE
+    assert fwd_ex(act=1, b1=256, b2=256) == moe.MOE_ERR_NO_DEVICE

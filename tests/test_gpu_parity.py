@@ -14,7 +14,7 @@ import torch
 
 import mixture_experts_expert_softmax_b200 as moe
 import oracle
-from moe_inputs import SHAPES, make_inputs, make_shape_inputs
+from moe_inputs import SHAPES, make_biases, make_inputs, make_shape_inputs
 from moe_testutil import assert_output_close, assert_weights_close
 
 pytestmark = pytest.mark.gpu
@@ -36,14 +36,16 @@ def gpu_route(logits_cpu, k, renorm=True):
     return ids.cpu().numpy(), w.cpu().numpy()
 
 
-def gpu_forward(hidden, w1, w2, w, ids):
+def gpu_forward(hidden, w1, w2, w, ids, act="silu", b1=None, b2=None):
     """Inputs may live on CPU or GPU; routing comes in as numpy."""
     dev = torch.device("cuda")
     # NaN-filled: every element of out must be written by the call
     out = torch.full((hidden.shape[0], hidden.shape[1]), float("nan"), device=dev)
     out = moe.moe_forward(hidden.to(dev), w1.to(dev), w2.to(dev),
                           torch.as_tensor(np.asarray(w, np.float32)).to(dev),
-                          torch.as_tensor(np.asarray(ids, np.int32)).to(dev), out=out)
+                          torch.as_tensor(np.asarray(ids, np.int32)).to(dev), out=out, act=act,
+                          b1=None if b1 is None else b1.to(dev),
+                          b2=None if b2 is None else b2.to(dev))
     torch.cuda.synchronize()
     return out.cpu().numpy()
 
@@ -274,6 +276,92 @@ def test_end_to_end_route_then_forward():
         assert_output_close(out.cpu().numpy(), ref, name)
 
 
+# ------------------------------------------------------------------ epilogue variants
+VARIANT_CASES = [
+    (64, 256, 128, 8, 2),      # tiny: one-kernel grouping, both GEMMs in one launch
+    (333, 384, 384, 16, 4),    # k > 2: separate GEMM launches, fp32 P, combine
+    (100, 256, 128, 128, 8),   # many experts below one tile
+]
+
+
+def _biases(which, E, H, I, seed):
+    b1, b2 = make_biases(E, H, I, seed=seed)
+    return (b1 if which in ("b1", "both") else None), (b2 if which in ("b2", "both") else None)
+
+
+@pytest.mark.parametrize("T,H,I,E,k", VARIANT_CASES)
+@pytest.mark.parametrize("act", ["silu", "gelu", "swigluoai"])
+@pytest.mark.parametrize("bias", ["none", "b1", "b2", "both"])
+def test_forward_variants(T, H, I, E, k, act, bias):
+    hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=T + 7)
+    b1, b2 = _biases(bias, E, H, I, seed=T)
+    ids, w = oracle.route(logits.numpy(), k, True)
+    ref = oracle.moe_token_loop(hidden, w1, w2, w, ids, act=act, b1=b1, b2=b2)
+    prev = moe.set_small_t_max(0)
+    try:
+        out = gpu_forward(hidden, w1, w2, w, ids, act, b1, b2)
+    finally:
+        moe.set_small_t_max(prev)
+    assert_output_close(out, ref, f"T={T} E={E} k={k} act={act} bias={bias}")
+    check_status_clean()
+
+
+@pytest.mark.parametrize("T", [1, 4])
+@pytest.mark.parametrize("act", ["silu", "gelu", "swigluoai"])
+def test_forward_variants_small_t(T, act):
+    H, I, E, k = 2048, 768, 128, 8
+    hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=50 + T)
+    b1, b2 = make_biases(E, H, I, seed=T)
+    ids, w = oracle.route(logits.numpy(), k, True)
+    ref = oracle.moe_token_loop(hidden, w1, w2, w, ids, act=act, b1=b1, b2=b2)
+    for bb1, bb2 in ((b1, b2), (None, None)):
+        r = ref if bb1 is not None else oracle.moe_token_loop(hidden, w1, w2, w, ids, act=act)
+        out = gpu_forward(hidden, w1, w2, w, ids, act, bb1, bb2)
+        assert_output_close(out, r, f"T={T} act={act} bias={bb1 is not None}")
+    check_status_clean()
+
+
+@pytest.mark.parametrize("small", [16, 0])
+def test_forward_swigluoai_clamps(small):
+    """Projections of a few units: many gate values above 7 and up values
+    beyond +-7, so both clips of swigluoai decide the result.  w2 is scaled
+    by 2^-7 (exact in bf16) so that the output, and with it the rounding of
+    the bf16 intermediate of the GEMM path (activations up to 56), stays at
+    the size the absolute tolerance was derived for."""
+    T, H, I, E, k = 12, 256, 128, 8, 2
+    hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=13, hidden_scale=12.0)
+    w2 = w2 * 2.0 ** -7
+    ids, w = oracle.route(logits.numpy(), k, True)
+    ref = oracle.moe_token_loop(hidden, w1, w2, w, ids, act="swigluoai")
+    g = hidden.double() @ w1[0, :I].double().T
+    assert (g > 7).float().mean() > 0.15  # the clip is really exercised
+    prev = moe.set_small_t_max(small)
+    try:
+        out = gpu_forward(hidden, w1, w2, w, ids, "swigluoai")
+    finally:
+        moe.set_small_t_max(prev)
+    assert_output_close(out, ref, f"small_t_max={small}")
+
+
+def test_forward_ex_default_equals_forward():
+    """moe_forward_ex with silu and no biases is moe_forward, bit for bit."""
+    T, H, I, E, k = 300, 512, 256, 8, 2
+    hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=17)
+    ids, w = oracle.route(logits.numpy(), k, True)
+    dev = torch.device("cuda")
+    args = [hidden.to(dev), w1.to(dev), w2.to(dev),
+            torch.as_tensor(w.astype(np.float32)).to(dev), torch.as_tensor(ids).to(dev)]
+    a = moe.moe_forward(*args)
+    b = torch.empty_like(a)
+    rc = moe._lib.moe_forward_ex(args[0].data_ptr(), args[1].data_ptr(), args[2].data_ptr(),
+                                 None, None, moe.MOE_ACT_SILU, args[3].data_ptr(),
+                                 args[4].data_ptr(), b.data_ptr(), T, H, I, E, k,
+                                 torch.cuda.current_stream().cuda_stream)
+    assert rc == moe.MOE_OK
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
 # ------------------------------------------------------------------ full-size workloads
 def _sample_rows(T, n, seed):
     rng = np.random.default_rng(seed)
@@ -299,6 +387,26 @@ def test_forward_full_size_workloads(name):
     assert_output_close(out.cpu().numpy()[rows], ref, name)
     check_status_clean()
     # properties that hold at any size: every row written and finite
+    assert torch.isfinite(out).all()
+
+
+@pytest.mark.parametrize("name,act", [("decode", "gelu"), ("prefill_8e", "swigluoai"),
+                                      ("prefill_thin", "gelu"), ("prefill_big", "swigluoai")])
+def test_forward_full_size_variants(name, act):
+    """The variant epilogues in the launch configuration of each workload
+    (prefill_big: GEMM1 and GEMM2 as two launches), on sampled tokens."""
+    s = SHAPES[name]
+    hidden, w1, w2, logits = make_shape_inputs(s, device="cuda")
+    b1, b2 = make_biases(s.E, s.H, s.I, seed=2, device="cuda")
+    ids_r, w_r = oracle.route(logits.cpu().numpy(), s.k, True)
+    out = moe.moe_forward(hidden, w1, w2, torch.as_tensor(w_r.astype(np.float32)).cuda(),
+                          torch.as_tensor(ids_r).cuda(), act=act, b1=b1, b2=b2)
+    torch.cuda.synchronize()
+    rows = np.arange(s.T) if s.T <= 64 else _sample_rows(s.T, 10, 3)
+    ref = oracle.moe_token_loop(hidden.cpu(), w1.cpu(), w2.cpu(), w_r, ids_r, rows=rows, act=act,
+                                b1=b1.cpu(), b2=b2.cpu())
+    assert_output_close(out.cpu().numpy()[rows], ref, f"{name} {act}")
+    check_status_clean()
     assert torch.isfinite(out).all()
 
 
