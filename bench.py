@@ -1,14 +1,15 @@
 """Benchmark of the fused MoE forward on B200 (one JSON line on stdout).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload prefill_8e] [--no-shapes]
+                    [--workload prefill_8e] [--shapes workloads|table|none]
 
 A step is one pass of the whole hot path over one batch: moe_route (softmax,
 top-k, renormalisation) then moe_forward (permutation, GEMM1+SwiGLU, GEMM2,
 combine -- or the small-T GEMV path) on synthetic inputs with the shapes and
 distributions of the atrex-bench #009 "fused_moe" workload.  The headline
 workload is "prefill, few large experts" (T=1979, H=2048, I=2048, E=8,
-top-k 2); the other shapes are reported under "per_shape".
+top-k 2); the other workloads are reported under "per_shape" (--shapes table:
+every row of the atrex-bench #009 shapes table, plus a two-token decode).
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
 device synchronise on both sides; each step is timed with CUDA events on the
@@ -40,7 +41,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from moe_inputs import SHAPES, MoEShape, make_shape_inputs  # noqa: E402
+from moe_inputs import (SHAPES, TABLE_SHAPES, MoEShape, make_shape_inputs,  # noqa: E402
+                        PAGE_T_PROD_US as TABLE_T_PROD_US)
 
 METRIC = "fused-MoE µs/call, TFLOP/s and % of roofline per shape; T=1 decode HBM GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -294,8 +296,10 @@ def run_ours(args, ws, rank, local):
     d2h = h_out.numel() * 4
 
     per_shape = {}
-    if not args.no_shapes:
-        per_shape = measure_shapes(moe, dev, peaks, flush, stream)
+    if args.shapes == "workloads":
+        per_shape = measure_shapes(moe, dev, peaks, flush, stream, SHAPES, PAGE_T_PROD_US)
+    elif args.shapes == "table":
+        per_shape = measure_shapes(moe, dev, peaks, flush, stream, TABLE_SHAPES, TABLE_T_PROD_US)
 
     line = {
         "metric": METRIC,
@@ -337,9 +341,9 @@ def run_ours(args, ws, rank, local):
     return line
 
 
-def measure_shapes(moe, dev, peaks, flush, stream, K=10, W=3):
+def measure_shapes(moe, dev, peaks, flush, stream, shapes, page_us, K=10, W=3):
     res = {}
-    for name, s in SHAPES.items():
+    for name, s in shapes.items():
         hidden, w1, w2, logits = make_shape_inputs(s, seed=0, device=str(dev))
         ids, wts = moe.moe_route(logits, s.k, True)
         out = torch.empty(s.T, s.H, dtype=torch.float32, device=dev)
@@ -361,8 +365,8 @@ def measure_shapes(moe, dev, peaks, flush, stream, K=10, W=3):
                      "hbm_gbs": round(algorithmic_bytes(s, n_active) / (us * 1e-6) / 1e9, 1),
                      "roofline_bound": bound, "roofline_us": round(t_roof, 2),
                      "roofline_frac": round(t_roof / us, 4)}
-        if name in PAGE_T_PROD_US:
-            res[name]["page_t_prod_us"] = PAGE_T_PROD_US[name]
+        if name in page_us:
+            res[name]["page_t_prod_us"] = page_us[name]
         del hidden, w1, w2, logits, ids, wts, out
         torch.cuda.empty_cache()
     return res
@@ -454,12 +458,17 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(SHAPES), default="prefill_8e")
-    ap.add_argument("--no-shapes", action="store_true", help="skip the per-shape table")
+    ap.add_argument("--shapes", choices=["workloads", "table", "none"], default="workloads",
+                    help="per-shape table: the five workloads, every row of the page's "
+                         "shapes table, or none")
+    ap.add_argument("--no-shapes", action="store_true", help="same as --shapes none")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.no_shapes:
+        args.shapes = "none"
     ws, rank, local = dist_env()
     if args.impl == "reference":
         line = run_reference(args, ws, rank)

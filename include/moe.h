@@ -207,7 +207,8 @@ int moe_get_device_status(void *stream, uint32_t *status);
 /*
  * Tuning and debug switches (host-side, process-wide):
  *   moe_set_small_t_max(n)  -- moe_forward uses the GEMV path when T <= n
- *                              (default 16, also read from MOE_SMALL_T_MAX);
+ *                              (default 8, at most 16, also read from
+ *                              MOE_SMALL_T_MAX);
  *                              n = 0 forces the grouped-GEMM path.
  *   moe_set_sync_each_stage(on) -- synchronise and check for errors after
  *                              every launch (also MOE_SYNC_EACH_STAGE=1);

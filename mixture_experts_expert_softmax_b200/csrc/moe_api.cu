@@ -65,7 +65,10 @@ cudaEvent_t get_event() {
 int small_t_max() {
   if (g_small_t_max < 0) {
     const char *v = std::getenv("MOE_SMALL_T_MAX");
-    g_small_t_max = v ? std::max(0, std::atoi(v)) : 16;
+    // up to 8 tokens the GEMV path streams the chosen experts' weights
+    // faster than the grouped GEMMs; at 16 the GEMMs win (B200 timings of
+    // the E = 8 / top-2 and E = 128 / top-8 shapes)
+    g_small_t_max = v ? std::max(0, std::atoi(v)) : 8;
     if (g_small_t_max > 16) g_small_t_max = 16;
   }
   return g_small_t_max;

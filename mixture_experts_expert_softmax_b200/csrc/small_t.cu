@@ -50,6 +50,7 @@ constexpr size_t kActCacheMax = 48 * 1024;
 constexpr uint64_t kW2WaitNs = 2000000000ull;
 constexpr int kMaxH = 4096;
 constexpr int kMaxI = 12288;
+constexpr int kMaxSlots = 16;   // w2 ring slots (one chosen expert's rows each)
 
 struct Lists {
   uint32_t bitmap[32];
@@ -204,21 +205,80 @@ __device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long
   return v;
 }
 
-// Dynamic shared memory of a CTA: the single token's vector in bf16 [H]
-// (one-token kernel only); the CTA's w2 rows of every chosen expert in bf16
-// [nd_max][rows_per_cta][I] when they fit (w2_smem); act in fp32 [T*k][I]
-// when it fits (phase 2); the dot products [rows_per_cta][T*k].
+// Phase 1 for a group of NQ tokens (at most NQ live: nq) routed to one
+// expert: the warp streams the (gate row g, up row u) pair once, dots both
+// with the NQ token vectors (staged in shared memory, sx), and lane 0
+// stores the activations of the group's pairs.  NQ is a template constant so that the accumulators stay
+// in registers and no instruction is spent on token slots that do not
+// exist; nq < NQ only wastes the predicated slots of the last group.
+template <int NQ, int kU>
+__device__ __forceinline__ void phase1_group(const uint4 *__restrict__ g,
+                                             const uint4 *__restrict__ u, const uint4 *sx,
+                                             const int *plist,
+                                             int nq, int k, int H8, int I, int i, float bg,
+                                             float bu, bool bias, int act_kind,
+                                             float *__restrict__ act) {
+  const int lane = threadIdx.x & 31;
+  int xo[NQ];  // offsets of the token vectors (T <= 16 tokens, H8 <= 512 chunks)
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) xo[q] = plist[q < nq ? q : 0] / k * H8;
+  float ag[NQ], au[NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) ag[q] = au[q] = 0.f;
+  for (int base = 0; base < H8; base += 32 * kU) {
+    uint4 gv[kU], uv[kU];
+#pragma unroll
+    for (int j = 0; j < kU; ++j) {
+      const int c = base + lane + 32 * j;
+      if (c < H8) {
+        gv[j] = __ldcs(g + c);
+        uv[j] = __ldcs(u + c);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kU; ++j) {
+      const int c = base + lane + 32 * j;
+      if (c < H8) {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          if (q < nq) {
+            const uint4 xv = sx[xo[q] + c];
+            ag[q] = fma8_bf16(gv[j], xv, ag[q]);
+            au[q] = fma8_bf16(uv[j], xv, au[q]);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    if (q < nq) {
+      const float gs = warp_sum(ag[q]);
+      const float us = warp_sum(au[q]);
+      if (lane == 0)
+        act[static_cast<size_t>(plist[q]) * I + i] =
+            bias ? gated_rt(act_kind, gs + bg, us + bu) : gated_rt(act_kind, gs, us);
+    }
+  }
+}
+
+// Dynamic shared memory of a CTA: the token vectors in bf16 [T][H]; a ring of `slots` buffers, each holding this
+// CTA's w2 rows of one chosen expert in bf16 [rows_per_cta][I] (no ring when
+// one expert's rows do not fit: phase 2 then reads w2 through L2); act in
+// fp32 [T*k][I] when it fits; the dot products [rows_per_cta][T*k].
 struct SmemLayout {
   size_t w2_off, act_off, dots_off, total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(bool one_token, int TK, int H, int I,
-                                                  int rows_per_cta, int nd_max, int w2_smem,
-                                                  int cache_act) {
+__host__ __device__ inline size_t w2_slot_bytes(int rows_per_cta, int I) {
+  return (static_cast<size_t>(rows_per_cta) * I * 2 + 127) & ~static_cast<size_t>(127);
+}
+
+__host__ __device__ inline SmemLayout smem_layout(int T, int TK, int H, int I,
+                                                  int rows_per_cta, int slots, int cache_act) {
   SmemLayout s;
-  s.w2_off = one_token ? static_cast<size_t>(H) * 2 : 0;
-  s.act_off =
-      s.w2_off + (w2_smem ? static_cast<size_t>(nd_max) * rows_per_cta * I * 2 : 0);
+  s.w2_off = static_cast<size_t>(T) * H * 2;
+  s.act_off = s.w2_off + static_cast<size_t>(slots) * w2_slot_bytes(rows_per_cta, I);
   s.dots_off = s.act_off + (cache_act ? static_cast<size_t>(TK) * I * sizeof(float) : 0);
   s.total = s.dots_off + static_cast<size_t>(rows_per_cta) * TK * sizeof(float);
   return s;
@@ -234,19 +294,20 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
                    const float *__restrict__ b2, int act_kind, const float *__restrict__ topk_w,
                    const int32_t *__restrict__ ids, float *__restrict__ act,
                    float *__restrict__ out, int T, int k, int H, int I, int E, int rows_per_cta,
-                   int nd_max, int w2_smem, int cache_act, uint32_t *status,
+                   int slots, int cache_act, uint32_t *status,
                    unsigned long long *grid_sync,
                    unsigned long long sync_target, uint64_t limit) {
   constexpr int kU1 = kTokens == 1 ? 8 : 4;  // phase 1: chunks per lane and row in flight
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ Lists L;
-  __shared__ int s_abort;
-  __shared__ uint64_t w2_full;  // the CTA's w2 rows have landed (w2_smem)
+  __shared__ volatile int s_abort;
+  __shared__ uint64_t w2_full[kMaxSlots];   // a slot's rows have landed
+  __shared__ uint64_t w2_empty[kMaxSlots];  // every compute warp is done with a slot
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int TK = T * k;
   const int H8 = H / 8, I8 = I / 8;
-  const SmemLayout lay =
-      smem_layout(kTokens == 1, TK, H, I, rows_per_cta, nd_max, w2_smem, cache_act);
+  const SmemLayout lay = smem_layout(T, TK, H, I, rows_per_cta, slots, cache_act);
+  const size_t slot_stride = w2_slot_bytes(rows_per_cta, I);
   uint8_t *sx = smem;  // the token's vector (one-token kernel)
   uint8_t *sw2 = smem + lay.w2_off;
   float *sact = reinterpret_cast<float *>(smem + lay.act_off);
@@ -257,31 +318,35 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   if (warp == 0) build_lists(L, ids, TK, E);
   if (threadIdx.x == 32) {
     s_abort = 0;
-    mbar_init(&w2_full, 1);
+    for (int q = 0; q < slots; ++q) {
+      mbar_init(&w2_full[q], 1);
+      mbar_init(&w2_empty[q], kWarps);
+    }
     fence_mbar_init();
   }
-  if (kTokens == 1)
-    for (int c = threadIdx.x; c < H8; c += kThreads)
-      reinterpret_cast<uint4 *>(sx)[c] = __ldg(hidden + c);
+  for (int c = threadIdx.x; c < T * H8; c += kThreads)
+    reinterpret_cast<uint4 *>(sx)[c] = __ldg(hidden + c);
+  const uint4 *sx4 = reinterpret_cast<const uint4 *>(sx);
   __syncthreads();
   const int nd = L.n_distinct;
   const int nw = gridDim.x * kWarps;
   const int n1 = nd * I;
-  if (warp == kCopyWarp) {
-    // this CTA's w2 rows of every chosen expert, for phase 2
-    if (lane == 0) {
-      const uint32_t bytes = static_cast<uint32_t>(nrows) * I * 2;
-      if (w2_smem) {
-        // nd <= nd_max: the host sized the slots for the distinct experts a
-        // call can have
-        mbar_arrive_expect_tx(&w2_full, bytes * static_cast<uint32_t>(nd));
-        for (int d = 0; d < nd && nrows > 0; ++d)
-          bulk_load(sw2 + static_cast<size_t>(d) * rows_per_cta * I * 2,
-                    w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * I8, bytes, &w2_full);
-      } else {
-        for (int d = 0; d < nd && nrows > 0; ++d)
-          bulk_prefetch_l2(w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * I8, bytes);
+  // bytes of one expert's rows of this CTA (nrows may be 0 for the last CTAs)
+  const uint32_t w2_bytes = static_cast<uint32_t>(nrows) * I * 2;
+  const bool ring = slots > 0 && nrows > 0;
+  if (warp == kCopyWarp && lane == 0 && nrows > 0) {
+    // the first experts' w2 rows, for phase 2, stream in alongside w1; the
+    // rest follow in phase 2 as slots free up.  Without a ring, ask L2 to
+    // prefetch them.
+    if (ring) {
+      for (int d = 0; d < nd && d < slots; ++d) {
+        mbar_arrive_expect_tx(&w2_full[d], w2_bytes);
+        bulk_load(sw2 + d * slot_stride, w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * I8,
+                  w2_bytes, &w2_full[d]);
       }
+    } else {
+      for (int d = 0; d < nd; ++d)
+        bulk_prefetch_l2(w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * I8, w2_bytes);
     }
   }
 
@@ -329,49 +394,16 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
         for (int q = 0; q < np; ++q) act[static_cast<size_t>(L.plist[p0 + q]) * I + i] = a;
       }
     } else {
-      // the tokens routed to e, kMaxT accumulator pairs at a time
-      for (int q0 = 0; q0 < np; q0 += kMaxT) {
-        const int nq = min(kMaxT, np - q0);
-        float ag[kMaxT], au[kMaxT];
-#pragma unroll
-        for (int q = 0; q < kMaxT; ++q) ag[q] = au[q] = 0.f;
-        for (int base = 0; base < H8; base += 32 * kU1) {
-          uint4 gv[kU1], uv[kU1];
-#pragma unroll
-          for (int j = 0; j < kU1; ++j) {
-            const int c = base + lane + 32 * j;
-            if (c < H8) {
-              gv[j] = __ldcs(g + c);
-              uv[j] = __ldcs(u + c);
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < kU1; ++j) {
-            const int c = base + lane + 32 * j;
-            if (c < H8) {
-#pragma unroll
-              for (int q = 0; q < kMaxT; ++q) {
-                if (q < nq) {
-                  const int t = L.plist[p0 + q0 + q] / k;
-                  const uint4 xv = __ldg(hidden + static_cast<size_t>(t) * H8 + c);
-                  ag[q] = fma8_bf16(gv[j], xv, ag[q]);
-                  au[q] = fma8_bf16(uv[j], xv, au[q]);
-                }
-              }
-            }
-          }
-        }
-#pragma unroll
-        for (int q = 0; q < kMaxT; ++q) {
-          if (q < nq) {
-            const float gs = warp_sum(ag[q]);
-            const float us = warp_sum(au[q]);
-            if (lane == 0)
-              act[static_cast<size_t>(L.plist[p0 + q0 + q]) * I + i] =
-                  b1 != nullptr ? gated_rt(act_kind, gs + bg, us + bu)
-                                : gated_rt(act_kind, gs, us);
-          }
-        }
+      // the tokens routed to e, in groups of at most 4 (the row pair is
+      // re-read from L2 for each further group)
+      for (int q0 = 0; q0 < np; q0 += 4) {
+        const int nq = min(4, np - q0);
+        const int *pl = L.plist + p0 + q0;
+        const bool bias = b1 != nullptr;
+        if (nq == 1)
+          phase1_group<1, 8>(g, u, sx4, pl, nq, k, H8, I, i, bg, bu, bias, act_kind, act);
+        else
+          phase1_group<4, 4>(g, u, sx4, pl, nq, k, H8, I, i, bg, bu, bias, act_kind, act);
       }
     }
   }
@@ -394,16 +426,13 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     }
     __threadfence();
   }
-  // the CTA's w2 rows: one thread waits (bounded) so that the decision to
-  // go on is the same for every thread; then each thread observes the
-  // completed phase itself, which orders the copied data before its reads
-  if (w2_smem && threadIdx.x == 0 && !s_abort && !mbar_wait(&w2_full, 0, kW2WaitNs)) {
-    s_abort = 1;
-    atomicOr(status, kStatusTimeout);
-  }
   __syncthreads();
-  if (s_abort) return;
-  if (w2_smem) mbar_wait(&w2_full, 0, kW2WaitNs);
+  if (s_abort) {
+    // let the bulk copies already issued land before the CTA exits
+    if (warp == kCopyWarp && lane == 0 && ring)
+      for (int d = 0; d < nd && d < slots; ++d) mbar_wait(&w2_full[d], 0, kW2WaitNs);
+    return;
+  }
 
   // ------------------------------------------------------------ phase 2
   const float4 *act4 = reinterpret_cast<const float4 *>(act);
@@ -415,47 +444,88 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     __syncthreads();
     act4 = d4;
   }
-  // items (distinct expert d, its pair q, group of kR2 local rows): the act
-  // chunks of the pair are loaded once and shared by kR2 independent dot
-  // products with w2[e][h0 + r, :] (on chip), one per row of the group
   const int rgroups = (nrows + kR2 - 1) / kR2;
-  const int n2 = L.dstart[nd] * rgroups;
-  for (int item = warp; item < n2 && warp < kWarps; item += kWarps) {
-    const int pq = item / rgroups, rg = item - pq * rgroups;  // pq: position in plist
-    const int pair = L.plist[pq];
-    const int d = L.pd[pair];
-    const int r0 = rg * kR2;
-    const float4 *a = act4 + static_cast<size_t>(pair) * (I / 4);
-    unsigned long long v[kR2];  // two fp32 partial sums each
+  if (warp == kCopyWarp) {
+    // refill the ring: expert d goes into slot d % slots once every compute
+    // warp has finished with expert d - slots
+    if (lane == 0 && ring) {
+      int issued = min(nd, slots);
+      for (int d = slots; d < nd; ++d) {
+        const int q = d % slots;
+        if (!mbar_wait(&w2_empty[q], ((d / slots) - 1) & 1, kW2WaitNs, &s_abort)) {
+          s_abort = 1;
+          atomicOr(status, kStatusTimeout);
+          break;
+        }
+        mbar_arrive_expect_tx(&w2_full[q], w2_bytes);
+        bulk_load(sw2 + q * slot_stride, w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * I8,
+                  w2_bytes, &w2_full[q]);
+        issued = d + 1;
+      }
+      if (s_abort) {
+        // the last load of each slot must land before the CTA exits
+        for (int d = max(0, issued - slots); d < issued; ++d)
+          mbar_wait(&w2_full[d % slots], (d / slots) & 1, kW2WaitNs);
+      }
+    }
+  } else if (rgroups > 0) {
+    // experts in order; the items (pair of the expert, group of kR2 local
+    // rows) are dealt round-robin over the compute warps, continuing from
+    // one expert to the next.  The act chunks of a pair are loaded once and
+    // shared by kR2 independent dot products with w2[e][h0 + r, :].
+    int before = 0;  // items of the experts before d
+    for (int d = 0; d < nd; ++d) {
+      const int q = ring ? d % slots : 0;
+      if (ring && !mbar_wait(&w2_full[q], (d / slots) & 1, kW2WaitNs, &s_abort)) {
+        s_abort = 1;
+        atomicOr(status, kStatusTimeout);
+        break;
+      }
+      const uint4 *ws = reinterpret_cast<const uint4 *>(sw2 + q * slot_stride);
+      const uint4 *wg = w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * I8;
+      const int p0 = L.dstart[d];
+      const int n_items = (L.dstart[d + 1] - p0) * rgroups;
+      int it = warp - before % kWarps;
+      if (it < 0) it += kWarps;
+      for (; it < n_items; it += kWarps) {
+        const int pq = p0 + it / rgroups, rg = it % rgroups;  // pq: position in plist
+        const int pair = L.plist[pq];
+        const int r0 = rg * kR2;
+        const float4 *a = act4 + static_cast<size_t>(pair) * (I / 4);
+        unsigned long long v[kR2];  // two fp32 partial sums each
 #pragma unroll
-    for (int rr = 0; rr < kR2; ++rr) v[rr] = 0ull;
-    for (int base = 0; base < I8; base += 32 * kU2) {
+        for (int rr = 0; rr < kR2; ++rr) v[rr] = 0ull;
+        for (int base = 0; base < I8; base += 32 * kU2) {
 #pragma unroll
-      for (int j = 0; j < kU2; ++j) {
-        const int c = base + lane + 32 * j;
-        if (c < I8) {
-          const float4 a0 = cache_act ? a[2 * c] : __ldcg(a + 2 * c);
-          const float4 a1 = cache_act ? a[2 * c + 1] : __ldcg(a + 2 * c + 1);
+          for (int j = 0; j < kU2; ++j) {
+            const int c = base + lane + 32 * j;
+            if (c < I8) {
+              const float4 a0 = cache_act ? a[2 * c] : __ldcg(a + 2 * c);
+              const float4 a1 = cache_act ? a[2 * c + 1] : __ldcg(a + 2 * c + 1);
+              uint4 wv[kR2];
 #pragma unroll
-          for (int rr = 0; rr < kR2; ++rr) {
-            const int r = r0 + rr;
-            if (r < nrows) {
-              const uint4 wv =
-                  w2_smem ? reinterpret_cast<const uint4 *>(sw2)[(d * rows_per_cta + r) * I8 + c]
-                          : __ldg(w2 + (static_cast<size_t>(L.dexp[d]) * H + h0 + r) * I8 + c);
-              fma8_f32x2(wv, a0, a1, v[rr]);
+              for (int rr = 0; rr < kR2; ++rr)
+                if (r0 + rr < nrows)
+                  wv[rr] = ring ? ws[(r0 + rr) * I8 + c] : __ldg(wg + (r0 + rr) * I8 + c);
+#pragma unroll
+              for (int rr = 0; rr < kR2; ++rr)
+                if (r0 + rr < nrows) fma8_f32x2(wv[rr], a0, a1, v[rr]);
             }
           }
         }
-      }
-    }
 #pragma unroll
-    for (int rr = 0; rr < kR2; ++rr) {
-      const float sv = warp_sum(sum_f32x2(v[rr]));
-      if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
+        for (int rr = 0; rr < kR2; ++rr) {
+          const float sv = warp_sum(sum_f32x2(v[rr]));
+          if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
+        }
+      }
+      before += n_items;
+      __syncwarp();
+      if (ring && lane == 0) mbar_arrive(&w2_empty[q]);
     }
   }
   __syncthreads();
+  if (s_abort) return;
   // out[t, h] = sum over j in ascending order of w[t, j] * dot(t*k + j)
   for (int x = threadIdx.x; x < T * nrows; x += kThreads) {
     const int t = x / nrows, r = x - t * nrows;
@@ -478,25 +548,34 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
 }
 
 struct SmallTConfig {
-  int rows_per_cta, nd_max, w2_smem, cache_act;
+  int rows_per_cta, slots, cache_act;
   size_t smem;
 };
 
-// What goes into `budget` bytes of dynamic shared memory, in order of gain:
-// the CTA's w2 rows, then the act cache.
+// What goes into `budget` bytes of dynamic shared memory: as many w2 ring
+// slots as there can be distinct experts (at most kMaxSlots), and the act
+// cache when it fits beside them -- unless it would leave fewer than two
+// slots (no overlap of copies and dot products) where dropping it gives more.
 SmallTConfig small_t_config(int T, int TK, int H, int I, int E, int grid, size_t budget) {
   SmallTConfig c;
   c.rows_per_cta = (H + grid - 1) / grid;
-  c.nd_max = std::min(TK, E);
-  c.w2_smem = 1;
-  c.cache_act = 1;
-  auto size = [&] {
-    return smem_layout(T == 1, TK, H, I, c.rows_per_cta, c.nd_max, c.w2_smem, c.cache_act).total;
+  const int want = std::min(std::min(TK, E), kMaxSlots);
+  auto size = [&](int slots, int cache) {
+    return smem_layout(T, TK, H, I, c.rows_per_cta, slots, cache).total;
   };
-  if (static_cast<size_t>(TK) * I * sizeof(float) > kActCacheMax || size() > budget)
+  auto fit = [&](int cache) {
+    int n = want;
+    while (n > 0 && size(n, cache) > budget) --n;
+    return n;
+  };
+  c.cache_act = static_cast<size_t>(TK) * I * sizeof(float) <= kActCacheMax ? 1 : 0;
+  c.slots = fit(c.cache_act);
+  if (c.cache_act && c.slots < std::min(want, 2) && fit(0) > c.slots) {
     c.cache_act = 0;
-  if (size() > budget) c.w2_smem = 0;
-  c.smem = size();
+    c.slots = fit(0);
+  }
+  if (c.cache_act && size(c.slots, 1) > budget) c.cache_act = 0;
+  c.smem = size(c.slots, c.cache_act);
   return c;
 }
 
@@ -582,7 +661,7 @@ cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uin
                          reinterpret_cast<const uint4 *>(hidden),
                          reinterpret_cast<const uint4 *>(w1), reinterpret_cast<const uint4 *>(w2),
                          b1, b2, act_kind, topk_weights, topk_ids, act, out, static_cast<int>(T), k, H, I, E,
-                         cfg.rows_per_cta, cfg.nd_max, cfg.w2_smem, cfg.cache_act, status,
+                         cfg.rows_per_cta, cfg.slots, cfg.cache_act, status,
                          grid_sync, target,
                          wait_limit_ns);
   if (e == cudaSuccess) *arrivals = target;

@@ -55,6 +55,47 @@ SHAPES = {
 }
 
 
+# The "Shapes" table of atrex-bench #009: (row, T, H, I, E, top-k, T_Prod in
+# microseconds of the production op on the page's "XPU-A" hardware, context
+# only).  Rows 4, 8, 19 and 22 are four of the workloads above.
+PAGE_TABLE = (
+    (0, 135, 2048, 2048, 8, 2, 232.70),
+    (1, 277, 2048, 2048, 8, 2, 249.80),
+    (2, 668, 2048, 2048, 8, 2, 477.10),
+    (3, 1023, 2048, 2048, 8, 2, 539.00),
+    (4, 1979, 2048, 2048, 8, 2, 772.50),
+    (5, 4195, 2048, 2048, 8, 2, 1600.0),
+    (6, 7689, 2048, 2048, 8, 2, 2680.0),
+    (7, 15809, 2048, 2048, 8, 2, 5370.0),
+    (8, 1, 2048, 768, 128, 8, 116.90),
+    (9, 2400, 2048, 768, 128, 8, 2160.0),
+    (10, 4195, 2048, 768, 128, 8, 2980.0),
+    (11, 8192, 2048, 768, 128, 8, 4990.0),
+    (12, 15809, 2048, 768, 128, 8, 9090.0),
+    (13, 25632, 2048, 768, 128, 8, 14480.0),
+    (14, 45936, 2048, 768, 128, 8, 25710.0),
+    (15, 520, 4096, 384, 128, 8, 595.80),
+    (16, 1019, 4096, 384, 128, 8, 882.90),
+    (17, 2044, 4096, 384, 128, 8, 1610.0),
+    (18, 3936, 4096, 384, 128, 8, 2800.0),
+    (19, 8192, 4096, 384, 128, 8, 5690.0),
+    (20, 4098, 4096, 4096, 8, 2, 5330.0),
+    (21, 8179, 4096, 4096, 8, 2, 10100.0),
+    (22, 15381, 4096, 4096, 8, 2, 18640.0),
+)
+
+# Every row of the table as a shape, plus a two-token decode (the batch of
+# two rows that the Rust page's decode kernels process).
+TABLE_SHAPES = {
+    f"row{r:02d}": MoEShape(f"atrex-bench #009 shapes row {r}: T={T} H={H} I={I} E={E} k={k}",
+                            T, H, I, E, k)
+    for r, T, H, I, E, k, _ in PAGE_TABLE
+}
+TABLE_SHAPES["decode_t2"] = MoEShape("decode, two tokens T=2 H=2048 I=768 E=128 k=8",
+                                     2, 2048, 768, 128, 8)
+PAGE_T_PROD_US = {f"row{r:02d}": t for r, *_, t in PAGE_TABLE}
+
+
 def make_inputs(T: int, H: int, I: int, E: int, seed: int = 0,
                 hidden_scale: float = 0.1, device: str = "cpu"):
     """Draw (hidden [T,H] bf16, w1 [E,2I,H] bf16, w2 [E,H,I] bf16,

@@ -14,7 +14,7 @@ import torch
 
 import mixture_experts_expert_softmax_b200 as moe
 import oracle
-from moe_inputs import SHAPES, make_biases, make_inputs, make_shape_inputs
+from moe_inputs import SHAPES, TABLE_SHAPES, make_biases, make_inputs, make_shape_inputs
 from moe_testutil import assert_output_close, assert_weights_close
 
 pytestmark = pytest.mark.gpu
@@ -25,9 +25,11 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     torch.cuda.set_device(0)
-    moe.set_small_t_max(16)
+    # every batch of up to 16 tokens takes the small-T path unless a test
+    # forces the GEMM path (the default threshold is lower)
+    prev = moe.set_small_t_max(16)
     yield
-    moe.set_small_t_max(16)
+    moe.set_small_t_max(prev)
 
 
 def gpu_route(logits_cpu, k, renorm=True):
@@ -387,6 +389,30 @@ def test_forward_full_size_workloads(name):
     assert_output_close(out.cpu().numpy()[rows], ref, name)
     check_status_clean()
     # properties that hold at any size: every row written and finite
+    assert torch.isfinite(out).all()
+
+
+TABLE_ONLY = [n for n, s in TABLE_SHAPES.items()
+              if (s.T, s.H, s.I, s.E, s.k) not in
+              {(w.T, w.H, w.I, w.E, w.k) for w in SHAPES.values()}]
+
+
+@pytest.mark.parametrize("name", TABLE_ONLY)
+def test_forward_table_rows(name):
+    """The other rows of the page's shapes table (and a two-token decode) at
+    full size: routing bit-exact, sampled tokens against the oracle."""
+    s = TABLE_SHAPES[name]
+    hidden, w1, w2, logits = make_shape_inputs(s, seed=1, device="cuda")
+    ids_r, w_r = oracle.route(logits.cpu().numpy(), s.k, True)
+    ids_g, w_g = moe.moe_route(logits, s.k, True)
+    out = moe.moe_forward(hidden, w1, w2, torch.as_tensor(w_r.astype(np.float32)).cuda(),
+                          torch.as_tensor(ids_r).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(ids_g.cpu().numpy(), ids_r)
+    rows = np.arange(s.T) if s.T <= 16 else _sample_rows(s.T, 6, 4)
+    ref = oracle.moe_token_loop(hidden.cpu(), w1.cpu(), w2.cpu(), w_r, ids_r, rows=rows)
+    assert_output_close(out.cpu().numpy()[rows], ref, name)
+    check_status_clean()
     assert torch.isfinite(out).all()
 
 
