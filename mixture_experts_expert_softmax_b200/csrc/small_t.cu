@@ -262,6 +262,43 @@ __device__ __forceinline__ void phase1_group(const uint4 *__restrict__ g,
   }
 }
 
+// Phase 2 item: the kR2 dot products of w2 rows r0.. r0+kR2-1 of this CTA
+// (ws: in shared memory, else wg: through L2) with act of one pair; the act
+// chunks are loaded once for the kR2 independent sums.  Lane 0 writes
+// sdots[r][pair].
+__device__ __forceinline__ void phase2_item(const uint4 *ws, const uint4 *__restrict__ wg,
+                                            const float4 *a4, int cache_act, int pair, int r0,
+                                            int nrows, int I, int TK, float *sdots) {
+  const int lane = threadIdx.x & 31;
+  const int I8 = I / 8;
+  const float4 *a = a4 + static_cast<size_t>(pair) * (I / 4);
+  unsigned long long v[kR2];  // two fp32 partial sums each
+#pragma unroll
+  for (int rr = 0; rr < kR2; ++rr) v[rr] = 0ull;
+  for (int base = 0; base < I8; base += 32 * kU2) {
+#pragma unroll
+    for (int j = 0; j < kU2; ++j) {
+      const int c = base + lane + 32 * j;
+      if (c < I8) {
+        const float4 a0 = cache_act ? a[2 * c] : __ldcg(a + 2 * c);
+        const float4 a1 = cache_act ? a[2 * c + 1] : __ldcg(a + 2 * c + 1);
+#pragma unroll
+        for (int rr = 0; rr < kR2; ++rr) {
+          if (r0 + rr < nrows) {
+            const uint4 wv = ws != nullptr ? ws[(r0 + rr) * I8 + c] : __ldg(wg + (r0 + rr) * I8 + c);
+            fma8_f32x2(wv, a0, a1, v[rr]);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int rr = 0; rr < kR2; ++rr) {
+    const float sv = warp_sum(sum_f32x2(v[rr]));
+    if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
+  }
+}
+
 // Dynamic shared memory of a CTA: the token vectors in bf16 [T][H]; a ring of `slots` buffers, each holding this
 // CTA's w2 rows of one chosen expert in bf16 [rows_per_cta][I] (no ring when
 // one expert's rows do not fit: phase 2 then reads w2 through L2); act in
@@ -468,60 +505,50 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
           mbar_wait(&w2_full[d % slots], (d / slots) & 1, kW2WaitNs);
       }
     }
-  } else if (rgroups > 0) {
-    // experts in order; the items (pair of the expert, group of kR2 local
-    // rows) are dealt round-robin over the compute warps, continuing from
-    // one expert to the next.  The act chunks of a pair are loaded once and
-    // shared by kR2 independent dot products with w2[e][h0 + r, :].
-    int before = 0;  // items of the experts before d
-    for (int d = 0; d < nd; ++d) {
-      const int q = ring ? d % slots : 0;
-      if (ring && !mbar_wait(&w2_full[q], (d / slots) & 1, kW2WaitNs, &s_abort)) {
+  } else if (rgroups > 0 && (!ring || nd <= slots)) {
+    // every chosen expert's rows are on chip (or read through L2): wait for
+    // the copies once, then deal all items (pair, group of kR2 local rows)
+    // round-robin over the compute warps
+    for (int d = 0; ring && d < nd; ++d) {
+      if (!mbar_wait(&w2_full[d], 0, kW2WaitNs, &s_abort)) {
         s_abort = 1;
         atomicOr(status, kStatusTimeout);
         break;
       }
-      const uint4 *ws = reinterpret_cast<const uint4 *>(sw2 + q * slot_stride);
-      const uint4 *wg = w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * I8;
+    }
+    const int n_items = L.dstart[nd] * rgroups;
+    for (int it = warp; it < n_items && !s_abort; it += kWarps) {
+      const int pq = it / rgroups, rg = it - pq * rgroups;  // pq: position in plist
+      const int pair = L.plist[pq];
+      const int d = L.pd[pair];
+      phase2_item(ring ? reinterpret_cast<const uint4 *>(sw2 + d * slot_stride) : nullptr,
+                  w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * I8, act4, cache_act, pair,
+                  rg * kR2, nrows, I, TK, sdots);
+    }
+  } else if (rgroups > 0) {
+    // more experts than slots: take the experts in order, waiting for each
+    // one's slot and releasing it after this warp's share of its items (the
+    // round-robin continues from one expert to the next)
+    int before = 0;  // items of the experts before d
+    for (int d = 0; d < nd; ++d) {
+      const int q = d % slots;
+      if (!mbar_wait(&w2_full[q], (d / slots) & 1, kW2WaitNs, &s_abort)) {
+        s_abort = 1;
+        atomicOr(status, kStatusTimeout);
+        break;
+      }
       const int p0 = L.dstart[d];
       const int n_items = (L.dstart[d + 1] - p0) * rgroups;
       int it = warp - before % kWarps;
       if (it < 0) it += kWarps;
       for (; it < n_items; it += kWarps) {
-        const int pq = p0 + it / rgroups, rg = it % rgroups;  // pq: position in plist
-        const int pair = L.plist[pq];
-        const int r0 = rg * kR2;
-        const float4 *a = act4 + static_cast<size_t>(pair) * (I / 4);
-        unsigned long long v[kR2];  // two fp32 partial sums each
-#pragma unroll
-        for (int rr = 0; rr < kR2; ++rr) v[rr] = 0ull;
-        for (int base = 0; base < I8; base += 32 * kU2) {
-#pragma unroll
-          for (int j = 0; j < kU2; ++j) {
-            const int c = base + lane + 32 * j;
-            if (c < I8) {
-              const float4 a0 = cache_act ? a[2 * c] : __ldcg(a + 2 * c);
-              const float4 a1 = cache_act ? a[2 * c + 1] : __ldcg(a + 2 * c + 1);
-              uint4 wv[kR2];
-#pragma unroll
-              for (int rr = 0; rr < kR2; ++rr)
-                if (r0 + rr < nrows)
-                  wv[rr] = ring ? ws[(r0 + rr) * I8 + c] : __ldg(wg + (r0 + rr) * I8 + c);
-#pragma unroll
-              for (int rr = 0; rr < kR2; ++rr)
-                if (r0 + rr < nrows) fma8_f32x2(wv[rr], a0, a1, v[rr]);
-            }
-          }
-        }
-#pragma unroll
-        for (int rr = 0; rr < kR2; ++rr) {
-          const float sv = warp_sum(sum_f32x2(v[rr]));
-          if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
-        }
+        const int pq = p0 + it / rgroups, rg = it % rgroups;
+        phase2_item(reinterpret_cast<const uint4 *>(sw2 + q * slot_stride), nullptr, act4,
+                    cache_act, L.plist[pq], rg * kR2, nrows, I, TK, sdots);
       }
       before += n_items;
       __syncwarp();
-      if (ring && lane == 0) mbar_arrive(&w2_empty[q]);
+      if (lane == 0) mbar_arrive(&w2_empty[q]);
     }
   }
   __syncthreads();
