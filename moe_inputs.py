@@ -123,5 +123,30 @@ def make_biases(E: int, H: int, I: int, seed: int = 0, b1_scale: float = 0.1,
     return b1, b2
 
 
+def make_fp8_weights(E: int, H: int, I: int, block: int, seed: int = 0, device: str = "cpu"):
+    """Sub-channel-quantised expert weights for the FP8 forward: randn
+    weights with the fan-in scaling of make_inputs, cut into blocks of
+    `block` consecutive contraction elements per output row; each block gets
+    the fp32 scale max|w| / 448 (the largest E4M3 value) and its codes are
+    torch's float8_e4m3fn conversion of w / scale.  Returns (q1 uint8
+    [E,2I,H], s1 fp32 [E,2I,H/block], q2 uint8 [E,H,I], s2 fp32
+    [E,H,I/block]).  This only prepares inputs (a checkpoint would hold
+    them); the forward reads codes and scales as given."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    kw = dict(generator=g, device=device)
+
+    def quant(w):
+        K = w.shape[-1]
+        wb = w.reshape(*w.shape[:-1], K // block, block)
+        sc = (wb.abs().amax(-1) / 448.0).clamp_min(1e-30)
+        q = (wb / sc.unsqueeze(-1)).to(torch.float8_e4m3fn).view(torch.uint8)
+        return q.reshape(w.shape).contiguous(), sc.float().contiguous()
+
+    q1, s1 = quant(torch.randn(E, 2 * I, H, dtype=torch.float32, **kw) * (H ** -0.5))
+    q2, s2 = quant(torch.randn(E, H, I, dtype=torch.float32, **kw) * (I ** -0.5))
+    return q1, s1, q2, s2
+
+
 def make_shape_inputs(shape: MoEShape, seed: int = 0, device: str = "cpu"):
     return make_inputs(shape.T, shape.H, shape.I, shape.E, seed=seed, device=device)

@@ -58,8 +58,15 @@ def _load(mutation: int = 0) -> ctypes.CDLL:
                                              P, i64, P]
     lib.oracle_moe_expert_loop_ex.argtypes = [P, P, P, P, P, i32, P, P, i64, i64, i64, i32, i32,
                                               P]
+    lib.oracle_moe_token_loop_fp8.argtypes = [P, P, P, P, P, i64, P, P, i64, i64, i64, i32, i32,
+                                              P, i64, P]
+    lib.oracle_moe_expert_loop_fp8.argtypes = [P, P, P, P, P, i64, P, P, i64, i64, i64, i32,
+                                               i32, P]
+    lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_to_double.restype = ctypes.c_double
     for f in ("oracle_route", "oracle_permute", "oracle_moe_token_loop",
               "oracle_moe_expert_loop", "oracle_moe_token_loop_ex", "oracle_moe_expert_loop_ex",
+              "oracle_moe_token_loop_fp8", "oracle_moe_expert_loop_fp8",
               "oracle_max_threads", "oracle_mutation"):
         getattr(lib, f).restype = ctypes.c_int
     lib.oracle_set_threads.argtypes = [i32]
@@ -182,4 +189,66 @@ def moe_expert_loop(hidden, w1, w2, topk_w, ids, mutation: int = 0,
         None if b2a is None else _ptr(b2a), a, _ptr(tw), _ptr(ti), T, H, I, E, k, _ptr(out))
     if rc != 0:
         raise RuntimeError("oracle_moe_expert_loop failed")
+    return out[:T]
+
+
+# ------------------------------------------------------------ FP8 weights
+def e4m3_to_double(code: int, mutation: int = 0) -> float:
+    """The value of one OCP FP8 E4M3 ("e4m3fn") code."""
+    return _load(mutation).oracle_e4m3_to_double(int(code) & 0xFF)
+
+
+def _fp8_args(hidden, q1, s1, q2, s2, block, topk_w, ids):
+    hb = _bf16_bits(hidden)
+    T, H = hb.shape
+    q1a = np.ascontiguousarray(np.asarray(q1, dtype=np.uint8))
+    q2a = np.ascontiguousarray(np.asarray(q2, dtype=np.uint8))
+    E, twoI, H1 = q1a.shape
+    I = twoI // 2
+    block = int(block)
+    if H1 != H or twoI != 2 * I or q2a.shape != (E, H, I):
+        raise ValueError("shape mismatch between hidden, q1 [E,2I,H] and q2 [E,H,I]")
+    if block < 1 or H % block or I % block:
+        raise ValueError("block must divide H and I")
+    s1a = np.ascontiguousarray(np.asarray(s1, dtype=np.float32).reshape(E, 2 * I, H // block))
+    s2a = np.ascontiguousarray(np.asarray(s2, dtype=np.float32).reshape(E, H, I // block))
+    tw = np.ascontiguousarray(np.asarray(topk_w, dtype=np.float64))
+    ti = np.ascontiguousarray(np.asarray(ids, dtype=np.int32))
+    k = ti.shape[1] if ti.ndim == 2 else 1
+    if tw.shape != (T, k) or ti.shape != (T, k):
+        raise ValueError("topk weights/ids must both be [T, k]")
+    return hb, q1a, s1a, q2a, s2a, block, tw, ti, T, H, I, E, k
+
+
+def moe_token_loop_fp8(hidden, q1, s1, q2, s2, block, topk_w, ids, rows=None,
+                       mutation: int = 0):
+    """Formulation A on FP8 E4M3 weights (uint8 codes q1 [E,2I,H], q2
+    [E,H,I]) with fp32 scales per row and block of `block` contraction
+    elements (s1 [E,2I,H/block], s2 [E,H,I/block]); silu, no biases."""
+    hb, q1a, s1a, q2a, s2a, block, tw, ti, T, H, I, E, k = _fp8_args(
+        hidden, q1, s1, q2, s2, block, topk_w, ids)
+    if rows is None:
+        rr, nrows, n = None, -1, T
+    else:
+        rr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        nrows = n = rr.shape[0]
+    out = np.empty((max(n, 1), H), np.float64)
+    rc = _load(mutation).oracle_moe_token_loop_fp8(
+        _ptr(hb), _ptr(q1a), _ptr(s1a), _ptr(q2a), _ptr(s2a), block, _ptr(tw), _ptr(ti), T, H,
+        I, E, k, None if rr is None else _ptr(rr), nrows, _ptr(out))
+    if rc != 0:
+        raise RuntimeError("oracle_moe_token_loop_fp8 failed")
+    return out[:n]
+
+
+def moe_expert_loop_fp8(hidden, q1, s1, q2, s2, block, topk_w, ids, mutation: int = 0):
+    """Formulation B on FP8 E4M3 weights (arguments as moe_token_loop_fp8)."""
+    hb, q1a, s1a, q2a, s2a, block, tw, ti, T, H, I, E, k = _fp8_args(
+        hidden, q1, s1, q2, s2, block, topk_w, ids)
+    out = np.empty((max(T, 1), H), np.float64)
+    rc = _load(mutation).oracle_moe_expert_loop_fp8(
+        _ptr(hb), _ptr(q1a), _ptr(s1a), _ptr(q2a), _ptr(s2a), block, _ptr(tw), _ptr(ti), T, H,
+        I, E, k, _ptr(out))
+    if rc != 0:
+        raise RuntimeError("oracle_moe_expert_loop_fp8 failed")
     return out[:T]

@@ -39,6 +39,15 @@
  *     g' = min(g, 7); b1 (fp32 [E, 2I]: gate bias, then up bias) is added to
  *     the two projections before the activation, b2 (fp32 [E, H]) to the
  *     expert output before the top-k weighting.
+ *   - sub-channel quantised weights (0.13.2 page: w1_scale, w2_scale,
+ *     subc_quant_wsz; ref_moe multiplies each weight, widened to f32, by the
+ *     scale of its block of subc_quant_wsz contraction elements): the codes
+ *     are OCP FP8 E4M3 ("e4m3fn": exponent bias 7, no infinities, 0x7f and
+ *     0xff are NaN), w1 [E, 2I, H] and w2 [E, H, I] in the layout above; a
+ *     scale belongs to one output row and one block of `block` consecutive
+ *     contraction elements: w1_scale [E, 2I, H / block], w2_scale
+ *     [E, H, I / block].  The dequantised weight is code * scale, exact in
+ *     double.
  */
 #include <math.h>
 #include <stdint.h>
@@ -63,6 +72,24 @@ static double bf16_to_double(uint16_t b)
     memcpy(&f, &u, sizeof f);
     return (double)f;
 }
+
+/* OCP FP8 E4M3 ("e4m3fn"): sign, 4 exponent bits (bias 7), 3 mantissa
+ * bits; exponent 0 is subnormal (m/8 * 2^-6); S.1111.111 is NaN; there are
+ * no infinities.  Planted mistake 10 uses bias 8. */
+static double e4m3_to_double(uint8_t c)
+{
+    const int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    const int bias = MUTATED(10) ? 8 : 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, 1 - bias);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - bias);
+    return s ? -v : v;
+}
+
+double oracle_e4m3_to_double(uint8_t c) { return e4m3_to_double(c); }
 
 static double silu(double z) { return z / (1.0 + exp(-z)); }
 
@@ -195,6 +222,37 @@ int oracle_permute(const int32_t *ids, int64_t n, int E,
 }
 
 /*
+ * The expert weights: bf16 (w1, w2) or FP8 E4M3 codes with per-block scales
+ * (q1, s1, q2, s2, block).  W1(e, r, h) is row r of w1[e] at contraction
+ * index h, W2(e, h, i) likewise for w2[e].
+ */
+typedef struct {
+    const uint16_t *w1, *w2;
+    const uint8_t *q1, *q2;
+    const float *s1, *s2;
+    int64_t block;
+} Weights;
+
+static double W1(const Weights *W, int e, int64_t r, int64_t h, int64_t H, int64_t I)
+{
+    const size_t row = (size_t)e * 2 * I + (size_t)r;
+    if (W->w1) return bf16_to_double(W->w1[row * H + h]);
+    /* planted mistake 9 picks the scale block by h modulo the block count */
+    const int64_t nb = H / W->block;
+    const int64_t b = MUTATED(9) ? h % nb : h / W->block;
+    return e4m3_to_double(W->q1[row * H + h]) * (double)W->s1[row * nb + b];
+}
+
+static double W2(const Weights *W, int e, int64_t h, int64_t i, int64_t H, int64_t I)
+{
+    const size_t row = (size_t)e * H + (size_t)h;
+    if (W->w2) return bf16_to_double(W->w2[row * I + i]);
+    const int64_t nb = I / W->block;
+    const int64_t b = MUTATED(9) ? i % nb : i / W->block;
+    return e4m3_to_double(W->q2[row * I + i]) * (double)W->s2[row * nb + b];
+}
+
+/*
  * One expert's gated FFN on one token, in double:
  *   g_i = W1[e][i,:] . x + b1[e][i], u_i = W1[e][I+i,:] . x + b1[e][I+i],
  *   a_i = act(g_i, u_i), y_h = W2[e][h,:] . a + b2[e][h]
@@ -203,20 +261,17 @@ int oracle_permute(const int32_t *ids, int64_t n, int E,
  * shape [2I, H]; the first I outputs are gate, the next I are up;
  * F.linear(act, w2_e) with w2_e of shape [H, I].
  */
-static void expert_ffn(const uint16_t *w1, const uint16_t *w2, const float *b1,
+static void expert_ffn(const Weights *W, const float *b1,
                        const float *b2, int act, int e, int64_t H, int64_t I,
                        const double *x, double *a, double *y)
 {
-    const uint16_t *W1 = w1 + (size_t)e * 2 * I * H;
-    const uint16_t *W2 = w2 + (size_t)e * H * I;
     for (int64_t i = 0; i < I; ++i) {
-        const uint16_t *rg = W1 + (size_t)i * H;
-        const uint16_t *ru = W1 + (size_t)(I + i) * H;
-        if (MUTATED(1)) { const uint16_t *tmp = rg; rg = ru; ru = tmp; }
+        int64_t rg = i, ru = I + i;
+        if (MUTATED(1)) { int64_t tmp = rg; rg = ru; ru = tmp; }
         double g = 0.0, u = 0.0;
         for (int64_t h = 0; h < H; ++h) {
-            g += bf16_to_double(rg[h]) * x[h];
-            u += bf16_to_double(ru[h]) * x[h];
+            g += W1(W, e, rg, h, H, I) * x[h];
+            u += W1(W, e, ru, h, H, I) * x[h];
         }
         if (b1) {
             double bg = (double)b1[(size_t)e * 2 * I + i];
@@ -232,8 +287,7 @@ static void expert_ffn(const uint16_t *w1, const uint16_t *w2, const float *b1,
         for (int64_t i = 0; i < I; ++i) {
             /* planted mistake 2 reads W2 as if it were stored [I, H]
              * (only meaningful when H == I, which the test uses) */
-            double wv = MUTATED(2) ? bf16_to_double(W2[(size_t)i * H + h])
-                                   : bf16_to_double(W2[(size_t)h * I + i]);
+            double wv = MUTATED(2) ? W2(W, e, i, h, I, H) : W2(W, e, h, i, H, I);
             acc += wv * a[i];
         }
         y[h] = acc + (b2 && !MUTATED(7) ? (double)b2[(size_t)e * H + h] : 0.0);
@@ -254,11 +308,10 @@ static void add_b2_unweighted(const float *b2, int e, int64_t H, double *o)
  * skipped.  hidden [T,H], w1 [E,2I,H], w2 [E,H,I] are bf16 bit patterns;
  * topk_w [T,k] double; out is [nrows or T, H] double, overwritten.
  */
-int oracle_moe_token_loop_ex(const uint16_t *hidden, const uint16_t *w1,
-                             const uint16_t *w2, const float *b1, const float *b2,
-                             int act, const double *topk_w, const int32_t *ids,
-                             int64_t T, int64_t H, int64_t I, int E, int k,
-                             const int64_t *rows, int64_t nrows, double *out)
+static int token_loop(const uint16_t *hidden, const Weights *W, const float *b1,
+                      const float *b2, int act, const double *topk_w, const int32_t *ids,
+                      int64_t T, int64_t H, int64_t I, int E, int k,
+                      const int64_t *rows, int64_t nrows, double *out)
 {
     if (act < ACT_SILU || act > ACT_SWIGLUOAI) return -1;
     if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1) return -1;
@@ -283,7 +336,7 @@ int oracle_moe_token_loop_ex(const uint16_t *hidden, const uint16_t *w1,
                 for (int j = 0; j < k; ++j) {
                     int e = ids[t * k + j];
                     if (e < 0 || e >= E) continue;
-                    expert_ffn(w1, w2, b1, b2, act, e, H, I, x, a, y);
+                    expert_ffn(W, b1, b2, act, e, H, I, x, a, y);
                     double wj = topk_w[t * k + j];
                     for (int64_t h = 0; h < H; ++h) o[h] += wj * y[h];
                     add_b2_unweighted(b2, e, H, o);
@@ -293,6 +346,33 @@ int oracle_moe_token_loop_ex(const uint16_t *hidden, const uint16_t *w1,
         free(x); free(a); free(y);
     }
     return err ? -1 : 0;
+}
+
+int oracle_moe_token_loop_ex(const uint16_t *hidden, const uint16_t *w1,
+                             const uint16_t *w2, const float *b1, const float *b2,
+                             int act, const double *topk_w, const int32_t *ids,
+                             int64_t T, int64_t H, int64_t I, int E, int k,
+                             const int64_t *rows, int64_t nrows, double *out)
+{
+    const Weights W = {w1, w2, NULL, NULL, NULL, NULL, 0};
+    return token_loop(hidden, &W, b1, b2, act, topk_w, ids, T, H, I, E, k, rows, nrows, out);
+}
+
+/*
+ * Formulation A on FP8 E4M3 weights with per-block scales (silu, no
+ * biases): q1 [E, 2I, H] codes, s1 [E, 2I, H / block]; q2 [E, H, I] codes,
+ * s2 [E, H, I / block].  block must divide H and I.
+ */
+int oracle_moe_token_loop_fp8(const uint16_t *hidden, const uint8_t *q1, const float *s1,
+                              const uint8_t *q2, const float *s2, int64_t block,
+                              const double *topk_w, const int32_t *ids, int64_t T,
+                              int64_t H, int64_t I, int E, int k, const int64_t *rows,
+                              int64_t nrows, double *out)
+{
+    if (block < 1 || H % block != 0 || I % block != 0) return -1;
+    const Weights W = {NULL, NULL, q1, q2, s1, s2, block};
+    return token_loop(hidden, &W, NULL, NULL, ACT_SILU, topk_w, ids, T, H, I, E, k, rows,
+                      nrows, out);
 }
 
 int oracle_moe_token_loop(const uint16_t *hidden, const uint16_t *w1,
@@ -312,10 +392,9 @@ int oracle_moe_token_loop(const uint16_t *hidden, const uint16_t *w1,
  * A token routed twice to e thus gets the summed weight.  Same argument
  * layout as formulation A (all T rows).
  */
-int oracle_moe_expert_loop_ex(const uint16_t *hidden, const uint16_t *w1,
-                              const uint16_t *w2, const float *b1, const float *b2,
-                              int act, const double *topk_w, const int32_t *ids,
-                              int64_t T, int64_t H, int64_t I, int E, int k, double *out)
+static int expert_loop(const uint16_t *hidden, const Weights *W, const float *b1,
+                       const float *b2, int act, const double *topk_w, const int32_t *ids,
+                       int64_t T, int64_t H, int64_t I, int E, int k, double *out)
 {
     if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1) return -1;
     if (act < ACT_SILU || act > ACT_SWIGLUOAI) return -1;
@@ -343,7 +422,7 @@ int oracle_moe_expert_loop_ex(const uint16_t *hidden, const uint16_t *w1,
                 for (int64_t t = 0; t < T; ++t) {
                     if (what[t] == 0.0) continue;
                     for (int64_t h = 0; h < H; ++h) x[h] = bf16_to_double(hidden[(size_t)t * H + h]);
-                    expert_ffn(w1, w2, b1, b2, act, e, H, I, x, a, y);
+                    expert_ffn(W, b1, b2, act, e, H, I, x, a, y);
                     double *o = out + (size_t)t * H;
                     for (int64_t h = 0; h < H; ++h) o[h] += what[t] * y[h];
                 }
@@ -353,6 +432,26 @@ int oracle_moe_expert_loop_ex(const uint16_t *hidden, const uint16_t *w1,
     }
     free(what);
     return err ? -1 : 0;
+}
+
+int oracle_moe_expert_loop_ex(const uint16_t *hidden, const uint16_t *w1,
+                              const uint16_t *w2, const float *b1, const float *b2,
+                              int act, const double *topk_w, const int32_t *ids,
+                              int64_t T, int64_t H, int64_t I, int E, int k, double *out)
+{
+    const Weights W = {w1, w2, NULL, NULL, NULL, NULL, 0};
+    return expert_loop(hidden, &W, b1, b2, act, topk_w, ids, T, H, I, E, k, out);
+}
+
+/* Formulation B on FP8 E4M3 weights with per-block scales (as above). */
+int oracle_moe_expert_loop_fp8(const uint16_t *hidden, const uint8_t *q1, const float *s1,
+                               const uint8_t *q2, const float *s2, int64_t block,
+                               const double *topk_w, const int32_t *ids, int64_t T,
+                               int64_t H, int64_t I, int E, int k, double *out)
+{
+    if (block < 1 || H % block != 0 || I % block != 0) return -1;
+    const Weights W = {NULL, NULL, q1, q2, s1, s2, block};
+    return expert_loop(hidden, &W, NULL, NULL, ACT_SILU, topk_w, ids, T, H, I, E, k, out);
 }
 
 int oracle_moe_expert_loop(const uint16_t *hidden, const uint16_t *w1,

@@ -28,3 +28,15 @@ def test_draws_are_seeded():
     assert not torch.equal(a[0], c[0])
     b1, b2 = make_biases(2, 128, 128, seed=1)
     assert b1.shape == (2, 256) and b2.shape == (2, 128) and b1.dtype == torch.float32
+
+
+def test_fp8_weights_shapes_and_range():
+    from moe_inputs import make_fp8_weights
+    q1, s1, q2, s2 = make_fp8_weights(2, 256, 128, 128, seed=3)
+    assert q1.dtype == torch.uint8 and q1.shape == (2, 256, 256)
+    assert s1.shape == (2, 256, 2) and s2.shape == (2, 256, 1)
+    assert q2.shape == (2, 256, 128) and s1.dtype == torch.float32
+    # no NaN codes, and every block uses the top of the E4M3 range
+    v = q1.view(torch.float8_e4m3fn).float()
+    assert not torch.isnan(v).any()
+    assert torch.allclose(v.abs().reshape(2, 256, 2, 128).amax(-1), torch.full((2, 256, 2), 448.0))

@@ -269,6 +269,62 @@ def pin_variants_formulations_agree(mutation=0):
     return bool(ok)
 
 
+# ------------------------------------------------ pins of the FP8 weights
+# (w1_scale / w2_scale / subc_quant_wsz of the 0.13.2 TPU page's ref_moe)
+
+
+def pin_e4m3_decoder(mutation=0):
+    """Every one of the 256 E4M3 codes against torch's float8_e4m3fn."""
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    got = np.array([oracle.e4m3_to_double(c, mutation=mutation) for c in codes])
+    nan = np.isnan(ref)
+    return bool(np.array_equal(nan, np.isnan(got)) and np.array_equal(ref[~nan], got[~nan]))
+
+
+def _fp8_case(T=9, H=512, I=256, E=4, k=2, block=128, seed=31):
+    """Codes and power-of-two scales that differ per block: the dequantised
+    weights are then exact in bf16, so the bf16 forward applies to them."""
+    rng = np.random.default_rng(seed)
+    hidden, _, _, logits = make_inputs(T, H, I, E, seed=seed)
+    q1 = rng.integers(0, 256, (E, 2 * I, H), dtype=np.uint8)
+    q2 = rng.integers(0, 256, (E, H, I), dtype=np.uint8)
+    q1[(q1 & 0x7F) == 0x7F] = 0  # no NaN codes
+    q2[(q2 & 0x7F) == 0x7F] = 0
+    s1 = np.exp2(rng.integers(-14, -8, (E, 2 * I, H // block))).astype(np.float32)
+    s2 = np.exp2(rng.integers(-14, -8, (E, H, I // block))).astype(np.float32)
+    ids, w = oracle.route(logits.numpy(), k, True)
+    return hidden, q1, s1, q2, s2, block, w, ids
+
+
+def _dequant_bf16(q, s, block):
+    """torch's E4M3 conversion times each block's scale (np.repeat spreads a
+    block's scale over its elements, as ref_moe's jnp.repeat does), as bf16."""
+    v = torch.from_numpy(q).view(torch.float8_e4m3fn).double()
+    v = v * torch.from_numpy(np.repeat(s.astype(np.float64), block, axis=-1))
+    bf = v.to(torch.bfloat16)
+    assert torch.equal(bf.double(), v)  # exact: power-of-two scales
+    return bf
+
+
+def pin_fp8_equals_bf16_of_dequantised(mutation=0):
+    hidden, q1, s1, q2, s2, block, w, ids = _fp8_case()
+    w1 = _dequant_bf16(q1, s1, block)
+    w2 = _dequant_bf16(q2, s2, block)
+    ref = oracle.moe_token_loop(hidden, w1, w2, w, ids)
+    a = oracle.moe_token_loop_fp8(hidden, q1, s1, q2, s2, block, w, ids, mutation=mutation)
+    b = oracle.moe_expert_loop_fp8(hidden, q1, s1, q2, s2, block, w, ids, mutation=mutation)
+    return bool(close(a, ref, 1e-12) and close(b, ref, 1e-12))
+
+
+def pin_fp8_w2_scale_linearity(mutation=0):
+    """Every w2 scale times 2 doubles the output exactly."""
+    hidden, q1, s1, q2, s2, block, w, ids = _fp8_case(seed=32)
+    a = oracle.moe_token_loop_fp8(hidden, q1, s1, q2, s2, block, w, ids, mutation=mutation)
+    b = oracle.moe_token_loop_fp8(hidden, q1, s1, q2, 2 * s2, block, w, ids, mutation=mutation)
+    return bool(np.array_equal(2 * a, b))
+
+
 # ---------------------------------------------------------------- tests
 
 def test_golden_route(golden_dir):
@@ -428,6 +484,24 @@ def test_variant_formulations_agree():
     assert pin_variants_formulations_agree()
 
 
+def test_e4m3_decoder_matches_torch():
+    assert pin_e4m3_decoder()
+
+
+def test_fp8_forward_equals_bf16_forward_of_dequantised_weights():
+    assert pin_fp8_equals_bf16_of_dequantised()
+
+
+def test_fp8_w2_scale_linearity():
+    assert pin_fp8_w2_scale_linearity()
+
+
+def test_fp8_block_must_divide():
+    hidden, q1, s1, q2, s2, block, w, ids = _fp8_case(T=2)
+    with pytest.raises(ValueError):
+        oracle.moe_token_loop_fp8(hidden, q1, s1, q2, s2, 96, w, ids)
+
+
 def test_unknown_activation_rejected():
     hidden, w1, w2, logits = make_inputs(2, 64, 32, 2, seed=25)
     ids, w = oracle.route(logits.numpy(), 1, True)
@@ -476,6 +550,8 @@ MUTATIONS = {
     6: "gate and up biases of b1 swapped",
     7: "b2 added once per expert after the top-k weighting",
     8: "gelu in its erf form instead of the tanh form",
+    9: "FP8 scale block chosen by the index modulo the block count",
+    10: "E4M3 exponent bias 8 instead of 7",
 }
 
 
@@ -495,6 +571,9 @@ def test_planted_mistakes_are_caught(mutation, golden_dir):
         "b1_zero_w1": pin_b1_with_zero_w1(mutation),
         "b2_zero_w2": pin_b2_with_zero_w2(mutation),
         "variants_agree": pin_variants_formulations_agree(mutation),
+        "e4m3_decoder": pin_e4m3_decoder(mutation),
+        "fp8_dequantised": pin_fp8_equals_bf16_of_dequantised(mutation),
+        "fp8_w2_linearity": pin_fp8_w2_scale_linearity(mutation),
     }
     assert oracle._load(mutation).oracle_mutation() == mutation
     caught = [k for k, v in results.items() if not v]
