@@ -140,6 +140,36 @@ int moe_forward_ex(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w
                    int64_t T, int H, int I, int E, int k, void *stream);
 
 /*
+ * moe_forward_fp8 -- moe_forward on sub-channel-quantised expert weights.
+ * Page: the 0.13.2 version of the TPU page (ref_moe with w1_scale,
+ * w2_scale and subc_quant_wsz): every weight is its code times the fp32
+ * scale of its block of `block` consecutive contraction elements.
+ *
+ *   w1        [E, 2I, H] FP8 E4M3 codes (OCP "e4m3fn", one byte each), rows
+ *             as in moe_forward (gate rows, then up rows)
+ *   w1_scale  [E, 2I, H / block] fp32: scale of row r, columns
+ *             b*block .. b*block + block - 1 (the page's w1_scale
+ *             [E, 2, H / block, 1, I] transposed to this row layout)
+ *   w2        [E, H, I] FP8 E4M3 codes
+ *   w2_scale  [E, H, I / block] fp32
+ *   block     a multiple of 128 that divides H and I (the page demands a
+ *             multiple of 256)
+ * Activation silu, no biases; other arguments, the output and the error
+ * codes are those of moe_forward, plus UNSUPPORTED for a block that is not
+ * a multiple of 128 or does not divide H and I, and INVALID_ARG for null
+ * scales or block < 1.
+ * Numerics: the small-T path (T <= the small-T limit) streams the codes and
+ * multiplies each 16-weight partial dot product (fp32) by its scale; the
+ * grouped-GEMM path first expands all E experts' weights to bf16
+ * (bf16_rn(code * scale), one rounding) into a second library-owned
+ * grow-only buffer of E * 3 * H * I * 2 bytes, then runs as moe_forward.
+ */
+int moe_forward_fp8(const uint16_t *hidden, const uint8_t *w1, const float *w1_scale,
+                    const uint8_t *w2, const float *w2_scale, int block,
+                    const float *topk_weights, const int32_t *topk_ids, float *out,
+                    int64_t T, int H, int I, int E, int k, void *stream);
+
+/*
  * moe_forward_small_noalloc -- the small-batch path of moe_forward (the two
  * GEMV kernels) in a form that never allocates device memory.  The pages
  * have no counterpart: it exists for callers that cannot allocate once they

@@ -43,7 +43,7 @@ EXPORTED = (
     "moe_get_device_status", "moe_set_small_t_max", "moe_set_sync_each_stage",
     "moe_set_wait_limit_ns", "moe_last_failed_stage", "moe_debug_wait_timeout",
     "moe_profile_enable", "moe_profile_reset", "moe_profile_read",
-    "moe_forward_small_noalloc", "moe_forward_ex",
+    "moe_forward_small_noalloc", "moe_forward_ex", "moe_forward_fp8",
 )
 
 
@@ -76,6 +76,7 @@ def _load() -> ctypes.CDLL:
         "moe_profile_read": ([I32, P, P, P], I32),
         "moe_forward_small_noalloc": ([P, P, P, P, P, P, I64, I32, I32, I32, I32, P], I32),
         "moe_forward_ex": ([P, P, P, P, P, I32, P, P, P, I64, I32, I32, I32, I32, P], I32),
+        "moe_forward_fp8": ([P, P, P, P, P, I32, P, P, P, I64, I32, I32, I32, I32, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -178,6 +179,38 @@ def moe_forward(hidden: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
     return out
 
 
+def moe_forward_fp8(hidden: torch.Tensor, w1: torch.Tensor, w1_scale: torch.Tensor,
+                    w2: torch.Tensor, w2_scale: torch.Tensor, block: int,
+                    topk_weights: torch.Tensor, topk_ids: torch.Tensor,
+                    out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Fused MoE forward on FP8 E4M3 expert weights: w1 [E,2I,H] and w2
+    [E,H,I] uint8 codes, w1_scale [E,2I,H/block] and w2_scale [E,H,I/block]
+    fp32 scales (one per row and block of `block` contraction elements)."""
+    _need(hidden, "hidden", torch.bfloat16)
+    T, H = hidden.shape
+    _need(w1, "w1", torch.uint8)
+    E, twoI, _ = w1.shape
+    I = twoI // 2
+    block = int(block)
+    if block < 1 or H % block or I % block:
+        raise ValueError(f"block must be positive and divide H={H} and I={I}")
+    _need(w1, "w1", torch.uint8, (E, 2 * I, H))
+    _need(w2, "w2", torch.uint8, (E, H, I))
+    _need(w1_scale, "w1_scale", torch.float32, (E, 2 * I, H // block))
+    _need(w2_scale, "w2_scale", torch.float32, (E, H, I // block))
+    k = topk_ids.shape[1] if topk_ids.dim() == 2 else 0
+    _need(topk_ids, "topk_ids", torch.int32, (T, k))
+    _need(topk_weights, "topk_weights", torch.float32, (T, k))
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.float32, device=hidden.device)
+    _need(out, "out", torch.float32, (T, H))
+    _check(_lib.moe_forward_fp8(hidden.data_ptr(), w1.data_ptr(), w1_scale.data_ptr(),
+                                w2.data_ptr(), w2_scale.data_ptr(), block,
+                                topk_weights.data_ptr(), topk_ids.data_ptr(), out.data_ptr(),
+                                T, H, I, E, k, _stream(stream)), "moe_forward_fp8")
+    return out
+
+
 def moe_forward_small_noalloc(hidden: torch.Tensor, w1: torch.Tensor, w2: torch.Tensor,
                               topk_weights: torch.Tensor, topk_ids: torch.Tensor,
                               out: torch.Tensor, stream=None) -> torch.Tensor:
@@ -268,7 +301,7 @@ def profile_read() -> dict[str, tuple[int, float]]:
 
 
 __all__ = [
-    "moe_route", "moe_forward", "moe_forward_small_noalloc", "moe_permute", "get_device_status", "set_small_t_max",
+    "moe_route", "moe_forward", "moe_forward_fp8", "moe_forward_small_noalloc", "moe_permute", "get_device_status", "set_small_t_max",
     "set_sync_each_stage", "set_wait_limit_ns", "last_failed_stage", "debug_wait_timeout",
     "profile_enable", "profile_reset", "profile_read", "error_string", "MoEError",
     "LIB_PATH", "EXPORTED", "ACTS",

@@ -31,6 +31,8 @@ struct DeviceState {
   unsigned long long small_t_arrivals = 0;  // small-T grid-barrier counter target
   void *ws = nullptr;          // grow-only workspace
   size_t ws_bytes = 0;
+  void *wq = nullptr;          // grow-only: bf16 copies of FP8 weights (GEMM path)
+  size_t wq_bytes = 0;
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -156,22 +158,24 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Make the workspace at least `bytes` large.
-int ensure_workspace(DeviceState &d, size_t bytes) {
-  if (bytes <= d.ws_bytes) return MOE_OK;
-  if (d.ws != nullptr) {
-    cudaFree(d.ws);  // synchronises the device
-    d.ws = nullptr;
-    d.ws_bytes = 0;
+// Make a grow-only device buffer at least `bytes` large.
+int ensure_buffer(void *&buf, size_t &have, size_t bytes) {
+  if (bytes <= have) return MOE_OK;
+  if (buf != nullptr) {
+    cudaFree(buf);  // synchronises the device
+    buf = nullptr;
+    have = 0;
   }
   const size_t want = align256(bytes);
-  if (cudaMalloc(&d.ws, want) != cudaSuccess) {
+  if (cudaMalloc(&buf, want) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_OOM;
   }
-  d.ws_bytes = want;
+  have = want;
   return MOE_OK;
 }
+
+int ensure_workspace(DeviceState &d, size_t bytes) { return ensure_buffer(d.ws, d.ws_bytes, bytes); }
 
 struct Carver {
   char *base;
@@ -265,12 +269,22 @@ static_assert(MOE_ACT_SILU == moe::kActSilu && MOE_ACT_GELU_TANH == moe::kActGel
                   MOE_ACT_SWIGLUOAI == moe::kActSwigluOai,
               "activation codes of the ABI and the kernels agree");
 
-// moe_forward and moe_forward_ex: the variant is (b1, b2, act); b1 and b2
-// may be null.
-int forward_impl(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2, const float *b1,
+// FP8 E4M3 weights: codes in the layouts of w1 and w2, fp32 scales per row
+// and block of `block` contraction elements.
+struct Fp8Weights {
+  const float *s1, *s2;
+  int block;
+};
+
+// moe_forward, moe_forward_ex and moe_forward_fp8: the variant is (b1, b2,
+// act); b1 and b2 may be null; fp8 non-null means w1/w2 hold E4M3 codes.
+int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const float *b1,
                  const float *b2, int act_kind, const float *topk_weights,
                  const int32_t *topk_ids, float *out, int64_t T, int H, int I, int E, int k,
-                 void *stream) {
+                 void *stream, const Fp8Weights *fp8 = nullptr) {
+  const uint16_t *hidden = static_cast<const uint16_t *>(hidden_);
+  const uint16_t *w1 = static_cast<const uint16_t *>(w1_);
+  const uint16_t *w2 = static_cast<const uint16_t *>(w2_);
   if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
   if (act_kind != MOE_ACT_SILU && act_kind != MOE_ACT_GELU_TANH && act_kind != MOE_ACT_SWIGLUOAI)
     return MOE_ERR_INVALID_ARG;
@@ -281,6 +295,12 @@ int forward_impl(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
       !aligned16(b1) || !aligned16(b2))
     return MOE_ERR_INVALID_ARG;
   if (H % 128 != 0 || I % 128 != 0 || E > kMaxExperts || k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+  if (fp8 != nullptr) {
+    if (T > 0 && (fp8->s1 == nullptr || fp8->s2 == nullptr)) return MOE_ERR_INVALID_ARG;
+    if (fp8->block < 1) return MOE_ERR_INVALID_ARG;
+    if (fp8->block % 128 != 0 || H % fp8->block != 0 || I % fp8->block != 0)
+      return MOE_ERR_UNSUPPORTED;
+  }
   const int64_t n = T * k;
   if (n >= (static_cast<int64_t>(1) << 31)) return MOE_ERR_UNSUPPORTED;
   if (T == 0) return MOE_OK;
@@ -297,10 +317,28 @@ int forward_impl(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
     Carver cv{static_cast<char *>(d->ws)};
     float *act = cv.take<float>(static_cast<size_t>(n) * I);
     return to_code(moe::launch_small_t(
-        hidden, w1, w2, b1, b2, act_kind, topk_weights, topk_ids, act, out, T, H, I, E, k,
+        hidden, w1, w2, fp8 ? fp8->s1 : nullptr, fp8 ? fp8->s2 : nullptr, fp8 ? fp8->block : 0,
+        b1, b2, act_kind, topk_weights, topk_ids, act, out, T, H, I, E, k,
         d->status,
         reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(d->status) + 64),
         &d->small_t_arrivals, static_cast<uint64_t>(g_wait_limit_ns), ctx.stream, hook));
+  }
+
+  cudaError_t e;
+  if (fp8 != nullptr) {
+    // the grouped GEMMs run on bf16 copies of all E experts' weights
+    const size_t n1 = static_cast<size_t>(E) * 2 * I * H, n2 = static_cast<size_t>(E) * H * I;
+    if ((rc = ensure_buffer(d->wq, d->wq_bytes, (n1 + n2) * 2)) != MOE_OK) return rc;
+    uint16_t *wd1 = static_cast<uint16_t *>(d->wq), *wd2 = wd1 + n1;
+    if ((e = moe::launch_dequant_e4m3(reinterpret_cast<const uint8_t *>(w1), fp8->s1,
+                                      static_cast<int64_t>(E) * 2 * I, H, fp8->block, wd1,
+                                      d->num_sms, ctx.stream, hook)) != cudaSuccess ||
+        (e = moe::launch_dequant_e4m3(reinterpret_cast<const uint8_t *>(w2), fp8->s2,
+                                      static_cast<int64_t>(E) * H, I, fp8->block, wd2,
+                                      d->num_sms, ctx.stream, hook)) != cudaSuccess)
+      return to_code(e);
+    w1 = wd1;
+    w2 = wd2;
   }
 
   // top-k <= 2: GEMM2 adds its rows straight into out and no P is needed
@@ -330,7 +368,6 @@ int forward_impl(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
 
   // grouping (and the sorted row copy): one kernel up to 8192 entries, the
   // three-kernel grouping and a separate copy above
-  cudaError_t e;
   if (moe::group_supported(n)) {
     e = moe::launch_group(topk_ids, n, E, k, expert_offsets, sorted_rows, inv, d->status, hidden,
                           H, xs, ready, static_cast<int>(n_ready), ready + n_ready, d->num_sms,
@@ -399,6 +436,15 @@ int moe_forward(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
                 int I, int E, int k, void *stream) {
   return forward_impl(hidden, w1, w2, nullptr, nullptr, MOE_ACT_SILU, topk_weights, topk_ids,
                       out, T, H, I, E, k, stream);
+}
+
+int moe_forward_fp8(const uint16_t *hidden, const uint8_t *w1, const float *w1_scale,
+                    const uint8_t *w2, const float *w2_scale, int block,
+                    const float *topk_weights, const int32_t *topk_ids, float *out, int64_t T,
+                    int H, int I, int E, int k, void *stream) {
+  const Fp8Weights q{w1_scale, w2_scale, block};
+  return forward_impl(hidden, w1, w2, nullptr, nullptr, MOE_ACT_SILU, topk_weights, topk_ids,
+                      out, T, H, I, E, k, stream, &q);
 }
 
 int moe_forward_ex(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,

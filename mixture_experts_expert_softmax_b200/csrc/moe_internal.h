@@ -111,6 +111,13 @@ cudaError_t launch_fused_gemm(const GroupedGemmArgs &a, bool with_gemm2, cudaStr
 inline int64_t fused_gemm_ready_count(int64_t n, int E) { return (n + 255) / 256 + E; }
 cudaError_t launch_wait_probe(uint32_t *status, uint64_t limit_ns, cudaStream_t s);
 
+// dequant.cu: out[r, c] = bf16(e4m3(q[r, c]) * scale[r, c / block]) for a
+// [rows, K] matrix of FP8 E4M3 codes (K and block multiples of 16, block
+// divides K; q and out 16-byte aligned).
+cudaError_t launch_dequant_e4m3(const uint8_t *q, const float *scale, int64_t rows, int K,
+                                int block, uint16_t *out, int num_sms, cudaStream_t s,
+                                const StageHook &hook);
+
 // combine.cu
 cudaError_t launch_combine(const float *P, const int32_t *inv, const float *topk_weights,
                            float *out, int64_t T, int H, int k, uint32_t *status, cudaStream_t s,
@@ -122,8 +129,12 @@ bool small_t_supported(int H, int I);
 // touch, 0 before the first launch; arrivals: the host's copy of the value
 // it reaches once every launch made so far has finished (advanced by the
 // call).  act: T*k*I fp32 scratch.
-// b1, b2, act_kind: the epilogue variant, as in GroupedGemmArgs.
-cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
+// b1, b2, act_kind: the epilogue variant, as in GroupedGemmArgs.  block == 0:
+// w1 [E, 2I, H] and w2 [E, H, I] are bf16; block > 0 (a multiple of 16 that
+// divides H and I): they are FP8 E4M3 codes with fp32 scales w1_scale
+// [E, 2I, H / block] and w2_scale [E, H, I / block].
+cudaError_t launch_small_t(const uint16_t *hidden, const void *w1, const void *w2,
+                           const float *w1_scale, const float *w2_scale, int block,
                            const float *b1, const float *b2, int act_kind,
                            const float *topk_weights, const int32_t *topk_ids, float *act,
                            float *out, int64_t T, int H, int I, int E, int k, uint32_t *status,

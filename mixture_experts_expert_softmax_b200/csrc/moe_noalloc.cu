@@ -91,7 +91,8 @@ extern "C" int moe_forward_small_noalloc(const uint16_t *hidden, const uint16_t 
   moe::StageHook hook;
   hook.pdl = true;
   const cudaError_t e =
-      moe::launch_small_t(hidden, w1, w2, nullptr, nullptr, moe::kActSilu, topk_weights,
+      moe::launch_small_t(hidden, w1, w2, nullptr, nullptr, 0, nullptr, nullptr, moe::kActSilu,
+                          topk_weights,
                           topk_ids, act, out, T, H, I, E, k, status,
                           grid_sync, &g_noalloc_arrivals[dev], 2000000000ull,
                           static_cast<cudaStream_t>(stream), hook);

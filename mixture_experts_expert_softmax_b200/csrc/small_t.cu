@@ -30,6 +30,9 @@
 // the decode dispatch of "metrale_model_layers/layers/moe/forward_k2.rs"
 // (gate-up, silu-down, weighted blend) with the activation fused into the
 // first phase and the blend into the second.
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include <algorithm>
 #include <mutex>
 
@@ -193,6 +196,66 @@ __device__ __forceinline__ float sum_f32x2(unsigned long long acc) {
          __uint_as_float(static_cast<uint32_t>(acc >> 32));
 }
 
+// Two E4M3 codes (low byte first) as floats, by the hardware conversion.
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two) {
+  const __half2_raw r =
+      __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xffffu), __NV_E4M3);
+  __half2 h;
+  memcpy(&h, &r, sizeof h);
+  return __half22float2(h);
+}
+
+// sum over q = 0..15 of e4m3(w[q]) * x[q] for 16 codes and 16 bf16 values
+// (x0: values 0..7, x1: 8..15), fp32 FMAs in order.
+__device__ __forceinline__ float dot16_e4m3_bf16(const uint4 &w, const uint4 &x0,
+                                                 const uint4 &x1) {
+  const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+  const uint32_t xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+  float acc = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 lo = e4m3x2_to_float2(wv[q]);
+    const float2 hi = e4m3x2_to_float2(wv[q] >> 16);
+    acc = fmaf(lo.x, __uint_as_float(xv[2 * q] << 16), acc);
+    acc = fmaf(lo.y, __uint_as_float(xv[2 * q] & 0xffff0000u), acc);
+    acc = fmaf(hi.x, __uint_as_float(xv[2 * q + 1] << 16), acc);
+    acc = fmaf(hi.y, __uint_as_float(xv[2 * q + 1] & 0xffff0000u), acc);
+  }
+  return acc;
+}
+
+// sum over q = 0..15 of e4m3(w[q]) * a[q] for 16 codes and 16 fp32 values
+__device__ __forceinline__ float dot16_e4m3_f32(const uint4 &w, const float4 &a0,
+                                                const float4 &a1, const float4 &a2,
+                                                const float4 &a3) {
+  float acc = 0.f;
+  float2 p = e4m3x2_to_float2(w.x);
+  acc = fmaf(p.x, a0.x, acc);
+  acc = fmaf(p.y, a0.y, acc);
+  p = e4m3x2_to_float2(w.x >> 16);
+  acc = fmaf(p.x, a0.z, acc);
+  acc = fmaf(p.y, a0.w, acc);
+  p = e4m3x2_to_float2(w.y);
+  acc = fmaf(p.x, a1.x, acc);
+  acc = fmaf(p.y, a1.y, acc);
+  p = e4m3x2_to_float2(w.y >> 16);
+  acc = fmaf(p.x, a1.z, acc);
+  acc = fmaf(p.y, a1.w, acc);
+  p = e4m3x2_to_float2(w.z);
+  acc = fmaf(p.x, a2.x, acc);
+  acc = fmaf(p.y, a2.y, acc);
+  p = e4m3x2_to_float2(w.z >> 16);
+  acc = fmaf(p.x, a2.z, acc);
+  acc = fmaf(p.y, a2.w, acc);
+  p = e4m3x2_to_float2(w.w);
+  acc = fmaf(p.x, a3.x, acc);
+  acc = fmaf(p.y, a3.y, acc);
+  p = e4m3x2_to_float2(w.w >> 16);
+  acc = fmaf(p.x, a3.z, acc);
+  acc = fmaf(p.y, a3.w, acc);
+  return acc;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -211,26 +274,28 @@ __device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long
 // stores the activations of the group's pairs.  NQ is a template constant so that the accumulators stay
 // in registers and no instruction is spent on token slots that do not
 // exist; nq < NQ only wastes the predicated slots of the last group.
-template <int NQ, int kU>
+template <int NQ, int kU, bool kFp8>
 __device__ __forceinline__ void phase1_group(const uint4 *__restrict__ g,
                                              const uint4 *__restrict__ u, const uint4 *sx,
                                              const int *plist,
                                              int nq, int k, int H8, int I, int i, float bg,
                                              float bu, bool bias, int act_kind,
-                                             float *__restrict__ act) {
+                                             float *__restrict__ act, const float *sg,
+                                             const float *su, int cpb) {
   const int lane = threadIdx.x & 31;
+  const int HC = kFp8 ? H8 / 2 : H8;  // 16-byte weight chunks per row
   int xo[NQ];  // offsets of the token vectors (T <= 16 tokens, H8 <= 512 chunks)
 #pragma unroll
   for (int q = 0; q < NQ; ++q) xo[q] = plist[q < nq ? q : 0] / k * H8;
   float ag[NQ], au[NQ];
 #pragma unroll
   for (int q = 0; q < NQ; ++q) ag[q] = au[q] = 0.f;
-  for (int base = 0; base < H8; base += 32 * kU) {
+  for (int base = 0; base < HC; base += 32 * kU) {
     uint4 gv[kU], uv[kU];
 #pragma unroll
     for (int j = 0; j < kU; ++j) {
       const int c = base + lane + 32 * j;
-      if (c < H8) {
+      if (c < HC) {
         gv[j] = __ldcs(g + c);
         uv[j] = __ldcs(u + c);
       }
@@ -238,13 +303,26 @@ __device__ __forceinline__ void phase1_group(const uint4 *__restrict__ g,
 #pragma unroll
     for (int j = 0; j < kU; ++j) {
       const int c = base + lane + 32 * j;
-      if (c < H8) {
+      if (c < HC) {
+        if (kFp8) {
+          // 16 codes per chunk, all in one scale block
+          const float sgc = __ldg(sg + c / cpb), suc = __ldg(su + c / cpb);
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          if (q < nq) {
-            const uint4 xv = sx[xo[q] + c];
-            ag[q] = fma8_bf16(gv[j], xv, ag[q]);
-            au[q] = fma8_bf16(uv[j], xv, au[q]);
+          for (int q = 0; q < NQ; ++q) {
+            if (q < nq) {
+              const uint4 x0 = sx[xo[q] + 2 * c], x1 = sx[xo[q] + 2 * c + 1];
+              ag[q] = fmaf(dot16_e4m3_bf16(gv[j], x0, x1), sgc, ag[q]);
+              au[q] = fmaf(dot16_e4m3_bf16(uv[j], x0, x1), suc, au[q]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            if (q < nq) {
+              const uint4 xv = sx[xo[q] + c];
+              ag[q] = fma8_bf16(gv[j], xv, ag[q]);
+              au[q] = fma8_bf16(uv[j], xv, au[q]);
+            }
           }
         }
       }
@@ -266,36 +344,74 @@ __device__ __forceinline__ void phase1_group(const uint4 *__restrict__ g,
 // (ws: in shared memory, else wg: through L2) with act of one pair; the act
 // chunks are loaded once for the kR2 independent sums.  Lane 0 writes
 // sdots[r][pair].
+// FP8 weights: 16 codes per chunk, each chunk's partial sum times the scale
+// of its row and block (s2r: the scales of row r0, ipb per row).
+template <bool kFp8>
 __device__ __forceinline__ void phase2_item(const uint4 *ws, const uint4 *__restrict__ wg,
                                             const float4 *a4, int cache_act, int pair, int r0,
-                                            int nrows, int I, int TK, float *sdots) {
+                                            int nrows, int I, int TK, float *sdots,
+                                            const float *s2r, int ipb, int cpb) {
   const int lane = threadIdx.x & 31;
   const int I8 = I / 8;
   const float4 *a = a4 + static_cast<size_t>(pair) * (I / 4);
-  unsigned long long v[kR2];  // two fp32 partial sums each
+  if constexpr (kFp8) {
+    const int IC = I / 16;
+    float v[kR2];
 #pragma unroll
-  for (int rr = 0; rr < kR2; ++rr) v[rr] = 0ull;
-  for (int base = 0; base < I8; base += 32 * kU2) {
+    for (int rr = 0; rr < kR2; ++rr) v[rr] = 0.f;
+    for (int base = 0; base < IC; base += 32 * kU2) {
 #pragma unroll
-    for (int j = 0; j < kU2; ++j) {
-      const int c = base + lane + 32 * j;
-      if (c < I8) {
-        const float4 a0 = cache_act ? a[2 * c] : __ldcg(a + 2 * c);
-        const float4 a1 = cache_act ? a[2 * c + 1] : __ldcg(a + 2 * c + 1);
+      for (int j = 0; j < kU2; ++j) {
+        const int c = base + lane + 32 * j;
+        if (c < IC) {
+          const float4 a0 = cache_act ? a[4 * c] : __ldcg(a + 4 * c);
+          const float4 a1 = cache_act ? a[4 * c + 1] : __ldcg(a + 4 * c + 1);
+          const float4 a2 = cache_act ? a[4 * c + 2] : __ldcg(a + 4 * c + 2);
+          const float4 a3 = cache_act ? a[4 * c + 3] : __ldcg(a + 4 * c + 3);
 #pragma unroll
-        for (int rr = 0; rr < kR2; ++rr) {
-          if (r0 + rr < nrows) {
-            const uint4 wv = ws != nullptr ? ws[(r0 + rr) * I8 + c] : __ldg(wg + (r0 + rr) * I8 + c);
-            fma8_f32x2(wv, a0, a1, v[rr]);
+          for (int rr = 0; rr < kR2; ++rr) {
+            if (r0 + rr < nrows) {
+              const uint4 wv =
+                  ws != nullptr ? ws[(r0 + rr) * IC + c] : __ldg(wg + (r0 + rr) * IC + c);
+              v[rr] = fmaf(dot16_e4m3_f32(wv, a0, a1, a2, a3), __ldg(s2r + rr * ipb + c / cpb),
+                           v[rr]);
+            }
           }
         }
       }
     }
-  }
 #pragma unroll
-  for (int rr = 0; rr < kR2; ++rr) {
-    const float sv = warp_sum(sum_f32x2(v[rr]));
-    if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
+    for (int rr = 0; rr < kR2; ++rr) {
+      const float sv = warp_sum(v[rr]);
+      if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
+    }
+  } else {
+    unsigned long long v[kR2];  // two fp32 partial sums each
+#pragma unroll
+    for (int rr = 0; rr < kR2; ++rr) v[rr] = 0ull;
+    for (int base = 0; base < I8; base += 32 * kU2) {
+#pragma unroll
+      for (int j = 0; j < kU2; ++j) {
+        const int c = base + lane + 32 * j;
+        if (c < I8) {
+          const float4 a0 = cache_act ? a[2 * c] : __ldcg(a + 2 * c);
+          const float4 a1 = cache_act ? a[2 * c + 1] : __ldcg(a + 2 * c + 1);
+#pragma unroll
+          for (int rr = 0; rr < kR2; ++rr) {
+            if (r0 + rr < nrows) {
+              const uint4 wv =
+                  ws != nullptr ? ws[(r0 + rr) * I8 + c] : __ldg(wg + (r0 + rr) * I8 + c);
+              fma8_f32x2(wv, a0, a1, v[rr]);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int rr = 0; rr < kR2; ++rr) {
+      const float sv = warp_sum(sum_f32x2(v[rr]));
+      if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
+    }
   }
 }
 
@@ -307,27 +423,32 @@ struct SmemLayout {
   size_t w2_off, act_off, dots_off, total;
 };
 
-__host__ __device__ inline size_t w2_slot_bytes(int rows_per_cta, int I) {
-  return (static_cast<size_t>(rows_per_cta) * I * 2 + 127) & ~static_cast<size_t>(127);
+// elem: bytes per weight (2: bf16, 1: FP8)
+__host__ __device__ inline size_t w2_slot_bytes(int rows_per_cta, int I, int elem) {
+  return (static_cast<size_t>(rows_per_cta) * I * elem + 127) & ~static_cast<size_t>(127);
 }
 
 __host__ __device__ inline SmemLayout smem_layout(int T, int TK, int H, int I,
-                                                  int rows_per_cta, int slots, int cache_act) {
+                                                  int rows_per_cta, int slots, int cache_act,
+                                                  int elem) {
   SmemLayout s;
   s.w2_off = static_cast<size_t>(T) * H * 2;
-  s.act_off = s.w2_off + static_cast<size_t>(slots) * w2_slot_bytes(rows_per_cta, I);
+  s.act_off = s.w2_off + static_cast<size_t>(slots) * w2_slot_bytes(rows_per_cta, I, elem);
   s.dots_off = s.act_off + (cache_act ? static_cast<size_t>(TK) * I * sizeof(float) : 0);
   s.total = s.dots_off + static_cast<size_t>(rows_per_cta) * TK * sizeof(float);
   return s;
 }
 
-// kTokens: 1 (decode: the token vector lives in shared memory as bf16 and 8
-// chunks per lane and row are in flight) or kMaxT (up to 16 tokens per
-// expert, token vectors read through L1, 4 chunks in flight).
-template <int kTokens>
+// kTokens: 1 (decode: 8 chunks per lane and row in flight) or kMaxT (up to
+// 16 tokens, taken per expert in groups).  kFp8: the weights are FP8 E4M3
+// codes (16 per 16-byte chunk) with fp32 scales s1 [E, 2I, H / block] and
+// s2 [E, H, I / block]; every chunk's partial dot product is multiplied by
+// the scale of its row and block before it is added.
+template <int kTokens, bool kFp8>
 __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     small_t_kernel(const uint4 *__restrict__ hidden, const uint4 *__restrict__ w1,
-                   const uint4 *__restrict__ w2, const float *__restrict__ b1,
+                   const uint4 *__restrict__ w2, const float *__restrict__ s1,
+                   const float *__restrict__ s2, int block, const float *__restrict__ b1,
                    const float *__restrict__ b2, int act_kind, const float *__restrict__ topk_w,
                    const int32_t *__restrict__ ids, float *__restrict__ act,
                    float *__restrict__ out, int T, int k, int H, int I, int E, int rows_per_cta,
@@ -342,9 +463,13 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   __shared__ uint64_t w2_empty[kMaxSlots];  // every compute warp is done with a slot
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int TK = T * k;
-  const int H8 = H / 8, I8 = I / 8;
-  const SmemLayout lay = smem_layout(T, TK, H, I, rows_per_cta, slots, cache_act);
-  const size_t slot_stride = w2_slot_bytes(rows_per_cta, I);
+  const int H8 = H / 8;
+  constexpr int kElem = kFp8 ? 1 : 2;
+  const int HC = H * kElem / 16, IC = I * kElem / 16;  // 16-byte weight chunks per row
+  const int cpb = kFp8 ? block / 16 : 1;                // chunks per scale block
+  const int hpb = kFp8 ? H / block : 0, ipb = kFp8 ? I / block : 0;  // blocks per row
+  const SmemLayout lay = smem_layout(T, TK, H, I, rows_per_cta, slots, cache_act, kElem);
+  const size_t slot_stride = w2_slot_bytes(rows_per_cta, I, kElem);
   uint8_t *sx = smem;  // the token's vector (one-token kernel)
   uint8_t *sw2 = smem + lay.w2_off;
   float *sact = reinterpret_cast<float *>(smem + lay.act_off);
@@ -369,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   const int nw = gridDim.x * kWarps;
   const int n1 = nd * I;
   // bytes of one expert's rows of this CTA (nrows may be 0 for the last CTAs)
-  const uint32_t w2_bytes = static_cast<uint32_t>(nrows) * I * 2;
+  const uint32_t w2_bytes = static_cast<uint32_t>(nrows) * I * kElem;
   const bool ring = slots > 0 && nrows > 0;
   if (warp == kCopyWarp && lane == 0 && nrows > 0) {
     // the first experts' w2 rows, for phase 2, stream in alongside w1; the
@@ -378,12 +503,12 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     if (ring) {
       for (int d = 0; d < nd && d < slots; ++d) {
         mbar_arrive_expect_tx(&w2_full[d], w2_bytes);
-        bulk_load(sw2 + d * slot_stride, w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * I8,
+        bulk_load(sw2 + d * slot_stride, w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * IC,
                   w2_bytes, &w2_full[d]);
       }
     } else {
       for (int d = 0; d < nd; ++d)
-        bulk_prefetch_l2(w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * I8, w2_bytes);
+        bulk_prefetch_l2(w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * IC, w2_bytes);
     }
   }
 
@@ -391,8 +516,11 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   for (int task = blockIdx.x * kWarps + warp; task < n1 && warp < kWarps; task += nw) {
     const int d = task / I, i = task - d * I;
     const int p0 = L.dstart[d], np = L.dstart[d + 1] - p0;
-    const uint4 *g = w1 + (static_cast<size_t>(L.dexp[d]) * 2 * I + i) * H8;
-    const uint4 *u = g + static_cast<size_t>(I) * H8;
+    const uint4 *g = w1 + (static_cast<size_t>(L.dexp[d]) * 2 * I + i) * HC;
+    const uint4 *u = g + static_cast<size_t>(I) * HC;
+    // FP8: the scale rows of the gate and up rows
+    const float *sg = kFp8 ? s1 + (static_cast<size_t>(L.dexp[d]) * 2 * I + i) * hpb : nullptr;
+    const float *su = kFp8 ? sg + static_cast<size_t>(I) * hpb : nullptr;
     // the variant's bias of this row pair (0 without b1)
     float bg = 0.f, bu = 0.f;
     if (b1 != nullptr) {
@@ -403,12 +531,12 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       // one token: its pairs on e (more than one only for repeated ids) share
       // the same dot products
       float ag = 0.f, au = 0.f;
-      for (int base = 0; base < H8; base += 32 * kU1) {
+      for (int base = 0; base < HC; base += 32 * kU1) {
         uint4 gv[kU1], uv[kU1];
 #pragma unroll
         for (int j = 0; j < kU1; ++j) {
           const int c = base + lane + 32 * j;
-          if (c < H8) {
+          if (c < HC) {
             gv[j] = __ldcs(g + c);
             uv[j] = __ldcs(u + c);
           }
@@ -416,10 +544,16 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
 #pragma unroll
         for (int j = 0; j < kU1; ++j) {
           const int c = base + lane + 32 * j;
-          if (c < H8) {
-            const uint4 xv = reinterpret_cast<const uint4 *>(sx)[c];
-            ag = fma8_bf16(gv[j], xv, ag);
-            au = fma8_bf16(uv[j], xv, au);
+          if (c < HC) {
+            if (kFp8) {
+              const uint4 x0 = sx4[2 * c], x1 = sx4[2 * c + 1];
+              ag = fmaf(dot16_e4m3_bf16(gv[j], x0, x1), __ldg(sg + c / cpb), ag);
+              au = fmaf(dot16_e4m3_bf16(uv[j], x0, x1), __ldg(su + c / cpb), au);
+            } else {
+              const uint4 xv = sx4[c];
+              ag = fma8_bf16(gv[j], xv, ag);
+              au = fma8_bf16(uv[j], xv, au);
+            }
           }
         }
       }
@@ -438,9 +572,11 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
         const int *pl = L.plist + p0 + q0;
         const bool bias = b1 != nullptr;
         if (nq == 1)
-          phase1_group<1, 8>(g, u, sx4, pl, nq, k, H8, I, i, bg, bu, bias, act_kind, act);
+          phase1_group<1, 8, kFp8>(g, u, sx4, pl, nq, k, H8, I, i, bg, bu, bias, act_kind, act,
+                                   sg, su, cpb);
         else
-          phase1_group<4, 4>(g, u, sx4, pl, nq, k, H8, I, i, bg, bu, bias, act_kind, act);
+          phase1_group<4, 4, kFp8>(g, u, sx4, pl, nq, k, H8, I, i, bg, bu, bias, act_kind, act,
+                                   sg, su, cpb);
       }
     }
   }
@@ -495,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
           break;
         }
         mbar_arrive_expect_tx(&w2_full[q], w2_bytes);
-        bulk_load(sw2 + q * slot_stride, w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * I8,
+        bulk_load(sw2 + q * slot_stride, w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * IC,
                   w2_bytes, &w2_full[q]);
         issued = d + 1;
       }
@@ -521,9 +657,10 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       const int pq = it / rgroups, rg = it - pq * rgroups;  // pq: position in plist
       const int pair = L.plist[pq];
       const int d = L.pd[pair];
-      phase2_item(ring ? reinterpret_cast<const uint4 *>(sw2 + d * slot_stride) : nullptr,
-                  w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * I8, act4, cache_act, pair,
-                  rg * kR2, nrows, I, TK, sdots);
+      const size_t row0 = static_cast<size_t>(L.dexp[d]) * H + h0;  // w2 row of local row 0
+      phase2_item<kFp8>(ring ? reinterpret_cast<const uint4 *>(sw2 + d * slot_stride) : nullptr,
+                        w2 + row0 * IC, act4, cache_act, pair, rg * kR2, nrows, I, TK, sdots,
+                        kFp8 ? s2 + (row0 + rg * kR2) * ipb : nullptr, ipb, cpb);
     }
   } else if (rgroups > 0) {
     // more experts than slots: take the experts in order, waiting for each
@@ -543,8 +680,10 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       if (it < 0) it += kWarps;
       for (; it < n_items; it += kWarps) {
         const int pq = p0 + it / rgroups, rg = it % rgroups;
-        phase2_item(reinterpret_cast<const uint4 *>(sw2 + q * slot_stride), nullptr, act4,
-                    cache_act, L.plist[pq], rg * kR2, nrows, I, TK, sdots);
+        const size_t row0 = static_cast<size_t>(L.dexp[d]) * H + h0;
+        phase2_item<kFp8>(reinterpret_cast<const uint4 *>(sw2 + q * slot_stride), nullptr, act4,
+                          cache_act, L.plist[pq], rg * kR2, nrows, I, TK, sdots,
+                          kFp8 ? s2 + (row0 + rg * kR2) * ipb : nullptr, ipb, cpb);
       }
       before += n_items;
       __syncwarp();
@@ -583,12 +722,13 @@ struct SmallTConfig {
 // slots as there can be distinct experts (at most kMaxSlots), and the act
 // cache when it fits beside them -- unless it would leave fewer than two
 // slots (no overlap of copies and dot products) where dropping it gives more.
-SmallTConfig small_t_config(int T, int TK, int H, int I, int E, int grid, size_t budget) {
+SmallTConfig small_t_config(int T, int TK, int H, int I, int E, int grid, size_t budget,
+                            int elem) {
   SmallTConfig c;
   c.rows_per_cta = (H + grid - 1) / grid;
   const int want = std::min(std::min(TK, E), kMaxSlots);
   auto size = [&](int slots, int cache) {
-    return smem_layout(T, TK, H, I, c.rows_per_cta, slots, cache).total;
+    return smem_layout(T, TK, H, I, c.rows_per_cta, slots, cache, elem).total;
   };
   auto fit = [&](int cache) {
     int n = want;
@@ -626,7 +766,8 @@ size_t smem_budget(int dev, const void *kern) {
 
 bool small_t_supported(int H, int I) { return H <= kMaxH && I <= kMaxI; }
 
-cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w2,
+cudaError_t launch_small_t(const uint16_t *hidden, const void *w1, const void *w2,
+                           const float *w1_scale, const float *w2_scale, int block,
                            const float *b1, const float *b2, int act_kind,
                            const float *topk_weights, const int32_t *topk_ids, float *act,
                            float *out, int64_t T, int H, int I, int E, int k, uint32_t *status,
@@ -647,12 +788,15 @@ cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uin
     if (!((ready_mask >> dev) & 1)) {
       // every CTA must be resident at once (the grid barrier): the grid is
       // the number of CTAs both kernels can keep on every SM
-      const size_t smem = std::min(smem_budget(dev, reinterpret_cast<const void *>(small_t_kernel<1>)),
-                                   smem_budget(dev, reinterpret_cast<const void *>(small_t_kernel<kMaxT>)));
+      const auto kerns = {small_t_kernel<1, false>, small_t_kernel<kMaxT, false>,
+                          small_t_kernel<1, true>, small_t_kernel<kMaxT, true>};
+      size_t smem = ~static_cast<size_t>(0);
+      for (auto kern : kerns)
+        smem = std::min(smem, smem_budget(dev, reinterpret_cast<const void *>(kern)));
       if (smem < 16384) return cudaErrorInvalidValue;
       budget_of[dev] = smem;
       int per_sm = kBlocksPerSm;
-      for (auto kern : {small_t_kernel<1>, small_t_kernel<kMaxT>}) {
+      for (auto kern : kerns) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem));
         if (e != cudaSuccess) return e;
@@ -667,8 +811,12 @@ cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uin
     }
   }
   const int grid = grid_of[dev];
+  const bool fp8 = block > 0;
+  if (fp8 && (w1_scale == nullptr || w2_scale == nullptr || block % 16 != 0 || H % block != 0 ||
+              I % block != 0))
+    return cudaErrorInvalidValue;
   const SmallTConfig cfg = small_t_config(static_cast<int>(T), static_cast<int>(T) * k, H, I, E,
-                                          grid, budget_of[dev]);
+                                          grid, budget_of[dev], fp8 ? 1 : 2);
   if (cfg.smem > budget_of[dev]) return cudaErrorInvalidValue;
   // each CTA adds one to the grid-sync counter per launch: the target is the
   // arrivals of all earlier launches plus this grid
@@ -683,11 +831,12 @@ cudaError_t launch_small_t(const uint16_t *hidden, const uint16_t *w1, const uin
   attr[0].val.cooperative = 1;
   lc.attrs = attr;
   lc.numAttrs = 1;
-  hook.begin("small_t");
-  e = cudaLaunchKernelEx(&lc, T == 1 ? small_t_kernel<1> : small_t_kernel<kMaxT>,
-                         reinterpret_cast<const uint4 *>(hidden),
+  hook.begin(fp8 ? "small_t_fp8" : "small_t");
+  auto kern = fp8 ? (T == 1 ? small_t_kernel<1, true> : small_t_kernel<kMaxT, true>)
+                  : (T == 1 ? small_t_kernel<1, false> : small_t_kernel<kMaxT, false>);
+  e = cudaLaunchKernelEx(&lc, kern, reinterpret_cast<const uint4 *>(hidden),
                          reinterpret_cast<const uint4 *>(w1), reinterpret_cast<const uint4 *>(w2),
-                         b1, b2, act_kind, topk_weights, topk_ids, act, out, static_cast<int>(T), k, H, I, E,
+                         w1_scale, w2_scale, block, b1, b2, act_kind, topk_weights, topk_ids, act, out, static_cast<int>(T), k, H, I, E,
                          cfg.rows_per_cta, cfg.slots, cfg.cache_act, status,
                          grid_sync, target,
                          wait_limit_ns);

@@ -103,6 +103,25 @@ def test_forward_ex_argument_checks(kw, code):
     assert fwd_ex(**kw) == code
 
 
+def fwd_fp8(s1=256, s2=256, block=128, **kw):
+    a = dict(FWD_OK, **kw)
+    return L.moe_forward_fp8(a["h"], a["w1"], s1, a["w2"], s2, block, a["w"], a["ids"], a["out"],
+                             a["T"], a["H"], a["I"], a["E"], a["k"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(s1=NULL), moe.MOE_ERR_INVALID_ARG),      # scales missing
+    (dict(s2=NULL), moe.MOE_ERR_INVALID_ARG),
+    (dict(block=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(block=64), moe.MOE_ERR_UNSUPPORTED),     # not a multiple of 128
+    (dict(block=256, I=128), moe.MOE_ERR_UNSUPPORTED),  # does not divide I
+    (dict(w1=260), moe.MOE_ERR_INVALID_ARG),       # codes not 16-byte aligned
+    (dict(T=0, h=NULL, out=NULL), moe.MOE_OK),
+])
+def test_forward_fp8_argument_checks(kw, code):
+    assert fwd_fp8(**kw) == code
+
+
 def test_binding_rejects_unknown_activation():
     import torch
     t = torch.empty(0)
@@ -134,3 +153,4 @@ def test_no_gpu_fails_loudly():
     assert L.moe_route(1, 4, 8, 2, 1, 1, 1, None) == moe.MOE_ERR_NO_DEVICE
     assert fwd() == moe.MOE_ERR_NO_DEVICE
     assert fwd_ex(act=1, b1=256, b2=256) == moe.MOE_ERR_NO_DEVICE
+    assert fwd_fp8() == moe.MOE_ERR_NO_DEVICE

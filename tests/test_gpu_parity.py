@@ -364,6 +364,60 @@ def test_forward_ex_default_equals_forward():
     assert torch.equal(a, b)
 
 
+# ------------------------------------------------------------------ FP8 weights
+def gpu_forward_fp8(hidden, q1, s1, q2, s2, block, w, ids):
+    dev = torch.device("cuda")
+    out = torch.full((hidden.shape[0], hidden.shape[1]), float("nan"), device=dev)
+    out = moe.moe_forward_fp8(hidden.to(dev), q1.to(dev), s1.to(dev), q2.to(dev), s2.to(dev),
+                              block, torch.as_tensor(np.asarray(w, np.float32)).to(dev),
+                              torch.as_tensor(np.asarray(ids, np.int32)).to(dev), out=out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+@pytest.mark.parametrize("T,H,I,E,k,block,path", [
+    (1, 2048, 768, 128, 8, 256, "small_t"),    # decode
+    (4, 2048, 768, 128, 8, 128, "small_t"),    # several tokens, blocks of 128
+    (3, 512, 256, 4, 2, 256, "small_t"),       # tokens sharing experts
+    (4, 2048, 768, 128, 8, 256, "gemm"),
+    (64, 256, 128, 8, 2, 128, "gemm"),         # tiny: one-launch GEMMs
+    (100, 384, 384, 16, 4, 128, "gemm"),       # k > 2: P and combine, half n-tile
+])
+def test_forward_fp8(T, H, I, E, k, block, path):
+    from moe_inputs import make_fp8_weights
+    hidden, _, _, logits = make_inputs(T, H, I, E, seed=60 + T)
+    q1, s1, q2, s2 = make_fp8_weights(E, H, I, block, seed=T)
+    ids, w = oracle.route(logits.numpy(), k, True)
+    ref = oracle.moe_token_loop_fp8(hidden, q1, s1, q2, s2, block, w, ids)
+    prev = moe.set_small_t_max(16 if path == "small_t" else 0)
+    try:
+        out = gpu_forward_fp8(hidden, q1, s1, q2, s2, block, w, ids)
+    finally:
+        moe.set_small_t_max(prev)
+    assert_output_close(out, ref, f"T={T} H={H} I={I} E={E} k={k} block={block} {path}")
+    check_status_clean()
+
+
+@pytest.mark.parametrize("name,block", [("decode", 256), ("prefill_8e", 256),
+                                        ("prefill_thin", 128)])
+def test_forward_fp8_full_size(name, block):
+    from moe_inputs import make_fp8_weights
+    s = SHAPES[name]
+    hidden, _, _, logits = make_shape_inputs(s, device="cuda")
+    q1, s1, q2, s2 = make_fp8_weights(s.E, s.H, s.I, block, seed=5, device="cuda")
+    ids_r, w_r = oracle.route(logits.cpu().numpy(), s.k, True)
+    out = moe.moe_forward_fp8(hidden, q1, s1, q2, s2, block,
+                              torch.as_tensor(w_r.astype(np.float32)).cuda(),
+                              torch.as_tensor(ids_r).cuda())
+    torch.cuda.synchronize()
+    rows = np.arange(s.T) if s.T <= 64 else _sample_rows(s.T, 6, 7)
+    ref = oracle.moe_token_loop_fp8(hidden.cpu(), q1.cpu(), s1.cpu(), q2.cpu(), s2.cpu(), block,
+                                    w_r, ids_r, rows=rows)
+    assert_output_close(out.cpu().numpy()[rows], ref, f"{name} fp8")
+    check_status_clean()
+    assert torch.isfinite(out).all()
+
+
 # ------------------------------------------------------------------ full-size workloads
 def _sample_rows(T, n, seed):
     rng = np.random.default_rng(seed)
