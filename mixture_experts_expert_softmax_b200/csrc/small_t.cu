@@ -206,54 +206,56 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two) {
 }
 
 // sum over q = 0..15 of e4m3(w[q]) * x[q] for 16 codes and 16 bf16 values
-// (x0: values 0..7, x1: 8..15), fp32 FMAs in order.
+// (x0: values 0..7, x1: 8..15): fp32 FMAs into two interleaved partial
+// sums (halving the dependent chain), added at the end.
 __device__ __forceinline__ float dot16_e4m3_bf16(const uint4 &w, const uint4 &x0,
                                                  const uint4 &x1) {
   const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
   const uint32_t xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-  float acc = 0.f;
+  float s0 = 0.f, s1 = 0.f;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const float2 lo = e4m3x2_to_float2(wv[q]);
     const float2 hi = e4m3x2_to_float2(wv[q] >> 16);
-    acc = fmaf(lo.x, __uint_as_float(xv[2 * q] << 16), acc);
-    acc = fmaf(lo.y, __uint_as_float(xv[2 * q] & 0xffff0000u), acc);
-    acc = fmaf(hi.x, __uint_as_float(xv[2 * q + 1] << 16), acc);
-    acc = fmaf(hi.y, __uint_as_float(xv[2 * q + 1] & 0xffff0000u), acc);
+    s0 = fmaf(lo.x, __uint_as_float(xv[2 * q] << 16), s0);
+    s1 = fmaf(lo.y, __uint_as_float(xv[2 * q] & 0xffff0000u), s1);
+    s0 = fmaf(hi.x, __uint_as_float(xv[2 * q + 1] << 16), s0);
+    s1 = fmaf(hi.y, __uint_as_float(xv[2 * q + 1] & 0xffff0000u), s1);
   }
-  return acc;
+  return s0 + s1;
 }
 
-// sum over q = 0..15 of e4m3(w[q]) * a[q] for 16 codes and 16 fp32 values
+// sum over q = 0..15 of e4m3(w[q]) * a[q] for 16 codes and 16 fp32 values,
+// two interleaved partial sums
 __device__ __forceinline__ float dot16_e4m3_f32(const uint4 &w, const float4 &a0,
                                                 const float4 &a1, const float4 &a2,
                                                 const float4 &a3) {
-  float acc = 0.f;
+  float s0 = 0.f, s1 = 0.f;
   float2 p = e4m3x2_to_float2(w.x);
-  acc = fmaf(p.x, a0.x, acc);
-  acc = fmaf(p.y, a0.y, acc);
+  s0 = fmaf(p.x, a0.x, s0);
+  s1 = fmaf(p.y, a0.y, s1);
   p = e4m3x2_to_float2(w.x >> 16);
-  acc = fmaf(p.x, a0.z, acc);
-  acc = fmaf(p.y, a0.w, acc);
+  s0 = fmaf(p.x, a0.z, s0);
+  s1 = fmaf(p.y, a0.w, s1);
   p = e4m3x2_to_float2(w.y);
-  acc = fmaf(p.x, a1.x, acc);
-  acc = fmaf(p.y, a1.y, acc);
+  s0 = fmaf(p.x, a1.x, s0);
+  s1 = fmaf(p.y, a1.y, s1);
   p = e4m3x2_to_float2(w.y >> 16);
-  acc = fmaf(p.x, a1.z, acc);
-  acc = fmaf(p.y, a1.w, acc);
+  s0 = fmaf(p.x, a1.z, s0);
+  s1 = fmaf(p.y, a1.w, s1);
   p = e4m3x2_to_float2(w.z);
-  acc = fmaf(p.x, a2.x, acc);
-  acc = fmaf(p.y, a2.y, acc);
+  s0 = fmaf(p.x, a2.x, s0);
+  s1 = fmaf(p.y, a2.y, s1);
   p = e4m3x2_to_float2(w.z >> 16);
-  acc = fmaf(p.x, a2.z, acc);
-  acc = fmaf(p.y, a2.w, acc);
+  s0 = fmaf(p.x, a2.z, s0);
+  s1 = fmaf(p.y, a2.w, s1);
   p = e4m3x2_to_float2(w.w);
-  acc = fmaf(p.x, a3.x, acc);
-  acc = fmaf(p.y, a3.y, acc);
+  s0 = fmaf(p.x, a3.x, s0);
+  s1 = fmaf(p.y, a3.y, s1);
   p = e4m3x2_to_float2(w.w >> 16);
-  acc = fmaf(p.x, a3.z, acc);
-  acc = fmaf(p.y, a3.w, acc);
-  return acc;
+  s0 = fmaf(p.x, a3.z, s0);
+  s1 = fmaf(p.y, a3.w, s1);
+  return s0 + s1;
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -292,12 +294,17 @@ __device__ __forceinline__ void phase1_group(const uint4 *__restrict__ g,
   for (int q = 0; q < NQ; ++q) ag[q] = au[q] = 0.f;
   for (int base = 0; base < HC; base += 32 * kU) {
     uint4 gv[kU], uv[kU];
+    float sgv[kU], suv[kU];  // FP8: the chunks' scales, loaded with the codes
 #pragma unroll
     for (int j = 0; j < kU; ++j) {
       const int c = base + lane + 32 * j;
       if (c < HC) {
         gv[j] = __ldcs(g + c);
         uv[j] = __ldcs(u + c);
+        if (kFp8) {
+          sgv[j] = __ldg(sg + c / cpb);
+          suv[j] = __ldg(su + c / cpb);
+        }
       }
     }
 #pragma unroll
@@ -306,13 +313,12 @@ __device__ __forceinline__ void phase1_group(const uint4 *__restrict__ g,
       if (c < HC) {
         if (kFp8) {
           // 16 codes per chunk, all in one scale block
-          const float sgc = __ldg(sg + c / cpb), suc = __ldg(su + c / cpb);
 #pragma unroll
           for (int q = 0; q < NQ; ++q) {
             if (q < nq) {
               const uint4 x0 = sx[xo[q] + 2 * c], x1 = sx[xo[q] + 2 * c + 1];
-              ag[q] = fmaf(dot16_e4m3_bf16(gv[j], x0, x1), sgc, ag[q]);
-              au[q] = fmaf(dot16_e4m3_bf16(uv[j], x0, x1), suc, au[q]);
+              ag[q] = fmaf(dot16_e4m3_bf16(gv[j], x0, x1), sgv[j], ag[q]);
+              au[q] = fmaf(dot16_e4m3_bf16(uv[j], x0, x1), suv[j], au[q]);
             }
           }
         } else {
@@ -360,6 +366,16 @@ __device__ __forceinline__ void phase2_item(const uint4 *ws, const uint4 *__rest
 #pragma unroll
     for (int rr = 0; rr < kR2; ++rr) v[rr] = 0.f;
     for (int base = 0; base < IC; base += 32 * kU2) {
+      // the scales of this lane's chunks, loaded ahead of the dot products
+      float sc[kU2][kR2];
+#pragma unroll
+      for (int j = 0; j < kU2; ++j) {
+        const int c = base + lane + 32 * j;
+#pragma unroll
+        for (int rr = 0; rr < kR2; ++rr)
+          // s2r may point into shared memory: a generic load
+          sc[j][rr] = c < IC && r0 + rr < nrows ? s2r[rr * ipb + c / cpb] : 0.f;
+      }
 #pragma unroll
       for (int j = 0; j < kU2; ++j) {
         const int c = base + lane + 32 * j;
@@ -373,8 +389,7 @@ __device__ __forceinline__ void phase2_item(const uint4 *ws, const uint4 *__rest
             if (r0 + rr < nrows) {
               const uint4 wv =
                   ws != nullptr ? ws[(r0 + rr) * IC + c] : __ldg(wg + (r0 + rr) * IC + c);
-              v[rr] = fmaf(dot16_e4m3_f32(wv, a0, a1, a2, a3), __ldg(s2r + rr * ipb + c / cpb),
-                           v[rr]);
+              v[rr] = fmaf(dot16_e4m3_f32(wv, a0, a1, a2, a3), sc[j][rr], v[rr]);
             }
           }
         }
@@ -455,7 +470,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
                    int slots, int cache_act, uint32_t *status,
                    unsigned long long *grid_sync,
                    unsigned long long sync_target, uint64_t limit) {
-  constexpr int kU1 = kTokens == 1 ? 8 : 4;  // phase 1: chunks per lane and row in flight
+  // phase 1: chunks per lane and row in flight (an FP8 chunk holds 16 codes)
+  constexpr int kU1 = kFp8 ? 4 : (kTokens == 1 ? 8 : 4);
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ Lists L;
   __shared__ volatile int s_abort;
@@ -533,12 +549,17 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       float ag = 0.f, au = 0.f;
       for (int base = 0; base < HC; base += 32 * kU1) {
         uint4 gv[kU1], uv[kU1];
+        float sgv[kU1], suv[kU1];  // FP8: the chunks' scales, loaded with the codes
 #pragma unroll
         for (int j = 0; j < kU1; ++j) {
           const int c = base + lane + 32 * j;
           if (c < HC) {
             gv[j] = __ldcs(g + c);
             uv[j] = __ldcs(u + c);
+            if (kFp8) {
+              sgv[j] = __ldg(sg + c / cpb);
+              suv[j] = __ldg(su + c / cpb);
+            }
           }
         }
 #pragma unroll
@@ -547,8 +568,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
           if (c < HC) {
             if (kFp8) {
               const uint4 x0 = sx4[2 * c], x1 = sx4[2 * c + 1];
-              ag = fmaf(dot16_e4m3_bf16(gv[j], x0, x1), __ldg(sg + c / cpb), ag);
-              au = fmaf(dot16_e4m3_bf16(uv[j], x0, x1), __ldg(su + c / cpb), au);
+              ag = fmaf(dot16_e4m3_bf16(gv[j], x0, x1), sgv[j], ag);
+              au = fmaf(dot16_e4m3_bf16(uv[j], x0, x1), suv[j], au);
             } else {
               const uint4 xv = sx4[c];
               ag = fma8_bf16(gv[j], xv, ag);
@@ -572,8 +593,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
         const int *pl = L.plist + p0 + q0;
         const bool bias = b1 != nullptr;
         if (nq == 1)
-          phase1_group<1, 8, kFp8>(g, u, sx4, pl, nq, k, H8, I, i, bg, bu, bias, act_kind, act,
-                                   sg, su, cpb);
+          phase1_group<1, kFp8 ? 4 : 8, kFp8>(g, u, sx4, pl, nq, k, H8, I, i, bg, bu, bias,
+                                              act_kind, act, sg, su, cpb);
         else
           phase1_group<4, 4, kFp8>(g, u, sx4, pl, nq, k, H8, I, i, bg, bu, bias, act_kind, act,
                                    sg, su, cpb);
@@ -658,9 +679,10 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       const int pair = L.plist[pq];
       const int d = L.pd[pair];
       const size_t row0 = static_cast<size_t>(L.dexp[d]) * H + h0;  // w2 row of local row 0
+      const float *s2r = kFp8 ? s2 + (row0 + rg * kR2) * ipb : nullptr;  // FP8 scales
       phase2_item<kFp8>(ring ? reinterpret_cast<const uint4 *>(sw2 + d * slot_stride) : nullptr,
                         w2 + row0 * IC, act4, cache_act, pair, rg * kR2, nrows, I, TK, sdots,
-                        kFp8 ? s2 + (row0 + rg * kR2) * ipb : nullptr, ipb, cpb);
+                        s2r, ipb, cpb);
     }
   } else if (rgroups > 0) {
     // more experts than slots: take the experts in order, waiting for each
