@@ -41,8 +41,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from moe_inputs import (SHAPES, TABLE_SHAPES, MoEShape, make_shape_inputs,  # noqa: E402
-                        PAGE_T_PROD_US as TABLE_T_PROD_US)
+from moe_inputs import (SHAPES, TABLE_SHAPES, MoEShape, make_fp8_weights,  # noqa: E402
+                        make_shape_inputs, PAGE_T_PROD_US as TABLE_T_PROD_US)
 
 METRIC = "fused-MoE µs/call, TFLOP/s and % of roofline per shape; T=1 decode HBM GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -65,9 +65,12 @@ def load_peaks():
         return dict(FALLBACK_PEAKS, source="fallback")
 
 
-def algorithmic_bytes(s: MoEShape, n_active: int) -> float:
-    """Activated expert weights + bf16 hidden + ids/weights + fp32 output."""
-    return n_active * 3.0 * s.H * s.I * 2 + s.T * s.H * 2 + s.T * s.k * 8 + s.T * s.H * 4
+def algorithmic_bytes(s: MoEShape, n_active: int, fp8_block: int = 0) -> float:
+    """Activated expert weights (bf16, or FP8 codes plus one fp32 scale per
+    block) + bf16 hidden + ids/weights + fp32 output."""
+    n_w = n_active * 3.0 * s.H * s.I
+    w_bytes = n_w * 2 if fp8_block == 0 else n_w + n_w / fp8_block * 4
+    return w_bytes + s.T * s.H * 2 + s.T * s.k * 8 + s.T * s.H * 4
 
 
 def roofline_us(s: MoEShape, n_active: int, peaks) -> tuple[float, str]:
@@ -207,6 +210,16 @@ def run_ours(args, ws, rank, local):
     peaks = load_peaks()
     s = SHAPES[args.workload]
     hidden, w1, w2, logits = make_shape_inputs(s, seed=0, device=str(dev))
+    fp8 = args.weights == "fp8"
+    if fp8:
+        q1, s1, q2, s2 = make_fp8_weights(s.E, s.H, s.I, args.fp8_block, seed=0, device=str(dev))
+        del w1, w2
+
+        def forward(h, wts_, ids_, out_):
+            moe.moe_forward_fp8(h, q1, s1, q2, s2, args.fp8_block, wts_, ids_, out_)
+    else:
+        def forward(h, wts_, ids_, out_):
+            moe.moe_forward(h, w1, w2, wts_, ids_, out_)
     stream = torch.cuda.current_stream()
     flush_buf = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_read = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -226,7 +239,7 @@ def run_ours(args, ws, rank, local):
         moe.moe_route(logits, s.k, True, ids, wts)
         if ev is not None:
             ev[1].record(stream)
-        moe.moe_forward(hidden, w1, w2, wts, ids, out)
+        forward(hidden, wts, ids, out)
         if ev is not None:
             ev[2].record(stream)
 
@@ -260,16 +273,16 @@ def run_ours(args, ws, rank, local):
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": round(achieved / peaks["bf16_tflops"], 4),
                 "peak_source": f"{peaks['source']} bf16 dense (burst)",
-                "traffic": traffic_from_profile(top, args.workload),
+                "traffic": None if fp8 else traffic_from_profile(top, args.workload),
                 "algorithmic_flops_per_launch": kernel_flops[top]}
     else:
-        gb = algorithmic_bytes(s, n_active)
+        gb = algorithmic_bytes(s, n_active, args.fp8_block if fp8 else 0)
         achieved = gb / (kernels[top]["avg_us"] * 1e-6) / 1e9
         roof = {"kernel": top, "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "peak_source": f"{peaks['source']} HBM copy",
-                "traffic": traffic_from_profile(top, args.workload)}
+                "traffic": None if fp8 else traffic_from_profile(top, args.workload)}
 
     # end to end through the public API with host buffers
     h_hidden = hidden.cpu().pin_memory()
@@ -284,7 +297,7 @@ def run_ours(args, ws, rank, local):
         d_hidden.copy_(h_hidden, non_blocking=True)
         d_logits.copy_(h_logits, non_blocking=True)
         moe.moe_route(d_logits, s.k, True, ids, wts)
-        moe.moe_forward(d_hidden, w1, w2, wts, ids, out)
+        forward(d_hidden, wts, ids, out)
         h_out.copy_(out, non_blocking=True)
         if ev is not None:
             ev[1].record(stream)
@@ -314,12 +327,15 @@ def run_ours(args, ws, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "fp8-e4m3 weights, bf16 activations" if fp8 else "bf16",
         "data": "synthetic (seeded randn, shapes and scales of atrex-bench #009 input.py)",
         "config": {"workload": s.name, "T": s.T, "H": s.H, "I": s.I, "E": s.E, "top_k": s.k,
                    "renorm": True, "active_experts": n_active,
+                   "weights": (f"fp8 e4m3 codes, fp32 scale per {args.fp8_block} contraction "
+                               "elements" if fp8 else "bf16"),
                    "l2": "flushed between steps (256 MiB write + 256 MiB read, untimed)",
-                   "step": "moe_route + moe_forward", "parallelism": f"replicas x{ws}"},
+                   "step": "moe_route + " + ("moe_forward_fp8" if fp8 else "moe_forward"),
+                   "parallelism": f"replicas x{ws}"},
         "roofline": roof,
         "kernels": {k: {"launches": v["launches"], "avg_us": round(v["avg_us"], 2)}
                     for k, v in kernels.items()},
@@ -337,7 +353,8 @@ def run_ours(args, ws, rank, local):
     if per_shape:
         line["per_shape"] = per_shape
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(s, hidden, w1, w2, logits, budget_s=args.cpu_seconds)
+        wa, wb = ((q1, s1, args.fp8_block), (q2, s2, args.fp8_block)) if fp8 else (w1, w2)
+        line["cpu_baseline"] = cpu_baseline(s, hidden, wa, wb, logits, budget_s=args.cpu_seconds)
     return line
 
 
@@ -374,12 +391,18 @@ def measure_shapes(moe, dev, peaks, flush, stream, shapes, page_us, K=10, W=3):
 
 # ------------------------------------------------------------------ oracle (CPU)
 def oracle_sample(s, hidden, w1, w2, logits, rows):
+    """Seconds of the oracle's forward on the listed tokens; w1/w2 are the
+    bf16 weights, or (codes, scales, block) triples of FP8 weights."""
     import oracle
     sel = torch.as_tensor(rows, dtype=torch.long)
     ids, w = oracle.route(logits[sel].numpy(), s.k, True)
     h = hidden[sel]
     t0 = time.perf_counter()
-    oracle.moe_token_loop(h, w1, w2, w, ids)
+    if isinstance(w1, tuple):
+        (q1, s1, block), (q2, s2, _) = w1, w2
+        oracle.moe_token_loop_fp8(h, q1, s1, q2, s2, block, w, ids)
+    else:
+        oracle.moe_token_loop(h, w1, w2, w, ids)
     return time.perf_counter() - t0
 
 
@@ -395,7 +418,12 @@ def calibrate_rows(s, hidden, w1, w2, logits, budget_s):
 
 def cpu_baseline(s, hidden, w1, w2, logits, budget_s=10.0):
     import oracle
-    hidden, w1, w2, logits = hidden.cpu(), w1.cpu(), w2.cpu(), logits.cpu()
+
+    def host(w):
+        return tuple(x.cpu() if torch.is_tensor(x) else x for x in w) if isinstance(w, tuple) \
+            else w.cpu()
+
+    hidden, w1, w2, logits = hidden.cpu(), host(w1), host(w2), logits.cpu()
     n, threads = calibrate_rows(s, hidden, w1, w2, logits, budget_s)
     rows = np.arange(n)
     dt = oracle_sample(s, hidden, w1, w2, logits, rows)
@@ -462,6 +490,10 @@ def main():
                     help="per-shape table: the five workloads, every row of the page's "
                          "shapes table, or none")
     ap.add_argument("--no-shapes", action="store_true", help="same as --shapes none")
+    ap.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
+                    help="expert weights: bf16, or FP8 E4M3 codes with fp32 scales per "
+                         "--fp8-block contraction elements (moe_forward_fp8)")
+    ap.add_argument("--fp8-block", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
