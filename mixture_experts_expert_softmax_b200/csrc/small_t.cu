@@ -9,20 +9,28 @@
 //   phase 1 (gate/up + SwiGLU): the work items are (distinct chosen expert,
 //     row i) row pairs -- gate row w1[e, i, :] and up row w1[e, I+i, :] --
 //     dealt round-robin to every warp of the grid.  A warp dots both rows
-//     with the hidden vector of each token routed to e and stores
-//     act[t*k + j, i] = silu(g) * u in fp32 (global memory) -- or the
-//     variant's activation of g + b1[e, i] and u + b1[e, I + i].
-//     Meanwhile the copy warp moves the w2 rows this CTA needs in phase 2
-//     into shared memory with bulk copies (or, when they do not fit, asks L2
-//     to prefetch them), so w2 streams from HBM alongside w1.  Bulk copies
-//     can stall the issuing warp for microseconds while the copy engine is
-//     busy, which is why a warp of its own issues them.
+//     with the vectors (staged in shared memory) of the tokens routed to e,
+//     in groups of up to four, and stores act[t*k + j, i] = silu(g) * u in
+//     fp32 (global memory) -- or the variant's activation of g + b1[e, i]
+//     and u + b1[e, I + i].  Meanwhile the copy warp moves the w2 rows this
+//     CTA needs in phase 2 into a ring of shared-memory slots (one chosen
+//     expert per slot) with bulk copies, so w2 streams from HBM alongside
+//     w1; when one expert's rows do not fit, it asks L2 to prefetch them.
+//     Bulk copies can stall the issuing warp for microseconds while the copy
+//     engine is busy, which is why a warp of its own issues them.
 //   grid barrier: every CTA has written its act values (bounded wait).
 //   phase 2 (down + weighted combine): each CTA owns a slice of output rows
-//     h; a warp dots w2[e][h, :] (now on chip) with act of every pair of e,
-//     one pair and four rows h at a time (four independent sums), and
-//     out[t, h] = sum_{j=0..k-1} w[t, j] * (dot_j + b2[e_j, h]) is summed in
-//     fixed j order (b2 only when given) -- deterministic, no extra buffer.
+//     h; a warp dots w2[e][h, :] (on chip) with act of every pair of e, one
+//     pair and four rows h at a time (four independent sums); with more
+//     chosen experts than slots, the copy warp refills a slot as soon as
+//     every compute warp has released it.  out[t, h] = sum_{j=0..k-1}
+//     w[t, j] * (dot_j + b2[e_j, h]) is summed in fixed j order (b2 only
+//     when given) -- deterministic, no extra buffer.
+//
+// FP8 weights (the sub-channel quantisation of the 0.13.2 page): w1 and w2
+// hold E4M3 codes, 16 per 16-byte chunk, converted by the hardware; each
+// chunk's fp32 partial dot product is multiplied by the scale of its row
+// and block before it is added, and the slots hold codes (half the bytes).
 //
 // Same function as ref_moe on the page "tpu_inference/kernels/fused_moe/v1/
 // kernel.py" (per token: x.[W_gate|W_up] -> silu(gate)*up -> .W2, weighted
