@@ -22,8 +22,6 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-__device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
-
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
@@ -144,15 +142,6 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *s
                : "memory");
 }
 
-// 1-D bulk copy shared -> global (bulk-group completion).  Both addresses
-// 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                   reinterpret_cast<uint64_t>(dst)),
-               "r"(smem_addr(src)), "r"(bytes)
-               : "memory");
-}
-
 // 1-D bulk reduction shared -> global: dst[i] += src[i] for bytes / 4 fp32
 // values, performed at L2 (bulk-group completion).  Both addresses 16-byte
 // aligned, bytes a multiple of 16.
@@ -190,15 +179,6 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint3
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
                : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void cp_async_wait_all() {
