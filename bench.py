@@ -73,9 +73,9 @@ def algorithmic_bytes(s: MoEShape, n_active: int, fp8_block: int = 0) -> float:
     return w_bytes + s.T * s.H * 2 + s.T * s.k * 8 + s.T * s.H * 4
 
 
-def roofline_us(s: MoEShape, n_active: int, peaks) -> tuple[float, str]:
+def roofline_us(s: MoEShape, n_active: int, peaks, fp8_block: int = 0) -> tuple[float, str]:
     t_flop = s.flops / (peaks["bf16_tflops"] * 1e12) * 1e6
-    t_mem = algorithmic_bytes(s, n_active) / (peaks["hbm_gbs"] * 1e9) * 1e6
+    t_mem = algorithmic_bytes(s, n_active, fp8_block) / (peaks["hbm_gbs"] * 1e9) * 1e6
     return (t_flop, "tensor") if t_flop >= t_mem else (t_mem, "hbm")
 
 
@@ -309,10 +309,13 @@ def run_ours(args, ws, rank, local):
     d2h = h_out.numel() * 4
 
     per_shape = {}
+    fb = args.fp8_block if fp8 else 0
     if args.shapes == "workloads":
-        per_shape = measure_shapes(moe, dev, peaks, flush, stream, SHAPES, PAGE_T_PROD_US)
+        per_shape = measure_shapes(moe, dev, peaks, flush, stream, SHAPES, PAGE_T_PROD_US,
+                                   fp8_block=fb)
     elif args.shapes == "table":
-        per_shape = measure_shapes(moe, dev, peaks, flush, stream, TABLE_SHAPES, TABLE_T_PROD_US)
+        per_shape = measure_shapes(moe, dev, peaks, flush, stream, TABLE_SHAPES, TABLE_T_PROD_US,
+                                   fp8_block=fb)
 
     line = {
         "metric": METRIC,
@@ -358,33 +361,45 @@ def run_ours(args, ws, rank, local):
     return line
 
 
-def measure_shapes(moe, dev, peaks, flush, stream, shapes, page_us, K=10, W=3):
+def measure_shapes(moe, dev, peaks, flush, stream, shapes, page_us, K=10, W=3, fp8_block=0):
+    """Forward-only time per shape; FP8 E4M3 weights when fp8_block > 0."""
     res = {}
     for name, s in shapes.items():
+        if fp8_block and (s.H % fp8_block or s.I % fp8_block or fp8_block % 128):
+            res[name] = {"skipped": f"block {fp8_block} does not divide H={s.H} and I={s.I}"}
+            continue
         hidden, w1, w2, logits = make_shape_inputs(s, seed=0, device=str(dev))
+        if fp8_block:
+            q1, s1, q2, s2 = make_fp8_weights(s.E, s.H, s.I, fp8_block, seed=0, device=str(dev))
         ids, wts = moe.moe_route(logits, s.k, True)
         out = torch.empty(s.T, s.H, dtype=torch.float32, device=dev)
 
         def step(ev):
             if ev is not None:
                 ev[0].record(stream)
-            moe.moe_forward(hidden, w1, w2, wts, ids, out)
+            if fp8_block:
+                moe.moe_forward_fp8(hidden, q1, s1, q2, s2, fp8_block, wts, ids, out)
+            else:
+                moe.moe_forward(hidden, w1, w2, wts, ids, out)
             if ev is not None:
                 ev[1].record(stream)
 
         t = time_steps(step, K, W, flush, stream, marks=1)
         us = statistics.median(x[0] for x in t) * 1e3
         n_active = int(torch.unique(ids).numel())
-        t_roof, bound = roofline_us(s, n_active, peaks)
+        t_roof, bound = roofline_us(s, n_active, peaks, fp8_block)
         res[name] = {"T": s.T, "H": s.H, "I": s.I, "E": s.E, "k": s.k,
                      "us_per_call": round(us, 2),
                      "tflops": round(s.flops / (us * 1e-6) / 1e12, 2),
-                     "hbm_gbs": round(algorithmic_bytes(s, n_active) / (us * 1e-6) / 1e9, 1),
+                     "hbm_gbs": round(algorithmic_bytes(s, n_active, fp8_block) / (us * 1e-6) / 1e9,
+                                      1),
                      "roofline_bound": bound, "roofline_us": round(t_roof, 2),
                      "roofline_frac": round(t_roof / us, 4)}
         if name in page_us:
             res[name]["page_t_prod_us"] = page_us[name]
         del hidden, w1, w2, logits, ids, wts, out
+        if fp8_block:
+            del q1, s1, q2, s2
         torch.cuda.empty_cache()
     return res
 
