@@ -32,6 +32,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 from datetime import timedelta
 
@@ -116,7 +117,9 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank_gpu{gpu_index}.csv")
+        # the raw samples (the JSON line carries their summary)
+        out_dir = os.environ.get("MOE_BENCH_CLOCKS_DIR", tempfile.gettempdir())
+        self.path = os.path.join(out_dir, f"moe_bench_clocks_gpu{gpu_index}_{os.getpid()}.csv")
 
     def __enter__(self):
         try:

@@ -23,7 +23,7 @@
  * double is exact).  Nothing is blocked, fused or reordered beyond what the
  * definitions state; OpenMP only splits independent tokens across threads.
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent or leave a choice open:
  *   - top-k order: largest logit first; equal logits go to the lowest expert
  *     index (the in-kernel argmax on the TPU page returns the lowest index).
  *     Ranking logits is ranking the exact softmax, since exp is monotone.
