@@ -470,6 +470,10 @@ def run_reference(args, ws, rank):
     import oracle
     s = SHAPES[args.workload]
     hidden, w1, w2, logits = make_shape_inputs(s, seed=0, device="cpu")
+    if args.weights == "fp8":
+        # the oracle's FP8 formulation on the same codes and scales
+        q1, s1, q2, s2 = make_fp8_weights(s.E, s.H, s.I, args.fp8_block, seed=0, device="cpu")
+        w1, w2 = (q1, s1, args.fp8_block), (q2, s2, args.fp8_block)
     per_step = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
     n, threads = calibrate_rows(s, hidden, w1, w2, logits, per_step)
     rows = np.arange(n)
@@ -487,7 +491,8 @@ def run_reference(args, ws, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded randn, shapes and scales of atrex-bench #009 input.py)",
         "config": {"workload": s.name, "T": s.T, "H": s.H, "I": s.I, "E": s.E, "top_k": s.k,
-                   "renorm": True, "step": f"oracle forward of a {n}-token sample"},
+                   "renorm": True, "weights": args.weights,
+                   "step": f"oracle forward of a {n}-token sample"},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads,
                          "kind": "oracle",
                          "sample": f"{n} of {s.T} tokens per step, fp64 per-token loop",
