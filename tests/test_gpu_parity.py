@@ -166,6 +166,19 @@ def test_forward_small_batches(T, path):
     check_status_clean()
 
 
+@pytest.mark.parametrize("T", [1, 3])
+def test_forward_small_batches_wide_hidden(T):
+    """The GEMV path at H = 4096, I = 384 (the thin experts): 28 output rows
+    per CTA, the last CTAs with a partial slice or none."""
+    H, I, E, k = 4096, 384, 128, 8
+    hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=70 + T)
+    ids, w = oracle.route(logits.numpy(), k, True)
+    ref = oracle.moe_token_loop(hidden, w1, w2, w, ids)
+    out = gpu_forward(hidden, w1, w2, w, ids)
+    assert_output_close(out, ref, f"T={T} H={H} I={I}")
+    check_status_clean()
+
+
 def test_forward_small_t_shared_and_duplicate_experts():
     """Several tokens on one expert, and one token routed twice to an expert."""
     T, H, I, E, k = 6, 512, 256, 4, 3
