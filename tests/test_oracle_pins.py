@@ -484,6 +484,19 @@ def test_variant_formulations_agree():
     assert pin_variants_formulations_agree()
 
 
+def test_e4m3_decoder_golden_values(golden_dir):
+    """Hand-derived E4M3 values (tests/golden/e4m3_codes.json)."""
+    with open(os.path.join(golden_dir, "e4m3_codes.json")) as f:
+        doc = json.load(f)
+    for code, want, why in doc["cases"]:
+        got = oracle.e4m3_to_double(int(code, 16))
+        if want == "nan":
+            assert math.isnan(got), (code, why)
+        else:
+            assert got == want and math.copysign(1.0, got) == math.copysign(1.0, want), \
+                (code, got, want, why)
+
+
 def test_e4m3_decoder_matches_torch():
     assert pin_e4m3_decoder()
 
