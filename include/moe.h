@@ -90,10 +90,10 @@ int moe_route(const float *logits, int64_t T, int E, int k, int renorm,
  *                          topk_weights[t, j] * FFN_{topk_ids[t, j]}(hidden[t]),
  *                 accumulated in fp32 (grouped-GEMM path, k <= 2: out is
  *                 zeroed and each rounded product w_j * y_j is added at L2,
- *                 which gives the same bits in either order; k > 2:
- *                 ascending j; small-T path: per column slice in ascending
- *                 expert order, then a fixed tree); a row with no valid id
- *                 is 0.
+ *                 which gives the same bits in either order; k > 2 and the
+ *                 small-T path: ascending j, one fused multiply-add per
+ *                 term, acc = fma(w_j, y_j, acc) from acc = 0); a row with
+ *                 no valid id is 0.
  * Numerics: bf16 inputs, fp32 accumulation; the SwiGLU intermediate is
  * rounded to bf16 before the second projection on the grouped-GEMM path
  * and kept in fp32 on the small-T path (T <= the small-T limit, H <= 4096
@@ -185,17 +185,26 @@ int moe_forward_fp8(const uint16_t *hidden, const uint8_t *w1, const float *w1_s
  *   - Limits: T <= MOE_NOALLOC_MAX_T and T*k*I <= MOE_NOALLOC_MAX_ACT, else
  *     MOE_ERR_SCRATCH_LIMIT and nothing is launched.  Other checks and
  *     codes as in moe_forward, plus UNSUPPORTED when H > 4096 or I > 12288
- *     (the largest rows the small-T kernels stage).
+ *     (the largest rows the small-T kernels stage) or when the shape's
+ *     token vectors and per-CTA buffers do not fit the kernel's shared
+ *     memory on this device.
  *   - The first call on each device, with that device current, looks up
  *     the array's device address (cudaGetSymbolAddress) and caches it; make
- *     that first call before any stream capture.
- *   - All calls share the one array, which keeps the last call's contents:
- *     calls whose kernels overlap on the GPU (e.g. on two streams without
- *     ordering) race on it.  Nothing in it has to be cleared between calls
- *     (its grid-barrier counter starts at zero when the library loads and
- *     every call advances it).
- *   - Expert ids outside [0, E) are skipped as in moe_forward, but the bad-id
- *     flag is not reported through moe_get_device_status.
+ *     that first call before any stream capture.  cudaDeviceReset between
+ *     calls is not supported (the cached address would be stale).
+ *   - All calls share the one array, which keeps the last call's contents.
+ *     Nothing in it has to be cleared between calls: every act value is
+ *     written before it is read in the same call, and the grid-barrier
+ *     counter in the array only ever advances by whole grids.  Calls whose
+ *     kernels overlap on the GPU (e.g. on two streams without ordering)
+ *     race on it: they mix each other's act values, and their CTAs count
+ *     towards each other's grid barrier, which can open a barrier early
+ *     (wrong output) or hold one until its 2 s limit (output unwritten).
+ *   - Failures on the device are not reported: expert ids outside [0, E)
+ *     are skipped as in moe_forward but flag nothing, and a grid-barrier or
+ *     copy wait that gives up after its 2 s limit leaves out unwritten
+ *     while the call has already returned MOE_OK.  moe_get_device_status
+ *     does not see this path's status word.
  *   - Calls no cudaMalloc, cudaFree or other allocating routine.
  */
 #define MOE_NOALLOC_MAX_T 16
@@ -206,9 +215,12 @@ int moe_forward_small_noalloc(const uint16_t *hidden, const uint16_t *w1, const 
 
 /*
  * moe_permute -- the expert grouping that moe_forward uses internally,
- * exported so that it can be checked bit for bit.  Pages: the TPU kernel
- * hands each expert its rows in (token, k) order (start_a2a_scatter);
- * Model.forward visits each expert's tokens in ascending order.
+ * exported so that it can be checked bit for bit: it runs the same grouping
+ * kernel that moe_forward runs for this many entries (one kernel up to 8192
+ * entries, a histogram / scan / scatter sequence above).  Pages: the TPU
+ * kernel hands each expert its rows in (token, k) order
+ * (start_a2a_scatter); Model.forward visits each expert's tokens in
+ * ascending order.
  *
  *   topk_ids        [T, k] int32 (flat index i = t*k + j)
  *   sorted_rows     [T*k] int32, written for positions < expert_offsets[E]:
@@ -218,11 +230,38 @@ int moe_forward_small_noalloc(const uint16_t *hidden, const uint16_t *w1, const 
  *   expert_offsets  [E+1] int32, written: exclusive prefix sum of the
  *                   per-expert counts; expert_offsets[E] = number of ids in
  *                   [0, E)
+ * Ids outside [0, E) are left out; unlike moe_forward, neither call raises
+ * MOE_STATUS_BAD_ID.
  * Errors: INVALID_ARG for null pointers, T < 0, k < 1, E < 1;
  *         UNSUPPORTED for E > 1024.
  */
 int moe_permute(const int32_t *topk_ids, int64_t T, int k, int E,
                 int32_t *sorted_rows, int32_t *expert_offsets, void *stream);
+
+/*
+ * moe_permute_ex -- moe_permute with everything the grouping stage of
+ * moe_forward produces, and a choice of grouping kernel (debug and test
+ * export).
+ *
+ *   inv     [T*k] int32 or NULL; written: inv[i] = the position of flat
+ *           index i in sorted_rows, or -1 when topk_ids[i] is outside [0, E)
+ *   hidden  [T, H] bf16 and xs [T*k, H] bf16, both NULL or both given
+ *           (16-byte aligned, H % 128 == 0): xs[r] = hidden[sorted_rows[r] / k]
+ *           for r < expert_offsets[E], the expert-sorted copy of the hidden
+ *           rows that moe_forward makes for top-k <= 2; later rows untouched
+ *   kernel  MOE_PERMUTE_AUTO: the kernel moe_forward uses for T*k entries;
+ *           MOE_PERMUTE_SINGLE: the one-kernel grouping (T*k <= 8192, else
+ *           UNSUPPORTED); MOE_PERMUTE_MULTI: histogram / scan / scatter
+ * Both kernels give identical results.  Errors: those of moe_permute, plus
+ * INVALID_ARG for an unknown kernel, only one of hidden / xs, or an
+ * unaligned hidden / xs.
+ */
+#define MOE_PERMUTE_AUTO 0
+#define MOE_PERMUTE_SINGLE 1
+#define MOE_PERMUTE_MULTI 2
+int moe_permute_ex(const int32_t *topk_ids, int64_t T, int k, int E,
+                   int32_t *sorted_rows, int32_t *expert_offsets, int32_t *inv,
+                   const uint16_t *hidden, int H, uint16_t *xs, int kernel, void *stream);
 
 /* Static, NUL-terminated description of an MOE_* return code. */
 const char *moe_error_string(int code);

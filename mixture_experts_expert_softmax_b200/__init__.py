@@ -32,6 +32,11 @@ MOE_NOALLOC_MAX_T = 16
 MOE_NOALLOC_MAX_ACT = 262144
 MOE_STATUS_TIMEOUT = 0x1
 MOE_STATUS_BAD_ID = 0x2
+MOE_PERMUTE_AUTO = 0
+MOE_PERMUTE_SINGLE = 1
+MOE_PERMUTE_MULTI = 2
+PERMUTE_KERNELS = {"auto": MOE_PERMUTE_AUTO, "single": MOE_PERMUTE_SINGLE,
+                   "multi": MOE_PERMUTE_MULTI}
 MOE_ACT_SILU = 0
 MOE_ACT_GELU_TANH = 1
 MOE_ACT_SWIGLUOAI = 2
@@ -43,7 +48,7 @@ EXPORTED = (
     "moe_get_device_status", "moe_set_small_t_max", "moe_set_sync_each_stage",
     "moe_set_wait_limit_ns", "moe_last_failed_stage", "moe_debug_wait_timeout",
     "moe_profile_enable", "moe_profile_reset", "moe_profile_read",
-    "moe_forward_small_noalloc", "moe_forward_ex", "moe_forward_fp8",
+    "moe_forward_small_noalloc", "moe_forward_ex", "moe_forward_fp8", "moe_permute_ex",
 )
 
 
@@ -64,6 +69,7 @@ def _load() -> ctypes.CDLL:
         "moe_route": ([P, I64, I32, I32, I32, P, P, P], I32),
         "moe_forward": ([P, P, P, P, P, P, I64, I32, I32, I32, I32, P], I32),
         "moe_permute": ([P, I64, I32, I32, P, P, P], I32),
+        "moe_permute_ex": ([P, I64, I32, I32, P, P, P, P, I32, P, I32, P], I32),
         "moe_error_string": ([I32], ctypes.c_char_p),
         "moe_get_device_status": ([P, ctypes.POINTER(ctypes.c_uint32)], I32),
         "moe_set_small_t_max": ([I32], I32),
@@ -251,6 +257,36 @@ def moe_permute(topk_ids: torch.Tensor, E: int, sorted_rows: torch.Tensor | None
     return sorted_rows, expert_offsets
 
 
+def moe_permute_ex(topk_ids: torch.Tensor, E: int, kernel: str = "auto",
+                   hidden: torch.Tensor | None = None, stream=None):
+    """Everything the grouping stage of moe_forward produces, with a choice
+    of grouping kernel ("auto", "single" or "multi").  Returns (sorted_rows
+    int32 [T*k], expert_offsets int32 [E+1], inv int32 [T*k], xs) where xs
+    is the expert-sorted copy of the bf16 hidden rows [T*k, H] when hidden
+    is given (rows past expert_offsets[E] stay zero), else None."""
+    _need(topk_ids, "topk_ids", torch.int32)
+    if kernel not in PERMUTE_KERNELS:
+        raise ValueError(f"kernel must be one of {sorted(PERMUTE_KERNELS)}, got {kernel!r}")
+    T, k = topk_ids.shape
+    dev = topk_ids.device
+    sorted_rows = torch.full((T * k,), -1, dtype=torch.int32, device=dev)
+    expert_offsets = torch.empty((E + 1,), dtype=torch.int32, device=dev)
+    inv = torch.full((T * k,), -2, dtype=torch.int32, device=dev)
+    xs, H = None, 0
+    if hidden is not None:
+        _need(hidden, "hidden", torch.bfloat16)
+        if hidden.shape[0] != T:
+            raise ValueError(f"hidden must have {T} rows, got {hidden.shape[0]}")
+        H = hidden.shape[1]
+        xs = torch.zeros((T * k, H), dtype=torch.bfloat16, device=dev)
+    _check(_lib.moe_permute_ex(topk_ids.data_ptr(), T, k, int(E), sorted_rows.data_ptr(),
+                               expert_offsets.data_ptr(), inv.data_ptr(),
+                               None if hidden is None else hidden.data_ptr(), H,
+                               None if xs is None else xs.data_ptr(),
+                               PERMUTE_KERNELS[kernel], _stream(stream)), "moe_permute_ex")
+    return sorted_rows, expert_offsets, inv, xs
+
+
 def get_device_status(stream=None) -> int:
     """Synchronise, return and clear the OR of MOE_STATUS_* bits."""
     v = ctypes.c_uint32(0)
@@ -301,7 +337,8 @@ def profile_read() -> dict[str, tuple[int, float]]:
 
 
 __all__ = [
-    "moe_route", "moe_forward", "moe_forward_fp8", "moe_forward_small_noalloc", "moe_permute", "get_device_status", "set_small_t_max",
+    "moe_route", "moe_forward", "moe_forward_fp8", "moe_forward_small_noalloc", "moe_permute",
+    "moe_permute_ex", "get_device_status", "set_small_t_max",
     "set_sync_each_stage", "set_wait_limit_ns", "last_failed_stage", "debug_wait_timeout",
     "profile_enable", "profile_reset", "profile_read", "error_string", "MoEError",
     "LIB_PATH", "EXPORTED", "ACTS",

@@ -28,7 +28,6 @@ struct DeviceState {
   bool usable = false;
   int num_sms = 0;
   uint32_t *status = nullptr;  // 256 B: status word at 0, small-T grid counter at 64
-  unsigned long long small_t_arrivals = 0;  // small-T grid-barrier counter target
   void *ws = nullptr;          // grow-only workspace
   size_t ws_bytes = 0;
   void *wq = nullptr;          // grow-only: bf16 copies of FP8 weights (GEMM path)
@@ -239,26 +238,53 @@ int moe_route(const float *logits, int64_t T, int E, int k, int renorm, int32_t 
   return to_code(hook.end(e));
 }
 
-int moe_permute(const int32_t *topk_ids, int64_t T, int k, int E, int32_t *sorted_rows,
-                int32_t *expert_offsets, void *stream) {
+int moe_permute_ex(const int32_t *topk_ids, int64_t T, int k, int E, int32_t *sorted_rows,
+                   int32_t *expert_offsets, int32_t *inv, const uint16_t *hidden, int H,
+                   uint16_t *xs, int kernel, void *stream) {
   if (T < 0 || k < 1 || E < 1) return MOE_ERR_INVALID_ARG;
   if (expert_offsets == nullptr || (T > 0 && (topk_ids == nullptr || sorted_rows == nullptr)))
     return MOE_ERR_INVALID_ARG;
-  if (E > kMaxExperts) return MOE_ERR_UNSUPPORTED;
+  if (kernel != MOE_PERMUTE_AUTO && kernel != MOE_PERMUTE_SINGLE && kernel != MOE_PERMUTE_MULTI)
+    return MOE_ERR_INVALID_ARG;
+  if ((hidden == nullptr) != (xs == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (xs != nullptr && (H < 1 || !aligned16(hidden) || !aligned16(xs)))
+    return MOE_ERR_INVALID_ARG;
+  if (E > kMaxExperts || (xs != nullptr && H % 128 != 0)) return MOE_ERR_UNSUPPORTED;
   const int64_t n = T * k;
   if (n >= (static_cast<int64_t>(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  const bool single = kernel == MOE_PERMUTE_SINGLE ||
+                      (kernel == MOE_PERMUTE_AUTO && moe::group_supported(n));
+  if (single && !moe::group_supported(n)) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState *d = nullptr;
   int rc = current_device(&d);
   if (rc != MOE_OK) return rc;
-  if ((rc = ensure_workspace(*d, permute_ws_bytes(n, E))) != MOE_OK) return rc;
+  // chunk counts of the three-kernel grouping, and the counters that the
+  // row copy zeroes for the fused GEMM (none here but the done flag)
+  if ((rc = ensure_workspace(*d, permute_ws_bytes(n, E) + 256)) != MOE_OK) return rc;
   Carver cv{static_cast<char *>(d->ws)};
   int32_t *chunk_counts = cv.take<int32_t>(std::max(moe::permute_num_chunks(n), 1) * static_cast<size_t>(E));
+  int *zero_done = cv.take<int>(1);
   CallCtx ctx{static_cast<cudaStream_t>(stream), "", nullptr};
   moe::StageHook hook = make_hook(&ctx);
-  cudaError_t e = moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets, sorted_rows,
-                                      nullptr, nullptr, ctx.stream, hook);
+  cudaError_t e;
+  if (single) {
+    e = moe::launch_group(topk_ids, n, E, k, expert_offsets, sorted_rows, inv, nullptr, hidden, H,
+                          xs, nullptr, 0, zero_done, d->num_sms, ctx.stream, hook);
+  } else {
+    e = moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets, sorted_rows, inv,
+                            nullptr, ctx.stream, hook);
+    if (e == cudaSuccess && xs != nullptr)
+      e = moe::launch_gather_rows(hidden, H, k, sorted_rows, expert_offsets, E, n, d->num_sms, xs,
+                                  zero_done, 0, zero_done, ctx.stream, hook);
+  }
   return to_code(e);
+}
+
+int moe_permute(const int32_t *topk_ids, int64_t T, int k, int E, int32_t *sorted_rows,
+                int32_t *expert_offsets, void *stream) {
+  return moe_permute_ex(topk_ids, T, k, E, sorted_rows, expert_offsets, nullptr, nullptr, 0,
+                        nullptr, MOE_PERMUTE_AUTO, stream);
 }
 
 }  // extern "C"
@@ -311,7 +337,12 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
   CallCtx ctx{static_cast<cudaStream_t>(stream), "", nullptr};
   moe::StageHook hook = make_hook(&ctx);
 
+  bool small = false;
   if (T <= small_t_max() && moe::small_t_supported(H, I)) {
+    cudaError_t e = moe::small_t_fits(T, H, I, E, k, fp8 != nullptr, &small);
+    if (e != cudaSuccess) return to_code(e);
+  }
+  if (small) {
     const size_t need = align256(static_cast<size_t>(n) * I * sizeof(float));
     if ((rc = ensure_workspace(*d, need)) != MOE_OK) return rc;
     Carver cv{static_cast<char *>(d->ws)};
@@ -321,7 +352,7 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
         b1, b2, act_kind, topk_weights, topk_ids, act, out, T, H, I, E, k,
         d->status,
         reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(d->status) + 64),
-        &d->small_t_arrivals, static_cast<uint64_t>(g_wait_limit_ns), ctx.stream, hook));
+        static_cast<uint64_t>(g_wait_limit_ns), ctx.stream, hook));
   }
 
   cudaError_t e;

@@ -125,10 +125,13 @@ cudaError_t launch_combine(const float *P, const int32_t *inv, const float *topk
 
 // small_t.cu
 bool small_t_supported(int H, int I);
+// *fits: whether launch_small_t can run this shape in the shared memory of
+// the current device (sets the kernels up for the device on first use).
+cudaError_t small_t_fits(int64_t T, int H, int I, int E, int k, bool fp8, bool *fits);
 // grid_sync: a 64-bit device counter that only this launcher's kernels
-// touch, 0 before the first launch; arrivals: the host's copy of the value
-// it reaches once every launch made so far has finished (advanced by the
-// call).  act: T*k*I fp32 scratch.
+// touch, 0 before the first launch (each launch advances it by its grid
+// size; launches on one counter must not overlap).  act: T*k*I fp32
+// scratch.
 // b1, b2, act_kind: the epilogue variant, as in GroupedGemmArgs.  block == 0:
 // w1 [E, 2I, H] and w2 [E, H, I] are bf16; block > 0 (a multiple of 16 that
 // divides H and I): they are FP8 E4M3 codes with fp32 scales w1_scale
@@ -138,7 +141,7 @@ cudaError_t launch_small_t(const uint16_t *hidden, const void *w1, const void *w
                            const float *b1, const float *b2, int act_kind,
                            const float *topk_weights, const int32_t *topk_ids, float *act,
                            float *out, int64_t T, int H, int I, int E, int k, uint32_t *status,
-                           unsigned long long *grid_sync, unsigned long long *arrivals,
-                           uint64_t wait_limit_ns, cudaStream_t s, const StageHook &hook);
+                           unsigned long long *grid_sync, uint64_t wait_limit_ns,
+                           cudaStream_t s, const StageHook &hook);
 
 }  // namespace moe

@@ -29,13 +29,13 @@ constexpr size_t kScratchBytes =
 
 // [0, 256): status word the kernel may raise bits in (not reported back) at
 // byte 0, and at byte 64 the kernel's grid-barrier counter, which starts at
-// zero when the module loads and is advanced by every call;
+// zero when the module loads and only ever advances (each launch adds its
+// grid size and derives its own barrier target from the value it reads);
 // [256, ...): the act scratch, T*k*I fp32 values.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 std::mutex g_noalloc_mu;
 void *g_noalloc_addr[kNoAllocMaxDevices] = {};
-unsigned long long g_noalloc_arrivals[kNoAllocMaxDevices] = {};
 
 }  // namespace
 
@@ -68,6 +68,15 @@ extern "C" int moe_forward_small_noalloc(const uint16_t *hidden, const uint16_t 
   }
   if (major != 10 || minor != 0) return MOE_ERR_NO_DEVICE;
 
+  // shapes whose token vectors and per-CTA buffers do not fit the kernel's
+  // shared memory are not a CUDA failure but a limit of this path
+  bool fits = false;
+  if (moe::small_t_fits(T, H, I, E, k, false, &fits) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  if (!fits) return MOE_ERR_UNSUPPORTED;
+
   void *base = nullptr;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   {
@@ -83,7 +92,7 @@ extern "C" int moe_forward_small_noalloc(const uint16_t *hidden, const uint16_t 
   }
   // Nothing has to be cleared between calls: every act value the second
   // phase reads is written by the first phase of the same call, and the
-  // grid-barrier counter only ever advances.
+  // grid-barrier counter only ever advances by whole grids.
   uint32_t *status = static_cast<uint32_t *>(base);
   unsigned long long *grid_sync =
       reinterpret_cast<unsigned long long *>(static_cast<char *>(base) + 64);
@@ -94,8 +103,7 @@ extern "C" int moe_forward_small_noalloc(const uint16_t *hidden, const uint16_t 
       moe::launch_small_t(hidden, w1, w2, nullptr, nullptr, 0, nullptr, nullptr, moe::kActSilu,
                           topk_weights,
                           topk_ids, act, out, T, H, I, E, k, status,
-                          grid_sync, &g_noalloc_arrivals[dev], 2000000000ull,
-                          static_cast<cudaStream_t>(stream), hook);
+                          grid_sync, 2000000000ull, static_cast<cudaStream_t>(stream), hook);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;

@@ -476,8 +476,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
                    const int32_t *__restrict__ ids, float *__restrict__ act,
                    float *__restrict__ out, int T, int k, int H, int I, int E, int rows_per_cta,
                    int slots, int cache_act, uint32_t *status,
-                   unsigned long long *grid_sync,
-                   unsigned long long sync_target, uint64_t limit) {
+                   unsigned long long *grid_sync, uint64_t limit) {
   // phase 1: chunks per lane and row in flight (an FP8 chunk holds 16 codes)
   constexpr int kU1 = kFp8 ? 4 : (kTokens == 1 ? 8 : 4);
   extern __shared__ __align__(16) uint8_t smem[];
@@ -611,14 +610,19 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   }
 
   // ------------------------------------------------------------ grid barrier
-  // Every CTA adds one per launch; the host passes the counter value that
-  // means every CTA of this launch has written its act values.
+  // Every CTA adds one per launch and every launch on this counter has the
+  // same grid, so between launches the counter is a multiple of gridDim.x:
+  // the value a CTA read decides which launch it belongs to, and the
+  // barrier opens when the counter reaches the end of that launch's block
+  // of arrivals.  (Derived here, not passed in, so that the target is right
+  // whatever was launched before on the counter.)
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
-    atomicAdd(grid_sync, 1ull);
+    const unsigned long long old = atomicAdd(grid_sync, 1ull);
+    const unsigned long long target = (old / gridDim.x + 1) * gridDim.x;
     const uint64_t t0 = global_timer_ns();
-    while (ld_acquire_gpu(grid_sync) < sync_target) {
+    while (ld_acquire_gpu(grid_sync) < target) {
       if (global_timer_ns() - t0 > limit) {
         s_abort = 1;
         atomicOr(status, kStatusTimeout);
@@ -796,61 +800,82 @@ size_t smem_budget(int dev, const void *kern) {
 
 bool small_t_supported(int H, int I) { return H <= kMaxH && I <= kMaxI; }
 
+namespace {
+
+std::mutex g_setup_mu;
+uint64_t g_ready_mask = 0;
+int g_grid_of[64] = {};
+size_t g_budget_of[64] = {};
+
+// Once per device: the shared-memory budget all four instantiations can
+// use and the cooperative grid (the CTAs both kernels keep resident on
+// every SM: the grid barrier needs every CTA resident at once).
+cudaError_t small_t_setup(int dev) {
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  if ((g_ready_mask >> dev) & 1) return cudaSuccess;
+  int sms = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const auto kerns = {small_t_kernel<1, false>, small_t_kernel<kMaxT, false>,
+                      small_t_kernel<1, true>, small_t_kernel<kMaxT, true>};
+  size_t smem = ~static_cast<size_t>(0);
+  for (auto kern : kerns)
+    smem = std::min(smem, smem_budget(dev, reinterpret_cast<const void *>(kern)));
+  if (smem < 16384) return cudaErrorInvalidValue;
+  int per_sm = kBlocksPerSm;
+  for (auto kern : kerns) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    per_sm = std::min(per_sm, n);
+  }
+  if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+  g_budget_of[dev] = smem;
+  g_grid_of[dev] = per_sm * sms;
+  g_ready_mask |= 1ull << dev;
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t small_t_fits(int64_t T, int H, int I, int E, int k, bool fp8, bool *fits) {
+  *fits = false;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if ((e = small_t_setup(dev)) != cudaSuccess) return e;
+  if (!small_t_supported(H, I) || T < 1 || T > kMaxT || T * k > kMaxPairs) return cudaSuccess;
+  const SmallTConfig cfg = small_t_config(static_cast<int>(T), static_cast<int>(T) * k, H, I, E,
+                                          g_grid_of[dev], g_budget_of[dev], fp8 ? 1 : 2);
+  *fits = cfg.smem <= g_budget_of[dev];
+  return cudaSuccess;
+}
+
 cudaError_t launch_small_t(const uint16_t *hidden, const void *w1, const void *w2,
                            const float *w1_scale, const float *w2_scale, int block,
                            const float *b1, const float *b2, int act_kind,
                            const float *topk_weights, const int32_t *topk_ids, float *act,
                            float *out, int64_t T, int H, int I, int E, int k, uint32_t *status,
-                           unsigned long long *grid_sync, unsigned long long *arrivals,
-                           uint64_t wait_limit_ns, cudaStream_t s, const StageHook &hook) {
-  static std::mutex mu;
-  static uint64_t ready_mask = 0;
-  static int grid_of[64] = {};
-  static size_t budget_of[64] = {};
-  int dev = 0, sms = 0;
+                           unsigned long long *grid_sync, uint64_t wait_limit_ns,
+                           cudaStream_t s, const StageHook &hook) {
+  int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  if (!small_t_supported(H, I) || dev >= 64 || T < 1 || T > kMaxT || T * k > kMaxPairs)
+  if (!small_t_supported(H, I) || dev < 0 || dev >= 64 || T < 1 || T > kMaxT || T * k > kMaxPairs)
     return cudaErrorInvalidValue;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    if (!((ready_mask >> dev) & 1)) {
-      // every CTA must be resident at once (the grid barrier): the grid is
-      // the number of CTAs both kernels can keep on every SM
-      const auto kerns = {small_t_kernel<1, false>, small_t_kernel<kMaxT, false>,
-                          small_t_kernel<1, true>, small_t_kernel<kMaxT, true>};
-      size_t smem = ~static_cast<size_t>(0);
-      for (auto kern : kerns)
-        smem = std::min(smem, smem_budget(dev, reinterpret_cast<const void *>(kern)));
-      if (smem < 16384) return cudaErrorInvalidValue;
-      budget_of[dev] = smem;
-      int per_sm = kBlocksPerSm;
-      for (auto kern : kerns) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        int n = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, smem);
-        if (e != cudaSuccess) return e;
-        per_sm = std::min(per_sm, n);
-      }
-      if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
-      grid_of[dev] = per_sm * sms;
-      ready_mask |= 1ull << dev;
-    }
-  }
-  const int grid = grid_of[dev];
+  if ((e = small_t_setup(dev)) != cudaSuccess) return e;
+  const int grid = g_grid_of[dev];
   const bool fp8 = block > 0;
   if (fp8 && (w1_scale == nullptr || w2_scale == nullptr || block % 16 != 0 || H % block != 0 ||
               I % block != 0))
     return cudaErrorInvalidValue;
   const SmallTConfig cfg = small_t_config(static_cast<int>(T), static_cast<int>(T) * k, H, I, E,
-                                          grid, budget_of[dev], fp8 ? 1 : 2);
-  if (cfg.smem > budget_of[dev]) return cudaErrorInvalidValue;
-  // each CTA adds one to the grid-sync counter per launch: the target is the
-  // arrivals of all earlier launches plus this grid
-  const unsigned long long target = *arrivals + static_cast<unsigned long long>(grid);
+                                          grid, g_budget_of[dev], fp8 ? 1 : 2);
+  if (cfg.smem > g_budget_of[dev]) return cudaErrorInvalidValue;
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(grid);
   lc.blockDim = dim3(kThreads);
@@ -868,9 +893,7 @@ cudaError_t launch_small_t(const uint16_t *hidden, const void *w1, const void *w
                          reinterpret_cast<const uint4 *>(w1), reinterpret_cast<const uint4 *>(w2),
                          w1_scale, w2_scale, block, b1, b2, act_kind, topk_weights, topk_ids, act, out, static_cast<int>(T), k, H, I, E,
                          cfg.rows_per_cta, cfg.slots, cfg.cache_act, status,
-                         grid_sync, target,
-                         wait_limit_ns);
-  if (e == cudaSuccess) *arrivals = target;
+                         grid_sync, wait_limit_ns);
   return hook.end(e);
 }
 

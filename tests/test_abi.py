@@ -135,6 +135,27 @@ def test_permute_argument_checks():
     assert L.moe_permute(1, 4, 2, 4096, 1, 1, None) == moe.MOE_ERR_UNSUPPORTED
 
 
+def perm_ex(ids=256, T=4, k=2, E=8, rows=256, offs=256, inv=NULL, h=NULL, H=0, xs=NULL,
+            kernel=0):
+    return L.moe_permute_ex(ids, T, k, E, rows, offs, inv, h, H, xs, kernel, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ids=NULL), moe.MOE_ERR_INVALID_ARG),
+    (dict(offs=NULL), moe.MOE_ERR_INVALID_ARG),
+    (dict(kernel=3), moe.MOE_ERR_INVALID_ARG),           # unknown grouping kernel
+    (dict(h=256, H=256), moe.MOE_ERR_INVALID_ARG),        # hidden without xs
+    (dict(xs=256, H=256), moe.MOE_ERR_INVALID_ARG),       # xs without hidden
+    (dict(h=264, xs=256, H=256), moe.MOE_ERR_INVALID_ARG),  # hidden not 16-byte aligned
+    (dict(h=256, xs=256, H=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(h=256, xs=256, H=200), moe.MOE_ERR_UNSUPPORTED),  # H % 128
+    (dict(E=2000), moe.MOE_ERR_UNSUPPORTED),
+    (dict(T=4097, k=2, kernel=1), moe.MOE_ERR_UNSUPPORTED),  # > 8192 entries, one kernel
+])
+def test_permute_ex_argument_checks(kw, code):
+    assert perm_ex(**kw) == code
+
+
 def test_debug_switches_roundtrip():
     prev = moe.set_small_t_max(5)
     assert moe.set_small_t_max(prev) == 5

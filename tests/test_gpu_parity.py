@@ -97,29 +97,108 @@ def test_route_empty():
 
 
 # ------------------------------------------------------------------ permutation
-@pytest.mark.parametrize("T,k,E", [(1, 1, 1), (5, 2, 3), (1024, 2, 8), (1025, 2, 8),
-                                   (4096, 8, 128), (3000, 7, 1024), (8192, 8, 128),
-                                   (15381, 2, 8), (100, 16, 1000)])
-def test_permute_bit_exact(T, k, E):
-    g = torch.Generator().manual_seed(T + 7 * E)
-    ids = torch.randint(-1, E + 1, (T, k), generator=g, dtype=torch.int32)
-    rows_r, offs_r = oracle.permute(ids.numpy(), E)
-    rows_g, offs_g = moe.moe_permute(ids.cuda(), E)
-    torch.cuda.synchronize()
-    offs_g = offs_g.cpu().numpy()
-    assert np.array_equal(offs_g, offs_r)
+def _perm_ids(kind, T, k, E, seed):
+    """Expert ids for the grouping tests: uniform with ids outside [0, E)
+    mixed in, routed (softmax top-k of randn logits, distinct per token),
+    every id on one expert, or a heavily skewed mix."""
+    g = torch.Generator().manual_seed(seed)
+    if kind == "uniform_invalid":
+        return torch.randint(-1, E + 1, (T, k), generator=g, dtype=torch.int32).numpy()
+    if kind == "routed":
+        ids, _ = oracle.route(torch.randn(T, E, generator=g).numpy(), k, True)
+        return ids
+    if kind == "one_expert":
+        return np.full((T, k), E - 1, np.int32)
+    if kind == "skewed":
+        # three quarters of the ids on expert 0, the rest spread, a few invalid
+        ids = torch.randint(0, E, (T, k), generator=g, dtype=torch.int32).numpy()
+        u = torch.rand(T, k, generator=g).numpy()
+        ids[u < 0.75] = 0
+        ids[u > 0.995] = -5
+        return ids
+    raise ValueError(kind)
+
+
+def _oracle_inverse(rows_r, n):
+    inv = np.full(n, -1, np.int64)
+    inv[rows_r] = np.arange(rows_r.size)
+    return inv
+
+
+PERMUTE_CASES = [
+    # (ids kind, T, k, E)
+    ("uniform_invalid", 1, 1, 1),
+    ("uniform_invalid", 5, 2, 3),
+    ("uniform_invalid", 1024, 2, 8),
+    ("uniform_invalid", 1025, 2, 8),
+    ("routed", 64, 2, 8),             # the tiny workload's routing
+    ("routed", 1979, 2, 8),           # the 8-expert prefill's routing
+    ("routed", 1024, 8, 128),         # exactly 8192 entries
+    ("uniform_invalid", 4096, 2, 8),  # exactly 8192 entries, invalid ids
+    ("one_expert", 4096, 2, 8),       # every entry on one expert
+    ("one_expert", 1, 16, 1024),
+    ("skewed", 2000, 4, 64),
+    ("uniform_invalid", 512, 16, 1024),  # E = 1024, 8192 entries
+    ("uniform_invalid", 4097, 2, 8),  # 8194 entries: only the three-kernel grouping
+    ("routed", 8192, 8, 128),         # the thin prefill's routing
+    ("uniform_invalid", 3000, 7, 1024),
+    ("skewed", 15381, 2, 8),
+    ("uniform_invalid", 100, 16, 1000),
+]
+
+
+@pytest.mark.parametrize("kind,T,k,E", PERMUTE_CASES)
+def test_permute_bit_exact_both_kernels(kind, T, k, E):
+    """sorted_rows, expert_offsets and the inverse permutation bit for bit
+    against the oracle's stable counting sort, from the kernel moe_forward
+    uses (auto) and from each grouping kernel that can take this size."""
+    ids = _perm_ids(kind, T, k, E, seed=T + 7 * E + k)
+    n = T * k
+    rows_r, offs_r = oracle.permute(ids, E)
+    inv_r = _oracle_inverse(rows_r, n)
     nv = int(offs_r[-1])
-    assert np.array_equal(rows_g.cpu().numpy()[:nv], rows_r[:nv])
+    kernels = ["auto", "multi"] + (["single"] if n <= 8192 else [])
+    ids_d = torch.as_tensor(ids).cuda()
+    for kern in kernels:
+        rows_g, offs_g, inv_g, _ = moe.moe_permute_ex(ids_d, E, kernel=kern)
+        torch.cuda.synchronize()
+        assert np.array_equal(offs_g.cpu().numpy(), offs_r), kern
+        rows_g = rows_g.cpu().numpy()
+        assert np.array_equal(rows_g[:nv], rows_r[:nv]), kern
+        assert np.all(rows_g[nv:] == -1), kern  # positions past the valid ids untouched
+        assert np.array_equal(inv_g.cpu().numpy(), inv_r), kern
+    # the plain export runs the same grouping
+    rows_p, offs_p = moe.moe_permute(ids_d, E)
+    torch.cuda.synchronize()
+    assert np.array_equal(offs_p.cpu().numpy(), offs_r)
+    assert np.array_equal(rows_p.cpu().numpy()[:nv], rows_r[:nv])
 
 
-def test_permute_of_routed_workload():
-    s = SHAPES["prefill_thin"]
-    logits = torch.randn(s.T, s.E, generator=torch.Generator().manual_seed(0))
-    ids, _ = oracle.route(logits.numpy(), s.k, True)
-    rows_r, offs_r = oracle.permute(ids, s.E)
-    rows_g, offs_g = moe.moe_permute(torch.as_tensor(ids).cuda(), s.E)
-    assert np.array_equal(offs_g.cpu().numpy(), offs_r)
-    assert np.array_equal(rows_g.cpu().numpy(), rows_r)
+@pytest.mark.parametrize("kind,T,k,E,H", [
+    ("routed", 64, 2, 8, 256),
+    ("routed", 1979, 2, 8, 2048),
+    ("uniform_invalid", 4096, 2, 8, 128),   # 8192 entries: one kernel, many CTAs
+    ("routed", 4097, 2, 8, 256),            # three kernels and the separate row copy
+    ("one_expert", 300, 1, 4, 384),
+])
+def test_permute_sorted_row_copy(kind, T, k, E, H):
+    """The expert-sorted copy of the hidden rows the top-k <= 2 GEMM path
+    loads (xs[r] = hidden[sorted_rows[r] // k]), bit for bit, from every
+    grouping kernel that can take this size."""
+    ids = _perm_ids(kind, T, k, E, seed=3 * T + H)
+    hidden = (torch.randn(T, H, generator=torch.Generator().manual_seed(T)) * 0.1).to(torch.bfloat16)
+    rows_r, offs_r = oracle.permute(ids, E)
+    nv = int(offs_r[-1])
+    want = hidden[torch.as_tensor(rows_r[:nv] // k, dtype=torch.long)]
+    kernels = ["auto", "multi"] + (["single"] if T * k <= 8192 else [])
+    for kern in kernels:
+        _, offs_g, _, xs = moe.moe_permute_ex(torch.as_tensor(ids).cuda(), E, kernel=kern,
+                                              hidden=hidden.cuda())
+        torch.cuda.synchronize()
+        assert np.array_equal(offs_g.cpu().numpy(), offs_r), kern
+        xs = xs.cpu()
+        assert torch.equal(xs[:nv].view(torch.int16), want.view(torch.int16)), kern
+        assert torch.all(xs[nv:].view(torch.int16) == 0), kern
 
 
 # ------------------------------------------------------------------ forward
@@ -438,6 +517,31 @@ def _sample_rows(T, n, seed):
     return np.array(sorted(rows), np.int64)
 
 
+def _tail_tile_tokens(ids, E, k, tile=256):
+    """Tokens of every row in each expert's last, partial m-tile of the
+    expert-sorted order (where the GEMM epilogues mask rows)."""
+    rows_r, offs_r = oracle.permute(ids, E)
+    toks = set()
+    for e in range(E):
+        lo, hi = int(offs_r[e]), int(offs_r[e + 1])
+        full = lo + (hi - lo) // tile * tile
+        toks.update((rows_r[full:hi] // k).tolist())
+    return toks
+
+
+def full_size_rows(s, ids):
+    """Rows of a full-size workload compared with the oracle: every row up
+    to the thin prefill (8192 tokens, ~30 s of oracle time on 16 cores);
+    for the large prefill every token in an expert's last partial m-tile,
+    the first and last token, and 2000 random tokens."""
+    if s.T <= 8192:
+        return np.arange(s.T)
+    rng = np.random.default_rng(11)
+    toks = _tail_tile_tokens(ids, s.E, s.k) | {0, s.T - 1}
+    toks |= set(rng.choice(s.T, size=2000, replace=False).tolist())
+    return np.array(sorted(toks), np.int64)
+
+
 @pytest.mark.parametrize("name", ["decode", "prefill_8e", "prefill_thin", "prefill_big"])
 def test_forward_full_size_workloads(name):
     s = SHAPES[name]
@@ -451,7 +555,8 @@ def test_forward_full_size_workloads(name):
     out = moe.moe_forward(hidden, w1, w2, torch.as_tensor(w_r.astype(np.float32)).cuda(),
                           torch.as_tensor(ids_r).cuda())
     torch.cuda.synchronize()
-    rows = np.arange(s.T) if s.T <= 64 else _sample_rows(s.T, 14, 1)
+    rows = full_size_rows(s, ids_r)
+    print(f"{name}: {rows.size} of {s.T} rows compared with the oracle")
     ref = oracle.moe_token_loop(hidden.cpu(), w1.cpu(), w2.cpu(), w_r, ids_r, rows=rows)
     assert_output_close(out.cpu().numpy()[rows], ref, name)
     check_status_clean()
