@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(kGroupThreads)
     if (e >= 0 && (peers & lt) == 0) my_hist[e] += static_cast<uint16_t>(__popc(peers));
     if (pos >= 0) s_sorted[pos] = i;
     if (publish && i < n) {
-      inv[i] = pos;
+      if (inv != nullptr) inv[i] = pos;
       if (pos >= 0) sorted_rows[pos] = i;
     }
     __syncwarp();
