@@ -119,9 +119,11 @@ def _perm_ids(kind, T, k, E, seed):
     raise ValueError(kind)
 
 
-def _oracle_inverse(rows_r, n):
+def _oracle_inverse(rows_r, nv, n):
+    """inv[i] = position of flat index i among the nv grouped entries, -1
+    for an entry whose id is outside [0, E)."""
     inv = np.full(n, -1, np.int64)
-    inv[rows_r] = np.arange(rows_r.size)
+    inv[rows_r[:nv]] = np.arange(nv)
     return inv
 
 
@@ -155,8 +157,8 @@ def test_permute_bit_exact_both_kernels(kind, T, k, E):
     ids = _perm_ids(kind, T, k, E, seed=T + 7 * E + k)
     n = T * k
     rows_r, offs_r = oracle.permute(ids, E)
-    inv_r = _oracle_inverse(rows_r, n)
     nv = int(offs_r[-1])
+    inv_r = _oracle_inverse(rows_r, nv, n)
     kernels = ["auto", "multi"] + (["single"] if n <= 8192 else [])
     ids_d = torch.as_tensor(ids).cuda()
     for kern in kernels:
