@@ -7,50 +7,59 @@
 //     version of the page below): gelu (tanh form) or swigluoai in place of
 //     silu, and a bias b1[e] added to g and u before the activation.
 //   GEMM2: y = act . w2[e]^T (fp32 in TMEM), plus the bias b2[e] when given
-//     (before the top-k weight).  For top-k <= 2 the epilogue
-//     adds w_j * y_j of each row straight into out[token] with bulk
-//     reductions at L2 (out was zeroed first); out[t] = 0 + a + b is the
-//     same in either arrival order, so the result is still deterministic.
-//     For larger k it stores y as fp32 rows of P in the same expert-sorted
-//     order and combine.cu forms sum_j w_j * y_j in fixed j order.
+//     (before the top-k weight), then the top-k weighted sum into out:
+//     - top-k <= 2: the epilogue adds w_j * y_j of each row straight into
+//       out[token] with bulk reductions at L2 (out was zeroed first);
+//       out[t] = 0 + a + b is the same in either arrival order, so the
+//       result is deterministic.
+//     - top-k > 2 (ordered): each token's contributions go into out in
+//       ascending expert order -- the order of the per-expert loop of
+//       atrex-bench #009 Model.forward -- the first one stored, the others
+//       added at L2 with bulk reductions, each after the previous one has
+//       landed (a turn counter per token and 128-column block).  No
+//       per-(token, slot) buffer and no separate combine pass.
 // This is the expert FFN of ref_moe on the page "tpu_inference/kernels/
 // fused_moe/v1/kernel.py" (gate = w1, up = w3, then act . w2) in the weight
 // layout of atrex-bench #009 (w1 [E, 2I, H], w2 [E, H, I], both applied as
 // F.linear, i.e. K-major).
 //
 // Work unit: an m-tile of one expert's rows times one 256-column n-tile of
-// the accumulator.  Tiles run expert-major, then n-tile, then m-tile, so
-// CTAs working together share a weight tile through L2; the grid is
-// persistent and loops over tiles.
+// the accumulator.  Tiles are numbered expert-major, then n-tile, then
+// m-tile, so CTAs working together share a weight tile through L2 (the
+// ordered GEMM2 takes its n-tiles in column groups first, so that the part
+// of out it adds into stays in L2).  Tiles are handed out dynamically: the
+// first thread of each CTA (pair) claims the next tile number from a global
+// counter and publishes it through a small queue in shared memory to every
+// role of the CTA(s).  Tiles are claimed in number order, and every wait
+// across tiles (GEMM2 rows on the act rows of GEMM1 tiles, an ordered
+// contribution on the previous expert's) points to a tile with a smaller
+// number, which a running CTA has already claimed: progress never depends on
+// a CTA that has not started, whatever else occupies the GPU.
 //
 // Three kernels share the code (MODE):
 //   kModeFused   one launch on CTA pairs (a cluster of 2, M = 256,
-//                cta_group::2) that runs every GEMM1 tile and then every
-//                GEMM2 tile.  Its A rows come from copies in expert-sorted
-//                order (hidden rows gathered by gather_rows_kernel, and act),
-//                so rank r of the pair loads A rows 128r..128r+127 and half
-//                of the B tile with TMA into its own shared memory; rank 0
-//                issues the MMAs and each CTA receives its 128 accumulator
-//                rows in its own TMEM.  For GEMM1 rank 0 loads the n-tile's
-//                128 gate rows of w1 and rank 1 the matching 128 up rows, so
-//                one accumulator holds gate and up side by side.  A GEMM2
-//                tile waits (bounded) until the epilogues of all GEMM1 tiles
-//                of its m-tile have published their act rows through a
-//                per-m-tile counter: the static tile order puts every GEMM1
-//                tile of a CTA before its GEMM2 tiles, so no wait can form a
-//                cycle, and GEMM2 tiles fill the last, partial wave of GEMM1.
+//                cta_group::2) that runs every GEMM1 tile and then (with
+//                run_gemm2) every GEMM2 tile.  Its A rows come from copies in
+//                expert-sorted order (hidden rows copied by the grouping
+//                stage, and act), so rank r of the pair loads A rows
+//                128r..128r+127 and half of the B tile with TMA into its own
+//                shared memory; rank 0 issues the MMAs and each CTA receives
+//                its 128 accumulator rows in its own TMEM.  For GEMM1 rank 0
+//                loads the n-tile's 128 gate rows of w1 and rank 1 the
+//                matching 128 up rows, so one accumulator holds gate and up
+//                side by side.  A GEMM2 tile waits (bounded) until the
+//                epilogues of all GEMM1 tiles of its m-tile have published
+//                their act rows through a per-m-tile counter.
 //   kModeGemm1   GEMM1 alone on single CTAs (M = 128, cta_group::1) that
 //                gather their A rows by token index with cp.async (whose
 //                completion can only be signalled to the CTA's own barriers)
 //                and load gate and up rows themselves: no row copy needed.
-//   kModeGemm2   GEMM2 alone on CTA pairs, after kModeGemm1.
+//   kModeGemm2   GEMM2 alone on CTA pairs.
 // The GEMM2 epilogue stages each warp's 32 rows x 32 columns in shared
-// memory and writes them with one asynchronous TMA tile store into P (a
-// block that straddles the end of an expert's rows is written row by row
-// instead), or, fused with the combine, scales row r by its top-k weight
-// and issues one 128-byte bulk reduce-add per row into out[token]: large
-// operations, because the TMA engine's cost per operation, not the bytes,
-// bounds this epilogue.
+// memory and scales row r by its top-k weight; it issues one 128-byte bulk
+// reduce-add (or, first in the order, bulk copy) per row into out[token]:
+// large operations, because the TMA engine's cost per operation, not the
+// bytes, bounds this epilogue.
 //
 // Shared memory: the barriers and the expert / tile offset tables sit in
 // front, then (1024-byte aligned, as the 128-byte swizzle needs) the stage
@@ -58,19 +67,20 @@
 // as many as fit, up to kMaxStages, given the expert count.
 //
 // Warp roles (416 threads per CTA):
-//   warps 0-3  producers.  kModeGemm1: the 128 threads gather the A rows with
-//              16-byte cp.async into the 128-byte-swizzled K-major layout and
-//              arrive on the stage barrier asynchronously when they land;
-//              thread 0 issues the two TMA boxes of w1.  CTA pairs: thread 0
-//              of each CTA issues TMA for its A rows and half of B, counted
-//              on rank 0's barrier.
+//   warps 0-3  producers.  Thread 0 of rank 0 is also the tile scheduler.
+//              kModeGemm1: the 128 threads gather the A rows with 16-byte
+//              cp.async into the 128-byte-swizzled K-major layout and arrive
+//              on the stage barrier asynchronously when they land; thread 0
+//              issues the two TMA boxes of w1.  CTA pairs: thread 0 of each
+//              CTA issues TMA for its A rows and half of B, counted on rank
+//              0's barrier.
 //   warp 4     allocates 512 TMEM columns (two accumulators); one thread (on
 //              rank 0) issues the MMAs and commits each stage back to the
 //              producers and each finished tile to the epilogues.
 //   warps 5-12 epilogue, two warps per 32-lane TMEM quarter (a warp can only
 //              read the quarter warp_id % 4), each taking half of the tile's
-//              columns: tcgen05.ld, SwiGLU + bf16 store, or the fp32 TMA
-//              store / bulk reductions, then release the accumulator.
+//              columns: tcgen05.ld, SwiGLU + bf16 store, or the weighted
+//              bulk reductions into out, then release the accumulator.
 // Every wait is bounded; a wait that gives up raises the timeout bit of the
 // status word and makes every role of the CTA leave its loop.
 #include <algorithm>
@@ -92,13 +102,12 @@ constexpr int kTmemCols = 2 * kAccN;  // double-buffered accumulator
 constexpr int kABytes = BM * BK * 2;  // 16 KB
 constexpr int kMaxE = 1024;
 constexpr int kMaxStages = 6;
+constexpr int kTQ = 8;  // depth of the tile queue
 constexpr uint16_t kBothCtas = 0x3;
-// Per-warp staging of the GEMM2 epilogue: one 32-row x 32-column fp32 block,
-// 128-byte swizzled for the TMA store, or 32 plain rows at a 144-byte pitch
-// for the reductions (16-byte writes of 8 consecutive lanes then hit 8
+// Per-warp staging of the GEMM2 epilogue: 32 rows of 32 fp32 values at a
+// 144-byte pitch (16-byte writes of 8 consecutive lanes then hit 8
 // different bank groups: bank conflicts here would take shared-memory
-// bandwidth from the tensor core's operand reads).  A 1024-byte multiple
-// keeps every warp's block swizzle-aligned.
+// bandwidth from the tensor core's operand reads).
 constexpr int kRedPitch = 144;
 constexpr int kEpiWarpBytes = 5 * 1024;
 static_assert(32 * kRedPitch <= kEpiWarpBytes, "staging");
@@ -106,6 +115,9 @@ constexpr size_t kSmemMax = 232448;  // opt-in maximum per block on sm_100
 // act rows of an m-tile are complete when every epilogue warp of both CTAs
 // has published each of its n-tiles
 constexpr int kReadyPerTile = 2 * kEpiWarps;
+// out is zeroed (top-k <= 2) in chunks of this many float4, claimed by the
+// epilogue warps of whichever CTAs run first
+constexpr int64_t kZeroChunk4 = 4096;
 
 enum { kModeGemm1 = 0, kModeGemm2 = 1, kModeFused = 2 };
 
@@ -141,10 +153,19 @@ struct __align__(8) Bars {
   uint64_t acc_full[2];        // accumulator ready for the epilogue
   uint64_t acc_empty[2];       // epilogues (of both CTAs) drained the accumulator
   uint64_t drain;              // every MMA has completed
+  uint64_t tq_full[kTQ];       // tile queue slot written by the scheduler
+  uint64_t tq_empty[kTQ];      // (rank 0) every consumer of both CTAs has read the slot
+  int tq[kTQ];                 // tile numbers (-1: no more tiles)
+  int prod_tile;               // kModeGemm1: the tile broadcast to the 128 producer threads
   uint32_t tmem_base;
   int abort_flag;
   int32_t scan[32];            // per-warp partial sums of build_tile_offsets
 };
+
+// Readers of each queue slot: the MMA thread and the epilogue warps of rank
+// 0, and on a pair also rank 1's producer thread and epilogue warps.
+template <int CG>
+constexpr int queue_consumers() { return CG == 2 ? 2 * (1 + kEpiWarps) : 1 + kEpiWarps; }
 
 // Bytes in front of the aligned region: barriers, then exp_off and tile_off
 // (E + 1 entries each).
@@ -176,25 +197,38 @@ struct Params {
   const int32_t *sorted_rows;
   const int32_t *expert_offsets;
   __nv_bfloat16 *act;
-  float *P;
+  int64_t T;
   int H, I, E, k;
   int nt1, nt2;  // n-tiles per m-tile of GEMM1 (I / 128) and GEMM2 (ceil(H / 256))
   int stages;    // depth of the operand ring (<= kMaxStages)
   int run_gemm2; // kModeFused: 0 runs the GEMM1 tiles only (GEMM2 follows as
                  // its own kModeGemm2 launch)
+  int *sched;    // tile counter of this launch, zero at launch
   uint32_t *status;
   uint64_t wait_limit_ns;
-  // float4 count of out to zero before GEMM2 adds into it (0: none)
+  // out is zeroed before GEMM2 adds into it (top-k <= 2): zero_n4 float4 in
+  // chunks claimed through zero_claim; zero_done counts finished chunks
   float4 *zero_out;
   int64_t zero_n4;
-  // GEMM2 fused with the combine: out [T, H] and the top-k weights [T, k]
+  int *zero_claim;
+  int *zero_done;
+  // GEMM2's combine: out [T, H] and the top-k weights [T, k]
   float *out;
   const float *topk_weights;
-  int fuse_combine;
-  // kModeFused: per-m-tile act counters and the count of epilogue warps
-  // that finished zeroing out (both zero at launch)
+  int fuse_combine;  // top-k <= 2: add into zeroed out in any order
+  // top-k > 2: ordered contributions guarded by turn [T, H / 128] (zero at
+  // the GEMM2 launch), ranked with topk_ids [T, k]; GEMM2 tiles in column
+  // groups of ngroup n-tiles
+  int ordered;
+  int *turn;
+  const int32_t *topk_ids;
+  int ngroup;
+  // kModeGemm1 ahead of an ordered GEMM2: zero turn (turn_n ints) and the
+  // out rows of tokens without an expert id in [0, E)
+  int64_t turn_n;
+  int prepare_ordered;
+  // kModeFused: per-m-tile act counters (zero at launch)
   int *ready;
-  int *zero_done;
   // epilogue variant: activation (kAct*) and optional fp32 biases
   // b1 [E, 2I] (gate, then up) and b2 [E, H]
   const float *b1;
@@ -295,8 +329,18 @@ __device__ __forceinline__ void gated_pack32(const uint32_t (&g)[32], const uint
                         gated_f<ACT>(as_f32(g[2 * v + 1]), as_f32(u[2 * v + 1])));
 }
 
-// What one tile of the static schedule is: GEMM1 or GEMM2 (phase 1 or 2),
-// its place, and its global m-tile index.
+// Stage row `lane` of a 32-column block, scaled by wgt, at srow (16-byte
+// writes).
+__device__ __forceinline__ void stage_scaled32(uint8_t *srow, const uint32_t (&v)[32], float wgt) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<float4 *>(srow + 16 * j) =
+        make_float4(wgt * as_f32(v[4 * j]), wgt * as_f32(v[4 * j + 1]),
+                    wgt * as_f32(v[4 * j + 2]), wgt * as_f32(v[4 * j + 3]));
+}
+
+// What one tile number is: GEMM1 or GEMM2 (phase 1 or 2), its place, and
+// its global m-tile index.
 struct Work {
   int phase;
   int mi;
@@ -304,7 +348,7 @@ struct Work {
 };
 
 template <int MODE>
-__device__ __forceinline__ Work get_work(int t, int total1, const Params &p,
+__device__ __forceinline__ Work get_work(int t, int total1, int m_tiles, const Params &p,
                                          const int32_t *tile_off, const int32_t *exp_off) {
   Work w;
   int local = t, nt = p.nt1;
@@ -314,9 +358,66 @@ __device__ __forceinline__ Work get_work(int t, int total1, const Params &p,
     nt = p.nt2;
     if (MODE == kModeFused) local = t - total1;
   }
-  w.tl = decode_tile<tile_m<MODE>()>(local, nt, p.E, tile_off, exp_off);
+  if (w.phase == 2 && p.ngroup > 0) {
+    // column group g holds n-tiles [g * ngroup, min(nt2, (g + 1) * ngroup)):
+    // all of its tiles (expert-major) come before those of group g + 1
+    const int per = m_tiles * p.ngroup;
+    const int g = local / per;
+    const int ntg = min(p.ngroup, p.nt2 - g * p.ngroup);
+    w.tl = decode_tile<tile_m<MODE>()>(local - g * per, ntg, p.E, tile_off, exp_off);
+    w.tl.nt += g * p.ngroup;
+  } else {
+    w.tl = decode_tile<tile_m<MODE>()>(local, nt, p.E, tile_off, exp_off);
+  }
   w.mi = tile_off[w.tl.e] + w.tl.mt;
   return w;
+}
+
+// ---------------------------------------------------------------- tile queue
+// The scheduler (thread 0 of rank 0) writes its claimed tile number (-1
+// past the last tile) into slot seq % kTQ of both CTAs' queues once every
+// reader of that slot's previous use is done.  False if it gave up.  The
+// claim for the next tile is made as soon as this one is published, so
+// that its round trip to L2 overlaps this tile's loads.
+template <int CG>
+__device__ __forceinline__ bool publish_tile(Bars *bars, uint32_t seq, int total, int *sched,
+                                             int *claimed, uint64_t limit,
+                                             volatile int *abort_flag, int *tile) {
+  const int t = *claimed < total ? *claimed : -1;
+  const int q = static_cast<int>(seq % kTQ);
+  const uint32_t ph = (seq / kTQ) & 1;
+  if (!mbar_wait_cluster(&bars->tq_empty[q], ph ^ 1, limit, abort_flag)) return false;
+  bars->tq[q] = t;
+  mbar_arrive(&bars->tq_full[q]);
+  if (CG == 2) {
+    // the store is ordered before the remote arrive (release at cluster scope)
+    st_shared_cluster_s32(map_to_rank(smem_addr(&bars->tq[q]), 1), t);
+    mbar_arrive_cluster(map_to_rank(smem_addr(&bars->tq_full[q]), 1));
+  }
+  if (t >= 0) *claimed = atomicAdd(sched, 1);
+  *tile = t;
+  return true;
+}
+
+// A reader's side: the tile number of slot seq % kTQ.  Every lane of the
+// calling warp (or the single calling thread) waits and reads; the arrival
+// on rank 0's tq_empty is made once, by lane 0.  False if it gave up.
+__device__ __forceinline__ bool read_tile(Bars *bars, uint32_t seq, uint32_t rank,
+                                          uint32_t tq_empty0, uint64_t limit,
+                                          volatile int *abort_flag, bool arrive, int *tile) {
+  const int q = static_cast<int>(seq % kTQ);
+  const uint32_t ph = (seq / kTQ) & 1;
+  const bool ok = rank == 0 ? mbar_wait(&bars->tq_full[q], ph, limit, abort_flag)
+                            : mbar_wait_cluster(&bars->tq_full[q], ph, limit, abort_flag);
+  if (!ok) return false;
+  *tile = *reinterpret_cast<volatile int *>(&bars->tq[q]);
+  if (arrive) {
+    if (rank == 0)
+      mbar_arrive(&bars->tq_empty[q]);
+    else
+      mbar_arrive_cluster(tq_empty0 + 8u * q);
+  }
+  return true;
 }
 
 template <int MODE>
@@ -324,8 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a1,
                         const __grid_constant__ CUtensorMap tm_b1,
                         const __grid_constant__ CUtensorMap tm_a2,
-                        const __grid_constant__ CUtensorMap tm_b2,
-                        const __grid_constant__ CUtensorMap tm_out, const Params p) {
+                        const __grid_constant__ CUtensorMap tm_b2, const Params p) {
   using C = Cfg<MODE>;
   constexpr int CG = C::CG;
   constexpr int TM = tile_m<MODE>();
@@ -357,6 +457,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->acc_empty[a], kEpiWarps * CG);  // every epilogue warp of the pair
     }
     mbar_init(&bars->drain, 1);
+    for (int q = 0; q < kTQ; ++q) {
+      mbar_init(&bars->tq_full[q], 1);
+      mbar_init(&bars->tq_empty[q], queue_consumers<CG>());
+    }
     bars->abort_flag = 0;
     fence_mbar_init();
     if (MODE != kModeGemm2) prefetch_tmap(&tm_b1);
@@ -364,7 +468,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (MODE != kModeGemm1) {
       prefetch_tmap(&tm_a2);
       prefetch_tmap(&tm_b2);
-      if (!p.fuse_combine) prefetch_tmap(&tm_out);
     }
   }
   if (warp == kMmaWarp) {
@@ -379,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // both CTAs' barriers exist before any traffic crosses the pair
   if (CG == 2) cluster_sync();
   // Everything above overlaps the previous kernel under PDL; the routing
-  // permutation (and the A rows) are read only after this point.
+  // permutation, the counters and the A rows are read only after this point.
   grid_dep_wait();
   grid_dep_launch();
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_exp_off[i] = p.expert_offsets[i];
@@ -394,13 +497,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total1 = MODE == kModeGemm2 ? 0 : m_tiles * p.nt1;
   const int total =
       total1 + (MODE == kModeGemm1 || (MODE == kModeFused && !p.run_gemm2) ? 0 : m_tiles * p.nt2);
-  const int unit = CG == 2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int nunits = CG == 2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   volatile int *abort_flag = &bars->abort_flag;
   const uint64_t limit = p.wait_limit_ns;
   // rank 0's barriers as seen from this CTA
   const uint32_t full0 = CG == 2 ? map_to_rank(smem_addr(&bars->full[0]), 0) : 0u;
   const uint32_t acc_empty0 = CG == 2 ? map_to_rank(smem_addr(&bars->acc_empty[0]), 0) : 0u;
+  const uint32_t tq_empty0 =
+      CG == 2 ? map_to_rank(smem_addr(&bars->tq_empty[0]), 0) : smem_addr(&bars->tq_empty[0]);
 
   if (warp < 4) {
     // ------------------------------------------------------------ producers
@@ -410,9 +513,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int KB = p.H / BK;
       int s = 0;  // ring slot and its phase parity, advanced per k-block
       uint32_t ph = 0;
-      bool stop = false;
-      for (int t = unit; t < total && !stop; t += nunits) {
-        const Tile tl = get_work<MODE>(t, total1, p, s_tile_off, s_exp_off).tl;
+      // Every producer thread takes each tile through the two named barriers
+      // (a thread that gives up inside a tile still comes back to them), and
+      // all leave together when thread 0 hands out -1: past the last tile,
+      // or once the CTA has given up.
+      int claimed = threadIdx.x == 0 ? atomicAdd(p.sched, 1) : 0;  // thread 0: the scheduler
+      for (uint32_t seq = 0;; ++seq) {
+        if (threadIdx.x == 0) {
+          int t = -1;
+          if (!*abort_flag &&
+              !publish_tile<CG>(bars, seq, total, p.sched, &claimed, limit, abort_flag, &t)) {
+            give_up(p, abort_flag);
+            t = -1;
+          }
+          bars->prod_tile = t;
+        }
+        named_bar_sync(1, kProducerThreads);
+        const int t = *reinterpret_cast<volatile int *>(&bars->prod_tile);
+        // every producer thread has the tile before thread 0 may replace it
+        named_bar_sync(1, kProducerThreads);
+        if (t < 0) break;
+        const Tile tl = get_work<MODE>(t, total1, m_tiles, p, s_tile_off, s_exp_off).tl;
         const __nv_bfloat16 *src[8];
         uint32_t nbytes[8];
 #pragma unroll
@@ -431,7 +552,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < KB; ++kb, s = s + 1 == kStages ? 0 : s + 1, ph ^= s == 0) {
           if (!mbar_wait(&bars->empty[s], ph ^ 1, limit, abort_flag)) {
             give_up(p, abort_flag);
-            stop = true;
             break;
           }
           if (threadIdx.x == 0) {
@@ -451,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       cp_async_wait_all();
-      if (stop && threadIdx.x == 0) {
+      if (*abort_flag && threadIdx.x == 0) {
         // let TMA copies already issued land before the CTA can exit
         const uint64_t t0 = global_timer_ns();
         while (global_timer_ns() - t0 < 200000) {
@@ -461,10 +581,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0;  // ring slot and its phase parity, advanced per k-block
       uint32_t ph = 0;
       bool stop = false;
-      for (int t = unit; t < total && !stop; t += nunits) {
-        const Work w = get_work<MODE>(t, total1, p, s_tile_off, s_exp_off);
+      int claimed = leader ? atomicAdd(p.sched, 1) : 0;
+      for (uint32_t seq = 0; !stop; ++seq) {
+        int t = -1;
+        const bool ok =
+            leader ? publish_tile<CG>(bars, seq, total, p.sched, &claimed, limit, abort_flag, &t)
+                   : read_tile(bars, seq, rank, tq_empty0, limit, abort_flag, true, &t);
+        if (!ok) {
+          give_up(p, abort_flag);
+          break;
+        }
+        if (t < 0) break;
+        const Work w = get_work<MODE>(t, total1, m_tiles, p, s_tile_off, s_exp_off);
         if (MODE == kModeFused && w.phase == 2) {
-          // the act rows of this m-tile come from other CTAs' GEMM1 epilogues
+          // the act rows of this m-tile come from GEMM1 epilogues of tiles
+          // claimed before this one
           if (!wait_geq(p.ready + w.mi, kReadyPerTile * p.nt1, limit, abort_flag)) {
             give_up(p, abort_flag);
             break;
@@ -502,13 +633,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && leader) {
       // ---------------------------------------------------------- MMA issuer
       const uint32_t idesc = idesc_bf16_f32(TM, kAccN);
-      int s = 0, acc_it = 0;  // ring slot and its phase parity, advanced per k-block
+      int s = 0;  // ring slot and its phase parity, advanced per k-block
       uint32_t ph = 0;
       bool stop = false;
-      for (int t = unit; t < total && !stop; t += nunits, ++acc_it) {
-        const int KB = (get_work<MODE>(t, total1, p, s_tile_off, s_exp_off).phase == 1 ? p.H : p.I) / BK;
-        const int a = acc_it & 1;
-        const uint32_t aph = (acc_it >> 1) & 1;
+      for (uint32_t seq = 0; !stop; ++seq) {
+        int t = -1;
+        if (!read_tile(bars, seq, 0, tq_empty0, limit, abort_flag, true, &t)) {
+          give_up(p, abort_flag);
+          break;
+        }
+        if (t < 0) break;
+        const int KB =
+            (get_work<MODE>(t, total1, m_tiles, p, s_tile_off, s_exp_off).phase == 1 ? p.H : p.I) /
+            BK;
+        const int a = seq & 1;
+        const uint32_t aph = (seq >> 1) & 1;
         if (!mbar_wait(&bars->acc_empty[a], aph ^ 1, limit, abort_flag)) {
           give_up(p, abort_flag);
           break;
@@ -565,30 +704,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = ew >> 2;               // which half of the tile's columns
     const int row = q * 32 + lane;
     uint8_t *ebuf = sEpi + ew * kEpiWarpBytes;  // GEMM2: this warp's staging buffer
+    const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * kEpiWarps + ew;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kEpiWarps;
     if (MODE != kModeGemm2 && p.zero_n4 > 0) {
       // out must read zero before GEMM2 adds into it; this runs while the
-      // first tiles' MMAs are in flight
-      const int64_t nw = static_cast<int64_t>(gridDim.x) * kEpiWarps;
+      // first tiles' MMAs are in flight.  Chunks are claimed, so whichever
+      // CTAs run first zero all of out.
+      const int64_t n_chunks = (p.zero_n4 + kZeroChunk4 - 1) / kZeroChunk4;
       const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int64_t i = (static_cast<int64_t>(blockIdx.x) * kEpiWarps + ew) * 32 + lane;
-           i < p.zero_n4; i += nw * 32)
-        p.zero_out[i] = z;
-      if (MODE == kModeFused && p.run_gemm2) {
-        // publish: GEMM2 tiles of any CTA add into out only after every
-        // epilogue warp of the grid has zeroed its part
+      for (;;) {
+        int ch = 0;
+        if (lane == 0) ch = atomicAdd(p.zero_claim, 1);
+        ch = __shfl_sync(0xffffffffu, ch, 0);
+        if (ch >= n_chunks) break;
+        const int64_t i0 = static_cast<int64_t>(ch) * kZeroChunk4;
+        const int64_t i1 = min(i0 + kZeroChunk4, p.zero_n4);
+        for (int64_t i = i0 + lane; i < i1; i += 32) p.zero_out[i] = z;
         __threadfence();
         __syncwarp();
         if (lane == 0) atomicAdd(p.zero_done, 1);
       }
     }
+    if (MODE == kModeGemm1 && p.prepare_ordered) {
+      // the ordered GEMM2 launch that follows starts from zero turn
+      // counters, and never writes the rows of tokens without an expert id
+      // in [0, E): zero both here, while the first MMAs are in flight
+      for (int64_t i = gwarp * 32 + lane; i < p.turn_n; i += nwarps * 32) p.turn[i] = 0;
+      const int H4 = p.H / 4;
+      for (int64_t b = gwarp * 32; b < p.T; b += nwarps * 32) {
+        const int64_t t = b + lane;
+        bool empty = false;
+        if (t < p.T) {
+          empty = true;
+          for (int j = 0; j < p.k; ++j) {
+            const int e2 = __ldg(p.topk_ids + t * p.k + j);
+            if (e2 >= 0 && e2 < p.E) empty = false;
+          }
+        }
+        uint32_t m = __ballot_sync(0xffffffffu, empty);
+        while (m != 0) {
+          const int l = __ffs(static_cast<int>(m)) - 1;
+          m &= m - 1;
+          float4 *orow = reinterpret_cast<float4 *>(p.out) + (b + l) * H4;
+          for (int c = lane; c < H4; c += 32) orow[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+    }
+    const int64_t zero_chunks = (p.zero_n4 + kZeroChunk4 - 1) / kZeroChunk4;
     bool zero_seen = MODE != kModeFused || p.zero_n4 == 0 || !p.run_gemm2;
-    int acc_it = 0;
-    for (int t = unit; t < total; t += nunits, ++acc_it) {
-      const Work w = get_work<MODE>(t, total1, p, s_tile_off, s_exp_off);
+    for (uint32_t seq = 0;; ++seq) {
+      // waits are taken by every lane; their outcome is made warp-uniform
+      // before the warp-collective TMEM loads
+      int t = -1;
+      const bool got = read_tile(bars, seq, rank, tq_empty0, limit, abort_flag, lane == 0, &t);
+      if (!__all_sync(0xffffffffu, got)) {
+        give_up(p, abort_flag);
+        break;
+      }
+      t = __shfl_sync(0xffffffffu, t, 0);
+      if (t < 0) break;
+      const Work w = get_work<MODE>(t, total1, m_tiles, p, s_tile_off, s_exp_off);
       const Tile &tl = w.tl;
-      const int a = acc_it & 1;
-      const uint32_t aph = (acc_it >> 1) & 1;
-      if (!mbar_wait(&bars->acc_full[a], aph, limit, abort_flag)) {
+      const int a = seq & 1;
+      const uint32_t aph = (seq >> 1) & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->acc_full[a], aph, limit, abort_flag))) {
         give_up(p, abort_flag);
         break;
       }
@@ -629,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else if (p.fuse_combine) {
         if (!zero_seen) {
-          if (!wait_geq(p.zero_done, static_cast<int>(gridDim.x) * kEpiWarps, limit, abort_flag))
+          if (!wait_geq(p.zero_done, static_cast<int>(zero_chunks), limit, abort_flag))
             give_up(p, abort_flag);
           fence_proxy_async_global();
           zero_seen = true;
@@ -655,11 +834,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (col < p.H && valid && !*abort_flag) {
             // the previous reduction from this row must have read it
             bulk_wait_group_read<0>();
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<float4 *>(srow + 16 * j) =
-                  make_float4(wgt * as_f32(v[4 * j]), wgt * as_f32(v[4 * j + 1]),
-                              wgt * as_f32(v[4 * j + 2]), wgt * as_f32(v[4 * j + 3]));
+            stage_scaled32(srow, v, wgt);
             fence_proxy_async_smem();
             bulk_reduce_add_f32(orow + col, srow, 128);
             bulk_commit_group();
@@ -667,39 +842,65 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
         }
       } else {
-        // this warp's 32 rows: whole blocks go out through TMA stores
-        const bool whole = q * 32 + 32 <= my_rows;
-        const float *b2row = p.b2 ? p.b2 + static_cast<size_t>(tl.e) * p.H : nullptr;
+        // ordered (top-k > 2): this warp's rows, columns col0..col0+127
+        const int col0 = tl.nt * kAccN + half * (kAccN / 2);
+        const bool cols_ok = col0 < p.H;
+        int tok = 0, rank_p = 0;
+        float wgt = 0.f;
+        if (valid) {
+          const int slot = p.sorted_rows[my_row0 + row];
+          tok = slot / p.k;
+          const int j = slot - tok * p.k;
+          wgt = p.topk_weights[slot];
+          // this contribution's place among the token's: every slot whose
+          // expert is smaller, or the same expert in an earlier slot
+          const int32_t *tid = p.topk_ids + static_cast<size_t>(tok) * p.k;
+          for (int jj = 0; jj < p.k; ++jj) {
+            const int e2 = __ldg(tid + jj);
+            if (e2 >= 0 && e2 < p.E && (e2 < tl.e || (e2 == tl.e && jj < j))) ++rank_p;
+          }
+        }
+        // a token routed to this expert more than once has adjacent rows;
+        // those of this warp are taken in passes, earliest slot first
+        const uint32_t same = __match_any_sync(0xffffffffu, valid ? tok : -1 - lane);
+        const int depth = __popc(same & ((1u << lane) - 1u));
+        const int max_depth = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(depth));
+        int *tp = p.turn + static_cast<size_t>(tok) * (p.H >> 7) + (col0 >> 7);
+        float *orow = p.out + static_cast<size_t>(tok) * p.H + col0;
+        uint8_t *srow = ebuf + lane * kRedPitch;
+        const float *b2row = p.b2 ? p.b2 + static_cast<size_t>(tl.e) * p.H + col0 : nullptr;
+        for (int pass = 0; pass <= max_depth; ++pass) {
+          const bool mine = valid && cols_ok && depth == pass;
+          // the previous contribution (a tile claimed earlier) has landed
+          if (mine && rank_p > 0 && !wait_geq(tp, rank_p, limit, abort_flag))
+            give_up(p, abort_flag);
+          __syncwarp();
+          const bool go = mine && !*abort_flag;
+          if (go) fence_proxy_async_global();
 #pragma unroll 1
-        for (int c0 = half * (kAccN / 2); c0 < (half + 1) * (kAccN / 2); c0 += 32) {
-          uint32_t v[32];
-          tmem_ld_32cols(tbase + c0, v);
-          tmem_ld_wait();
-          const int col = tl.nt * kAccN + c0;
-          if (b2row && col < p.H) add_bias32(v, b2row + col);
-          if (col < p.H && whole) {
-            // the previous store from this buffer must have read it
-            if (lane == 0) bulk_wait_group_read<0>();
-            __syncwarp();
-            // row `lane` as 8 chunks of 16 bytes, 128-byte swizzle
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<uint4 *>(ebuf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                  make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_2d(&tm_out, ebuf, col, my_row0 + q * 32);
+          for (int c0 = 0; c0 < kAccN / 2; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld_32cols(tbase + half * (kAccN / 2) + c0, v);
+            tmem_ld_wait();
+            if (go) {
+              if (b2row) add_bias32(v, b2row + c0);
+              bulk_wait_group_read<0>();
+              stage_scaled32(srow, v, wgt);
+              fence_proxy_async_smem();
+              if (rank_p == 0)
+                bulk_store(orow + c0, srow, 128);
+              else
+                bulk_reduce_add_f32(orow + c0, srow, 128);
               bulk_commit_group();
             }
-          } else if (col < p.H && valid) {
-            // the block crosses the end of the expert's rows: plain stores
-            float4 *d4 = reinterpret_cast<float4 *>(
-                p.P + static_cast<size_t>(my_row0 + row) * p.H + col);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              d4[i] = make_float4(as_f32(v[4 * i]), as_f32(v[4 * i + 1]), as_f32(v[4 * i + 2]),
-                                  as_f32(v[4 * i + 3]));
+            __syncwarp();
+          }
+          if (go) {
+            // all four blocks are in global memory before the next
+            // contribution of this token may start
+            bulk_wait_group_all();
+            fence_proxy_async_global();
+            st_release_gpu(tp, rank_p + 1);
           }
           __syncwarp();
         }
@@ -768,24 +969,19 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major matrix [outer, inner] as a 2-D tensor map with a
-// (box_inner x box_rows) box and the 128-byte swizzle.
-bool make_map(CUtensorMap *m, CUtensorMapDataType dtype, int elem_bytes, const void *base,
-              uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_rows) {
+// Row-major bf16 matrix [outer, inner] as a 2-D tensor map with a
+// (64 x box_rows) box and the 128-byte swizzle.
+bool make_bf16_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
+                   uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {inner * elem_bytes};
-  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(m, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool make_bf16_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
-                   uint32_t box_rows) {
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, inner, outer, BK, box_rows);
 }
 
 int g_max_pairs[64] = {};  // 2-CTA clusters resident at once, per device
@@ -795,8 +991,7 @@ int grid_for(const GroupedGemmArgs &a, int n_tiles_n, int device) {
   constexpr int CG = Cfg<MODE>::CG;
   const int64_t rows = a.T * a.k;
   const int64_t max_tiles = ((rows + tile_m<MODE>() - 1) / tile_m<MODE>() + a.E) * n_tiles_n;
-  // never more units than can be resident together: the fused kernel's
-  // GEMM2 tiles wait for other CTAs' GEMM1 tiles
+  // one CTA (pair) per SM (pair) that can hold one: more would only queue
   int units = a.num_sms / CG;
   if (CG == 2 && device >= 0 && device < 64 && g_max_pairs[device] > 0)
     units = std::min(units, g_max_pairs[device]);
@@ -810,7 +1005,7 @@ Params base_params(const GroupedGemmArgs &a) {
   p.sorted_rows = a.sorted_rows;
   p.expert_offsets = a.expert_offsets;
   p.act = reinterpret_cast<__nv_bfloat16 *>(a.act);
-  p.P = a.P;
+  p.T = a.T;
   p.H = a.H;
   p.I = a.I;
   p.E = a.E;
@@ -819,15 +1014,18 @@ Params base_params(const GroupedGemmArgs &a) {
   p.nt2 = (a.H + kAccN - 1) / kAccN;  // H % 128 == 0: a last half tile is masked
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
-  p.fuse_combine = a.fuse_combine;
-  if (a.fuse_combine) {
-    p.out = a.out;
-    p.topk_weights = a.topk_weights;
+  p.out = a.out;
+  p.topk_weights = a.topk_weights;
+  p.topk_ids = a.topk_ids;
+  p.fuse_combine = a.ordered ? 0 : 1;
+  if (!a.ordered) {
     p.zero_out = reinterpret_cast<float4 *>(a.out);
     p.zero_n4 = a.T * a.H / 4;
   }
-  p.ready = a.ready;
-  p.zero_done = a.zero_done;
+  p.zero_claim = a.counters + kCounterZeroClaim;
+  p.zero_done = a.counters + kCounterZeroDone;
+  p.ready = a.counters + kCounterReady;
+  p.turn = a.turn;
   p.b1 = a.b1;
   p.b2 = a.b2;
   p.act_kind = a.act_kind;
@@ -874,28 +1072,28 @@ cudaError_t max_pairs(int *clusters) {
   return cudaOccupancyMaxActiveClusters(clusters, grouped_gemm_kernel<MODE>, &cfg);
 }
 
-// The maps GEMM2 uses: act [T*k, I] and w2 [E*H, I] with 64 x 128-row boxes,
-// and P [T*k, H] fp32 in 32 x 32 blocks (a stand-in map over act when P is
-// not written).
-bool gemm2_maps(const GroupedGemmArgs &a, CUtensorMap *tm_act, CUtensorMap *tm_w2,
-                CUtensorMap *tm_p) {
+// The maps GEMM2 uses: act [T*k, I] and w2 [E*H, I] with 64 x 128-row boxes.
+bool gemm2_maps(const GroupedGemmArgs &a, CUtensorMap *tm_act, CUtensorMap *tm_w2) {
   const uint64_t rows = static_cast<uint64_t>(a.T) * a.k;
-  if (!make_bf16_map(tm_act, a.act, static_cast<uint64_t>(a.I), rows, BM) ||
-      !make_bf16_map(tm_w2, a.w2, static_cast<uint64_t>(a.I), static_cast<uint64_t>(a.E) * a.H,
-                     Cfg<kModeGemm2>::kBRows))
-    return false;
-  if (a.P == nullptr) {
-    *tm_p = *tm_act;
-    return true;
-  }
-  return make_map(tm_p, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.P, static_cast<uint64_t>(a.H), rows,
-                  32, 32);
+  return make_bf16_map(tm_act, a.act, static_cast<uint64_t>(a.I), rows, BM) &&
+         make_bf16_map(tm_w2, a.w2, static_cast<uint64_t>(a.I), static_cast<uint64_t>(a.E) * a.H,
+                       Cfg<kModeGemm2>::kBRows);
 }
 
 // w1 [E*2I, H], box 64 x 128 rows (128 gate or 128 up rows of an n-tile)
 bool w1_map(const GroupedGemmArgs &a, CUtensorMap *tm_w1) {
   return make_bf16_map(tm_w1, a.w1, static_cast<uint64_t>(a.H),
                        static_cast<uint64_t>(a.E) * 2 * a.I, kAccN / 2);
+}
+
+// n-tiles per column group of the ordered GEMM2: the part of out that one
+// group adds into (T rows x 256 columns per n-tile, fp32) stays within
+// about 40 MB, a third of L2.
+int ordered_group_ntiles(const GroupedGemmArgs &a) {
+  const int64_t per_ntile = a.T * static_cast<int64_t>(kAccN) * 4;
+  const int64_t g = (static_cast<int64_t>(40) << 20) / std::max<int64_t>(per_ntile, 1);
+  const int nt2 = (a.H + kAccN - 1) / kAccN;
+  return static_cast<int>(std::min<int64_t>(std::max<int64_t>(g, 1), nt2));
 }
 
 }  // namespace
@@ -933,48 +1131,59 @@ cudaError_t launch_gemm1_swiglu(const GroupedGemmArgs &a, cudaStream_t s, const 
   int dev = 0;
   cudaGetDevice(&dev);
   Params p = base_params(a);
+  p.sched = a.counters + kCounterSched0;
+  p.zero_n4 = 0;  // nothing is added into out before the GEMM2 launch
+  if (a.ordered) {
+    p.prepare_ordered = 1;
+    p.turn_n = a.T * (a.H / 128);
+  }
   p.stages = stages_for<kModeGemm1>(a.E);
   cudaLaunchAttribute attr[2];
   const cudaLaunchConfig_t cfg =
       launch_config<kModeGemm1>(grid_for<kModeGemm1>(a, p.nt1, dev),
                                 smem_bytes<kModeGemm1>(a.E, p.stages), s, hook.pdl, attr);
   hook.begin("gemm1_swiglu");
-  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm1>, tm_w1, tm_w1, tm_w1,
-                                     tm_w1, tm_w1, p);
+  cudaError_t e =
+      cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm1>, tm_w1, tm_w1, tm_w1, tm_w1, p);
   return hook.end(e);
 }
 
 cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s, const StageHook &hook) {
-  CUtensorMap tm_act, tm_w2, tm_p;
-  if (!gemm2_maps(a, &tm_act, &tm_w2, &tm_p)) return cudaErrorInvalidValue;
+  CUtensorMap tm_act, tm_w2;
+  if (!gemm2_maps(a, &tm_act, &tm_w2)) return cudaErrorInvalidValue;
   int dev = 0;
   cudaGetDevice(&dev);
   Params p = base_params(a);
-  p.zero_out = nullptr;  // zeroed by GEMM1
+  p.sched = a.counters + kCounterSched1;
+  p.zero_out = nullptr;  // zeroed by the GEMM1 launch
   p.zero_n4 = 0;
+  if (a.ordered) {
+    p.ordered = 1;
+    p.ngroup = ordered_group_ntiles(a);
+  }
   p.stages = stages_for<kModeGemm2>(a.E);
   cudaLaunchAttribute attr[2];
   const cudaLaunchConfig_t cfg =
       launch_config<kModeGemm2>(grid_for<kModeGemm2>(a, p.nt2, dev),
                                 smem_bytes<kModeGemm2>(a.E, p.stages), s, hook.pdl, attr);
   hook.begin("gemm2");
-  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm2>, tm_act, tm_w2, tm_act,
-                                     tm_w2, tm_p, p);
+  cudaError_t e =
+      cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm2>, tm_act, tm_w2, tm_act, tm_w2, p);
   return hook.end(e);
 }
 
 cudaError_t launch_fused_gemm(const GroupedGemmArgs &a, bool with_gemm2, cudaStream_t s,
                               const StageHook &hook) {
-  if (a.xs == nullptr || (with_gemm2 && (a.ready == nullptr || a.zero_done == nullptr)))
-    return cudaErrorInvalidValue;
-  CUtensorMap tm_xs, tm_w1, tm_act, tm_w2, tm_p;
+  if (a.xs == nullptr || a.ordered) return cudaErrorInvalidValue;
+  CUtensorMap tm_xs, tm_w1, tm_act, tm_w2;
   if (!make_bf16_map(&tm_xs, a.xs, static_cast<uint64_t>(a.H), static_cast<uint64_t>(a.T) * a.k,
                      BM) ||
-      !w1_map(a, &tm_w1) || !gemm2_maps(a, &tm_act, &tm_w2, &tm_p))
+      !w1_map(a, &tm_w1) || !gemm2_maps(a, &tm_act, &tm_w2))
     return cudaErrorInvalidValue;
   int dev = 0;
   cudaGetDevice(&dev);
   Params p = base_params(a);
+  p.sched = a.counters + kCounterSched0;
   p.run_gemm2 = with_gemm2 ? 1 : 0;
   p.stages = stages_for<kModeFused>(a.E, with_gemm2);
   cudaLaunchAttribute attr[2];
@@ -982,8 +1191,8 @@ cudaError_t launch_fused_gemm(const GroupedGemmArgs &a, bool with_gemm2, cudaStr
       grid_for<kModeFused>(a, with_gemm2 ? p.nt1 + p.nt2 : p.nt1, dev),
       smem_bytes<kModeFused>(a.E, p.stages, with_gemm2), s, hook.pdl, attr);
   hook.begin(with_gemm2 ? "gemm_fused" : "gemm1_swiglu");
-  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeFused>, tm_xs, tm_w1, tm_act,
-                                     tm_w2, tm_p, p);
+  cudaError_t e =
+      cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeFused>, tm_xs, tm_w1, tm_act, tm_w2, p);
   return hook.end(e);
 }
 

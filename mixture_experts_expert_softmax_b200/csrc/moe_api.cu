@@ -259,24 +259,22 @@ int moe_permute_ex(const int32_t *topk_ids, int64_t T, int k, int E, int32_t *so
   DeviceState *d = nullptr;
   int rc = current_device(&d);
   if (rc != MOE_OK) return rc;
-  // chunk counts of the three-kernel grouping, and the counters that the
-  // row copy zeroes for the fused GEMM (none here but the done flag)
-  if ((rc = ensure_workspace(*d, permute_ws_bytes(n, E) + 256)) != MOE_OK) return rc;
+  // chunk counts of the three-kernel grouping
+  if ((rc = ensure_workspace(*d, permute_ws_bytes(n, E))) != MOE_OK) return rc;
   Carver cv{static_cast<char *>(d->ws)};
   int32_t *chunk_counts = cv.take<int32_t>(std::max(moe::permute_num_chunks(n), 1) * static_cast<size_t>(E));
-  int *zero_done = cv.take<int>(1);
   CallCtx ctx{static_cast<cudaStream_t>(stream), "", nullptr};
   moe::StageHook hook = make_hook(&ctx);
   cudaError_t e;
   if (single) {
     e = moe::launch_group(topk_ids, n, E, k, expert_offsets, sorted_rows, inv, nullptr, hidden, H,
-                          xs, nullptr, 0, zero_done, d->num_sms, ctx.stream, hook);
+                          xs, nullptr, 0, d->num_sms, ctx.stream, hook);
   } else {
     e = moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets, sorted_rows, inv,
-                            nullptr, ctx.stream, hook);
+                            nullptr, nullptr, 0, ctx.stream, hook);
     if (e == cudaSuccess && xs != nullptr)
       e = moe::launch_gather_rows(hidden, H, k, sorted_rows, expert_offsets, E, n, d->num_sms, xs,
-                                  zero_done, 0, zero_done, ctx.stream, hook);
+                                  nullptr, 0, ctx.stream, hook);
   }
   return to_code(e);
 }
@@ -372,19 +370,19 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
     w2 = wd2;
   }
 
-  // top-k <= 2: GEMM2 adds its rows straight into out and no P is needed
-  const bool fuse_combine = k <= 2;
   // Copying the hidden rows into expert-sorted order costs k row copies per
   // token and lets GEMM1 run on CTA pairs with TMA operands; with few slots
-  // per token that pays off.
+  // per token that pays off.  With more slots GEMM2 orders each token's
+  // contributions (turn counters) instead of adding them in any order.
   const bool gather_rows = k <= 2;
-  const int64_t n_ready = moe::fused_gemm_ready_count(n, E);
+  const bool ordered = k > 2;
+  const int64_t n_counters = moe::gemm_counter_count(n, E);
+  const size_t n_turn = ordered ? static_cast<size_t>(T) * (H / 128) : 0;
   const size_t need = permute_ws_bytes(n, E) + align256(static_cast<size_t>(n) * 4) +
                       align256(static_cast<size_t>(n) * I * 2) +
-                      (gather_rows ? align256(static_cast<size_t>(n) * H * 2) +
-                                         align256(static_cast<size_t>(n_ready + 1) * 4)
-                                   : 0) +
-                      (fuse_combine ? 0 : align256(static_cast<size_t>(n) * H * sizeof(float)));
+                      align256(static_cast<size_t>(n_counters) * 4) +
+                      (gather_rows ? align256(static_cast<size_t>(n) * H * 2) : 0) +
+                      (ordered ? align256(n_turn * 4) : 0);
   if ((rc = ensure_workspace(*d, need)) != MOE_OK) return rc;
   Carver cv{static_cast<char *>(d->ws)};
   int32_t *chunk_counts =
@@ -393,25 +391,25 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
   int32_t *inv = cv.take<int32_t>(std::max<int64_t>(n, 1));
   int32_t *expert_offsets = cv.take<int32_t>(E + 1);
   uint16_t *act = cv.take<uint16_t>(static_cast<size_t>(n) * I);
-  float *P = fuse_combine ? nullptr : cv.take<float>(static_cast<size_t>(n) * H);
+  int *counters = cv.take<int>(static_cast<size_t>(n_counters));
   uint16_t *xs = gather_rows ? cv.take<uint16_t>(static_cast<size_t>(n) * H) : nullptr;
-  int *ready = gather_rows ? cv.take<int>(static_cast<size_t>(n_ready) + 1) : nullptr;
+  int *turn = ordered ? cv.take<int>(n_turn) : nullptr;
 
   // grouping (and the sorted row copy): one kernel up to 8192 entries, the
-  // three-kernel grouping and a separate copy above
+  // three-kernel grouping and a separate copy above; either zeroes the
+  // GEMMs' counters
   if (moe::group_supported(n)) {
     e = moe::launch_group(topk_ids, n, E, k, expert_offsets, sorted_rows, inv, d->status, hidden,
-                          H, xs, ready, static_cast<int>(n_ready), ready + n_ready, d->num_sms,
-                          ctx.stream, hook);
+                          H, xs, counters, static_cast<int>(n_counters), d->num_sms, ctx.stream,
+                          hook);
     if (e != cudaSuccess) return to_code(e);
   } else {
     e = moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets, sorted_rows, inv,
-                            d->status, ctx.stream, hook);
+                            d->status, counters, static_cast<int>(n_counters), ctx.stream, hook);
     if (e != cudaSuccess) return to_code(e);
     if (gather_rows &&
         (e = moe::launch_gather_rows(hidden, H, k, sorted_rows, expert_offsets, E, n, d->num_sms,
-                                     xs, ready, static_cast<int>(n_ready), ready + n_ready,
-                                     ctx.stream, hook)) != cudaSuccess)
+                                     xs, nullptr, 0, ctx.stream, hook)) != cudaSuccess)
       return to_code(e);
   }
   moe::GroupedGemmArgs ga = {};
@@ -422,7 +420,12 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
   ga.expert_offsets = expert_offsets;
   ga.xs = xs;
   ga.act = act;
-  ga.P = P;
+  ga.out = out;
+  ga.topk_weights = topk_weights;
+  ga.topk_ids = topk_ids;
+  ga.ordered = ordered ? 1 : 0;
+  ga.turn = turn;
+  ga.counters = counters;
   ga.T = T;
   ga.H = H;
   ga.I = I;
@@ -431,15 +434,10 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
   ga.num_sms = d->num_sms;
   ga.status = d->status;
   ga.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns);
-  ga.out = out;
-  ga.topk_weights = topk_weights;
-  ga.fuse_combine = fuse_combine ? 1 : 0;
   ga.b1 = b1;
   ga.b2 = b2;
   ga.act_kind = act_kind;
   if (gather_rows) {
-    ga.ready = ready;
-    ga.zero_done = ready + n_ready;
     // One launch for both GEMMs fills GEMM1's last partial wave with GEMM2
     // tiles; with many waves that gain is small and two launches, each with
     // the deepest operand ring its shared memory allows, run faster.
@@ -453,9 +451,7 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
     if ((e = moe::launch_gemm1_swiglu(ga, ctx.stream, hook)) != cudaSuccess) return to_code(e);
     if ((e = moe::launch_gemm2(ga, ctx.stream, hook)) != cudaSuccess) return to_code(e);
   }
-  if (fuse_combine) return MOE_OK;
-  e = moe::launch_combine(P, inv, topk_weights, out, T, H, k, d->status, ctx.stream, hook);
-  return to_code(e);
+  return MOE_OK;
 }
 
 }  // namespace

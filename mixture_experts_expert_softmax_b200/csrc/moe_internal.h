@@ -43,32 +43,48 @@ cudaError_t launch_route(const float *logits, int64_t T, int E, int k, int renor
                          float *weights, cudaStream_t s);
 
 // permute.cu
+// Every grouping launcher also zeroes zero[0..zero_n), the counters of the
+// GEMM launches that follow (their tile schedulers, the act readiness
+// counters of the one-launch GEMM); zero may be null when zero_n is 0.
 int permute_num_chunks(int64_t n);
 cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int32_t *chunk_counts,
                            int32_t *expert_offsets, int32_t *sorted_rows, int32_t *inv,
-                           uint32_t *status, cudaStream_t s, const StageHook &hook);
+                           uint32_t *status, int *zero, int zero_n, cudaStream_t s,
+                           const StageHook &hook);
 
 // Stable grouping of n <= 8192 entries in one kernel (the same result as
 // launch_permute), with the expert-sorted copy of the hidden rows when xs
-// is given (then also zeroing the fused GEMM's counters, as
-// launch_gather_rows does).  group_setup raises the kernel's shared-memory
-// limit once per device.
+// is given.  group_setup raises the kernel's shared-memory limit once per
+// device.
 bool group_supported(int64_t n);
 cudaError_t group_setup();
 cudaError_t launch_group(const int32_t *ids, int64_t n, int E, int k, int32_t *expert_offsets,
                          int32_t *sorted_rows, int32_t *inv, uint32_t *status,
-                         const uint16_t *hidden, int H, uint16_t *xs, int *ready, int n_ready,
-                         int *zero_done, int num_sms, cudaStream_t s, const StageHook &hook);
+                         const uint16_t *hidden, int H, uint16_t *xs, int *zero, int zero_n,
+                         int num_sms, cudaStream_t s, const StageHook &hook);
 
 // Expert-sorted copy of the hidden rows, xs[r] = hidden[sorted_rows[r] / k]
-// for r < expert_offsets[E] (device value); n = T*k bounds the grid.  Also
-// zeroes the fused GEMM's counters: ready[0..n_ready) and *zero_done.
+// for r < expert_offsets[E] (device value); n = T*k bounds the grid.
 cudaError_t launch_gather_rows(const uint16_t *hidden, int H, int k, const int32_t *sorted_rows,
                                const int32_t *expert_offsets, int E, int64_t n, int num_sms,
-                               uint16_t *xs, int *ready, int n_ready, int *zero_done,
-                               cudaStream_t s, const StageHook &hook);
+                               uint16_t *xs, int *zero, int zero_n, cudaStream_t s,
+                               const StageHook &hook);
 
 // grouped_gemm.cu
+// Counters of the GEMM launches of one forward, in one int block that the
+// grouping stage zeroes: the tile scheduler of the first and of the second
+// GEMM launch, the claimed and finished chunks of zeroing out, then one act
+// readiness counter per 256-row m-tile of the one-launch GEMM.
+constexpr int kCounterSched0 = 0;
+constexpr int kCounterSched1 = 1;
+constexpr int kCounterZeroClaim = 2;
+constexpr int kCounterZeroDone = 3;
+constexpr int kCounterReady = 4;
+inline int64_t fused_gemm_ready_count(int64_t n, int E) { return (n + 255) / 256 + E; }
+inline int64_t gemm_counter_count(int64_t n, int E) {
+  return kCounterReady + fused_gemm_ready_count(n, E);
+}
+
 struct GroupedGemmArgs {
   const uint16_t *hidden;  // [T, H] bf16
   const uint16_t *w1;      // [E, 2I, H] bf16
@@ -79,16 +95,16 @@ struct GroupedGemmArgs {
   // or null: GEMM1 then runs on single CTAs and gathers its A rows itself
   const uint16_t *xs;
   uint16_t *act;  // [T*k, I] bf16, expert-sorted rows
-  float *P;       // [T*k, H] fp32, expert-sorted rows (unused when fuse_combine)
-  // fuse_combine (k <= 2): GEMM1 zeroes out, and GEMM2 adds w * y of each
-  // row straight into out[token] instead of writing P.
   float *out;                 // [T, H] fp32
   const float *topk_weights;  // [T, k] fp32
-  int fuse_combine;
-  // launch_fused_gemm: one counter per 256-row m-tile (at most
-  // fused_gemm_ready_count(T*k, E)) and one more, all zero at launch
-  int *ready;
-  int *zero_done;
+  const int32_t *topk_ids;    // [T, k] int32
+  // 0 (top-k <= 2): GEMM1 zeroes out and GEMM2 adds w * y of each row into
+  // it in any order.  1 (top-k > 2): GEMM1 zeroes turn and the rows of
+  // tokens without a valid id; GEMM2 stores, then adds, each token's
+  // contributions in ascending expert order.
+  int ordered;
+  int *turn;      // ordered: [T, H / 128] int
+  int *counters;  // gemm_counter_count(T*k, E) ints, zero at the first GEMM launch
   // epilogue variant: activation (kAct* of common.cuh) and optional fp32
   // biases b1 [E, 2I] (gate, then up) and b2 [E, H], 16-byte aligned
   const float *b1;
@@ -104,11 +120,9 @@ cudaError_t grouped_gemm_setup(int device);
 cudaError_t launch_gemm1_swiglu(const GroupedGemmArgs &a, cudaStream_t s, const StageHook &hook);
 cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s, const StageHook &hook);
 // GEMM1 + SwiGLU on CTA pairs from the expert-sorted rows xs, and (with_gemm2)
-// GEMM2 in the same launch, which needs ready and zero_done.  Without it,
-// launch_gemm2 follows.
+// GEMM2 in the same launch.  Without it, launch_gemm2 follows.
 cudaError_t launch_fused_gemm(const GroupedGemmArgs &a, bool with_gemm2, cudaStream_t s,
                               const StageHook &hook);
-inline int64_t fused_gemm_ready_count(int64_t n, int E) { return (n + 255) / 256 + E; }
 cudaError_t launch_wait_probe(uint32_t *status, uint64_t limit_ns, cudaStream_t s);
 
 // dequant.cu: out[r, c] = bf16(e4m3(q[r, c]) * scale[r, c / block]) for a
@@ -117,11 +131,6 @@ cudaError_t launch_wait_probe(uint32_t *status, uint64_t limit_ns, cudaStream_t 
 cudaError_t launch_dequant_e4m3(const uint8_t *q, const float *scale, int64_t rows, int K,
                                 int block, uint16_t *out, int num_sms, cudaStream_t s,
                                 const StageHook &hook);
-
-// combine.cu
-cudaError_t launch_combine(const float *P, const int32_t *inv, const float *topk_weights,
-                           float *out, int64_t T, int H, int k, uint32_t *status, cudaStream_t s,
-                           const StageHook &hook);
 
 // small_t.cu
 bool small_t_supported(int H, int I);

@@ -45,13 +45,14 @@ __global__ void __launch_bounds__(kPermThreads)
 
 // One CTA of 1024 threads.  Turns chunk_counts into per-chunk exclusive
 // bases (in place) and writes expert_offsets[E+1] (exclusive scan of the
-// per-expert totals).
+// per-expert totals).  Also zeroes the GEMMs' counters zero[0..zero_n).
 __global__ void __launch_bounds__(1024)
     permute_scan_kernel(int32_t *__restrict__ chunk_counts, int n_chunks, int E,
-                        int32_t *__restrict__ expert_offsets) {
+                        int32_t *__restrict__ expert_offsets, int *zero, int zero_n) {
   __shared__ int32_t s_warp_cnt[32];
   grid_dep_wait();
   grid_dep_launch();
+  for (int x = threadIdx.x; x < zero_n; x += blockDim.x) zero[x] = 0;
   const int e = threadIdx.x;
   int32_t total = 0;
   if (e < E) {
@@ -153,10 +154,10 @@ __global__ void __launch_bounds__(kPermThreads)
 // entries and counts it into its own 16-bit histogram row, a scan over
 // (expert, warp) turns the counts into bases, and a second pass ranks each
 // warp step with __match_any_sync -- so the result equals the three-kernel
-// grouping above.  CTA 0 publishes it (expert_offsets, sorted_rows, inv);
-// all CTAs then copy their share of rows from their own copy of the
-// permutation, with no grid-wide synchronisation.  Only CTA 0 runs when
-// nothing is copied.
+// grouping above.  CTA 0 publishes it (expert_offsets, sorted_rows, inv)
+// and zeroes the GEMMs' counters zero[0..zero_n); all CTAs then copy their
+// share of rows from their own copy of the permutation, with no grid-wide
+// synchronisation.  Only CTA 0 runs when nothing is copied.
 constexpr int kGroupThreads = 1024;
 constexpr int kGroupWarps = kGroupThreads / 32;
 constexpr int64_t kGroupMaxN = 8192;  // above this the multi-CTA kernels are faster
@@ -172,7 +173,7 @@ __global__ void __launch_bounds__(kGroupThreads)
     group_kernel(const int32_t *__restrict__ ids, int n, int E, int k,
                  int32_t *__restrict__ expert_offsets, int32_t *__restrict__ sorted_rows,
                  int32_t *__restrict__ inv, uint32_t *status, const uint4 *__restrict__ hidden,
-                 int H8, uint4 *__restrict__ xs, int *ready, int n_ready, int *zero_done) {
+                 int H8, uint4 *__restrict__ xs, int *zero, int zero_n) {
   extern __shared__ __align__(16) unsigned char group_smem[];
   int32_t *s_sorted = reinterpret_cast<int32_t *>(group_smem);      // [n]
   int32_t *s_tot = s_sorted + ((n + 3) & ~3);                         // [E]
@@ -283,10 +284,8 @@ __global__ void __launch_bounds__(kGroupThreads)
     }
     __syncwarp();
   }
-  if (publish && ready != nullptr) {
-    for (int x = tid; x < n_ready; x += kGroupThreads) ready[x] = 0;
-    if (tid == 0) *zero_done = 0;
-  }
+  if (publish)
+    for (int x = tid; x < zero_n; x += kGroupThreads) zero[x] = 0;
   if (xs == nullptr) return;
   __syncthreads();
   const int nv = s_nvalid;
@@ -303,18 +302,16 @@ __global__ void __launch_bounds__(kGroupThreads)
 // sorted order, xs[r] = hidden[sorted_rows[r] / k], so that GEMM1 can load
 // its A tiles with TMA.  One warp per row, 16-byte chunks; rows past
 // expert_offsets[E] (entries with invalid ids) are not written.  Block 0
-// also zeroes the fused GEMM's counters.
+// also zeroes the GEMMs' counters zero[0..zero_n).
 __global__ void __launch_bounds__(256)
     gather_rows_kernel(const uint4 *__restrict__ hidden, int H8, int k,
                        const int32_t *__restrict__ sorted_rows,
                        const int32_t *__restrict__ expert_offsets, int E,
-                       uint4 *__restrict__ xs, int *ready, int n_ready, int *zero_done) {
+                       uint4 *__restrict__ xs, int *zero, int zero_n) {
   grid_dep_wait();
   grid_dep_launch();
-  if (blockIdx.x == 0) {
-    for (int i = threadIdx.x; i < n_ready; i += blockDim.x) ready[i] = 0;
-    if (threadIdx.x == 0) *zero_done = 0;
-  }
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < zero_n; i += blockDim.x) zero[i] = 0;
   const int64_t n_valid = expert_offsets[E];
   const int lane = threadIdx.x & 31;
   const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -332,16 +329,16 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_gather_rows(const uint16_t *hidden, int H, int k, const int32_t *sorted_rows,
                                const int32_t *expert_offsets, int E, int64_t n, int num_sms,
-                               uint16_t *xs, int *ready, int n_ready, int *zero_done,
-                               cudaStream_t s, const StageHook &hook) {
+                               uint16_t *xs, int *zero, int zero_n, cudaStream_t s,
+                               const StageHook &hook) {
   const int64_t want = (n + 7) / 8;  // 8 warps per CTA, one row each per pass
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;
   const int blocks = static_cast<int>(want < cap ? want : cap);
   hook.begin("gather_rows");
   cudaError_t e = launch_pdl(gather_rows_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, s,
                              hook.pdl, reinterpret_cast<const uint4 *>(hidden), H / 8, k,
-                             sorted_rows, expert_offsets, E, reinterpret_cast<uint4 *>(xs), ready,
-                             n_ready, zero_done);
+                             sorted_rows, expert_offsets, E, reinterpret_cast<uint4 *>(xs), zero,
+                             zero_n);
   return hook.end(e);
 }
 
@@ -356,8 +353,8 @@ cudaError_t group_setup() {
 
 cudaError_t launch_group(const int32_t *ids, int64_t n, int E, int k, int32_t *expert_offsets,
                          int32_t *sorted_rows, int32_t *inv, uint32_t *status,
-                         const uint16_t *hidden, int H, uint16_t *xs, int *ready, int n_ready,
-                         int *zero_done, int num_sms, cudaStream_t s, const StageHook &hook) {
+                         const uint16_t *hidden, int H, uint16_t *xs, int *zero, int zero_n,
+                         int num_sms, cudaStream_t s, const StageHook &hook) {
   int grid = 1;
   if (xs != nullptr) {
     const int64_t want = (n + kGroupWarps - 1) / kGroupWarps;  // one row per warp
@@ -370,13 +367,14 @@ cudaError_t launch_group(const int32_t *ids, int64_t n, int E, int k, int32_t *e
                                group_smem_bytes(static_cast<int>(n), E), s, hook.pdl, ids,
                                static_cast<int>(n), E, k, expert_offsets, sorted_rows, inv, status,
                                reinterpret_cast<const uint4 *>(hidden), H / 8,
-                               reinterpret_cast<uint4 *>(xs), ready, n_ready, zero_done);
+                               reinterpret_cast<uint4 *>(xs), zero, zero_n);
   return hook.end(err);
 }
 
 cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int32_t *chunk_counts,
                            int32_t *expert_offsets, int32_t *sorted_rows, int32_t *inv,
-                           uint32_t *status, cudaStream_t s, const StageHook &hook) {
+                           uint32_t *status, int *zero, int zero_n, cudaStream_t s,
+                           const StageHook &hook) {
   const int n_chunks = permute_num_chunks(n);
   cudaError_t err;
   if (n_chunks > 0) {
@@ -389,7 +387,7 @@ cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int32_t *chunk_
   }
   hook.begin("permute_scan");
   err = launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, s, hook.pdl, chunk_counts,
-                   n_chunks, E, expert_offsets);
+                   n_chunks, E, expert_offsets, zero, zero_n);
   if ((err = hook.end(err)) != cudaSuccess) return err;
   if (n_chunks > 0) {
     hook.begin("permute_scatter");

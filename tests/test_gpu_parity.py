@@ -279,7 +279,8 @@ def test_forward_small_t_shared_and_duplicate_experts():
 @pytest.mark.parametrize("small,k", [(16, 2), (0, 2), (0, 4)])
 def test_forward_invalid_ids_are_skipped_and_flagged(small, k):
     """k = 2 on the GEMM path flags bad ids in the grouping (GEMM2 adds into
-    out); k = 4 also goes through the separate combine."""
+    zeroed out); k = 4 orders the contributions, and GEMM1 zeroes the row of
+    the token without a valid id."""
     T, H, I, E = 12, 256, 128, 8
     hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=11)
     ids, w = oracle.route(logits.numpy(), k, True)
@@ -317,7 +318,8 @@ def test_forward_zero_token_gives_zero_row(small):
 def test_forward_deterministic(T, H, I, E, k):
     """Identical bits on repeated calls: with k <= 2 GEMM2 adds two rounded
     products onto zero in whatever order the tiles finish (a commutative
-    sum), with k > 2 the combine sums in fixed order."""
+    sum), with k > 2 each token's contributions are added in ascending
+    expert order, whatever order the tiles finish in."""
     hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=5)
     ids, w = oracle.route(logits.numpy(), k, True)
     prev = moe.set_small_t_max(0)
@@ -328,6 +330,39 @@ def test_forward_deterministic(T, H, I, E, k):
     finally:
         moe.set_small_t_max(prev)
     assert np.array_equal(a, b) and np.array_equal(a, c)
+
+
+@pytest.mark.parametrize("T,H,I,E,k", [(1979, 2048, 2048, 8, 2), (2000, 1024, 384, 64, 8)])
+def test_forward_beside_other_work(T, H, I, E, k):
+    """The forward while another stream keeps the SMs busy with matrix
+    products: tiles are claimed by whichever CTAs run, so the result must be
+    exact and no bounded wait may run out (which would raise the timeout
+    bit), however few CTAs are resident at first."""
+    hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=31)
+    ids, w = oracle.route(logits.numpy(), k, True)
+    dev = torch.device("cuda")
+    args = [hidden.to(dev), w1.to(dev), w2.to(dev),
+            torch.as_tensor(w.astype(np.float32)).to(dev), torch.as_tensor(ids).to(dev)]
+    prev = moe.set_small_t_max(0)
+    try:
+        alone = moe.moe_forward(*args)
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream()
+        a = torch.randn(4096, 4096, device=dev, dtype=torch.bfloat16)
+        outs = []
+        for _ in range(3):
+            with torch.cuda.stream(side):
+                for _ in range(20):
+                    a = (a @ a).clamp_(-1, 1)
+            outs.append(moe.moe_forward(*args))
+        torch.cuda.synchronize()
+    finally:
+        moe.set_small_t_max(prev)
+    check_status_clean()
+    for o in outs:
+        assert torch.equal(o, alone)
+    ref = oracle.moe_token_loop(hidden, w1, w2, w, ids, rows=np.arange(0, T, 7))
+    assert_output_close(alone.cpu().numpy()[::7], ref, f"T={T} k={k}")
 
 
 def test_forward_gemm_duplicate_slots_top2():
@@ -375,7 +410,7 @@ def test_end_to_end_route_then_forward():
 # ------------------------------------------------------------------ epilogue variants
 VARIANT_CASES = [
     (64, 256, 128, 8, 2),      # tiny: one-kernel grouping, both GEMMs in one launch
-    (333, 384, 384, 16, 4),    # k > 2: separate GEMM launches, fp32 P, combine
+    (333, 384, 384, 16, 4),    # k > 2: separate GEMM launches, ordered contributions
     (100, 256, 128, 128, 8),   # many experts below one tile
 ]
 
@@ -475,7 +510,7 @@ def gpu_forward_fp8(hidden, q1, s1, q2, s2, block, w, ids):
     (3, 512, 256, 4, 2, 256, "small_t"),       # tokens sharing experts
     (4, 2048, 768, 128, 8, 256, "gemm"),
     (64, 256, 128, 8, 2, 128, "gemm"),         # tiny: one-launch GEMMs
-    (100, 384, 384, 16, 4, 128, "gemm"),       # k > 2: P and combine, half n-tile
+    (100, 384, 384, 16, 4, 128, "gemm"),       # k > 2: ordered contributions, half n-tile
 ])
 def test_forward_fp8(T, H, I, E, k, block, path):
     from moe_inputs import make_fp8_weights
@@ -653,6 +688,7 @@ def test_sync_each_stage_mode_and_profiler():
         moe.profile_enable(False)
         moe.set_sync_each_stage(prev)
     prof = moe.profile_read()
-    for kname in ("permute", "gemm1_swiglu", "gemm2", "combine"):
+    for kname in ("permute", "gemm1_swiglu", "gemm2"):
         assert prof[kname][0] == 1 and prof[kname][1] > 0
+    assert "combine" not in prof
     assert_output_close(out, oracle.moe_token_loop(hidden, w1, w2, w, ids))
