@@ -5,7 +5,8 @@
 
 A step is one pass of the whole hot path over one batch: moe_route (softmax,
 top-k, renormalisation) then moe_forward (grouping, GEMM1+SwiGLU, GEMM2 with
-the weighted top-k sum -- or the small-T GEMV path) on synthetic inputs with the shapes and
+the weighted top-k sum, plus a fixed-order combine pass for top-k > 2 -- or
+the small-T GEMV path) on synthetic inputs with the shapes and
 distributions of the atrex-bench #009 "fused_moe" workload.  The headline
 workload is "prefill, few large experts" (T=1979, H=2048, I=2048, E=8,
 top-k 2); the other workloads are reported under "per_shape" (--shapes table:

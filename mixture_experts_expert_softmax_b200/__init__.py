@@ -49,6 +49,7 @@ EXPORTED = (
     "moe_set_wait_limit_ns", "moe_last_failed_stage", "moe_debug_wait_timeout",
     "moe_profile_enable", "moe_profile_reset", "moe_profile_read",
     "moe_forward_small_noalloc", "moe_forward_ex", "moe_forward_fp8", "moe_permute_ex",
+    "moe_timeline",
 )
 
 
@@ -70,6 +71,7 @@ def _load() -> ctypes.CDLL:
         "moe_forward": ([P, P, P, P, P, P, I64, I32, I32, I32, I32, P], I32),
         "moe_permute": ([P, I64, I32, I32, P, P, P], I32),
         "moe_permute_ex": ([P, I64, I32, I32, P, P, P, P, I32, P, I32, P], I32),
+        "moe_timeline": ([P, I64], I32),
         "moe_error_string": ([I32], ctypes.c_char_p),
         "moe_get_device_status": ([P, ctypes.POINTER(ctypes.c_uint32)], I32),
         "moe_set_small_t_max": ([I32], I32),
@@ -287,6 +289,61 @@ def moe_permute_ex(topk_ids: torch.Tensor, E: int, kernel: str = "auto",
     return sorted_rows, expert_offsets, inv, xs
 
 
+TIMELINE_KINDS = {1: "gemm1", 2: "gemm2", 3: "gemm_fused", 4: "small_t"}
+TIMELINE_ROLES = {0: "producer", 1: "mma", 2: "epilogue", 3: "phase1", 4: "barrier",
+                  5: "phase2"}
+_timeline_buf = None
+
+
+def timeline_start(capacity: int = 1 << 16, device=None) -> None:
+    """Record the kernels' per-tile / per-phase timeline (moe_timeline) into
+    a fresh device buffer until timeline_stop()."""
+    global _timeline_buf
+    _timeline_buf = torch.zeros(4 + 4 * int(capacity), dtype=torch.int64,
+                                device=device or torch.device("cuda"))
+    _check(_lib.moe_timeline(_timeline_buf.data_ptr(), int(capacity)), "moe_timeline")
+
+
+def timeline_stop() -> list[dict]:
+    """Stop recording; synchronise and return the records as dicts
+    {kind, role, cta, sub, id, t0, t1} (nanoseconds of %globaltimer)."""
+    global _timeline_buf
+    _check(_lib.moe_timeline(None, 0), "moe_timeline")
+    if _timeline_buf is None:
+        return []
+    torch.cuda.synchronize()
+    raw = _timeline_buf.cpu()
+    _timeline_buf = None
+    n = min(int(raw[0]), (raw.numel() - 4) // 4)
+    rec = raw[4:4 + 4 * n].view(n, 4).tolist()
+    out = []
+    for tag, ident, t0, t1 in rec:
+        tag &= (1 << 64) - 1
+        out.append({"kind": TIMELINE_KINDS.get(tag >> 56, str(tag >> 56)),
+                    "role": TIMELINE_ROLES.get((tag >> 48) & 0xff, str((tag >> 48) & 0xff)),
+                    "cta": (tag >> 16) & 0xffffffff, "sub": tag & 0xffff, "id": ident,
+                    "t0": t0 & ((1 << 64) - 1), "t1": t1 & ((1 << 64) - 1)})
+    return out
+
+
+def timeline_summary(records: list[dict]) -> dict:
+    """Per (kind, role): record count, mean and max duration (us), and the
+    span from the earliest t0 to the latest t1 (us); per kind also the
+    share of that span the busiest and the idlest CTA spent in its MMA or
+    phase records."""
+    import collections
+    out: dict = {}
+    by = collections.defaultdict(list)
+    for r in records:
+        by[(r["kind"], r["role"])].append(r)
+    for (kind, role), rs in sorted(by.items()):
+        d = [(r["t1"] - r["t0"]) / 1e3 for r in rs]
+        out[f"{kind}/{role}"] = {
+            "n": len(rs), "mean_us": round(sum(d) / len(d), 3), "max_us": round(max(d), 3),
+            "span_us": round((max(r["t1"] for r in rs) - min(r["t0"] for r in rs)) / 1e3, 3)}
+    return out
+
+
 def get_device_status(stream=None) -> int:
     """Synchronise, return and clear the OR of MOE_STATUS_* bits."""
     v = ctypes.c_uint32(0)
@@ -341,5 +398,6 @@ __all__ = [
     "moe_permute_ex", "get_device_status", "set_small_t_max",
     "set_sync_each_stage", "set_wait_limit_ns", "last_failed_stage", "debug_wait_timeout",
     "profile_enable", "profile_reset", "profile_read", "error_string", "MoEError",
+    "timeline_start", "timeline_stop", "timeline_summary",
     "LIB_PATH", "EXPORTED", "ACTS",
 ]

@@ -113,10 +113,6 @@ __device__ __forceinline__ int ld_acquire_gpu(const int *p) {
   return v;
 }
 
-__device__ __forceinline__ void st_release_gpu(int *p, int v) {
-  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 // Bounded wait until *p >= target (acquire at GPU scope): false when the
 // limit passes or *abort becomes non-zero first.
 __device__ __forceinline__ bool wait_geq(const int *p, int target, uint64_t limit_ns,
@@ -189,15 +185,6 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *s
 // aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_reduce_add_f32(float *dst, const void *src, uint32_t bytes) {
   asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
-                   reinterpret_cast<uint64_t>(dst)),
-               "r"(smem_addr(src)), "r"(bytes)
-               : "memory");
-}
-
-// 1-D bulk copy shared -> global (bulk-group completion).  Both addresses
-// 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
                    reinterpret_cast<uint64_t>(dst)),
                "r"(smem_addr(src)), "r"(bytes)
                : "memory");
@@ -402,6 +389,31 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t *bar, uint16_t cta_mas
       " [%0], %1;" ::"r"(smem_addr(bar)),
       "h"(cta_mask)
       : "memory");
+}
+
+// ---------------------------------------------------------------- timeline
+// Debug timeline (moe_timeline): buf[0] counts the records written so far;
+// record i is buf[4 + 4i .. 4 + 4i + 3] = {tag, id, t0, t1}, with %globaltimer
+// nanoseconds t0 <= t1 and tag = kind << 56 | role << 48 | cta << 16 | sub.
+// Records past `cap` are counted but not written.  buf == null: off.
+enum : uint32_t {
+  kTlGemm1 = 1, kTlGemm2 = 2, kTlFused = 3, kTlSmallT = 4,  // kinds
+  kTlProducer = 0, kTlMma = 1, kTlEpilogue = 2,             // roles (GEMM kernels)
+  kTlPhase1 = 3, kTlBarrier = 4, kTlPhase2 = 5              // roles (small-T kernel)
+};
+
+__device__ __forceinline__ void timeline_rec(uint64_t *buf, int64_t cap, uint32_t kind,
+                                             uint32_t role, uint32_t sub, uint64_t id,
+                                             uint64_t t0, uint64_t t1) {
+  if (buf == nullptr) return;
+  const unsigned long long i = atomicAdd(reinterpret_cast<unsigned long long *>(buf), 1ull);
+  if (static_cast<int64_t>(i) >= cap) return;
+  uint64_t *r = buf + 4 + 4 * i;
+  r[0] = static_cast<uint64_t>(kind) << 56 | static_cast<uint64_t>(role) << 48 |
+         static_cast<uint64_t>(blockIdx.x & 0xffffffffu) << 16 | (sub & 0xffffu);
+  r[1] = id;
+  r[2] = t0;
+  r[3] = t1;
 }
 
 // ---------------------------------------------------------------- PDL

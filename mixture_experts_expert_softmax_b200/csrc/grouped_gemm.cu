@@ -12,12 +12,9 @@
 //       out[token] with bulk reductions at L2 (out was zeroed first);
 //       out[t] = 0 + a + b is the same in either arrival order, so the
 //       result is deterministic.
-//     - top-k > 2 (ordered): each token's contributions go into out in
-//       ascending expert order -- the order of the per-expert loop of
-//       atrex-bench #009 Model.forward -- the first one stored, the others
-//       added at L2 with bulk reductions, each after the previous one has
-//       landed (a turn counter per token and 128-column block).  No
-//       per-(token, slot) buffer and no separate combine pass.
+//     - top-k > 2: the epilogue stores y as fp32 rows of P in the same
+//       expert-sorted order (TMA tile stores) and combine.cu forms
+//       sum_j w_j * y_j in fixed j order.
 // This is the expert FFN of ref_moe on the page "tpu_inference/kernels/
 // fused_moe/v1/kernel.py" (gate = w1, up = w3, then act . w2) in the weight
 // layout of atrex-bench #009 (w1 [E, 2I, H], w2 [E, H, I], both applied as
@@ -25,16 +22,15 @@
 //
 // Work unit: an m-tile of one expert's rows times one 256-column n-tile of
 // the accumulator.  Tiles are numbered expert-major, then n-tile, then
-// m-tile, so CTAs working together share a weight tile through L2 (the
-// ordered GEMM2 takes its n-tiles in column groups first, so that the part
-// of out it adds into stays in L2).  Tiles are handed out dynamically: the
+// m-tile, so CTAs working together share a weight tile through L2.  Tiles
+// are handed out dynamically: the
 // first thread of each CTA (pair) claims the next tile number from a global
 // counter and publishes it through a small queue in shared memory to every
 // role of the CTA(s).  Tiles are claimed in number order, and every wait
-// across tiles (GEMM2 rows on the act rows of GEMM1 tiles, an ordered
-// contribution on the previous expert's) points to a tile with a smaller
-// number, which a running CTA has already claimed: progress never depends on
-// a CTA that has not started, whatever else occupies the GPU.
+// across tiles (GEMM2 rows on the act rows of GEMM1 tiles) points to a tile
+// with a smaller number, which a running CTA has already claimed: progress
+// never depends on a CTA that has not started, whatever else occupies the
+// GPU.
 //
 // Three kernels share the code (MODE):
 //   kModeFused   one launch on CTA pairs (a cluster of 2, M = 256,
@@ -56,10 +52,12 @@
 //                and load gate and up rows themselves: no row copy needed.
 //   kModeGemm2   GEMM2 alone on CTA pairs.
 // The GEMM2 epilogue stages each warp's 32 rows x 32 columns in shared
-// memory and scales row r by its top-k weight; it issues one 128-byte bulk
-// reduce-add (or, first in the order, bulk copy) per row into out[token]:
-// large operations, because the TMA engine's cost per operation, not the
-// bytes, bounds this epilogue.
+// memory and writes them with one asynchronous TMA tile store into P (a
+// block that straddles the end of an expert's rows is written row by row
+// instead), or, fused with the combine, scales row r by its top-k weight
+// and issues one 128-byte bulk reduce-add per row into out[token]: large
+// operations, because the TMA engine's cost per operation, not the bytes,
+// bounds this epilogue.
 //
 // Shared memory: the barriers and the expert / tile offset tables sit in
 // front, then (1024-byte aligned, as the 128-byte swizzle needs) the stage
@@ -79,8 +77,8 @@
 //              producers and each finished tile to the epilogues.
 //   warps 5-12 epilogue, two warps per 32-lane TMEM quarter (a warp can only
 //              read the quarter warp_id % 4), each taking half of the tile's
-//              columns: tcgen05.ld, SwiGLU + bf16 store, or the weighted
-//              bulk reductions into out, then release the accumulator.
+//              columns: tcgen05.ld, SwiGLU + bf16 store, or the fp32 TMA
+//              store / bulk reductions, then release the accumulator.
 // Every wait is bounded; a wait that gives up raises the timeout bit of the
 // status word and makes every role of the CTA leave its loop.
 #include <algorithm>
@@ -104,10 +102,12 @@ constexpr int kMaxE = 1024;
 constexpr int kMaxStages = 6;
 constexpr int kTQ = 8;  // depth of the tile queue
 constexpr uint16_t kBothCtas = 0x3;
-// Per-warp staging of the GEMM2 epilogue: 32 rows of 32 fp32 values at a
-// 144-byte pitch (16-byte writes of 8 consecutive lanes then hit 8
+// Per-warp staging of the GEMM2 epilogue: one 32-row x 32-column fp32 block,
+// 128-byte swizzled for the TMA store, or 32 plain rows at a 144-byte pitch
+// for the reductions (16-byte writes of 8 consecutive lanes then hit 8
 // different bank groups: bank conflicts here would take shared-memory
-// bandwidth from the tensor core's operand reads).
+// bandwidth from the tensor core's operand reads).  A 1024-byte multiple
+// keeps every warp's block swizzle-aligned.
 constexpr int kRedPitch = 144;
 constexpr int kEpiWarpBytes = 5 * 1024;
 static_assert(32 * kRedPitch <= kEpiWarpBytes, "staging");
@@ -212,21 +212,12 @@ struct Params {
   int64_t zero_n4;
   int *zero_claim;
   int *zero_done;
-  // GEMM2's combine: out [T, H] and the top-k weights [T, k]
+  // GEMM2 fused with the combine (top-k <= 2): out [T, H] and the top-k
+  // weights [T, k]; otherwise GEMM2 writes P [T*k, H] fp32
   float *out;
   const float *topk_weights;
-  int fuse_combine;  // top-k <= 2: add into zeroed out in any order
-  // top-k > 2: ordered contributions guarded by turn [T, H / 128] (zero at
-  // the GEMM2 launch), ranked with topk_ids [T, k]; GEMM2 tiles in column
-  // groups of ngroup n-tiles
-  int ordered;
-  int *turn;
-  const int32_t *topk_ids;
-  int ngroup;
-  // kModeGemm1 ahead of an ordered GEMM2: zero turn (turn_n ints) and the
-  // out rows of tokens without an expert id in [0, E)
-  int64_t turn_n;
-  int prepare_ordered;
+  int fuse_combine;
+  float *P;
   // kModeFused: per-m-tile act counters (zero at launch)
   int *ready;
   // epilogue variant: activation (kAct*) and optional fp32 biases
@@ -234,6 +225,10 @@ struct Params {
   const float *b1;
   const float *b2;
   int act_kind;
+  // debug timeline (see timeline_rec): null when off
+  uint64_t *tl_buf;
+  int64_t tl_cap;
+  uint32_t tl_kind;
 };
 
 struct Tile {
@@ -348,7 +343,7 @@ struct Work {
 };
 
 template <int MODE>
-__device__ __forceinline__ Work get_work(int t, int total1, int m_tiles, const Params &p,
+__device__ __forceinline__ Work get_work(int t, int total1, const Params &p,
                                          const int32_t *tile_off, const int32_t *exp_off) {
   Work w;
   int local = t, nt = p.nt1;
@@ -358,17 +353,7 @@ __device__ __forceinline__ Work get_work(int t, int total1, int m_tiles, const P
     nt = p.nt2;
     if (MODE == kModeFused) local = t - total1;
   }
-  if (w.phase == 2 && p.ngroup > 0) {
-    // column group g holds n-tiles [g * ngroup, min(nt2, (g + 1) * ngroup)):
-    // all of its tiles (expert-major) come before those of group g + 1
-    const int per = m_tiles * p.ngroup;
-    const int g = local / per;
-    const int ntg = min(p.ngroup, p.nt2 - g * p.ngroup);
-    w.tl = decode_tile<tile_m<MODE>()>(local - g * per, ntg, p.E, tile_off, exp_off);
-    w.tl.nt += g * p.ngroup;
-  } else {
-    w.tl = decode_tile<tile_m<MODE>()>(local, nt, p.E, tile_off, exp_off);
-  }
+  w.tl = decode_tile<tile_m<MODE>()>(local, nt, p.E, tile_off, exp_off);
   w.mi = tile_off[w.tl.e] + w.tl.mt;
   return w;
 }
@@ -425,7 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a1,
                         const __grid_constant__ CUtensorMap tm_b1,
                         const __grid_constant__ CUtensorMap tm_a2,
-                        const __grid_constant__ CUtensorMap tm_b2, const Params p) {
+                        const __grid_constant__ CUtensorMap tm_b2,
+                        const __grid_constant__ CUtensorMap tm_out, const Params p) {
   using C = Cfg<MODE>;
   constexpr int CG = C::CG;
   constexpr int TM = tile_m<MODE>();
@@ -468,6 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (MODE != kModeGemm1) {
       prefetch_tmap(&tm_a2);
       prefetch_tmap(&tm_b2);
+      if (!p.fuse_combine) prefetch_tmap(&tm_out);
     }
   }
   if (warp == kMmaWarp) {
@@ -533,7 +520,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // every producer thread has the tile before thread 0 may replace it
         named_bar_sync(1, kProducerThreads);
         if (t < 0) break;
-        const Tile tl = get_work<MODE>(t, total1, m_tiles, p, s_tile_off, s_exp_off).tl;
+        const uint64_t tl_t0 = p.tl_buf ? global_timer_ns() : 0;
+        const Tile tl = get_work<MODE>(t, total1, p, s_tile_off, s_exp_off).tl;
         const __nv_bfloat16 *src[8];
         uint32_t nbytes[8];
 #pragma unroll
@@ -569,6 +557,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           // counts as this thread's arrival on full[s] once its copies land
           cp_async_arrive_noinc(&bars->full[s]);
         }
+        if (threadIdx.x == 0)
+          timeline_rec(p.tl_buf, p.tl_cap, p.tl_kind, kTlProducer, rank, t, tl_t0,
+                       global_timer_ns());
       }
       cp_async_wait_all();
       if (*abort_flag && threadIdx.x == 0) {
@@ -592,7 +583,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         if (t < 0) break;
-        const Work w = get_work<MODE>(t, total1, m_tiles, p, s_tile_off, s_exp_off);
+        const uint64_t tl_t0 = p.tl_buf ? global_timer_ns() : 0;
+        const Work w = get_work<MODE>(t, total1, p, s_tile_off, s_exp_off);
         if (MODE == kModeFused && w.phase == 2) {
           // the act rows of this m-tile come from GEMM1 epilogues of tiles
           // claimed before this one
@@ -622,6 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d_pair(sA + s * kABytes, am, full0 + 8u * s, kb * BK, a_row);
           tma_load_2d_pair(sB + s * kBBytes, bm, full0 + 8u * s, kb * BK, b_row);
         }
+        timeline_rec(p.tl_buf, p.tl_cap, p.tl_kind, kTlProducer, rank, t, tl_t0,
+                     global_timer_ns());
       }
       if (*abort_flag) {
         const uint64_t t0 = global_timer_ns();
@@ -644,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (t < 0) break;
         const int KB =
-            (get_work<MODE>(t, total1, m_tiles, p, s_tile_off, s_exp_off).phase == 1 ? p.H : p.I) /
+            (get_work<MODE>(t, total1, p, s_tile_off, s_exp_off).phase == 1 ? p.H : p.I) /
             BK;
         const int a = seq & 1;
         const uint32_t aph = (seq >> 1) & 1;
@@ -653,6 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after_sync();
+        const uint64_t tl_t0 = p.tl_buf ? global_timer_ns() : 0;
         const uint32_t d_tmem = tmem_base + a * kAccN;
         for (int kb = 0; kb < KB; ++kb, s = s + 1 == kStages ? 0 : s + 1, ph ^= s == 0) {
           if (!mbar_wait(&bars->full[s], ph, limit, abort_flag)) {
@@ -685,6 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           else
             umma_commit(&bars->acc_full[a]);
         }
+        timeline_rec(p.tl_buf, p.tl_cap, p.tl_kind, kTlMma, 0, t, tl_t0, global_timer_ns());
       }
       // every MMA must be complete before TMEM is released
       if (CG == 2)
@@ -725,31 +721,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) atomicAdd(p.zero_done, 1);
       }
     }
-    if (MODE == kModeGemm1 && p.prepare_ordered) {
-      // the ordered GEMM2 launch that follows starts from zero turn
-      // counters, and never writes the rows of tokens without an expert id
-      // in [0, E): zero both here, while the first MMAs are in flight
-      for (int64_t i = gwarp * 32 + lane; i < p.turn_n; i += nwarps * 32) p.turn[i] = 0;
-      const int H4 = p.H / 4;
-      for (int64_t b = gwarp * 32; b < p.T; b += nwarps * 32) {
-        const int64_t t = b + lane;
-        bool empty = false;
-        if (t < p.T) {
-          empty = true;
-          for (int j = 0; j < p.k; ++j) {
-            const int e2 = __ldg(p.topk_ids + t * p.k + j);
-            if (e2 >= 0 && e2 < p.E) empty = false;
-          }
-        }
-        uint32_t m = __ballot_sync(0xffffffffu, empty);
-        while (m != 0) {
-          const int l = __ffs(static_cast<int>(m)) - 1;
-          m &= m - 1;
-          float4 *orow = reinterpret_cast<float4 *>(p.out) + (b + l) * H4;
-          for (int c = lane; c < H4; c += 32) orow[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      }
-    }
     const int64_t zero_chunks = (p.zero_n4 + kZeroChunk4 - 1) / kZeroChunk4;
     bool zero_seen = MODE != kModeFused || p.zero_n4 == 0 || !p.run_gemm2;
     for (uint32_t seq = 0;; ++seq) {
@@ -763,18 +734,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       t = __shfl_sync(0xffffffffu, t, 0);
       if (t < 0) break;
-      const Work w = get_work<MODE>(t, total1, m_tiles, p, s_tile_off, s_exp_off);
+      const Work w = get_work<MODE>(t, total1, p, s_tile_off, s_exp_off);
       const Tile &tl = w.tl;
       const int a = seq & 1;
       const uint32_t aph = (seq >> 1) & 1;
+      const int my_row0 = tl.row0 + static_cast<int>(rank) * BM;
+      const int my_rows = min(BM, max(0, tl.rows - static_cast<int>(rank) * BM));
+      const bool valid = row < my_rows;
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->acc_full[a], aph, limit, abort_flag))) {
         give_up(p, abort_flag);
         break;
       }
       tc_fence_after_sync();
-      const int my_row0 = tl.row0 + static_cast<int>(rank) * BM;
-      const int my_rows = min(BM, max(0, tl.rows - static_cast<int>(rank) * BM));
-      const bool valid = row < my_rows;
+      const uint64_t tl_t0 = p.tl_buf && ew == 0 ? global_timer_ns() : 0;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kAccN;
       if (w.phase == 1) {
         __nv_bfloat16 *dst =
@@ -842,65 +814,39 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
         }
       } else {
-        // ordered (top-k > 2): this warp's rows, columns col0..col0+127
-        const int col0 = tl.nt * kAccN + half * (kAccN / 2);
-        const bool cols_ok = col0 < p.H;
-        int tok = 0, rank_p = 0;
-        float wgt = 0.f;
-        if (valid) {
-          const int slot = p.sorted_rows[my_row0 + row];
-          tok = slot / p.k;
-          const int j = slot - tok * p.k;
-          wgt = p.topk_weights[slot];
-          // this contribution's place among the token's: every slot whose
-          // expert is smaller, or the same expert in an earlier slot
-          const int32_t *tid = p.topk_ids + static_cast<size_t>(tok) * p.k;
-          for (int jj = 0; jj < p.k; ++jj) {
-            const int e2 = __ldg(tid + jj);
-            if (e2 >= 0 && e2 < p.E && (e2 < tl.e || (e2 == tl.e && jj < j))) ++rank_p;
-          }
-        }
-        // a token routed to this expert more than once has adjacent rows;
-        // those of this warp are taken in passes, earliest slot first
-        const uint32_t same = __match_any_sync(0xffffffffu, valid ? tok : -1 - lane);
-        const int depth = __popc(same & ((1u << lane) - 1u));
-        const int max_depth = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(depth));
-        int *tp = p.turn + static_cast<size_t>(tok) * (p.H >> 7) + (col0 >> 7);
-        float *orow = p.out + static_cast<size_t>(tok) * p.H + col0;
-        uint8_t *srow = ebuf + lane * kRedPitch;
-        const float *b2row = p.b2 ? p.b2 + static_cast<size_t>(tl.e) * p.H + col0 : nullptr;
-        for (int pass = 0; pass <= max_depth; ++pass) {
-          const bool mine = valid && cols_ok && depth == pass;
-          // the previous contribution (a tile claimed earlier) has landed
-          if (mine && rank_p > 0 && !wait_geq(tp, rank_p, limit, abort_flag))
-            give_up(p, abort_flag);
-          __syncwarp();
-          const bool go = mine && !*abort_flag;
-          if (go) fence_proxy_async_global();
+        // this warp's 32 rows: whole blocks go out through TMA stores
+        const bool whole = q * 32 + 32 <= my_rows;
+        const float *b2row = p.b2 ? p.b2 + static_cast<size_t>(tl.e) * p.H : nullptr;
 #pragma unroll 1
-          for (int c0 = 0; c0 < kAccN / 2; c0 += 32) {
-            uint32_t v[32];
-            tmem_ld_32cols(tbase + half * (kAccN / 2) + c0, v);
-            tmem_ld_wait();
-            if (go) {
-              if (b2row) add_bias32(v, b2row + c0);
-              bulk_wait_group_read<0>();
-              stage_scaled32(srow, v, wgt);
-              fence_proxy_async_smem();
-              if (rank_p == 0)
-                bulk_store(orow + c0, srow, 128);
-              else
-                bulk_reduce_add_f32(orow + c0, srow, 128);
+        for (int c0 = half * (kAccN / 2); c0 < (half + 1) * (kAccN / 2); c0 += 32) {
+          uint32_t v[32];
+          tmem_ld_32cols(tbase + c0, v);
+          tmem_ld_wait();
+          const int col = tl.nt * kAccN + c0;
+          if (b2row && col < p.H) add_bias32(v, b2row + col);
+          if (col < p.H && whole) {
+            // the previous store from this buffer must have read it
+            if (lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
+            // row `lane` as 8 chunks of 16 bytes, 128-byte swizzle
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4 *>(ebuf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                  make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tm_out, ebuf, col, my_row0 + q * 32);
               bulk_commit_group();
             }
-            __syncwarp();
-          }
-          if (go) {
-            // all four blocks are in global memory before the next
-            // contribution of this token may start
-            bulk_wait_group_all();
-            fence_proxy_async_global();
-            st_release_gpu(tp, rank_p + 1);
+          } else if (col < p.H && valid) {
+            // the block crosses the end of the expert's rows: plain stores
+            float4 *d4 = reinterpret_cast<float4 *>(
+                p.P + static_cast<size_t>(my_row0 + row) * p.H + col);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              d4[i] = make_float4(as_f32(v[4 * i]), as_f32(v[4 * i + 1]), as_f32(v[4 * i + 2]),
+                                  as_f32(v[4 * i + 3]));
           }
           __syncwarp();
         }
@@ -912,6 +858,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_cluster(acc_empty0 + 8u * a);
         else
           mbar_arrive(&bars->acc_empty[a]);
+        if (ew == 0)
+          timeline_rec(p.tl_buf, p.tl_cap, p.tl_kind, kTlEpilogue, rank, t, tl_t0,
+                       global_timer_ns());
       }
       if (MODE == kModeFused && w.phase == 1 && p.run_gemm2) {
         // publish this warp's act rows of the m-tile to GEMM2 tiles (after
@@ -969,19 +918,24 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major bf16 matrix [outer, inner] as a 2-D tensor map with a
-// (64 x box_rows) box and the 128-byte swizzle.
-bool make_bf16_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
-                   uint32_t box_rows) {
+// Row-major matrix [outer, inner] as a 2-D tensor map with a
+// (box_inner x box_rows) box and the 128-byte swizzle.
+bool make_map(CUtensorMap *m, CUtensorMapDataType dtype, int elem_bytes, const void *base,
+              uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {inner * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), box_rows};
+  const cuuint64_t strides[1] = {inner * elem_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  return enc(m, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_bf16_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
+                   uint32_t box_rows) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, inner, outer, BK, box_rows);
 }
 
 int g_max_pairs[64] = {};  // 2-CTA clusters resident at once, per device
@@ -1016,19 +970,20 @@ Params base_params(const GroupedGemmArgs &a) {
   p.wait_limit_ns = a.wait_limit_ns;
   p.out = a.out;
   p.topk_weights = a.topk_weights;
-  p.topk_ids = a.topk_ids;
-  p.fuse_combine = a.ordered ? 0 : 1;
-  if (!a.ordered) {
+  p.fuse_combine = a.P == nullptr ? 1 : 0;
+  p.P = a.P;
+  if (p.fuse_combine) {
     p.zero_out = reinterpret_cast<float4 *>(a.out);
     p.zero_n4 = a.T * a.H / 4;
   }
   p.zero_claim = a.counters + kCounterZeroClaim;
   p.zero_done = a.counters + kCounterZeroDone;
   p.ready = a.counters + kCounterReady;
-  p.turn = a.turn;
   p.b1 = a.b1;
   p.b2 = a.b2;
   p.act_kind = a.act_kind;
+  p.tl_buf = a.timeline;
+  p.tl_cap = a.timeline_cap;
   return p;
 }
 
@@ -1072,28 +1027,28 @@ cudaError_t max_pairs(int *clusters) {
   return cudaOccupancyMaxActiveClusters(clusters, grouped_gemm_kernel<MODE>, &cfg);
 }
 
-// The maps GEMM2 uses: act [T*k, I] and w2 [E*H, I] with 64 x 128-row boxes.
-bool gemm2_maps(const GroupedGemmArgs &a, CUtensorMap *tm_act, CUtensorMap *tm_w2) {
+// The maps GEMM2 uses: act [T*k, I] and w2 [E*H, I] with 64 x 128-row boxes,
+// and P [T*k, H] fp32 in 32 x 32 blocks (a stand-in map over act when P is
+// not written).
+bool gemm2_maps(const GroupedGemmArgs &a, CUtensorMap *tm_act, CUtensorMap *tm_w2,
+                CUtensorMap *tm_p) {
   const uint64_t rows = static_cast<uint64_t>(a.T) * a.k;
-  return make_bf16_map(tm_act, a.act, static_cast<uint64_t>(a.I), rows, BM) &&
-         make_bf16_map(tm_w2, a.w2, static_cast<uint64_t>(a.I), static_cast<uint64_t>(a.E) * a.H,
-                       Cfg<kModeGemm2>::kBRows);
+  if (!make_bf16_map(tm_act, a.act, static_cast<uint64_t>(a.I), rows, BM) ||
+      !make_bf16_map(tm_w2, a.w2, static_cast<uint64_t>(a.I), static_cast<uint64_t>(a.E) * a.H,
+                     Cfg<kModeGemm2>::kBRows))
+    return false;
+  if (a.P == nullptr) {
+    *tm_p = *tm_act;
+    return true;
+  }
+  return make_map(tm_p, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.P, static_cast<uint64_t>(a.H), rows,
+                  32, 32);
 }
 
 // w1 [E*2I, H], box 64 x 128 rows (128 gate or 128 up rows of an n-tile)
 bool w1_map(const GroupedGemmArgs &a, CUtensorMap *tm_w1) {
   return make_bf16_map(tm_w1, a.w1, static_cast<uint64_t>(a.H),
                        static_cast<uint64_t>(a.E) * 2 * a.I, kAccN / 2);
-}
-
-// n-tiles per column group of the ordered GEMM2: the part of out that one
-// group adds into (T rows x 256 columns per n-tile, fp32) stays within
-// about 40 MB, a third of L2.
-int ordered_group_ntiles(const GroupedGemmArgs &a) {
-  const int64_t per_ntile = a.T * static_cast<int64_t>(kAccN) * 4;
-  const int64_t g = (static_cast<int64_t>(40) << 20) / std::max<int64_t>(per_ntile, 1);
-  const int nt2 = (a.H + kAccN - 1) / kAccN;
-  return static_cast<int>(std::min<int64_t>(std::max<int64_t>(g, 1), nt2));
 }
 
 }  // namespace
@@ -1132,11 +1087,8 @@ cudaError_t launch_gemm1_swiglu(const GroupedGemmArgs &a, cudaStream_t s, const 
   cudaGetDevice(&dev);
   Params p = base_params(a);
   p.sched = a.counters + kCounterSched0;
+  p.tl_kind = kTlGemm1;
   p.zero_n4 = 0;  // nothing is added into out before the GEMM2 launch
-  if (a.ordered) {
-    p.prepare_ordered = 1;
-    p.turn_n = a.T * (a.H / 128);
-  }
   p.stages = stages_for<kModeGemm1>(a.E);
   cudaLaunchAttribute attr[2];
   const cudaLaunchConfig_t cfg =
@@ -1144,23 +1096,20 @@ cudaError_t launch_gemm1_swiglu(const GroupedGemmArgs &a, cudaStream_t s, const 
                                 smem_bytes<kModeGemm1>(a.E, p.stages), s, hook.pdl, attr);
   hook.begin("gemm1_swiglu");
   cudaError_t e =
-      cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm1>, tm_w1, tm_w1, tm_w1, tm_w1, p);
+      cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm1>, tm_w1, tm_w1, tm_w1, tm_w1, tm_w1, p);
   return hook.end(e);
 }
 
 cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s, const StageHook &hook) {
-  CUtensorMap tm_act, tm_w2;
-  if (!gemm2_maps(a, &tm_act, &tm_w2)) return cudaErrorInvalidValue;
+  CUtensorMap tm_act, tm_w2, tm_p;
+  if (!gemm2_maps(a, &tm_act, &tm_w2, &tm_p)) return cudaErrorInvalidValue;
   int dev = 0;
   cudaGetDevice(&dev);
   Params p = base_params(a);
   p.sched = a.counters + kCounterSched1;
+  p.tl_kind = kTlGemm2;
   p.zero_out = nullptr;  // zeroed by the GEMM1 launch
   p.zero_n4 = 0;
-  if (a.ordered) {
-    p.ordered = 1;
-    p.ngroup = ordered_group_ntiles(a);
-  }
   p.stages = stages_for<kModeGemm2>(a.E);
   cudaLaunchAttribute attr[2];
   const cudaLaunchConfig_t cfg =
@@ -1168,22 +1117,23 @@ cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s, const StageHo
                                 smem_bytes<kModeGemm2>(a.E, p.stages), s, hook.pdl, attr);
   hook.begin("gemm2");
   cudaError_t e =
-      cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm2>, tm_act, tm_w2, tm_act, tm_w2, p);
+      cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm2>, tm_act, tm_w2, tm_act, tm_w2, tm_p, p);
   return hook.end(e);
 }
 
 cudaError_t launch_fused_gemm(const GroupedGemmArgs &a, bool with_gemm2, cudaStream_t s,
                               const StageHook &hook) {
-  if (a.xs == nullptr || a.ordered) return cudaErrorInvalidValue;
-  CUtensorMap tm_xs, tm_w1, tm_act, tm_w2;
+  if (a.xs == nullptr || a.P != nullptr) return cudaErrorInvalidValue;
+  CUtensorMap tm_xs, tm_w1, tm_act, tm_w2, tm_p;
   if (!make_bf16_map(&tm_xs, a.xs, static_cast<uint64_t>(a.H), static_cast<uint64_t>(a.T) * a.k,
                      BM) ||
-      !w1_map(a, &tm_w1) || !gemm2_maps(a, &tm_act, &tm_w2))
+      !w1_map(a, &tm_w1) || !gemm2_maps(a, &tm_act, &tm_w2, &tm_p))
     return cudaErrorInvalidValue;
   int dev = 0;
   cudaGetDevice(&dev);
   Params p = base_params(a);
   p.sched = a.counters + kCounterSched0;
+  p.tl_kind = with_gemm2 ? kTlFused : kTlGemm1;
   p.run_gemm2 = with_gemm2 ? 1 : 0;
   p.stages = stages_for<kModeFused>(a.E, with_gemm2);
   cudaLaunchAttribute attr[2];
@@ -1192,7 +1142,7 @@ cudaError_t launch_fused_gemm(const GroupedGemmArgs &a, bool with_gemm2, cudaStr
       smem_bytes<kModeFused>(a.E, p.stages, with_gemm2), s, hook.pdl, attr);
   hook.begin(with_gemm2 ? "gemm_fused" : "gemm1_swiglu");
   cudaError_t e =
-      cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeFused>, tm_xs, tm_w1, tm_act, tm_w2, p);
+      cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeFused>, tm_xs, tm_w1, tm_act, tm_w2, tm_p, p);
   return hook.end(e);
 }
 

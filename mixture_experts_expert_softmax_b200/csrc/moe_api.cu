@@ -38,6 +38,8 @@ DeviceState g_dev[kMaxDevices];
 int g_small_t_max = -1;  // -1: not read from the environment yet
 int g_sync_each = -1;
 int64_t g_wait_limit_ns = 2000000000LL;
+uint64_t *g_timeline = nullptr;  // debug timeline buffer (moe_timeline), device
+int64_t g_timeline_cap = 0;
 thread_local const char *g_failed_stage = "";
 
 // ---- profiler
@@ -350,7 +352,7 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
         b1, b2, act_kind, topk_weights, topk_ids, act, out, T, H, I, E, k,
         d->status,
         reinterpret_cast<unsigned long long *>(reinterpret_cast<char *>(d->status) + 64),
-        static_cast<uint64_t>(g_wait_limit_ns), ctx.stream, hook));
+        static_cast<uint64_t>(g_wait_limit_ns), ctx.stream, hook, g_timeline, g_timeline_cap));
   }
 
   cudaError_t e;
@@ -370,19 +372,18 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
     w2 = wd2;
   }
 
+  // top-k <= 2: GEMM2 adds its rows straight into out and no P is needed
+  const bool fuse_combine = k <= 2;
   // Copying the hidden rows into expert-sorted order costs k row copies per
   // token and lets GEMM1 run on CTA pairs with TMA operands; with few slots
-  // per token that pays off.  With more slots GEMM2 orders each token's
-  // contributions (turn counters) instead of adding them in any order.
+  // per token that pays off.
   const bool gather_rows = k <= 2;
-  const bool ordered = k > 2;
   const int64_t n_counters = moe::gemm_counter_count(n, E);
-  const size_t n_turn = ordered ? static_cast<size_t>(T) * (H / 128) : 0;
   const size_t need = permute_ws_bytes(n, E) + align256(static_cast<size_t>(n) * 4) +
                       align256(static_cast<size_t>(n) * I * 2) +
                       align256(static_cast<size_t>(n_counters) * 4) +
                       (gather_rows ? align256(static_cast<size_t>(n) * H * 2) : 0) +
-                      (ordered ? align256(n_turn * 4) : 0);
+                      (fuse_combine ? 0 : align256(static_cast<size_t>(n) * H * sizeof(float)));
   if ((rc = ensure_workspace(*d, need)) != MOE_OK) return rc;
   Carver cv{static_cast<char *>(d->ws)};
   int32_t *chunk_counts =
@@ -393,7 +394,7 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
   uint16_t *act = cv.take<uint16_t>(static_cast<size_t>(n) * I);
   int *counters = cv.take<int>(static_cast<size_t>(n_counters));
   uint16_t *xs = gather_rows ? cv.take<uint16_t>(static_cast<size_t>(n) * H) : nullptr;
-  int *turn = ordered ? cv.take<int>(n_turn) : nullptr;
+  float *P = fuse_combine ? nullptr : cv.take<float>(static_cast<size_t>(n) * H);
 
   // grouping (and the sorted row copy): one kernel up to 8192 entries, the
   // three-kernel grouping and a separate copy above; either zeroes the
@@ -422,9 +423,7 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
   ga.act = act;
   ga.out = out;
   ga.topk_weights = topk_weights;
-  ga.topk_ids = topk_ids;
-  ga.ordered = ordered ? 1 : 0;
-  ga.turn = turn;
+  ga.P = P;
   ga.counters = counters;
   ga.T = T;
   ga.H = H;
@@ -434,6 +433,8 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
   ga.num_sms = d->num_sms;
   ga.status = d->status;
   ga.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns);
+  ga.timeline = g_timeline;
+  ga.timeline_cap = g_timeline_cap;
   ga.b1 = b1;
   ga.b2 = b2;
   ga.act_kind = act_kind;
@@ -451,7 +452,9 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
     if ((e = moe::launch_gemm1_swiglu(ga, ctx.stream, hook)) != cudaSuccess) return to_code(e);
     if ((e = moe::launch_gemm2(ga, ctx.stream, hook)) != cudaSuccess) return to_code(e);
   }
-  return MOE_OK;
+  if (fuse_combine) return MOE_OK;
+  e = moe::launch_combine(P, inv, topk_weights, out, T, H, k, d->status, ctx.stream, hook);
+  return to_code(e);
 }
 
 }  // namespace
@@ -520,6 +523,15 @@ int64_t moe_set_wait_limit_ns(int64_t ns) {
 }
 
 const char *moe_last_failed_stage(void) { return g_failed_stage; }
+
+int moe_timeline(void *buf, int64_t capacity) {
+  if (buf != nullptr && (capacity < 1 || (reinterpret_cast<uintptr_t>(buf) & 7u) != 0))
+    return MOE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_timeline = static_cast<uint64_t *>(buf);
+  g_timeline_cap = buf != nullptr ? capacity : 0;
+  return MOE_OK;
+}
 
 int moe_debug_wait_timeout(int64_t limit_ns, void *stream) {
   if (limit_ns <= 0 || limit_ns > 10000000000LL) return MOE_ERR_INVALID_ARG;

@@ -97,13 +97,10 @@ struct GroupedGemmArgs {
   uint16_t *act;  // [T*k, I] bf16, expert-sorted rows
   float *out;                 // [T, H] fp32
   const float *topk_weights;  // [T, k] fp32
-  const int32_t *topk_ids;    // [T, k] int32
-  // 0 (top-k <= 2): GEMM1 zeroes out and GEMM2 adds w * y of each row into
-  // it in any order.  1 (top-k > 2): GEMM1 zeroes turn and the rows of
-  // tokens without a valid id; GEMM2 stores, then adds, each token's
-  // contributions in ascending expert order.
-  int ordered;
-  int *turn;      // ordered: [T, H / 128] int
+  // null (top-k <= 2): GEMM1 zeroes out and GEMM2 adds w * y of each row
+  // into it in any order; else GEMM2 writes [T*k, H] fp32 expert-sorted
+  // rows here for the fixed-order combine
+  float *P;
   int *counters;  // gemm_counter_count(T*k, E) ints, zero at the first GEMM launch
   // epilogue variant: activation (kAct* of common.cuh) and optional fp32
   // biases b1 [E, 2I] (gate, then up) and b2 [E, H], 16-byte aligned
@@ -115,6 +112,8 @@ struct GroupedGemmArgs {
   int num_sms;
   uint32_t *status;
   uint64_t wait_limit_ns;
+  uint64_t *timeline;  // debug timeline buffer (timeline_rec), or null
+  int64_t timeline_cap;
 };
 cudaError_t grouped_gemm_setup(int device);
 cudaError_t launch_gemm1_swiglu(const GroupedGemmArgs &a, cudaStream_t s, const StageHook &hook);
@@ -124,6 +123,11 @@ cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s, const StageHo
 cudaError_t launch_fused_gemm(const GroupedGemmArgs &a, bool with_gemm2, cudaStream_t s,
                               const StageHook &hook);
 cudaError_t launch_wait_probe(uint32_t *status, uint64_t limit_ns, cudaStream_t s);
+
+// combine.cu
+cudaError_t launch_combine(const float *P, const int32_t *inv, const float *topk_weights,
+                           float *out, int64_t T, int H, int k, uint32_t *status, cudaStream_t s,
+                           const StageHook &hook);
 
 // dequant.cu: out[r, c] = bf16(e4m3(q[r, c]) * scale[r, c / block]) for a
 // [rows, K] matrix of FP8 E4M3 codes (K and block multiples of 16, block
@@ -151,6 +155,7 @@ cudaError_t launch_small_t(const uint16_t *hidden, const void *w1, const void *w
                            const float *topk_weights, const int32_t *topk_ids, float *act,
                            float *out, int64_t T, int H, int I, int E, int k, uint32_t *status,
                            unsigned long long *grid_sync, uint64_t wait_limit_ns,
-                           cudaStream_t s, const StageHook &hook);
+                           cudaStream_t s, const StageHook &hook,
+                           uint64_t *timeline = nullptr, int64_t timeline_cap = 0);
 
 }  // namespace moe

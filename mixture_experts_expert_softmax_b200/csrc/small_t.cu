@@ -476,7 +476,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
                    const int32_t *__restrict__ ids, float *__restrict__ act,
                    float *__restrict__ out, int T, int k, int H, int I, int E, int rows_per_cta,
                    int slots, int cache_act, uint32_t *status,
-                   unsigned long long *grid_sync, uint64_t limit) {
+                   unsigned long long *grid_sync, uint64_t limit, uint64_t *tl_buf,
+                   int64_t tl_cap) {
   // phase 1: chunks per lane and row in flight (an FP8 chunk holds 16 codes)
   constexpr int kU1 = kFp8 ? 4 : (kTokens == 1 ? 8 : 4);
   extern __shared__ __align__(16) uint8_t smem[];
@@ -500,6 +501,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   const int h0 = blockIdx.x * rows_per_cta;
   const int nrows = max(0, min(H, h0 + rows_per_cta) - h0);
 
+  const uint64_t tl_start = tl_buf ? global_timer_ns() : 0;
   if (warp == 0) build_lists(L, ids, TK, E);
   if (threadIdx.x == 32) {
     s_abort = 0;
@@ -618,6 +620,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   // whatever was launched before on the counter.)
   __threadfence();
   __syncthreads();
+  const uint64_t tl_p1 = tl_buf ? global_timer_ns() : 0;
   if (threadIdx.x == 0) {
     const unsigned long long old = atomicAdd(grid_sync, 1ull);
     const unsigned long long target = (old / gridDim.x + 1) * gridDim.x;
@@ -633,6 +636,11 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     __threadfence();
   }
   __syncthreads();
+  const uint64_t tl_bar = tl_buf ? global_timer_ns() : 0;
+  if (threadIdx.x == 0) {
+    timeline_rec(tl_buf, tl_cap, kTlSmallT, kTlPhase1, 0, blockIdx.x, tl_start, tl_p1);
+    timeline_rec(tl_buf, tl_cap, kTlSmallT, kTlBarrier, 0, blockIdx.x, tl_p1, tl_bar);
+  }
   if (s_abort) {
     // let the bulk copies already issued land before the CTA exits
     if (warp == kCopyWarp && lane == 0 && ring)
@@ -739,6 +747,11 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       }
     }
     out[static_cast<size_t>(t) * H + h0 + r] = acc;
+  }
+  if (tl_buf != nullptr) {
+    __syncthreads();
+    if (threadIdx.x == 0)
+      timeline_rec(tl_buf, tl_cap, kTlSmallT, kTlPhase2, 0, blockIdx.x, tl_bar, global_timer_ns());
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     bool bad = false;
@@ -861,7 +874,8 @@ cudaError_t launch_small_t(const uint16_t *hidden, const void *w1, const void *w
                            const float *topk_weights, const int32_t *topk_ids, float *act,
                            float *out, int64_t T, int H, int I, int E, int k, uint32_t *status,
                            unsigned long long *grid_sync, uint64_t wait_limit_ns,
-                           cudaStream_t s, const StageHook &hook) {
+                           cudaStream_t s, const StageHook &hook, uint64_t *timeline,
+                           int64_t timeline_cap) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -893,7 +907,7 @@ cudaError_t launch_small_t(const uint16_t *hidden, const void *w1, const void *w
                          reinterpret_cast<const uint4 *>(w1), reinterpret_cast<const uint4 *>(w2),
                          w1_scale, w2_scale, block, b1, b2, act_kind, topk_weights, topk_ids, act, out, static_cast<int>(T), k, H, I, E,
                          cfg.rows_per_cta, cfg.slots, cfg.cache_act, status,
-                         grid_sync, wait_limit_ns);
+                         grid_sync, wait_limit_ns, timeline, timeline_cap);
   return hook.end(e);
 }
 

@@ -156,6 +156,13 @@ def test_permute_ex_argument_checks(kw, code):
     assert perm_ex(**kw) == code
 
 
+def test_timeline_argument_checks():
+    assert L.moe_timeline(256, 0) == moe.MOE_ERR_INVALID_ARG    # capacity < 1
+    assert L.moe_timeline(260, 16) == moe.MOE_ERR_INVALID_ARG   # not 8-byte aligned
+    assert L.moe_timeline(256, 16) == moe.MOE_OK                # set (no device access)
+    assert L.moe_timeline(None, 0) == moe.MOE_OK                # off
+
+
 def test_debug_switches_roundtrip():
     prev = moe.set_small_t_max(5)
     assert moe.set_small_t_max(prev) == 5

@@ -279,8 +279,7 @@ def test_forward_small_t_shared_and_duplicate_experts():
 @pytest.mark.parametrize("small,k", [(16, 2), (0, 2), (0, 4)])
 def test_forward_invalid_ids_are_skipped_and_flagged(small, k):
     """k = 2 on the GEMM path flags bad ids in the grouping (GEMM2 adds into
-    zeroed out); k = 4 orders the contributions, and GEMM1 zeroes the row of
-    the token without a valid id."""
+    out); k = 4 also goes through the separate combine."""
     T, H, I, E = 12, 256, 128, 8
     hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=11)
     ids, w = oracle.route(logits.numpy(), k, True)
@@ -318,8 +317,7 @@ def test_forward_zero_token_gives_zero_row(small):
 def test_forward_deterministic(T, H, I, E, k):
     """Identical bits on repeated calls: with k <= 2 GEMM2 adds two rounded
     products onto zero in whatever order the tiles finish (a commutative
-    sum), with k > 2 each token's contributions are added in ascending
-    expert order, whatever order the tiles finish in."""
+    sum), with k > 2 the combine sums in fixed order."""
     hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=5)
     ids, w = oracle.route(logits.numpy(), k, True)
     prev = moe.set_small_t_max(0)
@@ -410,7 +408,7 @@ def test_end_to_end_route_then_forward():
 # ------------------------------------------------------------------ epilogue variants
 VARIANT_CASES = [
     (64, 256, 128, 8, 2),      # tiny: one-kernel grouping, both GEMMs in one launch
-    (333, 384, 384, 16, 4),    # k > 2: separate GEMM launches, ordered contributions
+    (333, 384, 384, 16, 4),    # k > 2: separate GEMM launches, fp32 P, combine
     (100, 256, 128, 128, 8),   # many experts below one tile
 ]
 
@@ -510,7 +508,7 @@ def gpu_forward_fp8(hidden, q1, s1, q2, s2, block, w, ids):
     (3, 512, 256, 4, 2, 256, "small_t"),       # tokens sharing experts
     (4, 2048, 768, 128, 8, 256, "gemm"),
     (64, 256, 128, 8, 2, 128, "gemm"),         # tiny: one-launch GEMMs
-    (100, 384, 384, 16, 4, 128, "gemm"),       # k > 2: ordered contributions, half n-tile
+    (100, 384, 384, 16, 4, 128, "gemm"),       # k > 2: P and combine, half n-tile
 ])
 def test_forward_fp8(T, H, I, E, k, block, path):
     from moe_inputs import make_fp8_weights
@@ -655,6 +653,37 @@ def test_bounded_wait_times_out_without_hanging():
     check_status_clean()
 
 
+@pytest.mark.parametrize("T,k,kinds", [(300, 2, {"gemm_fused"}), (300, 4, {"gemm1", "gemm2"}),
+                                       (1, 8, {"small_t"})])
+def test_timeline_records(T, k, kinds):
+    """The debug timeline: every tile of the GEMM launches (or every CTA of
+    the small-batch kernel) leaves its records, t0 <= t1, and the forward's
+    result is the same with it on."""
+    H, I, E = 512, 256, 16
+    hidden, w1, w2, logits = [t.cuda() for t in make_inputs(T, H, I, E, seed=4)]
+    ids, w = moe.moe_route(logits, k, True)
+    ref = moe.moe_forward(hidden, w1, w2, w, ids)
+    moe.timeline_start(1 << 14)
+    try:
+        out = moe.moe_forward(hidden, w1, w2, w, ids)
+    finally:
+        recs = moe.timeline_stop()
+    assert torch.equal(out, ref)
+    assert recs and {r["kind"] for r in recs} == kinds
+    assert all(r["t0"] <= r["t1"] for r in recs)
+    if "small_t" in kinds:
+        ctas = {r["id"] for r in recs if r["role"] == "phase2"}
+        assert len(ctas) == torch.cuda.get_device_properties(0).multi_processor_count
+    else:
+        prod = [r for r in recs if r["role"] == "producer" and r["sub"] == 0]
+        assert len({r["id"] for r in prod}) == len(prod)  # each tile claimed once
+        assert len({r["id"] for r in recs if r["role"] == "mma"}) == len(prod)
+    summary = moe.timeline_summary(recs)
+    assert all(v["n"] > 0 for v in summary.values())
+    moe.moe_forward(hidden, w1, w2, w, ids)  # off again: nothing recorded, nothing breaks
+    torch.cuda.synchronize()
+
+
 def test_sync_each_stage_mode_and_profiler():
     s = SHAPES["tiny"]
     hidden, w1, w2, logits = make_shape_inputs(s)
@@ -688,7 +717,6 @@ def test_sync_each_stage_mode_and_profiler():
         moe.profile_enable(False)
         moe.set_sync_each_stage(prev)
     prof = moe.profile_read()
-    for kname in ("permute", "gemm1_swiglu", "gemm2"):
+    for kname in ("permute", "gemm1_swiglu", "gemm2", "combine"):
         assert prof[kname][0] == 1 and prof[kname][1] > 0
-    assert "combine" not in prof
     assert_output_close(out, oracle.moe_token_loop(hidden, w1, w2, w, ids))
