@@ -675,9 +675,12 @@ def test_timeline_records(T, k, kinds):
         ctas = {r["id"] for r in recs if r["role"] == "phase2"}
         assert len(ctas) == torch.cuda.get_device_properties(0).multi_processor_count
     else:
-        prod = [r for r in recs if r["role"] == "producer" and r["sub"] == 0]
-        assert len({r["id"] for r in prod}) == len(prod)  # each tile claimed once
-        assert len({r["id"] for r in recs if r["role"] == "mma"}) == len(prod)
+        for kind in kinds:  # each launch numbers its tiles from 0
+            prod = [r for r in recs if r["kind"] == kind and r["role"] == "producer"
+                    and r["sub"] == 0]
+            assert len({r["id"] for r in prod}) == len(prod)  # each tile claimed once
+            mma = {r["id"] for r in recs if r["kind"] == kind and r["role"] == "mma"}
+            assert mma == {r["id"] for r in prod}
     summary = moe.timeline_summary(recs)
     assert all(v["n"] > 0 for v in summary.values())
     moe.moe_forward(hidden, w1, w2, w, ids)  # off again: nothing recorded, nothing breaks
