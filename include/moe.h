@@ -305,21 +305,22 @@ int moe_debug_wait_timeout(int64_t limit_ns, void *stream);
 /*
  * moe_timeline -- debug timeline of the kernels' inner schedule.  While buf
  * (a zeroed DEVICE buffer of 32 + 32 * capacity bytes, 8-byte aligned,
- * owned by the caller) is set, the grouped-GEMM kernels append one record
- * per tile and role and the small-batch kernel one per CTA and phase:
- * buf as uint64_t[]: [0] = records appended (may exceed capacity; extra
- * ones are dropped), record i at [4 + 4i ..] = {tag, id, t0, t1} with
- * %globaltimer nanoseconds t0 <= t1 and tag = kind << 56 | role << 48 |
- * cta << 16 | sub:
+ * owned by the caller) is set, the grouped-GEMM kernels write one record
+ * per tile and role and the small-batch kernel one per CTA and phase into
+ * fixed slots of buf (as uint64_t[]): record i at [4 + 4i ..] = {tag, id,
+ * t0, t1} with %globaltimer nanoseconds t0 <= t1 and tag = kind << 56 |
+ * role << 48 | cta << 16 | sub (unused slots keep tag 0):
  *   kind 1 GEMM1 launch, 2 GEMM2 launch, 3 one-launch GEMM, 4 small-batch;
  *   role 0 producer (t0 tile start, t1 last operand load issued),
  *        1 MMA issuer (t0 accumulator free, t1 last MMA issued),
  *        2 epilogue, first epilogue warp (t0 accumulator full, t1 released),
- *        3/4/5 small-batch phase 1 / grid barrier / phase 2 (id = CTA);
+ *        3 / 4 small-batch phase 1 / grid barrier, 5 act staged on chip,
+ *        6 w2 rows on chip, 7 phase 2 (3-7: id = CTA);
  *   sub: the CTA's rank in its pair (roles 0 and 2); id: the tile number.
- * buf == NULL turns it off (the default).  Not synchronised with running
- * work: set it between calls.  Errors: INVALID_ARG for capacity < 1 or an
- * unaligned buf.
+ * Each call's records overwrite the previous call's; slots past capacity
+ * are dropped.  buf == NULL turns it off (the default).  Not synchronised
+ * with running work: set it between calls.  Errors: INVALID_ARG for
+ * capacity < 1 or an unaligned buf.
  */
 int moe_timeline(void *buf, int64_t capacity);
 

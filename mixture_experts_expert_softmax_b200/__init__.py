@@ -291,7 +291,7 @@ def moe_permute_ex(topk_ids: torch.Tensor, E: int, kernel: str = "auto",
 
 TIMELINE_KINDS = {1: "gemm1", 2: "gemm2", 3: "gemm_fused", 4: "small_t"}
 TIMELINE_ROLES = {0: "producer", 1: "mma", 2: "epilogue", 3: "phase1", 4: "barrier",
-                  5: "phase2"}
+                  5: "act_load", 6: "w2_wait", 7: "phase2"}
 _timeline_buf = None
 
 
@@ -314,8 +314,9 @@ def timeline_stop() -> list[dict]:
     torch.cuda.synchronize()
     raw = _timeline_buf.cpu()
     _timeline_buf = None
-    n = min(int(raw[0]), (raw.numel() - 4) // 4)
-    rec = raw[4:4 + 4 * n].view(n, 4).tolist()
+    n = (raw.numel() - 4) // 4
+    rec = raw[4:4 + 4 * n].view(n, 4)
+    rec = rec[rec[:, 0] != 0].tolist()  # slots nobody wrote
     out = []
     for tag, ident, t0, t1 in rec:
         tag &= (1 << 64) - 1

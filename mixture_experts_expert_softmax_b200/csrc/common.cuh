@@ -392,23 +392,25 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t *bar, uint16_t cta_mas
 }
 
 // ---------------------------------------------------------------- timeline
-// Debug timeline (moe_timeline): buf[0] counts the records written so far;
-// record i is buf[4 + 4i .. 4 + 4i + 3] = {tag, id, t0, t1}, with %globaltimer
-// nanoseconds t0 <= t1 and tag = kind << 56 | role << 48 | cta << 16 | sub.
-// Records past `cap` are counted but not written.  buf == null: off.
+// Debug timeline (moe_timeline): record i is buf[4 + 4i .. 4 + 4i + 3] =
+// {tag, id, t0, t1}, with %globaltimer nanoseconds t0 <= t1 and tag =
+// kind << 56 | role << 48 | cta << 16 | sub (never 0).  Every record has a
+// fixed slot (a launch's base plus its tile or CTA times the records per
+// tile or CTA), so writing one costs four plain stores; slots at or past
+// `cap` are not written.  buf == null: off.
 enum : uint32_t {
   kTlGemm1 = 1, kTlGemm2 = 2, kTlFused = 3, kTlSmallT = 4,  // kinds
   kTlProducer = 0, kTlMma = 1, kTlEpilogue = 2,             // roles (GEMM kernels)
-  kTlPhase1 = 3, kTlBarrier = 4, kTlPhase2 = 5              // roles (small-T kernel)
+  kTlPhase1 = 3, kTlBarrier = 4, kTlActLoad = 5, kTlW2Wait = 6, kTlPhase2 = 7  // small-T
 };
+constexpr int kTlPerTile = 5;  // producer x2 (pair ranks), MMA, epilogue x2
+constexpr int kTlPerCta = 5;   // small-T: phase 1, barrier, act load, w2 wait, phase 2
 
-__device__ __forceinline__ void timeline_rec(uint64_t *buf, int64_t cap, uint32_t kind,
-                                             uint32_t role, uint32_t sub, uint64_t id,
-                                             uint64_t t0, uint64_t t1) {
-  if (buf == nullptr) return;
-  const unsigned long long i = atomicAdd(reinterpret_cast<unsigned long long *>(buf), 1ull);
-  if (static_cast<int64_t>(i) >= cap) return;
-  uint64_t *r = buf + 4 + 4 * i;
+__device__ __forceinline__ void timeline_rec(uint64_t *buf, int64_t cap, int64_t slot,
+                                             uint32_t kind, uint32_t role, uint32_t sub,
+                                             uint64_t id, uint64_t t0, uint64_t t1) {
+  if (buf == nullptr || slot < 0 || slot >= cap) return;
+  uint64_t *r = buf + 4 + 4 * slot;
   r[0] = static_cast<uint64_t>(kind) << 56 | static_cast<uint64_t>(role) << 48 |
          static_cast<uint64_t>(blockIdx.x & 0xffffffffu) << 16 | (sub & 0xffffu);
   r[1] = id;

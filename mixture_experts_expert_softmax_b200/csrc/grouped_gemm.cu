@@ -225,9 +225,11 @@ struct Params {
   const float *b1;
   const float *b2;
   int act_kind;
-  // debug timeline (see timeline_rec): null when off
+  // debug timeline (see timeline_rec): null when off; this launch's records
+  // start at slot tl_base, kTlPerTile per tile
   uint64_t *tl_buf;
   int64_t tl_cap;
+  int64_t tl_base;
   uint32_t tl_kind;
 };
 
@@ -558,8 +560,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           cp_async_arrive_noinc(&bars->full[s]);
         }
         if (threadIdx.x == 0)
-          timeline_rec(p.tl_buf, p.tl_cap, p.tl_kind, kTlProducer, rank, t, tl_t0,
-                       global_timer_ns());
+          timeline_rec(p.tl_buf, p.tl_cap, p.tl_base + int64_t{t} * kTlPerTile + rank,
+                       p.tl_kind, kTlProducer, rank, t, tl_t0, global_timer_ns());
       }
       cp_async_wait_all();
       if (*abort_flag && threadIdx.x == 0) {
@@ -614,8 +616,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d_pair(sA + s * kABytes, am, full0 + 8u * s, kb * BK, a_row);
           tma_load_2d_pair(sB + s * kBBytes, bm, full0 + 8u * s, kb * BK, b_row);
         }
-        timeline_rec(p.tl_buf, p.tl_cap, p.tl_kind, kTlProducer, rank, t, tl_t0,
-                     global_timer_ns());
+        timeline_rec(p.tl_buf, p.tl_cap, p.tl_base + int64_t{t} * kTlPerTile + rank, p.tl_kind,
+                     kTlProducer, rank, t, tl_t0, global_timer_ns());
       }
       if (*abort_flag) {
         const uint64_t t0 = global_timer_ns();
@@ -680,7 +682,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           else
             umma_commit(&bars->acc_full[a]);
         }
-        timeline_rec(p.tl_buf, p.tl_cap, p.tl_kind, kTlMma, 0, t, tl_t0, global_timer_ns());
+        timeline_rec(p.tl_buf, p.tl_cap, p.tl_base + int64_t{t} * kTlPerTile + 2, p.tl_kind, kTlMma,
+                     0, t, tl_t0, global_timer_ns());
       }
       // every MMA must be complete before TMEM is released
       if (CG == 2)
@@ -859,8 +862,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         else
           mbar_arrive(&bars->acc_empty[a]);
         if (ew == 0)
-          timeline_rec(p.tl_buf, p.tl_cap, p.tl_kind, kTlEpilogue, rank, t, tl_t0,
-                       global_timer_ns());
+          timeline_rec(p.tl_buf, p.tl_cap, p.tl_base + int64_t{t} * kTlPerTile + 3 + rank,
+                       p.tl_kind, kTlEpilogue, rank, t, tl_t0, global_timer_ns());
       }
       if (MODE == kModeFused && w.phase == 1 && p.run_gemm2) {
         // publish this warp's act rows of the m-tile to GEMM2 tiles (after
@@ -984,6 +987,7 @@ Params base_params(const GroupedGemmArgs &a) {
   p.act_kind = a.act_kind;
   p.tl_buf = a.timeline;
   p.tl_cap = a.timeline_cap;
+  p.tl_base = 0;
   return p;
 }
 
@@ -1108,6 +1112,8 @@ cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s, const StageHo
   Params p = base_params(a);
   p.sched = a.counters + kCounterSched1;
   p.tl_kind = kTlGemm2;
+  // after the first launch's records: at most (m-tiles) * (GEMM1 n-tiles) tiles
+  p.tl_base = ((a.T * a.k + 255) / 128 + 2 * a.E) * (a.I / (kAccN / 2)) * kTlPerTile;
   p.zero_out = nullptr;  // zeroed by the GEMM1 launch
   p.zero_n4 = 0;
   p.stages = stages_for<kModeGemm2>(a.E);

@@ -637,9 +637,10 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   }
   __syncthreads();
   const uint64_t tl_bar = tl_buf ? global_timer_ns() : 0;
+  const int64_t tl_slot = static_cast<int64_t>(blockIdx.x) * kTlPerCta;
   if (threadIdx.x == 0) {
-    timeline_rec(tl_buf, tl_cap, kTlSmallT, kTlPhase1, 0, blockIdx.x, tl_start, tl_p1);
-    timeline_rec(tl_buf, tl_cap, kTlSmallT, kTlBarrier, 0, blockIdx.x, tl_p1, tl_bar);
+    timeline_rec(tl_buf, tl_cap, tl_slot, kTlSmallT, kTlPhase1, 0, blockIdx.x, tl_start, tl_p1);
+    timeline_rec(tl_buf, tl_cap, tl_slot + 1, kTlSmallT, kTlBarrier, 0, blockIdx.x, tl_p1, tl_bar);
   }
   if (s_abort) {
     // let the bulk copies already issued land before the CTA exits
@@ -658,6 +659,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     __syncthreads();
     act4 = d4;
   }
+  const uint64_t tl_act = tl_buf ? global_timer_ns() : 0;
+  if (threadIdx.x == 0)
+    timeline_rec(tl_buf, tl_cap, tl_slot + 2, kTlSmallT, kTlActLoad, 0, blockIdx.x, tl_bar, tl_act);
   const int rgroups = (nrows + kR2 - 1) / kR2;
   if (warp == kCopyWarp) {
     // refill the ring: expert d goes into slot d % slots once every compute
@@ -693,6 +697,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
         break;
       }
     }
+    if (warp == 0 && lane == 0)
+      timeline_rec(tl_buf, tl_cap, tl_slot + 3, kTlSmallT, kTlW2Wait, 0, blockIdx.x, tl_act,
+                   global_timer_ns());
     const int n_items = L.dstart[nd] * rgroups;
     for (int it = warp; it < n_items && !s_abort; it += kWarps) {
       const int pq = it / rgroups, rg = it - pq * rgroups;  // pq: position in plist
@@ -751,7 +758,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   if (tl_buf != nullptr) {
     __syncthreads();
     if (threadIdx.x == 0)
-      timeline_rec(tl_buf, tl_cap, kTlSmallT, kTlPhase2, 0, blockIdx.x, tl_bar, global_timer_ns());
+      timeline_rec(tl_buf, tl_cap, tl_slot + 4, kTlSmallT, kTlPhase2, 0, blockIdx.x, tl_bar,
+                   global_timer_ns());
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     bool bad = false;
