@@ -363,9 +363,11 @@ __device__ __forceinline__ Work get_work(int t, int total1, const Params &p,
 // ---------------------------------------------------------------- tile queue
 // The scheduler (thread 0 of rank 0) writes its claimed tile number (-1
 // past the last tile) into slot seq % kTQ of both CTAs' queues once every
-// reader of that slot's previous use is done.  False if it gave up.  The
-// claim for the next tile is made as soon as this one is published, so
-// that its round trip to L2 overlaps this tile's loads.
+// reader of that slot's previous use is done.  False if it gave up.  Every
+// tile, the first included, is claimed from the counter (a tile held by a
+// CTA that never started could stall the tiles that wait on it); the claim
+// for the next tile is made as soon as this one is published, so that its
+// round trip to L2 overlaps this tile's loads.
 template <int CG>
 __device__ __forceinline__ bool publish_tile(Bars *bars, uint32_t seq, int total, int *sched,
                                              int *claimed, uint64_t limit,
@@ -574,11 +576,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0;  // ring slot and its phase parity, advanced per k-block
       uint32_t ph = 0;
       bool stop = false;
+      // rank 0 publishes each tile one ahead of loading it, so that rank 1
+      // (which loads the other half of every stage) has it in time
       int claimed = leader ? atomicAdd(p.sched, 1) : 0;
+      int t_next = -1;
+      if (leader &&
+          !publish_tile<CG>(bars, 0, total, p.sched, &claimed, limit, abort_flag, &t_next)) {
+        give_up(p, abort_flag);
+        stop = true;
+      }
       for (uint32_t seq = 0; !stop; ++seq) {
-        int t = -1;
+        int t = t_next;
         const bool ok =
-            leader ? publish_tile<CG>(bars, seq, total, p.sched, &claimed, limit, abort_flag, &t)
+            leader ? (t < 0 || publish_tile<CG>(bars, seq + 1, total, p.sched, &claimed, limit,
+                                                abort_flag, &t_next))
                    : read_tile(bars, seq, rank, tq_empty0, limit, abort_flag, true, &t);
         if (!ok) {
           give_up(p, abort_flag);
