@@ -115,9 +115,10 @@ constexpr size_t kSmemMax = 232448;  // opt-in maximum per block on sm_100
 // act rows of an m-tile are complete when every epilogue warp of both CTAs
 // has published each of its n-tiles
 constexpr int kReadyPerTile = 2 * kEpiWarps;
-// out is zeroed (top-k <= 2) in chunks of this many float4, claimed by the
-// epilogue warps of whichever CTAs run first
-constexpr int64_t kZeroChunk4 = 4096;
+// out is zeroed (top-k <= 2) in one share per epilogue warp of the grid;
+// each warp takes its own share first (a flag per share, claimed with
+// atomicCAS: no contention), and a warp that waits for zeroing to finish
+// takes the shares nobody has taken (those of CTAs that have not started)
 
 enum { kModeGemm1 = 0, kModeGemm2 = 1, kModeFused = 2 };
 
@@ -162,10 +163,18 @@ struct __align__(8) Bars {
   int32_t scan[32];            // per-warp partial sums of build_tile_offsets
 };
 
-// Readers of each queue slot: the MMA thread and the epilogue warps of rank
-// 0, and on a pair also rank 1's producer thread and epilogue warps.
+// Readers that acknowledge each queue slot: the epilogue warps of every CTA
+// and, on a pair, rank 1's producer thread.  The MMA thread reads without
+// acknowledging: an mbarrier arrive has release semantics and would wait
+// for the tensor core to finish the MMAs it has just issued.  It needs no
+// acknowledgement, because the slot of tile seq is reused only for tile
+// seq + kTQ, which is published just before the loads of tile seq + kTQ - 1,
+// and those loads need ring slots that the MMA frees only once it has
+// committed stages of tile seq + kTQ - 4 or later (K >= 128: at least two
+// stages per tile, at most kMaxStages stages in flight).
 template <int CG>
-constexpr int queue_consumers() { return CG == 2 ? 2 * (1 + kEpiWarps) : 1 + kEpiWarps; }
+constexpr int queue_consumers() { return CG == 2 ? 1 + 2 * kEpiWarps : kEpiWarps; }
+static_assert(kTQ >= 2 + (kMaxStages + 1) / 2 + 2, "tile queue deeper than the MMA's lead");
 
 // Bytes in front of the aligned region: barriers, then exp_off and tile_off
 // (E + 1 entries each).
@@ -207,10 +216,11 @@ struct Params {
   uint32_t *status;
   uint64_t wait_limit_ns;
   // out is zeroed before GEMM2 adds into it (top-k <= 2): zero_n4 float4 in
-  // chunks claimed through zero_claim; zero_done counts finished chunks
+  // gridDim.x * kEpiWarps shares, each taken once through its flag in
+  // zero_flags; zero_done counts finished shares
   float4 *zero_out;
   int64_t zero_n4;
-  int *zero_claim;
+  int *zero_flags;
   int *zero_done;
   // GEMM2 fused with the combine (top-k <= 2): out [T, H] and the top-k
   // weights [T, k]; otherwise GEMM2 writes P [T*k, H] fp32
@@ -334,6 +344,22 @@ __device__ __forceinline__ void stage_scaled32(uint8_t *srow, const uint32_t (&v
     *reinterpret_cast<float4 *>(srow + 16 * j) =
         make_float4(wgt * as_f32(v[4 * j]), wgt * as_f32(v[4 * j + 1]),
                     wgt * as_f32(v[4 * j + 2]), wgt * as_f32(v[4 * j + 3]));
+}
+
+// Zero share `sh` of out (zero_n4 float4 in `shares` contiguous shares) if
+// no warp has taken it yet; the whole warp calls it.
+__device__ __forceinline__ void zero_share(const Params &p, int64_t sh, int64_t shares,
+                                           int lane) {
+  int mine = 0;
+  if (lane == 0) mine = atomicCAS(p.zero_flags + sh, 0, 1) == 0;
+  if (!__shfl_sync(0xffffffffu, mine, 0)) return;
+  const int64_t per = (p.zero_n4 + shares - 1) / shares;
+  const int64_t i0 = sh * per, i1 = min(i0 + per, p.zero_n4);
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int64_t i = i0 + lane; i < i1; i += 32) p.zero_out[i] = z;
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) atomicAdd(p.zero_done, 1);
 }
 
 // What one tile number is: GEMM1 or GEMM2 (phase 1 or 2), its place, and
@@ -645,7 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool stop = false;
       for (uint32_t seq = 0; !stop; ++seq) {
         int t = -1;
-        if (!read_tile(bars, seq, 0, tq_empty0, limit, abort_flag, true, &t)) {
+        if (!read_tile(bars, seq, 0, tq_empty0, limit, abort_flag, false, &t)) {
           give_up(p, abort_flag);
           break;
         }
@@ -716,26 +742,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *ebuf = sEpi + ew * kEpiWarpBytes;  // GEMM2: this warp's staging buffer
     const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * kEpiWarps + ew;
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kEpiWarps;
+    const int64_t zero_shares = nwarps;
     if (MODE != kModeGemm2 && p.zero_n4 > 0) {
       // out must read zero before GEMM2 adds into it; this runs while the
-      // first tiles' MMAs are in flight.  Chunks are claimed, so whichever
-      // CTAs run first zero all of out.
-      const int64_t n_chunks = (p.zero_n4 + kZeroChunk4 - 1) / kZeroChunk4;
-      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (;;) {
-        int ch = 0;
-        if (lane == 0) ch = atomicAdd(p.zero_claim, 1);
-        ch = __shfl_sync(0xffffffffu, ch, 0);
-        if (ch >= n_chunks) break;
-        const int64_t i0 = static_cast<int64_t>(ch) * kZeroChunk4;
-        const int64_t i1 = min(i0 + kZeroChunk4, p.zero_n4);
-        for (int64_t i = i0 + lane; i < i1; i += 32) p.zero_out[i] = z;
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) atomicAdd(p.zero_done, 1);
-      }
+      // first tiles' MMAs are in flight
+      zero_share(p, gwarp, zero_shares, lane);
     }
-    const int64_t zero_chunks = (p.zero_n4 + kZeroChunk4 - 1) / kZeroChunk4;
     bool zero_seen = MODE != kModeFused || p.zero_n4 == 0 || !p.run_gemm2;
     for (uint32_t seq = 0;; ++seq) {
       // waits are taken by every lane; their outcome is made warp-uniform
@@ -794,7 +806,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else if (p.fuse_combine) {
         if (!zero_seen) {
-          if (!wait_geq(p.zero_done, static_cast<int>(zero_chunks), limit, abort_flag))
+          // every share zeroed; first take any share whose CTA has not
+          // started, so that this never waits for a CTA that is not running
+          if (ld_acquire_gpu(p.zero_done) < static_cast<int>(zero_shares))
+            for (int64_t sh = 0; sh < zero_shares; ++sh) zero_share(p, sh, zero_shares, lane);
+          if (!wait_geq(p.zero_done, static_cast<int>(zero_shares), limit, abort_flag))
             give_up(p, abort_flag);
           fence_proxy_async_global();
           zero_seen = true;
@@ -990,9 +1006,9 @@ Params base_params(const GroupedGemmArgs &a) {
     p.zero_out = reinterpret_cast<float4 *>(a.out);
     p.zero_n4 = a.T * a.H / 4;
   }
-  p.zero_claim = a.counters + kCounterZeroClaim;
   p.zero_done = a.counters + kCounterZeroDone;
   p.ready = a.counters + kCounterReady;
+  p.zero_flags = p.ready + fused_gemm_ready_count(a.T * a.k, a.E);
   p.b1 = a.b1;
   p.b2 = a.b2;
   p.act_kind = a.act_kind;
