@@ -68,44 +68,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
   return true;
 }
 
-// mbar_wait with acquire at cluster scope: for barriers that a thread of the
-// other CTA of a pair arrives on after writing this CTA's shared memory.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
-                                                  uint64_t limit_ns,
-                                                  const volatile int *abort = nullptr) {
-  const uint32_t a = smem_addr(bar);
-  if (mbar_try_wait_cluster(a, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait_cluster(a, parity)) {
-    if (abort != nullptr && *abort != 0) return false;
-    if (global_timer_ns() - t0 > limit_ns) return false;
-  }
-  return true;
-}
-
-// 32-bit store into the shared memory of a CTA of the cluster (address from
-// map_to_rank).
-__device__ __forceinline__ void st_shared_cluster_s32(uint32_t cluster_addr, int v) {
-  asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
-
-// Named barrier over `count` threads (a multiple of 32) of this CTA.
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // ---------------------------------------------------------------- global flags
 __device__ __forceinline__ int ld_acquire_gpu(const int *p) {
   int v;

@@ -7,50 +7,46 @@
 //     version of the page below): gelu (tanh form) or swigluoai in place of
 //     silu, and a bias b1[e] added to g and u before the activation.
 //   GEMM2: y = act . w2[e]^T (fp32 in TMEM), plus the bias b2[e] when given
-//     (before the top-k weight), then the top-k weighted sum into out:
-//     - top-k <= 2: the epilogue adds w_j * y_j of each row straight into
-//       out[token] with bulk reductions at L2 (out was zeroed first);
-//       out[t] = 0 + a + b is the same in either arrival order, so the
-//       result is deterministic.
-//     - top-k > 2: the epilogue stores y as fp32 rows of P in the same
-//       expert-sorted order (TMA tile stores) and combine.cu forms
-//       sum_j w_j * y_j in fixed j order.
+//     (before the top-k weight).  For top-k <= 2 the epilogue
+//     adds w_j * y_j of each row straight into out[token] with bulk
+//     reductions at L2 (out was zeroed first); out[t] = 0 + a + b is the
+//     same in either arrival order, so the result is still deterministic.
+//     For larger k it stores y as fp32 rows of P in the same expert-sorted
+//     order and combine.cu forms sum_j w_j * y_j in fixed j order.
 // This is the expert FFN of ref_moe on the page "tpu_inference/kernels/
 // fused_moe/v1/kernel.py" (gate = w1, up = w3, then act . w2) in the weight
 // layout of atrex-bench #009 (w1 [E, 2I, H], w2 [E, H, I], both applied as
 // F.linear, i.e. K-major).
 //
 // Work unit: an m-tile of one expert's rows times one 256-column n-tile of
-// the accumulator.  Tiles are numbered expert-major, then n-tile, then
-// m-tile, so CTAs working together share a weight tile through L2.  Tiles
-// are handed out dynamically: the
-// first thread of each CTA (pair) claims the next tile number from a global
-// counter and publishes it through a small queue in shared memory to every
-// role of the CTA(s).  Tiles are claimed in number order, and every wait
-// across tiles (GEMM2 rows on the act rows of GEMM1 tiles) points to a tile
-// with a smaller number, which a running CTA has already claimed: progress
-// never depends on a CTA that has not started, whatever else occupies the
-// GPU.
+// the accumulator.  Tiles run expert-major, then n-tile, then m-tile, so
+// CTAs working together share a weight tile through L2; the grid is
+// persistent and loops over tiles.
 //
 // Three kernels share the code (MODE):
 //   kModeFused   one launch on CTA pairs (a cluster of 2, M = 256,
-//                cta_group::2) that runs every GEMM1 tile and then (with
-//                run_gemm2) every GEMM2 tile.  Its A rows come from copies in
-//                expert-sorted order (hidden rows copied by the grouping
-//                stage, and act), so rank r of the pair loads A rows
-//                128r..128r+127 and half of the B tile with TMA into its own
-//                shared memory; rank 0 issues the MMAs and each CTA receives
-//                its 128 accumulator rows in its own TMEM.  For GEMM1 rank 0
-//                loads the n-tile's 128 gate rows of w1 and rank 1 the
-//                matching 128 up rows, so one accumulator holds gate and up
-//                side by side.  A GEMM2 tile waits (bounded) until the
-//                epilogues of all GEMM1 tiles of its m-tile have published
-//                their act rows through a per-m-tile counter.
+//                cta_group::2) that runs every GEMM1 tile and then every
+//                GEMM2 tile.  Its A rows come from copies in expert-sorted
+//                order (hidden rows gathered by gather_rows_kernel, and act),
+//                so rank r of the pair loads A rows 128r..128r+127 and half
+//                of the B tile with TMA into its own shared memory; rank 0
+//                issues the MMAs and each CTA receives its 128 accumulator
+//                rows in its own TMEM.  For GEMM1 rank 0 loads the n-tile's
+//                128 gate rows of w1 and rank 1 the matching 128 up rows, so
+//                one accumulator holds gate and up side by side.  A GEMM2
+//                tile waits (bounded) until the epilogues of all GEMM1 tiles
+//                of its m-tile have published their act rows through a
+//                per-m-tile counter: the static tile order puts every GEMM1
+//                tile of a CTA before its GEMM2 tiles, so no wait can form a
+//                cycle, and GEMM2 tiles fill the last, partial wave of GEMM1.
+//                The launch is cooperative: every CTA is resident before any
+//                runs, so no wait depends on a CTA that other work on the
+//                GPU holds back.
 //   kModeGemm1   GEMM1 alone on single CTAs (M = 128, cta_group::1) that
 //                gather their A rows by token index with cp.async (whose
 //                completion can only be signalled to the CTA's own barriers)
 //                and load gate and up rows themselves: no row copy needed.
-//   kModeGemm2   GEMM2 alone on CTA pairs.
+//   kModeGemm2   GEMM2 alone on CTA pairs, after kModeGemm1.
 // The GEMM2 epilogue stages each warp's 32 rows x 32 columns in shared
 // memory and writes them with one asynchronous TMA tile store into P (a
 // block that straddles the end of an expert's rows is written row by row
@@ -65,13 +61,12 @@
 // as many as fit, up to kMaxStages, given the expert count.
 //
 // Warp roles (416 threads per CTA):
-//   warps 0-3  producers.  Thread 0 of rank 0 is also the tile scheduler.
-//              kModeGemm1: the 128 threads gather the A rows with 16-byte
-//              cp.async into the 128-byte-swizzled K-major layout and arrive
-//              on the stage barrier asynchronously when they land; thread 0
-//              issues the two TMA boxes of w1.  CTA pairs: thread 0 of each
-//              CTA issues TMA for its A rows and half of B, counted on rank
-//              0's barrier.
+//   warps 0-3  producers.  kModeGemm1: the 128 threads gather the A rows with
+//              16-byte cp.async into the 128-byte-swizzled K-major layout and
+//              arrive on the stage barrier asynchronously when they land;
+//              thread 0 issues the two TMA boxes of w1.  CTA pairs: thread 0
+//              of each CTA issues TMA for its A rows and half of B, counted
+//              on rank 0's barrier.
 //   warp 4     allocates 512 TMEM columns (two accumulators); one thread (on
 //              rank 0) issues the MMAs and commits each stage back to the
 //              producers and each finished tile to the epilogues.
@@ -100,7 +95,6 @@ constexpr int kTmemCols = 2 * kAccN;  // double-buffered accumulator
 constexpr int kABytes = BM * BK * 2;  // 16 KB
 constexpr int kMaxE = 1024;
 constexpr int kMaxStages = 6;
-constexpr int kTQ = 8;  // depth of the tile queue
 constexpr uint16_t kBothCtas = 0x3;
 // Per-warp staging of the GEMM2 epilogue: one 32-row x 32-column fp32 block,
 // 128-byte swizzled for the TMA store, or 32 plain rows at a 144-byte pitch
@@ -115,10 +109,6 @@ constexpr size_t kSmemMax = 232448;  // opt-in maximum per block on sm_100
 // act rows of an m-tile are complete when every epilogue warp of both CTAs
 // has published each of its n-tiles
 constexpr int kReadyPerTile = 2 * kEpiWarps;
-// out is zeroed (top-k <= 2) in one share per epilogue warp of the grid;
-// each warp takes its own share first (a flag per share, claimed with
-// atomicCAS: no contention), and a warp that waits for zeroing to finish
-// takes the shares nobody has taken (those of CTAs that have not started)
 
 enum { kModeGemm1 = 0, kModeGemm2 = 1, kModeFused = 2 };
 
@@ -154,27 +144,10 @@ struct __align__(8) Bars {
   uint64_t acc_full[2];        // accumulator ready for the epilogue
   uint64_t acc_empty[2];       // epilogues (of both CTAs) drained the accumulator
   uint64_t drain;              // every MMA has completed
-  uint64_t tq_full[kTQ];       // tile queue slot written by the scheduler
-  uint64_t tq_empty[kTQ];      // (rank 0) every consumer of both CTAs has read the slot
-  int tq[kTQ];                 // tile numbers (-1: no more tiles)
-  int prod_tile;               // kModeGemm1: the tile broadcast to the 128 producer threads
   uint32_t tmem_base;
   int abort_flag;
   int32_t scan[32];            // per-warp partial sums of build_tile_offsets
 };
-
-// Readers that acknowledge each queue slot: the epilogue warps of every CTA
-// and, on a pair, rank 1's producer thread.  The MMA thread reads without
-// acknowledging: an mbarrier arrive has release semantics and would wait
-// for the tensor core to finish the MMAs it has just issued.  It needs no
-// acknowledgement, because the slot of tile seq is reused only for tile
-// seq + kTQ, which is published just before the loads of tile seq + kTQ - 1,
-// and those loads need ring slots that the MMA frees only once it has
-// committed stages of tile seq + kTQ - 4 or later (K >= 128: at least two
-// stages per tile, at most kMaxStages stages in flight).
-template <int CG>
-constexpr int queue_consumers() { return CG == 2 ? 1 + 2 * kEpiWarps : kEpiWarps; }
-static_assert(kTQ >= 2 + (kMaxStages + 1) / 2 + 2, "tile queue deeper than the MMA's lead");
 
 // Bytes in front of the aligned region: barriers, then exp_off and tile_off
 // (E + 1 entries each).
@@ -206,30 +179,25 @@ struct Params {
   const int32_t *sorted_rows;
   const int32_t *expert_offsets;
   __nv_bfloat16 *act;
-  int64_t T;
+  float *P;
   int H, I, E, k;
   int nt1, nt2;  // n-tiles per m-tile of GEMM1 (I / 128) and GEMM2 (ceil(H / 256))
   int stages;    // depth of the operand ring (<= kMaxStages)
   int run_gemm2; // kModeFused: 0 runs the GEMM1 tiles only (GEMM2 follows as
                  // its own kModeGemm2 launch)
-  int *sched;    // tile counter of this launch, zero at launch
   uint32_t *status;
   uint64_t wait_limit_ns;
-  // out is zeroed before GEMM2 adds into it (top-k <= 2): zero_n4 float4 in
-  // gridDim.x * kEpiWarps shares, each taken once through its flag in
-  // zero_flags; zero_done counts finished shares
+  // float4 count of out to zero before GEMM2 adds into it (0: none)
   float4 *zero_out;
   int64_t zero_n4;
-  int *zero_flags;
-  int *zero_done;
-  // GEMM2 fused with the combine (top-k <= 2): out [T, H] and the top-k
-  // weights [T, k]; otherwise GEMM2 writes P [T*k, H] fp32
+  // GEMM2 fused with the combine: out [T, H] and the top-k weights [T, k]
   float *out;
   const float *topk_weights;
   int fuse_combine;
-  float *P;
-  // kModeFused: per-m-tile act counters (zero at launch)
+  // kModeFused: per-m-tile act counters and the count of epilogue warps
+  // that finished zeroing out (both zero at launch)
   int *ready;
+  int *zero_done;
   // epilogue variant: activation (kAct*) and optional fp32 biases
   // b1 [E, 2I] (gate, then up) and b2 [E, H]
   const float *b1;
@@ -336,34 +304,8 @@ __device__ __forceinline__ void gated_pack32(const uint32_t (&g)[32], const uint
                         gated_f<ACT>(as_f32(g[2 * v + 1]), as_f32(u[2 * v + 1])));
 }
 
-// Stage row `lane` of a 32-column block, scaled by wgt, at srow (16-byte
-// writes).
-__device__ __forceinline__ void stage_scaled32(uint8_t *srow, const uint32_t (&v)[32], float wgt) {
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-    *reinterpret_cast<float4 *>(srow + 16 * j) =
-        make_float4(wgt * as_f32(v[4 * j]), wgt * as_f32(v[4 * j + 1]),
-                    wgt * as_f32(v[4 * j + 2]), wgt * as_f32(v[4 * j + 3]));
-}
-
-// Zero share `sh` of out (zero_n4 float4 in `shares` contiguous shares) if
-// no warp has taken it yet; the whole warp calls it.
-__device__ __forceinline__ void zero_share(const Params &p, int64_t sh, int64_t shares,
-                                           int lane) {
-  int mine = 0;
-  if (lane == 0) mine = atomicCAS(p.zero_flags + sh, 0, 1) == 0;
-  if (!__shfl_sync(0xffffffffu, mine, 0)) return;
-  const int64_t per = (p.zero_n4 + shares - 1) / shares;
-  const int64_t i0 = sh * per, i1 = min(i0 + per, p.zero_n4);
-  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int64_t i = i0 + lane; i < i1; i += 32) p.zero_out[i] = z;
-  __threadfence();
-  __syncwarp();
-  if (lane == 0) atomicAdd(p.zero_done, 1);
-}
-
-// What one tile number is: GEMM1 or GEMM2 (phase 1 or 2), its place, and
-// its global m-tile index.
+// What one tile of the static schedule is: GEMM1 or GEMM2 (phase 1 or 2),
+// its place, and its global m-tile index.
 struct Work {
   int phase;
   int mi;
@@ -384,55 +326,6 @@ __device__ __forceinline__ Work get_work(int t, int total1, const Params &p,
   w.tl = decode_tile<tile_m<MODE>()>(local, nt, p.E, tile_off, exp_off);
   w.mi = tile_off[w.tl.e] + w.tl.mt;
   return w;
-}
-
-// ---------------------------------------------------------------- tile queue
-// The scheduler (thread 0 of rank 0) writes its claimed tile number (-1
-// past the last tile) into slot seq % kTQ of both CTAs' queues once every
-// reader of that slot's previous use is done.  False if it gave up.  Every
-// tile, the first included, is claimed from the counter (a tile held by a
-// CTA that never started could stall the tiles that wait on it); the claim
-// for the next tile is made as soon as this one is published, so that its
-// round trip to L2 overlaps this tile's loads.
-template <int CG>
-__device__ __forceinline__ bool publish_tile(Bars *bars, uint32_t seq, int total, int *sched,
-                                             int *claimed, uint64_t limit,
-                                             volatile int *abort_flag, int *tile) {
-  const int t = *claimed < total ? *claimed : -1;
-  const int q = static_cast<int>(seq % kTQ);
-  const uint32_t ph = (seq / kTQ) & 1;
-  if (!mbar_wait_cluster(&bars->tq_empty[q], ph ^ 1, limit, abort_flag)) return false;
-  bars->tq[q] = t;
-  mbar_arrive(&bars->tq_full[q]);
-  if (CG == 2) {
-    // the store is ordered before the remote arrive (release at cluster scope)
-    st_shared_cluster_s32(map_to_rank(smem_addr(&bars->tq[q]), 1), t);
-    mbar_arrive_cluster(map_to_rank(smem_addr(&bars->tq_full[q]), 1));
-  }
-  if (t >= 0) *claimed = atomicAdd(sched, 1);
-  *tile = t;
-  return true;
-}
-
-// A reader's side: the tile number of slot seq % kTQ.  Every lane of the
-// calling warp (or the single calling thread) waits and reads; the arrival
-// on rank 0's tq_empty is made once, by lane 0.  False if it gave up.
-__device__ __forceinline__ bool read_tile(Bars *bars, uint32_t seq, uint32_t rank,
-                                          uint32_t tq_empty0, uint64_t limit,
-                                          volatile int *abort_flag, bool arrive, int *tile) {
-  const int q = static_cast<int>(seq % kTQ);
-  const uint32_t ph = (seq / kTQ) & 1;
-  const bool ok = rank == 0 ? mbar_wait(&bars->tq_full[q], ph, limit, abort_flag)
-                            : mbar_wait_cluster(&bars->tq_full[q], ph, limit, abort_flag);
-  if (!ok) return false;
-  *tile = *reinterpret_cast<volatile int *>(&bars->tq[q]);
-  if (arrive) {
-    if (rank == 0)
-      mbar_arrive(&bars->tq_empty[q]);
-    else
-      mbar_arrive_cluster(tq_empty0 + 8u * q);
-  }
-  return true;
 }
 
 template <int MODE>
@@ -473,10 +366,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->acc_empty[a], kEpiWarps * CG);  // every epilogue warp of the pair
     }
     mbar_init(&bars->drain, 1);
-    for (int q = 0; q < kTQ; ++q) {
-      mbar_init(&bars->tq_full[q], 1);
-      mbar_init(&bars->tq_empty[q], queue_consumers<CG>());
-    }
     bars->abort_flag = 0;
     fence_mbar_init();
     if (MODE != kModeGemm2) prefetch_tmap(&tm_b1);
@@ -499,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // both CTAs' barriers exist before any traffic crosses the pair
   if (CG == 2) cluster_sync();
   // Everything above overlaps the previous kernel under PDL; the routing
-  // permutation, the counters and the A rows are read only after this point.
+  // permutation (and the A rows) are read only after this point.
   grid_dep_wait();
   grid_dep_launch();
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_exp_off[i] = p.expert_offsets[i];
@@ -514,13 +403,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total1 = MODE == kModeGemm2 ? 0 : m_tiles * p.nt1;
   const int total =
       total1 + (MODE == kModeGemm1 || (MODE == kModeFused && !p.run_gemm2) ? 0 : m_tiles * p.nt2);
+  const int unit = CG == 2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int nunits = CG == 2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   volatile int *abort_flag = &bars->abort_flag;
   const uint64_t limit = p.wait_limit_ns;
   // rank 0's barriers as seen from this CTA
   const uint32_t full0 = CG == 2 ? map_to_rank(smem_addr(&bars->full[0]), 0) : 0u;
   const uint32_t acc_empty0 = CG == 2 ? map_to_rank(smem_addr(&bars->acc_empty[0]), 0) : 0u;
-  const uint32_t tq_empty0 =
-      CG == 2 ? map_to_rank(smem_addr(&bars->tq_empty[0]), 0) : smem_addr(&bars->tq_empty[0]);
 
   if (warp < 4) {
     // ------------------------------------------------------------ producers
@@ -530,26 +419,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int KB = p.H / BK;
       int s = 0;  // ring slot and its phase parity, advanced per k-block
       uint32_t ph = 0;
-      // Every producer thread takes each tile through the two named barriers
-      // (a thread that gives up inside a tile still comes back to them), and
-      // all leave together when thread 0 hands out -1: past the last tile,
-      // or once the CTA has given up.
-      int claimed = threadIdx.x == 0 ? atomicAdd(p.sched, 1) : 0;  // thread 0: the scheduler
-      for (uint32_t seq = 0;; ++seq) {
-        if (threadIdx.x == 0) {
-          int t = -1;
-          if (!*abort_flag &&
-              !publish_tile<CG>(bars, seq, total, p.sched, &claimed, limit, abort_flag, &t)) {
-            give_up(p, abort_flag);
-            t = -1;
-          }
-          bars->prod_tile = t;
-        }
-        named_bar_sync(1, kProducerThreads);
-        const int t = *reinterpret_cast<volatile int *>(&bars->prod_tile);
-        // every producer thread has the tile before thread 0 may replace it
-        named_bar_sync(1, kProducerThreads);
-        if (t < 0) break;
+      bool stop = false;
+      for (int t = unit; t < total && !stop; t += nunits) {
         const uint64_t tl_t0 = p.tl_buf ? global_timer_ns() : 0;
         const Tile tl = get_work<MODE>(t, total1, p, s_tile_off, s_exp_off).tl;
         const __nv_bfloat16 *src[8];
@@ -570,6 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < KB; ++kb, s = s + 1 == kStages ? 0 : s + 1, ph ^= s == 0) {
           if (!mbar_wait(&bars->empty[s], ph ^ 1, limit, abort_flag)) {
             give_up(p, abort_flag);
+            stop = true;
             break;
           }
           if (threadIdx.x == 0) {
@@ -588,11 +460,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           cp_async_arrive_noinc(&bars->full[s]);
         }
         if (threadIdx.x == 0)
-          timeline_rec(p.tl_buf, p.tl_cap, p.tl_base + int64_t{t} * kTlPerTile + rank,
-                       p.tl_kind, kTlProducer, rank, t, tl_t0, global_timer_ns());
+          timeline_rec(p.tl_buf, p.tl_cap, p.tl_base + int64_t{t} * kTlPerTile + rank, p.tl_kind,
+                       kTlProducer, rank, t, tl_t0, global_timer_ns());
       }
       cp_async_wait_all();
-      if (*abort_flag && threadIdx.x == 0) {
+      if (stop && threadIdx.x == 0) {
         // let TMA copies already issued land before the CTA can exit
         const uint64_t t0 = global_timer_ns();
         while (global_timer_ns() - t0 < 200000) {
@@ -602,31 +474,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int s = 0;  // ring slot and its phase parity, advanced per k-block
       uint32_t ph = 0;
       bool stop = false;
-      // rank 0 publishes each tile one ahead of loading it, so that rank 1
-      // (which loads the other half of every stage) has it in time
-      int claimed = leader ? atomicAdd(p.sched, 1) : 0;
-      int t_next = -1;
-      if (leader &&
-          !publish_tile<CG>(bars, 0, total, p.sched, &claimed, limit, abort_flag, &t_next)) {
-        give_up(p, abort_flag);
-        stop = true;
-      }
-      for (uint32_t seq = 0; !stop; ++seq) {
-        int t = t_next;
-        const bool ok =
-            leader ? (t < 0 || publish_tile<CG>(bars, seq + 1, total, p.sched, &claimed, limit,
-                                                abort_flag, &t_next))
-                   : read_tile(bars, seq, rank, tq_empty0, limit, abort_flag, true, &t);
-        if (!ok) {
-          give_up(p, abort_flag);
-          break;
-        }
-        if (t < 0) break;
+      for (int t = unit; t < total && !stop; t += nunits) {
         const uint64_t tl_t0 = p.tl_buf ? global_timer_ns() : 0;
         const Work w = get_work<MODE>(t, total1, p, s_tile_off, s_exp_off);
         if (MODE == kModeFused && w.phase == 2) {
-          // the act rows of this m-tile come from GEMM1 epilogues of tiles
-          // claimed before this one
+          // the act rows of this m-tile come from other CTAs' GEMM1 epilogues
           if (!wait_geq(p.ready + w.mi, kReadyPerTile * p.nt1, limit, abort_flag)) {
             give_up(p, abort_flag);
             break;
@@ -666,21 +518,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && leader) {
       // ---------------------------------------------------------- MMA issuer
       const uint32_t idesc = idesc_bf16_f32(TM, kAccN);
-      int s = 0;  // ring slot and its phase parity, advanced per k-block
+      int s = 0, acc_it = 0;  // ring slot and its phase parity, advanced per k-block
       uint32_t ph = 0;
       bool stop = false;
-      for (uint32_t seq = 0; !stop; ++seq) {
-        int t = -1;
-        if (!read_tile(bars, seq, 0, tq_empty0, limit, abort_flag, false, &t)) {
-          give_up(p, abort_flag);
-          break;
-        }
-        if (t < 0) break;
-        const int KB =
-            (get_work<MODE>(t, total1, p, s_tile_off, s_exp_off).phase == 1 ? p.H : p.I) /
-            BK;
-        const int a = seq & 1;
-        const uint32_t aph = (seq >> 1) & 1;
+      for (int t = unit; t < total && !stop; t += nunits, ++acc_it) {
+        const int KB = (get_work<MODE>(t, total1, p, s_tile_off, s_exp_off).phase == 1 ? p.H : p.I) / BK;
+        const int a = acc_it & 1;
+        const uint32_t aph = (acc_it >> 1) & 1;
         if (!mbar_wait(&bars->acc_empty[a], aph ^ 1, limit, abort_flag)) {
           give_up(p, abort_flag);
           break;
@@ -740,39 +584,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = ew >> 2;               // which half of the tile's columns
     const int row = q * 32 + lane;
     uint8_t *ebuf = sEpi + ew * kEpiWarpBytes;  // GEMM2: this warp's staging buffer
-    const int64_t gwarp = static_cast<int64_t>(blockIdx.x) * kEpiWarps + ew;
-    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kEpiWarps;
-    const int64_t zero_shares = nwarps;
     if (MODE != kModeGemm2 && p.zero_n4 > 0) {
       // out must read zero before GEMM2 adds into it; this runs while the
       // first tiles' MMAs are in flight
-      zero_share(p, gwarp, zero_shares, lane);
+      const int64_t nw = static_cast<int64_t>(gridDim.x) * kEpiWarps;
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int64_t i = (static_cast<int64_t>(blockIdx.x) * kEpiWarps + ew) * 32 + lane;
+           i < p.zero_n4; i += nw * 32)
+        p.zero_out[i] = z;
+      if (MODE == kModeFused && p.run_gemm2) {
+        // publish: GEMM2 tiles of any CTA add into out only after every
+        // epilogue warp of the grid has zeroed its part
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(p.zero_done, 1);
+      }
     }
     bool zero_seen = MODE != kModeFused || p.zero_n4 == 0 || !p.run_gemm2;
-    for (uint32_t seq = 0;; ++seq) {
-      // waits are taken by every lane; their outcome is made warp-uniform
-      // before the warp-collective TMEM loads
-      int t = -1;
-      const bool got = read_tile(bars, seq, rank, tq_empty0, limit, abort_flag, lane == 0, &t);
-      if (!__all_sync(0xffffffffu, got)) {
-        give_up(p, abort_flag);
-        break;
-      }
-      t = __shfl_sync(0xffffffffu, t, 0);
-      if (t < 0) break;
+    int acc_it = 0;
+    for (int t = unit; t < total; t += nunits, ++acc_it) {
       const Work w = get_work<MODE>(t, total1, p, s_tile_off, s_exp_off);
       const Tile &tl = w.tl;
-      const int a = seq & 1;
-      const uint32_t aph = (seq >> 1) & 1;
-      const int my_row0 = tl.row0 + static_cast<int>(rank) * BM;
-      const int my_rows = min(BM, max(0, tl.rows - static_cast<int>(rank) * BM));
-      const bool valid = row < my_rows;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars->acc_full[a], aph, limit, abort_flag))) {
+      const int a = acc_it & 1;
+      const uint32_t aph = (acc_it >> 1) & 1;
+      if (!mbar_wait(&bars->acc_full[a], aph, limit, abort_flag)) {
         give_up(p, abort_flag);
         break;
       }
       tc_fence_after_sync();
       const uint64_t tl_t0 = p.tl_buf && ew == 0 ? global_timer_ns() : 0;
+      const int my_row0 = tl.row0 + static_cast<int>(rank) * BM;
+      const int my_rows = min(BM, max(0, tl.rows - static_cast<int>(rank) * BM));
+      const bool valid = row < my_rows;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * kAccN;
       if (w.phase == 1) {
         __nv_bfloat16 *dst =
@@ -806,11 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else if (p.fuse_combine) {
         if (!zero_seen) {
-          // every share zeroed; first take any share whose CTA has not
-          // started, so that this never waits for a CTA that is not running
-          if (ld_acquire_gpu(p.zero_done) < static_cast<int>(zero_shares))
-            for (int64_t sh = 0; sh < zero_shares; ++sh) zero_share(p, sh, zero_shares, lane);
-          if (!wait_geq(p.zero_done, static_cast<int>(zero_shares), limit, abort_flag))
+          if (!wait_geq(p.zero_done, static_cast<int>(gridDim.x) * kEpiWarps, limit, abort_flag))
             give_up(p, abort_flag);
           fence_proxy_async_global();
           zero_seen = true;
@@ -836,7 +675,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (col < p.H && valid && !*abort_flag) {
             // the previous reduction from this row must have read it
             bulk_wait_group_read<0>();
-            stage_scaled32(srow, v, wgt);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<float4 *>(srow + 16 * j) =
+                  make_float4(wgt * as_f32(v[4 * j]), wgt * as_f32(v[4 * j + 1]),
+                              wgt * as_f32(v[4 * j + 2]), wgt * as_f32(v[4 * j + 3]));
             fence_proxy_async_smem();
             bulk_reduce_add_f32(orow + col, srow, 128);
             bulk_commit_group();
@@ -975,7 +818,8 @@ int grid_for(const GroupedGemmArgs &a, int n_tiles_n, int device) {
   constexpr int CG = Cfg<MODE>::CG;
   const int64_t rows = a.T * a.k;
   const int64_t max_tiles = ((rows + tile_m<MODE>() - 1) / tile_m<MODE>() + a.E) * n_tiles_n;
-  // one CTA (pair) per SM (pair) that can hold one: more would only queue
+  // never more units than can be resident together: the fused kernel's
+  // GEMM2 tiles wait for other CTAs' GEMM1 tiles
   int units = a.num_sms / CG;
   if (CG == 2 && device >= 0 && device < 64 && g_max_pairs[device] > 0)
     units = std::min(units, g_max_pairs[device]);
@@ -989,7 +833,7 @@ Params base_params(const GroupedGemmArgs &a) {
   p.sorted_rows = a.sorted_rows;
   p.expert_offsets = a.expert_offsets;
   p.act = reinterpret_cast<__nv_bfloat16 *>(a.act);
-  p.T = a.T;
+  p.P = a.P;
   p.H = a.H;
   p.I = a.I;
   p.E = a.E;
@@ -998,29 +842,29 @@ Params base_params(const GroupedGemmArgs &a) {
   p.nt2 = (a.H + kAccN - 1) / kAccN;  // H % 128 == 0: a last half tile is masked
   p.status = a.status;
   p.wait_limit_ns = a.wait_limit_ns;
-  p.out = a.out;
-  p.topk_weights = a.topk_weights;
   p.fuse_combine = a.P == nullptr ? 1 : 0;
-  p.P = a.P;
   if (p.fuse_combine) {
+    p.out = a.out;
+    p.topk_weights = a.topk_weights;
     p.zero_out = reinterpret_cast<float4 *>(a.out);
     p.zero_n4 = a.T * a.H / 4;
   }
-  p.zero_done = a.counters + kCounterZeroDone;
   p.ready = a.counters + kCounterReady;
-  p.zero_flags = p.ready + fused_gemm_ready_count(a.T * a.k, a.E);
+  p.zero_done = a.counters + kCounterZeroDone;
   p.b1 = a.b1;
   p.b2 = a.b2;
   p.act_kind = a.act_kind;
   p.tl_buf = a.timeline;
   p.tl_cap = a.timeline_cap;
-  p.tl_base = 0;
   return p;
 }
 
+// cooperative: every CTA of the grid is resident before any of them runs
+// (the one-launch GEMM's GEMM2 tiles wait for other CTAs' GEMM1 tiles, so
+// those CTAs must not be held back by other work on the GPU).
 template <int MODE>
 cudaLaunchConfig_t launch_config(int grid, size_t smem, cudaStream_t s, bool pdl,
-                                 cudaLaunchAttribute (&attr)[2]) {
+                                 cudaLaunchAttribute (&attr)[3], bool cooperative = false) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
@@ -1039,6 +883,11 @@ cudaLaunchConfig_t launch_config(int grid, size_t smem, cudaStream_t s, bool pdl
     attr[n].val.programmaticStreamSerializationAllowed = 1;
     ++n;
   }
+  if (cooperative) {
+    attr[n].id = cudaLaunchAttributeCooperative;
+    attr[n].val.cooperative = 1;
+    ++n;
+  }
   cfg.attrs = attr;
   cfg.numAttrs = n;
   return cfg;
@@ -1053,7 +902,7 @@ cudaError_t set_smem_attr() {
 
 template <int MODE>
 cudaError_t max_pairs(int *clusters) {
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   cudaLaunchConfig_t cfg = launch_config<MODE>(2, kSmemMax, nullptr, false, attr);
   return cudaOccupancyMaxActiveClusters(clusters, grouped_gemm_kernel<MODE>, &cfg);
 }
@@ -1117,17 +966,15 @@ cudaError_t launch_gemm1_swiglu(const GroupedGemmArgs &a, cudaStream_t s, const 
   int dev = 0;
   cudaGetDevice(&dev);
   Params p = base_params(a);
-  p.sched = a.counters + kCounterSched0;
   p.tl_kind = kTlGemm1;
-  p.zero_n4 = 0;  // nothing is added into out before the GEMM2 launch
   p.stages = stages_for<kModeGemm1>(a.E);
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   const cudaLaunchConfig_t cfg =
       launch_config<kModeGemm1>(grid_for<kModeGemm1>(a, p.nt1, dev),
                                 smem_bytes<kModeGemm1>(a.E, p.stages), s, hook.pdl, attr);
   hook.begin("gemm1_swiglu");
-  cudaError_t e =
-      cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm1>, tm_w1, tm_w1, tm_w1, tm_w1, tm_w1, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm1>, tm_w1, tm_w1, tm_w1,
+                                     tm_w1, tm_w1, p);
   return hook.end(e);
 }
 
@@ -1137,26 +984,25 @@ cudaError_t launch_gemm2(const GroupedGemmArgs &a, cudaStream_t s, const StageHo
   int dev = 0;
   cudaGetDevice(&dev);
   Params p = base_params(a);
-  p.sched = a.counters + kCounterSched1;
+  p.zero_out = nullptr;  // zeroed by GEMM1
+  p.zero_n4 = 0;
   p.tl_kind = kTlGemm2;
   // after the first launch's records: at most (m-tiles) * (GEMM1 n-tiles) tiles
   p.tl_base = ((a.T * a.k + 255) / 128 + 2 * a.E) * (a.I / (kAccN / 2)) * kTlPerTile;
-  p.zero_out = nullptr;  // zeroed by the GEMM1 launch
-  p.zero_n4 = 0;
   p.stages = stages_for<kModeGemm2>(a.E);
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   const cudaLaunchConfig_t cfg =
       launch_config<kModeGemm2>(grid_for<kModeGemm2>(a, p.nt2, dev),
                                 smem_bytes<kModeGemm2>(a.E, p.stages), s, hook.pdl, attr);
   hook.begin("gemm2");
-  cudaError_t e =
-      cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm2>, tm_act, tm_w2, tm_act, tm_w2, tm_p, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeGemm2>, tm_act, tm_w2, tm_act,
+                                     tm_w2, tm_p, p);
   return hook.end(e);
 }
 
 cudaError_t launch_fused_gemm(const GroupedGemmArgs &a, bool with_gemm2, cudaStream_t s,
                               const StageHook &hook) {
-  if (a.xs == nullptr || a.P != nullptr) return cudaErrorInvalidValue;
+  if (a.xs == nullptr || (with_gemm2 && a.counters == nullptr)) return cudaErrorInvalidValue;
   CUtensorMap tm_xs, tm_w1, tm_act, tm_w2, tm_p;
   if (!make_bf16_map(&tm_xs, a.xs, static_cast<uint64_t>(a.H), static_cast<uint64_t>(a.T) * a.k,
                      BM) ||
@@ -1165,17 +1011,16 @@ cudaError_t launch_fused_gemm(const GroupedGemmArgs &a, bool with_gemm2, cudaStr
   int dev = 0;
   cudaGetDevice(&dev);
   Params p = base_params(a);
-  p.sched = a.counters + kCounterSched0;
   p.tl_kind = with_gemm2 ? kTlFused : kTlGemm1;
   p.run_gemm2 = with_gemm2 ? 1 : 0;
   p.stages = stages_for<kModeFused>(a.E, with_gemm2);
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   const cudaLaunchConfig_t cfg = launch_config<kModeFused>(
       grid_for<kModeFused>(a, with_gemm2 ? p.nt1 + p.nt2 : p.nt1, dev),
-      smem_bytes<kModeFused>(a.E, p.stages, with_gemm2), s, hook.pdl, attr);
+      smem_bytes<kModeFused>(a.E, p.stages, with_gemm2), s, hook.pdl, attr, with_gemm2);
   hook.begin(with_gemm2 ? "gemm_fused" : "gemm1_swiglu");
-  cudaError_t e =
-      cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeFused>, tm_xs, tm_w1, tm_act, tm_w2, tm_p, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeFused>, tm_xs, tm_w1, tm_act,
+                                     tm_w2, tm_p, p);
   return hook.end(e);
 }
 

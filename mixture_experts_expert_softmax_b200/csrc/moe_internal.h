@@ -72,19 +72,14 @@ cudaError_t launch_gather_rows(const uint16_t *hidden, int H, int k, const int32
 
 // grouped_gemm.cu
 // Counters of the GEMM launches of one forward, in one int block that the
-// grouping stage zeroes: the tile scheduler of the first and of the second
-// GEMM launch (each in a 128-byte line of its own, away from the others'
-// traffic), the finished shares of zeroing out, one act readiness counter
-// per 256-row m-tile of the one-launch GEMM, then one flag per share of
-// zeroing out (at most kMaxZeroShares: one per epilogue warp of the grid).
-constexpr int kCounterSched0 = 0;
-constexpr int kCounterSched1 = 32;
-constexpr int kCounterZeroDone = 64;
-constexpr int kCounterReady = 96;
-constexpr int kMaxZeroShares = 2048;
+// grouping stage zeroes: the number of epilogue warps of the one-launch GEMM
+// that have zeroed their part of out, then one act readiness counter per
+// 256-row m-tile.
+constexpr int kCounterZeroDone = 0;
+constexpr int kCounterReady = 32;
 inline int64_t fused_gemm_ready_count(int64_t n, int E) { return (n + 255) / 256 + E; }
 inline int64_t gemm_counter_count(int64_t n, int E) {
-  return kCounterReady + fused_gemm_ready_count(n, E) + kMaxZeroShares;
+  return kCounterReady + fused_gemm_ready_count(n, E);
 }
 
 struct GroupedGemmArgs {
