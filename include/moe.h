@@ -28,6 +28,17 @@
  *     allocates (and synchronises the device if it frees a smaller one).
  *     Calls on two different streams of one device must not overlap in time
  *     (they share that workspace).
+ *   - Two kernels expect all of their CTAs on the GPU at once: the
+ *     small-batch kernel (a cooperative launch, which the runtime only
+ *     starts when every CTA fits) and, for top-k <= 2 with at most about
+ *     twelve waves of tiles, the grouped GEMM that runs both projections in
+ *     one launch (its second-projection tiles wait for first-projection
+ *     tiles of other CTAs).  Work that another stream keeps on the SMs while
+ *     that GEMM runs -- a persistent kernel such as a running collective --
+ *     can hold some of its CTAs back; its waits then give up after the wait
+ *     limit (moe_set_wait_limit_ns, 2 s by default), out is invalid and
+ *     MOE_STATUS_TIMEOUT is raised.  Order such work before or after the
+ *     call on the stream.
  */
 #ifndef MOE_H
 #define MOE_H

@@ -39,9 +39,10 @@
 //                per-m-tile counter: the static tile order puts every GEMM1
 //                tile of a CTA before its GEMM2 tiles, so no wait can form a
 //                cycle, and GEMM2 tiles fill the last, partial wave of GEMM1.
-//                The launch is cooperative: every CTA is resident before any
-//                runs, so no wait depends on a CTA that other work on the
-//                GPU holds back.
+//                This needs every CTA of the grid resident at once (the grid
+//                never exceeds the occupancy query's cluster count): work that
+//                another stream keeps on the SMs meanwhile can hold CTAs back
+//                until a bounded wait gives up (MOE_STATUS_TIMEOUT).
 //   kModeGemm1   GEMM1 alone on single CTAs (M = 128, cta_group::1) that
 //                gather their A rows by token index with cp.async (whose
 //                completion can only be signalled to the CTA's own barriers)
@@ -859,12 +860,9 @@ Params base_params(const GroupedGemmArgs &a) {
   return p;
 }
 
-// cooperative: every CTA of the grid is resident before any of them runs
-// (the one-launch GEMM's GEMM2 tiles wait for other CTAs' GEMM1 tiles, so
-// those CTAs must not be held back by other work on the GPU).
 template <int MODE>
 cudaLaunchConfig_t launch_config(int grid, size_t smem, cudaStream_t s, bool pdl,
-                                 cudaLaunchAttribute (&attr)[3], bool cooperative = false) {
+                                 cudaLaunchAttribute (&attr)[3]) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
@@ -881,11 +879,6 @@ cudaLaunchConfig_t launch_config(int grid, size_t smem, cudaStream_t s, bool pdl
   if (pdl) {
     attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[n].val.programmaticStreamSerializationAllowed = 1;
-    ++n;
-  }
-  if (cooperative) {
-    attr[n].id = cudaLaunchAttributeCooperative;
-    attr[n].val.cooperative = 1;
     ++n;
   }
   cfg.attrs = attr;
@@ -1017,7 +1010,7 @@ cudaError_t launch_fused_gemm(const GroupedGemmArgs &a, bool with_gemm2, cudaStr
   cudaLaunchAttribute attr[3];
   const cudaLaunchConfig_t cfg = launch_config<kModeFused>(
       grid_for<kModeFused>(a, with_gemm2 ? p.nt1 + p.nt2 : p.nt1, dev),
-      smem_bytes<kModeFused>(a.E, p.stages, with_gemm2), s, hook.pdl, attr, with_gemm2);
+      smem_bytes<kModeFused>(a.E, p.stages, with_gemm2), s, hook.pdl, attr);
   hook.begin(with_gemm2 ? "gemm_fused" : "gemm1_swiglu");
   cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kModeFused>, tm_xs, tm_w1, tm_act,
                                      tm_w2, tm_p, p);
