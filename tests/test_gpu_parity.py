@@ -333,9 +333,9 @@ def test_forward_deterministic(T, H, I, E, k):
 @pytest.mark.parametrize("T,H,I,E,k", [(1979, 2048, 2048, 8, 2), (2000, 1024, 384, 64, 8)])
 def test_forward_beside_other_work(T, H, I, E, k):
     """The forward while another stream keeps the SMs busy with matrix
-    products: tiles are claimed by whichever CTAs run, so the result must be
-    exact and no bounded wait may run out (which would raise the timeout
-    bit), however few CTAs are resident at first."""
+    products (finite work: CTAs it holds back start when it ends, well
+    inside the wait limit): the result is bit-identical to the forward run
+    alone and no bounded wait runs out (which would raise the timeout bit)."""
     hidden, w1, w2, logits = make_inputs(T, H, I, E, seed=31)
     ids, w = oracle.route(logits.numpy(), k, True)
     dev = torch.device("cuda")
