@@ -326,7 +326,8 @@ int moe_debug_wait_timeout(int64_t limit_ns, void *stream);
  *        1 MMA issuer (t0 accumulator free, t1 last MMA issued),
  *        2 epilogue, first epilogue warp (t0 accumulator full, t1 released),
  *        3 / 4 small-batch phase 1 / grid barrier, 5 act staged on chip,
- *        6 w2 rows on chip, 7 phase 2 (3-7: id = CTA);
+ *        6 w2 rows on chip, 7 phase 2, 8 phase 2's dot products done
+ *        (3-8: id = CTA);
  *   sub: the CTA's rank in its pair (roles 0 and 2); id: the tile number.
  * Each call's records overwrite the previous call's; slots past capacity
  * are dropped.  buf == NULL turns it off (the default).  Not synchronised

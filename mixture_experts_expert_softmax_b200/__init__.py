@@ -291,7 +291,7 @@ def moe_permute_ex(topk_ids: torch.Tensor, E: int, kernel: str = "auto",
 
 TIMELINE_KINDS = {1: "gemm1", 2: "gemm2", 3: "gemm_fused", 4: "small_t"}
 TIMELINE_ROLES = {0: "producer", 1: "mma", 2: "epilogue", 3: "phase1", 4: "barrier",
-                  5: "act_load", 6: "w2_wait", 7: "phase2"}
+                  5: "act_load", 6: "w2_wait", 7: "phase2", 8: "phase2_dots"}
 _timeline_buf = None
 
 

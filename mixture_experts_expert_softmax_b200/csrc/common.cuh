@@ -363,10 +363,11 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t *bar, uint16_t cta_mas
 enum : uint32_t {
   kTlGemm1 = 1, kTlGemm2 = 2, kTlFused = 3, kTlSmallT = 4,  // kinds
   kTlProducer = 0, kTlMma = 1, kTlEpilogue = 2,             // roles (GEMM kernels)
-  kTlPhase1 = 3, kTlBarrier = 4, kTlActLoad = 5, kTlW2Wait = 6, kTlPhase2 = 7  // small-T
+  kTlPhase1 = 3, kTlBarrier = 4, kTlActLoad = 5, kTlW2Wait = 6, kTlPhase2 = 7,  // small-T
+  kTlItems = 8
 };
 constexpr int kTlPerTile = 5;  // producer x2 (pair ranks), MMA, epilogue x2
-constexpr int kTlPerCta = 5;   // small-T: phase 1, barrier, act load, w2 wait, phase 2
+constexpr int kTlPerCta = 6;   // small-T: phase 1, barrier, act, w2 wait, phase 2, dot products
 
 __device__ __forceinline__ void timeline_rec(uint64_t *buf, int64_t cap, int64_t slot,
                                              uint32_t kind, uint32_t role, uint32_t sub,

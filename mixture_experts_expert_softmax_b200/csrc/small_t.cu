@@ -483,6 +483,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ Lists L;
   __shared__ volatile int s_abort;
+  __shared__ int s_taken;  // phase-1 tasks of this CTA taken so far
   __shared__ uint64_t w2_full[kMaxSlots];   // a slot's rows have landed
   __shared__ uint64_t w2_empty[kMaxSlots];  // every compute warp is done with a slot
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -505,6 +506,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   if (warp == 0) build_lists(L, ids, TK, E);
   if (threadIdx.x == 32) {
     s_abort = 0;
+    s_taken = 0;
     for (int q = 0; q < slots; ++q) {
       mbar_init(&w2_full[q], 1);
       mbar_init(&w2_empty[q], kWarps);
@@ -516,7 +518,6 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   const uint4 *sx4 = reinterpret_cast<const uint4 *>(sx);
   __syncthreads();
   const int nd = L.n_distinct;
-  const int nw = gridDim.x * kWarps;
   const int n1 = nd * I;
   // bytes of one expert's rows of this CTA (nrows may be 0 for the last CTAs)
   const uint32_t w2_bytes = static_cast<uint32_t>(nrows) * I * kElem;
@@ -538,7 +539,17 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   }
 
   // ------------------------------------------------------------ phase 1
-  for (int task = blockIdx.x * kWarps + warp; task < n1 && warp < kWarps; task += nw) {
+  // This CTA's share of the (expert, row) tasks: a contiguous range of
+  // n1 / gridDim.x of them (within one), taken by its compute warps one at
+  // a time, so that every CTA streams the same number of bytes and no warp
+  // idles while another of its CTA still has two tasks to go.
+  const int task_lo = static_cast<int>(static_cast<int64_t>(blockIdx.x) * n1 / gridDim.x);
+  const int task_hi = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * n1 / gridDim.x);
+  for (;;) {
+    int task = 0;
+    if (lane == 0) task = task_lo + atomicAdd(&s_taken, 1);
+    task = __shfl_sync(0xffffffffu, task, 0);
+    if (task >= task_hi || warp >= kWarps) break;
     const int d = task / I, i = task - d * I;
     const int p0 = L.dstart[d], np = L.dstart[d + 1] - p0;
     const uint4 *g = w1 + (static_cast<size_t>(L.dexp[d]) * 2 * I + i) * HC;
@@ -740,6 +751,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     }
   }
   __syncthreads();
+  if (threadIdx.x == 0)
+    timeline_rec(tl_buf, tl_cap, tl_slot + 5, kTlSmallT, kTlItems, 0, blockIdx.x, tl_bar,
+                 global_timer_ns());
   if (s_abort) return;
   // out[t, h] = sum over j in ascending order of w[t, j] * dot(t*k + j)
   for (int x = threadIdx.x; x < T * nrows; x += kThreads) {
