@@ -545,11 +545,11 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   // idles while another of its CTA still has two tasks to go.
   const int task_lo = static_cast<int>(static_cast<int64_t>(blockIdx.x) * n1 / gridDim.x);
   const int task_hi = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * n1 / gridDim.x);
-  for (;;) {
+  for (; warp < kWarps;) {  // the copy warp takes no task
     int task = 0;
     if (lane == 0) task = task_lo + atomicAdd(&s_taken, 1);
     task = __shfl_sync(0xffffffffu, task, 0);
-    if (task >= task_hi || warp >= kWarps) break;
+    if (task >= task_hi) break;
     const int d = task / I, i = task - d * I;
     const int p0 = L.dstart[d], np = L.dstart[d + 1] - p0;
     const uint4 *g = w1 + (static_cast<size_t>(L.dexp[d]) * 2 * I + i) * HC;
