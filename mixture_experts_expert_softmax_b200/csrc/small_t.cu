@@ -711,7 +711,37 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     if (warp == 0 && lane == 0)
       timeline_rec(tl_buf, tl_cap, tl_slot + 3, kTlSmallT, kTlW2Wait, 0, blockIdx.x, tl_act,
                    global_timer_ns());
-    const int n_items = L.dstart[nd] * rgroups;
+    if (!kFp8) {
+      // each compute warp takes whole output rows: for every token, the dot
+      // products of the row with act of its pairs (independent loads, one
+      // pass) and the weighted sum in ascending j straight into out
+      const int I8 = I / 8;
+      for (int r = warp; r < nrows && !s_abort; r += kWarps) {
+        for (int t = 0; t < T; ++t) {
+          float acc = 0.f;
+          for (int j = 0; j < k; ++j) {
+            const int pair = t * k + j;
+            const int d = L.pd[pair];
+            if (d < 0) continue;
+            const uint4 *wrow =
+                ring ? reinterpret_cast<const uint4 *>(sw2 + d * slot_stride) + r * IC
+                     : w2 + (static_cast<size_t>(L.dexp[d]) * H + h0 + r) * IC;
+            const float4 *arow = act4 + static_cast<size_t>(pair) * (I / 4);
+            unsigned long long v = 0ull;  // two fp32 partial sums
+            for (int c = lane; c < I8; c += 32) {
+              const float4 a0 = cache_act ? arow[2 * c] : __ldcg(arow + 2 * c);
+              const float4 a1 = cache_act ? arow[2 * c + 1] : __ldcg(arow + 2 * c + 1);
+              fma8_f32x2(ring ? wrow[c] : __ldg(wrow + c), a0, a1, v);
+            }
+            float y = warp_sum(sum_f32x2(v));
+            if (b2 != nullptr) y += __ldg(b2 + static_cast<size_t>(L.ids[pair]) * H + h0 + r);
+            acc = fmaf(__ldg(topk_w + pair), y, acc);
+          }
+          if (lane == 0) out[static_cast<size_t>(t) * H + h0 + r] = acc;
+        }
+      }
+    }
+    const int n_items = kFp8 ? L.dstart[nd] * rgroups : 0;
     for (int it = warp; it < n_items && !s_abort; it += kWarps) {
       const int pq = it / rgroups, rg = it - pq * rgroups;  // pq: position in plist
       const int pair = L.plist[pq];
@@ -756,7 +786,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
                  global_timer_ns());
   if (s_abort) return;
   // out[t, h] = sum over j in ascending order of w[t, j] * dot(t*k + j)
-  for (int x = threadIdx.x; x < T * nrows; x += kThreads) {
+  const bool wrote = (!kFp8 && rgroups > 0 && (!ring || nd <= slots));
+  for (int x = wrote ? T * nrows : threadIdx.x; x < T * nrows; x += kThreads) {
     const int t = x / nrows, r = x - t * nrows;
     float acc = 0.f;
     for (int j = 0; j < k; ++j) {
