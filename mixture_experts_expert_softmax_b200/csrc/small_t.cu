@@ -483,7 +483,6 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ Lists L;
   __shared__ volatile int s_abort;
-  __shared__ int s_taken;  // phase-1 tasks of this CTA taken so far
   __shared__ uint64_t w2_full[kMaxSlots];   // a slot's rows have landed
   __shared__ uint64_t w2_empty[kMaxSlots];  // every compute warp is done with a slot
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -506,7 +505,6 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   if (warp == 0) build_lists(L, ids, TK, E);
   if (threadIdx.x == 32) {
     s_abort = 0;
-    s_taken = 0;
     for (int q = 0; q < slots; ++q) {
       mbar_init(&w2_full[q], 1);
       mbar_init(&w2_empty[q], kWarps);
@@ -518,6 +516,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   const uint4 *sx4 = reinterpret_cast<const uint4 *>(sx);
   __syncthreads();
   const int nd = L.n_distinct;
+  const int nw = gridDim.x * kWarps;
   const int n1 = nd * I;
   // bytes of one expert's rows of this CTA (nrows may be 0 for the last CTAs)
   const uint32_t w2_bytes = static_cast<uint32_t>(nrows) * I * kElem;
@@ -539,17 +538,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   }
 
   // ------------------------------------------------------------ phase 1
-  // This CTA's share of the (expert, row) tasks: a contiguous range of
-  // n1 / gridDim.x of them (within one), taken by its compute warps one at
-  // a time, so that every CTA streams the same number of bytes and no warp
-  // idles while another of its CTA still has two tasks to go.
-  const int task_lo = static_cast<int>(static_cast<int64_t>(blockIdx.x) * n1 / gridDim.x);
-  const int task_hi = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * n1 / gridDim.x);
-  for (; warp < kWarps;) {  // the copy warp takes no task
-    int task = 0;
-    if (lane == 0) task = task_lo + atomicAdd(&s_taken, 1);
-    task = __shfl_sync(0xffffffffu, task, 0);
-    if (task >= task_hi) break;
+  for (int task = blockIdx.x * kWarps + warp; task < n1 && warp < kWarps; task += nw) {
     const int d = task / I, i = task - d * I;
     const int p0 = L.dstart[d], np = L.dstart[d + 1] - p0;
     const uint4 *g = w1 + (static_cast<size_t>(L.dexp[d]) * 2 * I + i) * HC;
@@ -711,37 +700,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     if (warp == 0 && lane == 0)
       timeline_rec(tl_buf, tl_cap, tl_slot + 3, kTlSmallT, kTlW2Wait, 0, blockIdx.x, tl_act,
                    global_timer_ns());
-    if (!kFp8) {
-      // each compute warp takes whole output rows: for every token, the dot
-      // products of the row with act of its pairs (independent loads, one
-      // pass) and the weighted sum in ascending j straight into out
-      const int I8 = I / 8;
-      for (int r = warp; r < nrows && !s_abort; r += kWarps) {
-        for (int t = 0; t < T; ++t) {
-          float acc = 0.f;
-          for (int j = 0; j < k; ++j) {
-            const int pair = t * k + j;
-            const int d = L.pd[pair];
-            if (d < 0) continue;
-            const uint4 *wrow =
-                ring ? reinterpret_cast<const uint4 *>(sw2 + d * slot_stride) + r * IC
-                     : w2 + (static_cast<size_t>(L.dexp[d]) * H + h0 + r) * IC;
-            const float4 *arow = act4 + static_cast<size_t>(pair) * (I / 4);
-            unsigned long long v = 0ull;  // two fp32 partial sums
-            for (int c = lane; c < I8; c += 32) {
-              const float4 a0 = cache_act ? arow[2 * c] : __ldcg(arow + 2 * c);
-              const float4 a1 = cache_act ? arow[2 * c + 1] : __ldcg(arow + 2 * c + 1);
-              fma8_f32x2(ring ? wrow[c] : __ldg(wrow + c), a0, a1, v);
-            }
-            float y = warp_sum(sum_f32x2(v));
-            if (b2 != nullptr) y += __ldg(b2 + static_cast<size_t>(L.ids[pair]) * H + h0 + r);
-            acc = fmaf(__ldg(topk_w + pair), y, acc);
-          }
-          if (lane == 0) out[static_cast<size_t>(t) * H + h0 + r] = acc;
-        }
-      }
-    }
-    const int n_items = kFp8 ? L.dstart[nd] * rgroups : 0;
+    const int n_items = L.dstart[nd] * rgroups;
     for (int it = warp; it < n_items && !s_abort; it += kWarps) {
       const int pq = it / rgroups, rg = it - pq * rgroups;  // pq: position in plist
       const int pair = L.plist[pq];
@@ -786,8 +745,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
                  global_timer_ns());
   if (s_abort) return;
   // out[t, h] = sum over j in ascending order of w[t, j] * dot(t*k + j)
-  const bool wrote = (!kFp8 && rgroups > 0 && (!ring || nd <= slots));
-  for (int x = wrote ? T * nrows : threadIdx.x; x < T * nrows; x += kThreads) {
+  for (int x = threadIdx.x; x < T * nrows; x += kThreads) {
     const int t = x / nrows, r = x - t * nrows;
     float acc = 0.f;
     for (int j = 0; j < k; ++j) {
