@@ -274,6 +274,88 @@ int moe_permute_ex(const int32_t *topk_ids, int64_t T, int k, int E,
                    int32_t *sorted_rows, int32_t *expert_offsets, int32_t *inv,
                    const uint16_t *hidden, int H, uint16_t *xs, int kernel, void *stream);
 
+/*
+ * Expert parallelism (EP) over `world` ranks, one per GPU: rank r owns the
+ * experts [r * E / world, (r + 1) * E / world) (w1 / w2 hold only those
+ * E / world experts on each rank) and routes its own tokens.  A forward is
+ *   1. moe_ep_dispatch_plan: the send order (the (token, slot) rows grouped
+ *      by owner rank) and its per-rank counts;
+ *   2. an exchange of the counts (every rank learns where its rows land in
+ *      every receiver's buffer);
+ *   3. moe_ep_pack: the hidden rows and local expert ids, stored straight
+ *      into the receivers' buffers;
+ *   4. moe_forward on the received rows with top-k 1 and weight 1 (each row
+ *      its own expert's FFN output);
+ *   5. moe_ep_return: each output row stored straight into its sender's
+ *      buffer;
+ *   6. moe_ep_combine: out[t] = sum over j in ascending order of
+ *      w[t, j] * y[t, j], fp32.
+ * Pages: the TPU kernel's expert-parallel structure (all_reduce_metadata of
+ * the per-device expert counts, start_a2a_scatter, the expert FFNs,
+ * start_a2a_gather back to the token owner, the fixed-order bt_acc sum) and
+ * the 0.13.2 version's fused_ep_moe wrapper (a shard_map over the expert
+ * axis).  Steps 2 and the synchronisation between ranks are the caller's
+ * (the Python package's ep module does them with torch.distributed).  The
+ * destination buffers may be another GPU's memory mapped into this one: the
+ * copies only store to them.
+ */
+
+/*
+ * moe_ep_dispatch_plan -- the send order of this rank's (token, slot) rows.
+ *   topk_ids      [T, k] int32 (global expert ids)
+ *   send_rows     [T*k] int32, written for positions < send_offsets[world]:
+ *                 flat indices t*k + j grouped by owner rank, ascending
+ *                 within a rank
+ *   send_offsets  [world+1] int32, written: exclusive prefix sum of the rows
+ *                 sent to each rank
+ *   inv           [T*k] int32, written: the position of flat index i in
+ *                 send_rows, -1 for an id outside [0, E) (flagged with
+ *                 MOE_STATUS_BAD_ID)
+ * Errors: INVALID_ARG for null pointers, T < 0, k outside [1, E], world < 1;
+ *         UNSUPPORTED for E > 1024, world > 64 or E % world != 0.
+ */
+int moe_ep_dispatch_plan(const int32_t *topk_ids, int64_t T, int k, int E, int world,
+                         int32_t *send_rows, int32_t *send_offsets, int32_t *inv,
+                         void *stream);
+
+/*
+ * moe_ep_pack -- row r of the send order (destination d: the segment of
+ * send_offsets it falls in) is stored as row dst_row0[d] + r -
+ * send_offsets[d] of d's buffers: dst_x[d] [rows, H] bf16 gets the hidden
+ * row of its token, dst_eid[d] [rows] int32 its expert id minus d * E / world.
+ *   send_offsets, dst_row0  HOST arrays of world + 1 and world int64 values
+ *   dst_x, dst_eid          HOST arrays of world DEVICE pointers (16-byte
+ *                           aligned; unused, and may be NULL, for a rank
+ *                           that receives no rows)
+ * Errors: INVALID_ARG for null pointers, offsets that are not a prefix sum
+ *         starting at 0 or exceed T*k, negative rows, unaligned buffers;
+ *         UNSUPPORTED for H % 128 != 0, world > 64 or E % world != 0.
+ */
+int moe_ep_pack(const uint16_t *hidden, int H, const int32_t *topk_ids, int64_t T, int k, int E,
+                int world, const int32_t *send_rows, const int64_t *send_offsets,
+                uint16_t *const *dst_x, int32_t *const *dst_eid, const int64_t *dst_row0,
+                void *stream);
+
+/*
+ * moe_ep_return -- received row q (source s: the segment of recv_offsets it
+ * falls in) of y [recv_offsets[world], H] fp32 is stored as row
+ * dst_row0[s] + q - recv_offsets[s] of dst_y[s] (the source's buffer of its
+ * send order).  Arrays and errors as in moe_ep_pack.
+ */
+int moe_ep_return(const float *y, int H, int world, const int64_t *recv_offsets,
+                  float *const *dst_y, const int64_t *dst_row0, void *stream);
+
+/*
+ * moe_ep_combine -- out[t] = sum over j = 0..k-1 in ascending order of
+ * topk_weights[t, j] * y_back[inv[t*k + j]] (one fp32 fused multiply-add per
+ * term; slots with inv = -1 skipped and flagged), every row of out
+ * [T, H] fp32 written.  y_back [T*k, H] fp32 in the send order.
+ * Errors: INVALID_ARG for null pointers or unaligned y_back / out, T < 0,
+ *         k < 1; UNSUPPORTED for H % 128 != 0 or k > 16.
+ */
+int moe_ep_combine(const float *y_back, const int32_t *inv, const float *topk_weights, float *out,
+                   int64_t T, int H, int k, void *stream);
+
 /* Static, NUL-terminated description of an MOE_* return code. */
 const char *moe_error_string(int code);
 

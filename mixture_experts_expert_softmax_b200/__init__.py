@@ -49,7 +49,7 @@ EXPORTED = (
     "moe_set_wait_limit_ns", "moe_last_failed_stage", "moe_debug_wait_timeout",
     "moe_profile_enable", "moe_profile_reset", "moe_profile_read",
     "moe_forward_small_noalloc", "moe_forward_ex", "moe_forward_fp8", "moe_permute_ex",
-    "moe_timeline",
+    "moe_timeline", "moe_ep_dispatch_plan", "moe_ep_pack", "moe_ep_return", "moe_ep_combine",
 )
 
 
@@ -72,6 +72,10 @@ def _load() -> ctypes.CDLL:
         "moe_permute": ([P, I64, I32, I32, P, P, P], I32),
         "moe_permute_ex": ([P, I64, I32, I32, P, P, P, P, I32, P, I32, P], I32),
         "moe_timeline": ([P, I64], I32),
+        "moe_ep_dispatch_plan": ([P, I64, I32, I32, I32, P, P, P, P], I32),
+        "moe_ep_pack": ([P, I32, P, I64, I32, I32, I32, P, P, P, P, P, P], I32),
+        "moe_ep_return": ([P, I32, I32, P, P, P, P], I32),
+        "moe_ep_combine": ([P, P, P, P, I64, I32, I32, P], I32),
         "moe_error_string": ([I32], ctypes.c_char_p),
         "moe_get_device_status": ([P, ctypes.POINTER(ctypes.c_uint32)], I32),
         "moe_set_small_t_max": ([I32], I32),

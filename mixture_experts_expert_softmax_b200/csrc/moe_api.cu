@@ -485,6 +485,136 @@ int moe_forward_ex(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w
                       stream);
 }
 
+// ---------------------------------------------------------------- expert parallelism
+
+int moe_ep_dispatch_plan(const int32_t *topk_ids, int64_t T, int k, int E, int world,
+                         int32_t *send_rows, int32_t *send_offsets, int32_t *inv, void *stream) {
+  if (T < 0 || k < 1 || E < 1 || world < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (send_offsets == nullptr ||
+      (T > 0 && (topk_ids == nullptr || send_rows == nullptr || inv == nullptr)))
+    return MOE_ERR_INVALID_ARG;
+  if (E > kMaxExperts || world > moe::kEpMaxWorld || E % world != 0) return MOE_ERR_UNSUPPORTED;
+  const int64_t n = T * k;
+  if (n >= (static_cast<int64_t>(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState *d = nullptr;
+  int rc = current_device(&d);
+  if (rc != MOE_OK) return rc;
+  if ((rc = ensure_workspace(*d, permute_ws_bytes(n, world) +
+                                     align256(static_cast<size_t>(std::max<int64_t>(n, 1)) * 4))) !=
+      MOE_OK)
+    return rc;
+  Carver cv{static_cast<char *>(d->ws)};
+  int32_t *chunk_counts =
+      cv.take<int32_t>(std::max(moe::permute_num_chunks(n), 1) * static_cast<size_t>(world));
+  int32_t *owner = cv.take<int32_t>(std::max<int64_t>(n, 1));
+  CallCtx ctx{static_cast<cudaStream_t>(stream), "", nullptr};
+  moe::StageHook hook = make_hook(&ctx);
+  cudaError_t e = cudaSuccess;
+  if (n > 0) e = moe::launch_ep_owner(topk_ids, n, E, world, owner, ctx.stream, hook);
+  // the (token, slot) rows grouped by owner rank, stable: the send order
+  if (e == cudaSuccess) {
+    if (moe::group_supported(n))
+      e = moe::launch_group(owner, n, world, k, send_offsets, send_rows, inv, d->status, nullptr,
+                            0, nullptr, nullptr, 0, d->num_sms, ctx.stream, hook);
+    else
+      e = moe::launch_permute(owner, n, world, chunk_counts, send_offsets, send_rows, inv,
+                              d->status, nullptr, 0, ctx.stream, hook);
+  }
+  return to_code(e);
+}
+
+namespace {
+
+// Host route tables of moe_ep_pack / moe_ep_return into the kernels' form.
+int ep_routes(int world, const int64_t *offsets, const int64_t *row0, moe::EpRoutes *r) {
+  if (world < 1 || world > moe::kEpMaxWorld || offsets == nullptr || row0 == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  *r = moe::EpRoutes{};
+  for (int i = 0; i <= world; ++i) {
+    if (offsets[i] < 0 || (i > 0 && offsets[i] < offsets[i - 1])) return MOE_ERR_INVALID_ARG;
+    r->off[i] = offsets[i];
+  }
+  if (offsets[0] != 0) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < world; ++i) {
+    if (row0[i] < 0) return MOE_ERR_INVALID_ARG;
+    r->row0[i] = row0[i];
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+
+int moe_ep_pack(const uint16_t *hidden, int H, const int32_t *topk_ids, int64_t T, int k, int E,
+                int world, const int32_t *send_rows, const int64_t *send_offsets,
+                uint16_t *const *dst_x, int32_t *const *dst_eid, const int64_t *dst_row0,
+                void *stream) {
+  if (T < 0 || H < 1 || k < 1 || E < 1 || world < 1 || dst_x == nullptr || dst_eid == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (H % 128 != 0 || world > moe::kEpMaxWorld || E % world != 0) return MOE_ERR_UNSUPPORTED;
+  moe::EpRoutes r;
+  int rc = ep_routes(world, send_offsets, dst_row0, &r);
+  if (rc != MOE_OK) return rc;
+  if (r.off[world] > T * k) return MOE_ERR_INVALID_ARG;
+  if (r.off[world] == 0) return MOE_OK;
+  if (hidden == nullptr || topk_ids == nullptr || send_rows == nullptr || !aligned16(hidden))
+    return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < world; ++i) {
+    if (r.off[i + 1] == r.off[i]) continue;
+    if (dst_x[i] == nullptr || dst_eid[i] == nullptr || !aligned16(dst_x[i]))
+      return MOE_ERR_INVALID_ARG;
+    r.x[i] = dst_x[i];
+    r.eid[i] = dst_eid[i];
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState *d = nullptr;
+  if ((rc = current_device(&d)) != MOE_OK) return rc;
+  CallCtx ctx{static_cast<cudaStream_t>(stream), "", nullptr};
+  moe::StageHook hook = make_hook(&ctx);
+  return to_code(moe::launch_ep_pack(hidden, H, topk_ids, k, E, world, send_rows, r, d->num_sms,
+                                     ctx.stream, hook));
+}
+
+int moe_ep_return(const float *y, int H, int world, const int64_t *recv_offsets,
+                  float *const *dst_y, const int64_t *dst_row0, void *stream) {
+  if (H < 1 || world < 1 || dst_y == nullptr) return MOE_ERR_INVALID_ARG;
+  if (H % 128 != 0 || world > moe::kEpMaxWorld) return MOE_ERR_UNSUPPORTED;
+  moe::EpRoutes r;
+  int rc = ep_routes(world, recv_offsets, dst_row0, &r);
+  if (rc != MOE_OK) return rc;
+  if (r.off[world] == 0) return MOE_OK;
+  if (y == nullptr || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < world; ++i) {
+    if (r.off[i + 1] == r.off[i]) continue;
+    if (dst_y[i] == nullptr || !aligned16(dst_y[i])) return MOE_ERR_INVALID_ARG;
+    r.y[i] = dst_y[i];
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState *d = nullptr;
+  if ((rc = current_device(&d)) != MOE_OK) return rc;
+  CallCtx ctx{static_cast<cudaStream_t>(stream), "", nullptr};
+  moe::StageHook hook = make_hook(&ctx);
+  return to_code(moe::launch_ep_return(y, H, world, r, d->num_sms, ctx.stream, hook));
+}
+
+int moe_ep_combine(const float *y_back, const int32_t *inv, const float *topk_weights, float *out,
+                   int64_t T, int H, int k, void *stream) {
+  if (T < 0 || H < 1 || k < 1) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (y_back == nullptr || inv == nullptr || topk_weights == nullptr || out == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_back) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  if (H % 128 != 0 || k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState *d = nullptr;
+  int rc = current_device(&d);
+  if (rc != MOE_OK) return rc;
+  CallCtx ctx{static_cast<cudaStream_t>(stream), "", nullptr};
+  moe::StageHook hook = make_hook(&ctx);
+  return to_code(moe::launch_combine(y_back, inv, topk_weights, out, T, H, k, d->status,
+                                     ctx.stream, hook));
+}
+
 int moe_get_device_status(void *stream, uint32_t *status) {
   if (status == nullptr) return MOE_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(g_mu);

@@ -133,6 +133,27 @@ cudaError_t launch_dequant_e4m3(const uint8_t *q, const float *scale, int64_t ro
                                 int block, uint16_t *out, int num_sms, cudaStream_t s,
                                 const StageHook &hook);
 
+// ep.cu: expert parallelism over `world` ranks (experts in contiguous blocks
+// of E / world).  EpRoutes holds, for every peer rank, the segment offsets
+// of this rank's order (off, host values copied into the kernel's
+// parameters), the first row in the peer's buffer and the peer's buffers
+// (device pointers, possibly another GPU's memory mapped here).
+constexpr int kEpMaxWorld = 64;
+struct EpRoutes {
+  int64_t off[kEpMaxWorld + 1];
+  int64_t row0[kEpMaxWorld];
+  void *x[kEpMaxWorld];       // pack: bf16 hidden rows [rows, H]
+  int32_t *eid[kEpMaxWorld];  // pack: expert index within the peer's block
+  void *y[kEpMaxWorld];       // return: fp32 expert outputs [rows, H]
+};
+cudaError_t launch_ep_owner(const int32_t *ids, int64_t n, int E, int world, int32_t *owner,
+                            cudaStream_t s, const StageHook &hook);
+cudaError_t launch_ep_pack(const uint16_t *hidden, int H, const int32_t *ids, int k, int E,
+                           int world, const int32_t *send_rows, const EpRoutes &routes,
+                           int num_sms, cudaStream_t s, const StageHook &hook);
+cudaError_t launch_ep_return(const float *y, int H, int world, const EpRoutes &routes,
+                             int num_sms, cudaStream_t s, const StageHook &hook);
+
 // small_t.cu
 bool small_t_supported(int H, int I);
 // *fits: whether launch_small_t can run this shape in the shared memory of

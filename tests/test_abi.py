@@ -163,6 +163,38 @@ def test_timeline_argument_checks():
     assert L.moe_timeline(None, 0) == moe.MOE_OK                # off
 
 
+def test_ep_argument_checks():
+    i64 = ctypes.c_int64
+    offs = (i64 * 3)(0, 2, 5)
+    row0 = (i64 * 2)(0, 0)
+    ptrs = (ctypes.c_void_p * 2)(256, 256)
+    # dispatch plan
+    assert L.moe_ep_dispatch_plan(256, 4, 2, 8, 0, 256, 256, 256, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_ep_dispatch_plan(256, 4, 2, 8, 3, 256, 256, 256, None) == moe.MOE_ERR_UNSUPPORTED
+    assert L.moe_ep_dispatch_plan(256, 4, 2, 8, 65, 256, 256, 256, None) == moe.MOE_ERR_UNSUPPORTED
+    assert L.moe_ep_dispatch_plan(NULL, 4, 2, 8, 2, 256, 256, 256, None) == moe.MOE_ERR_INVALID_ARG
+    # pack: offsets must be a prefix sum from 0 within T*k
+    assert L.moe_ep_pack(256, 256, 256, 4, 2, 8, 2, 256, offs, ptrs, ptrs, row0,
+                         None) in (moe.MOE_ERR_NO_DEVICE, moe.MOE_OK)
+    bad = (i64 * 3)(1, 2, 5)
+    assert L.moe_ep_pack(256, 256, 256, 4, 2, 8, 2, 256, bad, ptrs, ptrs, row0,
+                         None) == moe.MOE_ERR_INVALID_ARG
+    down = (i64 * 3)(0, 4, 3)
+    assert L.moe_ep_pack(256, 256, 256, 4, 2, 8, 2, 256, down, ptrs, ptrs, row0,
+                         None) == moe.MOE_ERR_INVALID_ARG
+    big = (i64 * 3)(0, 4, 9)  # more rows than T*k
+    assert L.moe_ep_pack(256, 256, 256, 4, 2, 8, 2, 256, big, ptrs, ptrs, row0,
+                         None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_ep_pack(256, 200, 256, 4, 2, 8, 2, 256, offs, ptrs, ptrs, row0,
+                         None) == moe.MOE_ERR_UNSUPPORTED
+    # return and combine
+    assert L.moe_ep_return(256, 256, 2, bad, ptrs, row0, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_ep_return(264, 256, 2, offs, ptrs, row0, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_ep_combine(256, 256, 256, 256, 4, 200, 2, None) == moe.MOE_ERR_UNSUPPORTED
+    assert L.moe_ep_combine(NULL, 256, 256, 256, 4, 256, 2, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_ep_combine(NULL, NULL, NULL, NULL, 0, 256, 2, None) == moe.MOE_OK
+
+
 def test_debug_switches_roundtrip():
     prev = moe.set_small_t_max(5)
     assert moe.set_small_t_max(prev) == 5
