@@ -171,7 +171,7 @@ int moe_forward_ex(const uint16_t *hidden, const uint16_t *w1, const uint16_t *w
  * scales or block < 1.
  * Numerics: the small-T path (T <= the small-T limit) streams the codes and
  * multiplies each 16-weight partial dot product (fp32) by its scale; the
- * grouped-GEMM path first expands all E experts' weights to bf16
+ * grouped-GEMM path first expands the chosen experts' weights to bf16
  * (bf16_rn(code * scale), one rounding) into a second library-owned
  * grow-only buffer of E * 3 * H * I * 2 bytes, then runs as moe_forward.
  */

@@ -23,9 +23,12 @@ __device__ __forceinline__ uint32_t e4m3x2_scaled_bf16x2(uint32_t two, float sc)
   return pack_bf16x2(f.x * sc, f.y * sc);
 }
 
+// With expert_offsets (the grouping's [E+1] row offsets), the rows of an
+// expert that no token chose (rows_per_expert rows each) are skipped.
 __global__ void __launch_bounds__(256)
     dequant_e4m3_kernel(const uint4 *__restrict__ q, const float *__restrict__ scale,
-                        int64_t rows, int K, int block, uint4 *__restrict__ out) {
+                        int64_t rows, int K, int block, uint4 *__restrict__ out,
+                        const int32_t *__restrict__ expert_offsets, int64_t rows_per_expert) {
   grid_dep_wait();
   grid_dep_launch();
   const int kc = K / 16;  // 16-code chunks per row
@@ -34,6 +37,10 @@ __global__ void __launch_bounds__(256)
   for (int64_t x = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; x < n;
        x += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t r = x / kc;
+    if (expert_offsets != nullptr) {
+      const int64_t e = r / rows_per_expert;
+      if (__ldg(expert_offsets + e + 1) == __ldg(expert_offsets + e)) continue;
+    }
     const int c = static_cast<int>(x - r * kc);
     const float sc = __ldg(scale + r * nb + (c * 16) / block);
     const uint4 v = __ldcs(q + x);
@@ -55,7 +62,10 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_dequant_e4m3(const uint8_t *q, const float *scale, int64_t rows, int K,
                                 int block, uint16_t *out, int num_sms, cudaStream_t s,
-                                const StageHook &hook) {
+                                const StageHook &hook, const int32_t *expert_offsets,
+                                int64_t rows_per_expert) {
+  if (expert_offsets != nullptr && (rows_per_expert < 1 || rows % rows_per_expert != 0))
+    return cudaErrorInvalidValue;
   if (K % 16 != 0 || block % 16 != 0 || K % block != 0 || rows < 1) return cudaErrorInvalidValue;
   const int64_t n = rows * (K / 16);
   const int64_t want = (n + 255) / 256;
@@ -64,7 +74,7 @@ cudaError_t launch_dequant_e4m3(const uint8_t *q, const float *scale, int64_t ro
   hook.begin("dequant_fp8");
   cudaError_t e = launch_pdl(dequant_e4m3_kernel, dim3(blocks), dim3(256), 0, s, hook.pdl,
                              reinterpret_cast<const uint4 *>(q), scale, rows, K, block,
-                             reinterpret_cast<uint4 *>(out));
+                             reinterpret_cast<uint4 *>(out), expert_offsets, rows_per_expert);
   return hook.end(e);
 }
 

@@ -20,6 +20,9 @@ constexpr int kMaxTopK = 16;
 // above this many waves of GEMM tiles (per resident CTA pair) the two GEMMs
 // run as separate launches
 constexpr int64_t kFusedMaxWaves = 12;
+// bytes of w1 the grouping kernel asks L2 to prefetch for the GEMM's first
+// tiles (about the first wave's gate and up rows on the 8-expert prefill)
+constexpr int64_t kFirstWaveBytes = static_cast<int64_t>(40) << 20;
 
 std::mutex g_mu;  // guards the per-device state and the profiler
 
@@ -356,22 +359,6 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
   }
 
   cudaError_t e;
-  if (fp8 != nullptr) {
-    // the grouped GEMMs run on bf16 copies of all E experts' weights
-    const size_t n1 = static_cast<size_t>(E) * 2 * I * H, n2 = static_cast<size_t>(E) * H * I;
-    if ((rc = ensure_buffer(d->wq, d->wq_bytes, (n1 + n2) * 2)) != MOE_OK) return rc;
-    uint16_t *wd1 = static_cast<uint16_t *>(d->wq), *wd2 = wd1 + n1;
-    if ((e = moe::launch_dequant_e4m3(reinterpret_cast<const uint8_t *>(w1), fp8->s1,
-                                      static_cast<int64_t>(E) * 2 * I, H, fp8->block, wd1,
-                                      d->num_sms, ctx.stream, hook)) != cudaSuccess ||
-        (e = moe::launch_dequant_e4m3(reinterpret_cast<const uint8_t *>(w2), fp8->s2,
-                                      static_cast<int64_t>(E) * H, I, fp8->block, wd2,
-                                      d->num_sms, ctx.stream, hook)) != cudaSuccess)
-      return to_code(e);
-    w1 = wd1;
-    w2 = wd2;
-  }
-
   // top-k <= 2: GEMM2 adds its rows straight into out and no P is needed
   const bool fuse_combine = k <= 2;
   // Copying the hidden rows into expert-sorted order costs k row copies per
@@ -400,9 +387,13 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
   // three-kernel grouping and a separate copy above; either zeroes the
   // GEMMs' counters
   if (moe::group_supported(n)) {
+    // with the row copy, also bring the first GEMM tiles' w1 rows into L2
+    // (bf16 weights: the copies of FP8 weights are written after this)
+    const int64_t w1_expert = static_cast<int64_t>(2) * I * H * 2;
     e = moe::launch_group(topk_ids, n, E, k, expert_offsets, sorted_rows, inv, d->status, hidden,
                           H, xs, counters, static_cast<int>(n_counters), d->num_sms, ctx.stream,
-                          hook);
+                          hook, fp8 == nullptr ? w1 : nullptr, w1_expert, w1_expert * E,
+                          kFirstWaveBytes);
     if (e != cudaSuccess) return to_code(e);
   } else {
     e = moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets, sorted_rows, inv,
@@ -412,6 +403,24 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
         (e = moe::launch_gather_rows(hidden, H, k, sorted_rows, expert_offsets, E, n, d->num_sms,
                                      xs, nullptr, 0, ctx.stream, hook)) != cudaSuccess)
       return to_code(e);
+  }
+  if (fp8 != nullptr) {
+    // the grouped GEMMs run on bf16 copies of the chosen experts' weights
+    // (the others are left as they are: no row of theirs is read)
+    const size_t n1 = static_cast<size_t>(E) * 2 * I * H, n2 = static_cast<size_t>(E) * H * I;
+    if ((rc = ensure_buffer(d->wq, d->wq_bytes, (n1 + n2) * 2)) != MOE_OK) return rc;
+    uint16_t *wd1 = static_cast<uint16_t *>(d->wq), *wd2 = wd1 + n1;
+    if ((e = moe::launch_dequant_e4m3(reinterpret_cast<const uint8_t *>(w1), fp8->s1,
+                                      static_cast<int64_t>(E) * 2 * I, H, fp8->block, wd1,
+                                      d->num_sms, ctx.stream, hook, expert_offsets,
+                                      2 * I)) != cudaSuccess ||
+        (e = moe::launch_dequant_e4m3(reinterpret_cast<const uint8_t *>(w2), fp8->s2,
+                                      static_cast<int64_t>(E) * H, I, fp8->block, wd2,
+                                      d->num_sms, ctx.stream, hook, expert_offsets, H)) !=
+            cudaSuccess)
+      return to_code(e);
+    w1 = wd1;
+    w2 = wd2;
   }
   moe::GroupedGemmArgs ga = {};
   ga.hidden = hidden;
