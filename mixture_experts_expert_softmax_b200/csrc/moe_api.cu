@@ -20,9 +20,6 @@ constexpr int kMaxTopK = 16;
 // above this many waves of GEMM tiles (per resident CTA pair) the two GEMMs
 // run as separate launches
 constexpr int64_t kFusedMaxWaves = 12;
-// bytes of w1 the grouping kernel asks L2 to prefetch for the GEMM's first
-// tiles (about the first wave's gate and up rows on the 8-expert prefill)
-constexpr int64_t kFirstWaveBytes = static_cast<int64_t>(40) << 20;
 
 std::mutex g_mu;  // guards the per-device state and the profiler
 
@@ -387,13 +384,9 @@ int forward_impl(const void *hidden_, const void *w1_, const void *w2_, const fl
   // three-kernel grouping and a separate copy above; either zeroes the
   // GEMMs' counters
   if (moe::group_supported(n)) {
-    // with the row copy, also bring the first GEMM tiles' w1 rows into L2
-    // (bf16 weights: the copies of FP8 weights are written after this)
-    const int64_t w1_expert = static_cast<int64_t>(2) * I * H * 2;
     e = moe::launch_group(topk_ids, n, E, k, expert_offsets, sorted_rows, inv, d->status, hidden,
                           H, xs, counters, static_cast<int>(n_counters), d->num_sms, ctx.stream,
-                          hook, fp8 == nullptr ? w1 : nullptr, w1_expert, w1_expert * E,
-                          kFirstWaveBytes);
+                          hook);
     if (e != cudaSuccess) return to_code(e);
   } else {
     e = moe::launch_permute(topk_ids, n, E, chunk_counts, expert_offsets, sorted_rows, inv,

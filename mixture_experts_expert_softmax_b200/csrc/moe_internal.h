@@ -54,18 +54,14 @@ cudaError_t launch_permute(const int32_t *ids, int64_t n, int E, int32_t *chunk_
 
 // Stable grouping of n <= 8192 entries in one kernel (the same result as
 // launch_permute), with the expert-sorted copy of the hidden rows when xs
-// is given; then also, with `prefetch` (an [E, ...] weight array of
-// prefetch_expert_bytes per expert and prefetch_total bytes), an L2
-// prefetch of prefetch_bytes from the first chosen expert's weights on.
-// group_setup raises the kernel's shared-memory limit once per device.
+// is given.  group_setup raises the kernel's shared-memory limit once per
+// device.
 bool group_supported(int64_t n);
 cudaError_t group_setup();
 cudaError_t launch_group(const int32_t *ids, int64_t n, int E, int k, int32_t *expert_offsets,
                          int32_t *sorted_rows, int32_t *inv, uint32_t *status,
                          const uint16_t *hidden, int H, uint16_t *xs, int *zero, int zero_n,
-                         int num_sms, cudaStream_t s, const StageHook &hook,
-                         const void *prefetch = nullptr, int64_t prefetch_expert_bytes = 0,
-                         int64_t prefetch_total = 0, int64_t prefetch_bytes = 0);
+                         int num_sms, cudaStream_t s, const StageHook &hook);
 
 // Expert-sorted copy of the hidden rows, xs[r] = hidden[sorted_rows[r] / k]
 // for r < expert_offsets[E] (device value); n = T*k bounds the grid.

@@ -173,9 +173,7 @@ __global__ void __launch_bounds__(kGroupThreads)
     group_kernel(const int32_t *__restrict__ ids, int n, int E, int k,
                  int32_t *__restrict__ expert_offsets, int32_t *__restrict__ sorted_rows,
                  int32_t *__restrict__ inv, uint32_t *status, const uint4 *__restrict__ hidden,
-                 int H8, uint4 *__restrict__ xs, int *zero, int zero_n,
-                 const uint8_t *pf_base, int64_t pf_expert_bytes, int64_t pf_total,
-                 int64_t pf_bytes) {
+                 int H8, uint4 *__restrict__ xs, int *zero, int zero_n) {
   extern __shared__ __align__(16) unsigned char group_smem[];
   int32_t *s_sorted = reinterpret_cast<int32_t *>(group_smem);      // [n]
   int32_t *s_tot = s_sorted + ((n + 3) & ~3);                         // [E]
@@ -290,19 +288,6 @@ __global__ void __launch_bounds__(kGroupThreads)
     for (int x = tid; x < zero_n; x += kGroupThreads) zero[x] = 0;
   if (xs == nullptr) return;
   __syncthreads();
-  if (pf_base != nullptr) {
-    // the weights the first GEMM tiles will read (expert-major, from the
-    // first chosen expert on), brought into L2 while the rows are copied
-    int e0 = 0;
-    while (e0 + 1 < E && s_tot[e0 + 1] == 0) ++e0;  // s_tot holds the expert offsets
-    const int64_t start = static_cast<int64_t>(e0) * pf_expert_bytes;
-    const int64_t len = min(pf_bytes, pf_total - start);
-    constexpr int64_t kPfChunk = 32768;
-    for (int64_t c = static_cast<int64_t>(blockIdx.x) * kGroupThreads + tid; c * kPfChunk < len;
-         c += static_cast<int64_t>(gridDim.x) * kGroupThreads)
-      bulk_prefetch_l2(pf_base + start + c * kPfChunk,
-                       static_cast<uint32_t>(min(kPfChunk, len - c * kPfChunk)));
-  }
   const int nv = s_nvalid;
   for (int r = blockIdx.x * kGroupWarps + warp; r < nv; r += gridDim.x * kGroupWarps) {
     const int64_t tok = s_sorted[r] / k;
@@ -369,9 +354,7 @@ cudaError_t group_setup() {
 cudaError_t launch_group(const int32_t *ids, int64_t n, int E, int k, int32_t *expert_offsets,
                          int32_t *sorted_rows, int32_t *inv, uint32_t *status,
                          const uint16_t *hidden, int H, uint16_t *xs, int *zero, int zero_n,
-                         int num_sms, cudaStream_t s, const StageHook &hook,
-                         const void *prefetch, int64_t prefetch_expert_bytes,
-                         int64_t prefetch_total, int64_t prefetch_bytes) {
+                         int num_sms, cudaStream_t s, const StageHook &hook) {
   int grid = 1;
   if (xs != nullptr) {
     const int64_t want = (n + kGroupWarps - 1) / kGroupWarps;  // one row per warp
@@ -384,9 +367,7 @@ cudaError_t launch_group(const int32_t *ids, int64_t n, int E, int k, int32_t *e
                                group_smem_bytes(static_cast<int>(n), E), s, hook.pdl, ids,
                                static_cast<int>(n), E, k, expert_offsets, sorted_rows, inv, status,
                                reinterpret_cast<const uint4 *>(hidden), H / 8,
-                               reinterpret_cast<uint4 *>(xs), zero, zero_n,
-                               static_cast<const uint8_t *>(prefetch), prefetch_expert_bytes,
-                               prefetch_total, prefetch_bytes);
+                               reinterpret_cast<uint4 *>(xs), zero, zero_n);
   return hook.end(err);
 }
 
