@@ -312,6 +312,18 @@ def run_ours(args, ws, rank, local):
     h2d = h_hidden.numel() * 2 + h_logits.numel() * 4
     d2h = h_out.numel() * 4
 
+    if args.timeline and rank == 0:
+        # one more forward of the workload (cold L2) with the kernels'
+        # per-tile / per-phase records on, written with their summary
+        flush()
+        torch.cuda.synchronize(dev)
+        moe.timeline_start(1 << 16, device=dev)
+        forward(hidden, wts, ids, out)
+        recs = moe.timeline_stop()
+        with open(args.timeline, "w") as f:
+            json.dump({"workload": args.workload, "summary": moe.timeline_summary(recs),
+                       "records": recs}, f)
+
     per_shape = {}
     fb = args.fp8_block if fp8 else 0
     if args.shapes == "workloads":
@@ -520,6 +532,9 @@ def main():
     ap.add_argument("--fp8-block", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--timeline", metavar="PATH",
+                    help="after the timed steps, write the kernels' per-tile / per-phase "
+                         "records of one more forward (moe_timeline) to PATH as JSON")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -333,9 +333,11 @@ def timeline_stop() -> list[dict]:
 
 def timeline_summary(records: list[dict]) -> dict:
     """Per (kind, role): record count, mean and max duration (us), and the
-    span from the earliest t0 to the latest t1 (us); per kind also the
-    share of that span the busiest and the idlest CTA spent in its MMA or
-    phase records."""
+    span from the earliest t0 to the latest t1 (us).  Per GEMM kind also:
+    the MMA records binned by their start (10 us bins from the first MMA:
+    tiles started and their mean duration), each CTA's summed MMA time
+    (min / median / max), and the median gap between consecutive tiles of
+    one CTA's MMA thread."""
     import collections
     out: dict = {}
     by = collections.defaultdict(list)
@@ -346,6 +348,24 @@ def timeline_summary(records: list[dict]) -> dict:
         out[f"{kind}/{role}"] = {
             "n": len(rs), "mean_us": round(sum(d) / len(d), 3), "max_us": round(max(d), 3),
             "span_us": round((max(r["t1"] for r in rs) - min(r["t0"] for r in rs)) / 1e3, 3)}
+        if role != "mma":
+            continue
+        t0 = min(r["t0"] for r in rs)
+        bins = collections.defaultdict(list)
+        per_cta = collections.defaultdict(list)
+        for r in rs:
+            bins[int((r["t0"] - t0) / 1e4) * 10].append((r["t1"] - r["t0"]) / 1e3)
+            per_cta[r["cta"]].append(r)
+        busy = sorted(sum(r["t1"] - r["t0"] for r in v) / 1e3 for v in per_cta.values())
+        gaps = sorted((b["t0"] - a["t1"]) / 1e3 for v in per_cta.values()
+                      for a, b in zip(sorted(v, key=lambda r: r["t0"]),
+                                      sorted(v, key=lambda r: r["t0"])[1:]))
+        out[f"{kind}/mma"].update({
+            "by_start_10us": {k: [len(v), round(sum(v) / len(v), 2)]
+                              for k, v in sorted(bins.items())},
+            "cta_mma_us_min_med_max": [round(busy[0], 1), round(busy[len(busy) // 2], 1),
+                                       round(busy[-1], 1)],
+            "tile_gap_us_median": round(gaps[len(gaps) // 2], 3) if gaps else None})
     return out
 
 
