@@ -424,6 +424,10 @@ int moe_timeline(void *buf, int64_t capacity);
  * caller's stream.  moe_profile_read SYNCHRONISES the device, then for each
  * kernel name (up to max_names) writes its launch count, total milliseconds
  * and name, and returns how many names exist.  moe_profile_reset clears.
+ * Independently of this switch, every kernel launch of every entry point
+ * sits inside an NVTX range named after its stage ("route", "group_gather",
+ * "gemm_fused", "small_t", ...), pushed and popped on the calling thread;
+ * with no NVTX tool attached to the process those calls do nothing.
  */
 int moe_profile_enable(int on);
 int moe_profile_reset(void);

@@ -9,6 +9,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "moe.h"
 #include "moe_internal.h"
 
@@ -91,8 +93,12 @@ struct CallCtx {
   cudaEvent_t ev0;
 };
 
+// Every stage is also an NVTX range named after it (pushed before its
+// launch, popped after), so that a timeline tool attached to the process
+// groups each kernel under its stage; without a tool the calls do nothing.
 void hook_begin(void *c, const char *name) {
   CallCtx *ctx = static_cast<CallCtx *>(c);
+  nvtxRangePushA(name);
   ctx->cur = name;
   ctx->ev0 = nullptr;
   if (g_prof) {
@@ -113,6 +119,7 @@ cudaError_t hook_end(void *c, cudaError_t err) {
     if (err == cudaSuccess) err = cudaGetLastError();
   }
   if (err != cudaSuccess) g_failed_stage = ctx->cur;
+  nvtxRangePop();
   return err;
 }
 
