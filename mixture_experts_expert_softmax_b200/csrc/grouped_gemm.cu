@@ -106,6 +106,10 @@ constexpr uint16_t kBothCtas = 0x3;
 constexpr int kRedPitch = 144;
 constexpr int kEpiWarpBytes = 5 * 1024;
 static_assert(32 * kRedPitch <= kEpiWarpBytes, "staging");
+// The CTA's last tile of the combine-fused GEMM2 stages whole 128-column
+// half rows (512 bytes, at a 528-byte pitch: 8 consecutive lanes again hit
+// 8 different bank groups) in the idle operand ring, one reduction per row.
+constexpr int kBigPitch = 528;
 constexpr size_t kSmemMax = 232448;  // opt-in maximum per block on sm_100
 // act rows of an m-tile are complete when every epilogue warp of both CTAs
 // has published each of its n-tiles
@@ -666,8 +670,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint8_t *srow = ebuf + lane * kRedPitch;
         const float *b2row = p.b2 ? p.b2 + static_cast<size_t>(tl.e) * p.H : nullptr;
+        // The CTA's last tile: no MMA follows to hide this epilogue behind,
+        // and the TMA engine's cost per operation bounds it.  Every MMA has
+        // completed (acc_full) and every operand load has landed (each was
+        // consumed by one of those MMAs), so the operand ring is idle: each
+        // lane stages its row's 128 columns there and adds them with one
+        // 512-byte reduction instead of four 128-byte ones.
+        const int colh = tl.nt * kAccN + half * (kAccN / 2);
+        const bool wide = t + nunits >= total && colh + kAccN / 2 <= p.H &&
+                          kStages * (kABytes + kBBytes) >= kEpiWarps * 32 * kBigPitch;
+        if (wide) {
+          uint8_t *brow = sA + (ew * 32 + lane) * kBigPitch;
 #pragma unroll 1
-        for (int c0 = half * (kAccN / 2); c0 < (half + 1) * (kAccN / 2); c0 += 32) {
+          for (int c0 = 0; c0 < kAccN / 2; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld_32cols(tbase + half * (kAccN / 2) + c0, v);
+            tmem_ld_wait();
+            if (b2row) add_bias32(v, b2row + colh + c0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<float4 *>(brow + 4 * c0 + 16 * j) =
+                  make_float4(wgt * as_f32(v[4 * j]), wgt * as_f32(v[4 * j + 1]),
+                              wgt * as_f32(v[4 * j + 2]), wgt * as_f32(v[4 * j + 3]));
+          }
+          if (valid && !*abort_flag) {
+            fence_proxy_async_smem();
+            bulk_reduce_add_f32(orow + colh, brow, 4 * (kAccN / 2));
+            bulk_commit_group();
+          }
+          __syncwarp();
+        }
+#pragma unroll 1
+        for (int c0 = half * (kAccN / 2); !wide && c0 < (half + 1) * (kAccN / 2); c0 += 32) {
           uint32_t v[32];
           tmem_ld_32cols(tbase + c0, v);
           tmem_ld_wait();
