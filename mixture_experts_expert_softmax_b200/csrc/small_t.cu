@@ -438,12 +438,99 @@ __device__ __forceinline__ void phase2_item(const uint4 *ws, const uint4 *__rest
   }
 }
 
+// Phase 2 item with both operands on chip (w2 rows in a ring slot, act
+// staged in shared memory): the same kR2 dot products as phase2_item, in
+// the same order per lane (so the same sums), but every load of a block of
+// chunks is issued before the first FMA, so a warp waits for shared memory
+// once per block rather than once per load (with the loads behind the
+// operand-location branches, each one was its own round trip: ~1.4 us per
+// item).  Rows past nrows read the last row and are not stored.  FP8: sc0
+// holds the scales of the CTA's local row 0 (ipb per row; on chip when the
+// copy warp staged them, else in global memory).
+constexpr int kU2c = 3;  // bf16: chunks per lane per block (I = 768: one block)
+constexpr int kU2f = 1;  // FP8: chunks of 16 codes per lane per block
+template <bool kFp8>
+__device__ __forceinline__ void phase2_item_onchip(const uint4 *ws, const float4 *sa,
+                                                   const float *sc0, int pair, int r0,
+                                                   int nrows, int I, int TK, float *sdots,
+                                                   int ipb, int cpb) {
+  const int lane = threadIdx.x & 31;
+  int rows[kR2];
+#pragma unroll
+  for (int rr = 0; rr < kR2; ++rr) rows[rr] = min(r0 + rr, nrows - 1);
+  if constexpr (kFp8) {
+    const int IC = I / 16;
+    float v[kR2];
+#pragma unroll
+    for (int rr = 0; rr < kR2; ++rr) v[rr] = 0.f;
+    for (int base = 0; base < IC; base += 32 * kU2f) {
+      float4 a[kU2f][4];
+      uint4 wv[kU2f][kR2];
+      float sc[kU2f][kR2];
+#pragma unroll
+      for (int j = 0; j < kU2f; ++j) {
+        const int c = min(base + lane + 32 * j, IC - 1);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a[j][q] = sa[4 * c + q];
+#pragma unroll
+        for (int rr = 0; rr < kR2; ++rr) {
+          wv[j][rr] = ws[rows[rr] * IC + c];
+          sc[j][rr] = sc0[rows[rr] * ipb + c / cpb];  // generic: shared or global
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kU2f; ++j) {
+        if (base + lane + 32 * j < IC) {
+#pragma unroll
+          for (int rr = 0; rr < kR2; ++rr)
+            v[rr] = fmaf(dot16_e4m3_f32(wv[j][rr], a[j][0], a[j][1], a[j][2], a[j][3]),
+                         sc[j][rr], v[rr]);
+        }
+      }
+    }
+#pragma unroll
+    for (int rr = 0; rr < kR2; ++rr) {
+      const float sv = warp_sum(v[rr]);
+      if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
+    }
+  } else {
+    const int I8 = I / 8;
+    unsigned long long v[kR2];  // two fp32 partial sums each
+#pragma unroll
+    for (int rr = 0; rr < kR2; ++rr) v[rr] = 0ull;
+    for (int base = 0; base < I8; base += 32 * kU2c) {
+      float4 lo[kU2c], hi[kU2c];
+      uint4 wv[kU2c][kR2];
+#pragma unroll
+      for (int j = 0; j < kU2c; ++j) {
+        const int c = min(base + lane + 32 * j, I8 - 1);
+        lo[j] = sa[2 * c];
+        hi[j] = sa[2 * c + 1];
+#pragma unroll
+        for (int rr = 0; rr < kR2; ++rr) wv[j][rr] = ws[rows[rr] * I8 + c];
+      }
+#pragma unroll
+      for (int j = 0; j < kU2c; ++j) {
+        if (base + lane + 32 * j < I8) {
+#pragma unroll
+          for (int rr = 0; rr < kR2; ++rr) fma8_f32x2(wv[j][rr], lo[j], hi[j], v[rr]);
+        }
+      }
+    }
+#pragma unroll
+    for (int rr = 0; rr < kR2; ++rr) {
+      const float sv = warp_sum(sum_f32x2(v[rr]));
+      if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
+    }
+  }
+}
+
 // Dynamic shared memory of a CTA: the token vectors in bf16 [T][H]; a ring of `slots` buffers, each holding this
 // CTA's w2 rows of one chosen expert in bf16 [rows_per_cta][I] (no ring when
 // one expert's rows do not fit: phase 2 then reads w2 through L2); act in
 // fp32 [T*k][I] when it fits; the dot products [rows_per_cta][T*k].
 struct SmemLayout {
-  size_t w2_off, act_off, dots_off, total;
+  size_t w2_off, act_off, dots_off, scl_off, total;
 };
 
 // elem: bytes per weight (2: bf16, 1: FP8)
@@ -451,14 +538,17 @@ __host__ __device__ inline size_t w2_slot_bytes(int rows_per_cta, int I, int ele
   return (static_cast<size_t>(rows_per_cta) * I * elem + 127) & ~static_cast<size_t>(127);
 }
 
+// scl: fp32 w2 scales per row staged on chip (FP8: I / block, else 0), for
+// the first `slots` chosen experts
 __host__ __device__ inline SmemLayout smem_layout(int T, int TK, int H, int I,
                                                   int rows_per_cta, int slots, int cache_act,
-                                                  int elem) {
+                                                  int elem, int scl = 0) {
   SmemLayout s;
   s.w2_off = static_cast<size_t>(T) * H * 2;
   s.act_off = s.w2_off + static_cast<size_t>(slots) * w2_slot_bytes(rows_per_cta, I, elem);
   s.dots_off = s.act_off + (cache_act ? static_cast<size_t>(TK) * I * sizeof(float) : 0);
-  s.total = s.dots_off + static_cast<size_t>(rows_per_cta) * TK * sizeof(float);
+  s.scl_off = s.dots_off + static_cast<size_t>(rows_per_cta) * TK * sizeof(float);
+  s.total = s.scl_off + static_cast<size_t>(slots) * rows_per_cta * scl * sizeof(float);
   return s;
 }
 
@@ -475,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
                    const float *__restrict__ b2, int act_kind, const float *__restrict__ topk_w,
                    const int32_t *__restrict__ ids, float *__restrict__ act,
                    float *__restrict__ out, int T, int k, int H, int I, int E, int rows_per_cta,
-                   int slots, int cache_act, uint32_t *status,
+                   int slots, int cache_act, int stage_scl, uint32_t *status,
                    unsigned long long *grid_sync, uint64_t limit, uint64_t *tl_buf,
                    int64_t tl_cap) {
   // phase 1: chunks per lane and row in flight (an FP8 chunk holds 16 codes)
@@ -485,6 +575,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   __shared__ volatile int s_abort;
   __shared__ uint64_t w2_full[kMaxSlots];   // a slot's rows have landed
   __shared__ uint64_t w2_empty[kMaxSlots];  // every compute warp is done with a slot
+  __shared__ float s_topw[kMaxPairs];       // the top-k weights, for the final sum
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int TK = T * k;
   const int H8 = H / 8;
@@ -492,12 +583,14 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   const int HC = H * kElem / 16, IC = I * kElem / 16;  // 16-byte weight chunks per row
   const int cpb = kFp8 ? block / 16 : 1;                // chunks per scale block
   const int hpb = kFp8 ? H / block : 0, ipb = kFp8 ? I / block : 0;  // blocks per row
-  const SmemLayout lay = smem_layout(T, TK, H, I, rows_per_cta, slots, cache_act, kElem);
+  const SmemLayout lay =
+      smem_layout(T, TK, H, I, rows_per_cta, slots, cache_act, kElem, stage_scl ? ipb : 0);
   const size_t slot_stride = w2_slot_bytes(rows_per_cta, I, kElem);
   uint8_t *sx = smem;  // the token's vector (one-token kernel)
   uint8_t *sw2 = smem + lay.w2_off;
   float *sact = reinterpret_cast<float *>(smem + lay.act_off);
   float *sdots = reinterpret_cast<float *>(smem + lay.dots_off);
+  float *sscl = reinterpret_cast<float *>(smem + lay.scl_off);  // [slots][rows_per_cta][ipb]
   const int h0 = blockIdx.x * rows_per_cta;
   const int nrows = max(0, min(H, h0 + rows_per_cta) - h0);
 
@@ -513,6 +606,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   }
   for (int c = threadIdx.x; c < T * H8; c += kThreads)
     reinterpret_cast<uint4 *>(sx)[c] = __ldg(hidden + c);
+  // loaded now, while the weights stream, rather than at the end where the
+  // final sum would wait for them
+  for (int i = threadIdx.x; i < TK; i += kThreads) s_topw[i] = __ldg(topk_w + i);
   const uint4 *sx4 = reinterpret_cast<const uint4 *>(sx);
   __syncthreads();
   const int nd = L.n_distinct;
@@ -534,6 +630,19 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
     } else {
       for (int d = 0; d < nd; ++d)
         bulk_prefetch_l2(w2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * IC, w2_bytes);
+    }
+  }
+  if (kFp8 && stage_scl && warp == kCopyWarp && nrows > 0) {
+    // the w2 scales of this CTA's rows, for the experts that get a slot:
+    // read now, while the weights stream, so that no phase-2 item waits on
+    // a global load for them (they are read once, but each costs a round
+    // trip to memory where the phase-2 item needs it)
+    __syncwarp();
+    const int per = nrows * ipb;
+    for (int d = 0; d < nd && d < slots; ++d) {
+      const float *src = s2 + (static_cast<size_t>(L.dexp[d]) * H + h0) * ipb;
+      for (int x = lane; x < per; x += 32)
+        sscl[static_cast<size_t>(d) * rows_per_cta * ipb + x] = __ldg(src + x);
     }
   }
 
@@ -651,6 +760,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
 
   // ------------------------------------------------------------ phase 2
   const float4 *act4 = reinterpret_cast<const float4 *>(act);
+  // every operand on chip (w2 rows in the ring, act staged below):
+  // phase2_item_onchip
+  const bool onchip = ring && cache_act;
   if (cache_act) {
     // act was written by other CTAs in this launch: read it from L2
     const int n4 = TK * I / 4;
@@ -707,9 +819,17 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       const int d = L.pd[pair];
       const size_t row0 = static_cast<size_t>(L.dexp[d]) * H + h0;  // w2 row of local row 0
       const float *s2r = kFp8 ? s2 + (row0 + rg * kR2) * ipb : nullptr;  // FP8 scales
-      phase2_item<kFp8>(ring ? reinterpret_cast<const uint4 *>(sw2 + d * slot_stride) : nullptr,
-                        w2 + row0 * IC, act4, cache_act, pair, rg * kR2, nrows, I, TK, sdots,
-                        s2r, ipb, cpb);
+      if (onchip)
+        phase2_item_onchip<kFp8>(
+            reinterpret_cast<const uint4 *>(sw2 + d * slot_stride),
+            act4 + static_cast<size_t>(pair) * (I / 4),
+            !kFp8 ? nullptr
+                  : stage_scl ? sscl + static_cast<size_t>(d) * rows_per_cta * ipb : s2 + row0 * ipb,
+            pair, rg * kR2, nrows, I, TK, sdots, ipb, cpb);
+      else
+        phase2_item<kFp8>(ring ? reinterpret_cast<const uint4 *>(sw2 + d * slot_stride) : nullptr,
+                          w2 + row0 * IC, act4, cache_act, pair, rg * kR2, nrows, I, TK, sdots,
+                          s2r, ipb, cpb);
     }
   } else if (rgroups > 0) {
     // more experts than slots: take the experts in order, waiting for each
@@ -730,9 +850,18 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       for (; it < n_items; it += kWarps) {
         const int pq = p0 + it / rgroups, rg = it % rgroups;
         const size_t row0 = static_cast<size_t>(L.dexp[d]) * H + h0;
-        phase2_item<kFp8>(reinterpret_cast<const uint4 *>(sw2 + q * slot_stride), nullptr, act4,
-                          cache_act, L.plist[pq], rg * kR2, nrows, I, TK, sdots,
-                          kFp8 ? s2 + (row0 + rg * kR2) * ipb : nullptr, ipb, cpb);
+        if (onchip)
+          phase2_item_onchip<kFp8>(
+              reinterpret_cast<const uint4 *>(sw2 + q * slot_stride),
+              act4 + static_cast<size_t>(L.plist[pq]) * (I / 4),
+              !kFp8                     ? nullptr
+              : stage_scl && d < slots ? sscl + static_cast<size_t>(d) * rows_per_cta * ipb
+                                       : s2 + row0 * ipb,
+              L.plist[pq], rg * kR2, nrows, I, TK, sdots, ipb, cpb);
+        else
+          phase2_item<kFp8>(reinterpret_cast<const uint4 *>(sw2 + q * slot_stride), nullptr,
+                            act4, cache_act, L.plist[pq], rg * kR2, nrows, I, TK, sdots,
+                            kFp8 ? s2 + (row0 + rg * kR2) * ipb : nullptr, ipb, cpb);
       }
       before += n_items;
       __syncwarp();
@@ -753,7 +882,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       if (L.pd[pair] >= 0) {
         float y = sdots[r * TK + pair];
         if (b2 != nullptr) y += __ldg(b2 + static_cast<size_t>(L.ids[pair]) * H + h0 + r);
-        acc = fmaf(__ldg(topk_w + pair), y, acc);
+        acc = fmaf(s_topw[pair], y, acc);
       }
     }
     out[static_cast<size_t>(t) * H + h0 + r] = acc;
@@ -772,7 +901,7 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
 }
 
 struct SmallTConfig {
-  int rows_per_cta, slots, cache_act;
+  int rows_per_cta, slots, cache_act, stage_scl;
   size_t smem;
 };
 
@@ -780,8 +909,11 @@ struct SmallTConfig {
 // slots as there can be distinct experts (at most kMaxSlots), and the act
 // cache when it fits beside them -- unless it would leave fewer than two
 // slots (no overlap of copies and dot products) where dropping it gives more.
+// scl: FP8 w2 scales per row (I / block; 0 for bf16), staged on chip when
+// they fit beside the rest (at most kSclStageMax bytes).
+constexpr size_t kSclStageMax = 16 * 1024;
 SmallTConfig small_t_config(int T, int TK, int H, int I, int E, int grid, size_t budget,
-                            int elem) {
+                            int elem, int scl) {
   SmallTConfig c;
   c.rows_per_cta = (H + grid - 1) / grid;
   const int want = std::min(std::min(TK, E), kMaxSlots);
@@ -801,6 +933,10 @@ SmallTConfig small_t_config(int T, int TK, int H, int I, int E, int grid, size_t
   }
   if (c.cache_act && size(c.slots, 1) > budget) c.cache_act = 0;
   c.smem = size(c.slots, c.cache_act);
+  const size_t with_scl =
+      smem_layout(T, TK, H, I, c.rows_per_cta, c.slots, c.cache_act, elem, scl).total;
+  c.stage_scl = scl > 0 && c.slots > 0 && with_scl - c.smem <= kSclStageMax && with_scl <= budget;
+  if (c.stage_scl) c.smem = with_scl;
   return c;
 }
 
@@ -873,8 +1009,9 @@ cudaError_t small_t_fits(int64_t T, int H, int I, int E, int k, bool fp8, bool *
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if ((e = small_t_setup(dev)) != cudaSuccess) return e;
   if (!small_t_supported(H, I) || T < 1 || T > kMaxT || T * k > kMaxPairs) return cudaSuccess;
+  // scales are staged only when they fit, so the bf16-sized layout decides
   const SmallTConfig cfg = small_t_config(static_cast<int>(T), static_cast<int>(T) * k, H, I, E,
-                                          g_grid_of[dev], g_budget_of[dev], fp8 ? 1 : 2);
+                                          g_grid_of[dev], g_budget_of[dev], fp8 ? 1 : 2, 0);
   *fits = cfg.smem <= g_budget_of[dev];
   return cudaSuccess;
 }
@@ -899,7 +1036,8 @@ cudaError_t launch_small_t(const uint16_t *hidden, const void *w1, const void *w
               I % block != 0))
     return cudaErrorInvalidValue;
   const SmallTConfig cfg = small_t_config(static_cast<int>(T), static_cast<int>(T) * k, H, I, E,
-                                          grid, g_budget_of[dev], fp8 ? 1 : 2);
+                                          grid, g_budget_of[dev], fp8 ? 1 : 2,
+                                          fp8 ? I / block : 0);
   if (cfg.smem > g_budget_of[dev]) return cudaErrorInvalidValue;
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(grid);
@@ -917,7 +1055,7 @@ cudaError_t launch_small_t(const uint16_t *hidden, const void *w1, const void *w
   e = cudaLaunchKernelEx(&lc, kern, reinterpret_cast<const uint4 *>(hidden),
                          reinterpret_cast<const uint4 *>(w1), reinterpret_cast<const uint4 *>(w2),
                          w1_scale, w2_scale, block, b1, b2, act_kind, topk_weights, topk_ids, act, out, static_cast<int>(T), k, H, I, E,
-                         cfg.rows_per_cta, cfg.slots, cfg.cache_act, status,
+                         cfg.rows_per_cta, cfg.slots, cfg.cache_act, cfg.stage_scl, status,
                          grid_sync, wait_limit_ns, timeline, timeline_cap);
   return hook.end(e);
 }
