@@ -106,9 +106,9 @@ int moe_route(const float *logits, int64_t T, int E, int k, int renorm,
  *                 term, acc = fma(w_j, y_j, acc) from acc = 0); a row with
  *                 no valid id is 0.
  * Numerics: bf16 inputs, fp32 accumulation; the SwiGLU intermediate is
- * rounded to bf16 before the second projection on the grouped-GEMM path
- * and kept in fp32 on the small-T path (T <= the small-T limit, H <= 4096
- * and I <= 12288).  The combine is deterministic: repeated calls give
+ * rounded to bf16 before the second projection on both paths (grouped
+ * GEMMs, and the small-T path: T <= the small-T limit, H <= 4096 and
+ * I <= 12288).  The combine is deterministic: repeated calls give
  * identical bits.
  * hidden, w1, w2 and out must start on a 16-byte boundary.
  * Errors: INVALID_ARG for null pointers, hidden/w1/w2/out not 16-byte
@@ -189,10 +189,11 @@ int moe_forward_fp8(const uint16_t *hidden, const uint8_t *w1, const float *w1_s
  * synchronisation of cudaFree when a workspace grows.
  *
  * Arguments, layouts, numerics and the result are those of moe_forward on
- * its small-T path (fp32 SwiGLU intermediate, fixed-order fp32 combine).
+ * its small-T path (bf16 SwiGLU intermediate, fixed-order fp32 combine).
  * Its only scratch is a fixed __device__ array of this library:
- * 256 bytes + MOE_NOALLOC_MAX_ACT fp32 values (1 MiB), which every GPU that
- * loads the library holds until the process exits.
+ * 256 bytes + MOE_NOALLOC_MAX_ACT fp32-sized values (1 MiB; the bf16
+ * intermediate uses half of it), which every GPU that loads the library
+ * holds until the process exits.
  *   - Limits: T <= MOE_NOALLOC_MAX_T and T*k*I <= MOE_NOALLOC_MAX_ACT, else
  *     MOE_ERR_SCRATCH_LIMIT and nothing is launched.  Other checks and
  *     codes as in moe_forward, plus UNSUPPORTED when H > 4096 or I > 12288

@@ -6,7 +6,7 @@
 // reservation at start-up, or a latency-critical decode loop that cannot
 // afford the device-wide synchronisation that cudaFree performs when the
 // regular entry points grow their workspace.  Such callers pass inputs and
-// outputs as usual; the only scratch this path needs (the fp32 SwiGLU
+// outputs as usual; the only scratch this path needs (the bf16 SwiGLU
 // intermediate of at most MOE_NOALLOC_MAX_ACT values, plus a status word)
 // lives in a fixed __device__ array of this file, which every GPU that loads
 // the library keeps until the process exits.

@@ -10,8 +10,9 @@
 //     row i) row pairs -- gate row w1[e, i, :] and up row w1[e, I+i, :] --
 //     dealt round-robin to every warp of the grid.  A warp dots both rows
 //     with the vectors (staged in shared memory) of the tokens routed to e,
-//     in groups of up to four, and stores act[t*k + j, i] = silu(g) * u in
-//     fp32 (global memory) -- or the variant's activation of g + b1[e, i]
+//     in groups of up to four, and stores act[t*k + j, i] = silu(g) * u
+//     rounded to bf16 (global memory; the grouped-GEMM path keeps the same
+//     intermediate in bf16) -- or the variant's activation of g + b1[e, i]
 //     and u + b1[e, I + i].  Meanwhile the copy warp moves the w2 rows this
 //     CTA needs in phase 2 into a ring of shared-memory slots (one chosen
 //     expert per slot) with bulk copies, so w2 streams from HBM alongside
@@ -39,6 +40,7 @@
 // (gate-up, silu-down, weighted blend) with the activation fused into the
 // first phase and the blend into the second.
 #include <cuda_fp16.h>
+#include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
 #include <algorithm>
@@ -165,45 +167,6 @@ __device__ __forceinline__ float fma8_bf16(const uint4 &w, const uint4 &x, float
   return acc;
 }
 
-// Two fp32 sums in one 64-bit register (even and odd terms), advanced with
-// the packed fma.rn.f32x2: acc += w[q] * x[q] for 8 bf16 weights and 8 fp32
-// values (x0 = terms 0..3, x1 = terms 4..7).
-__device__ __forceinline__ void fma8_f32x2(const uint4 &w, const float4 &x0, const float4 &x1,
-                                           unsigned long long &acc) {
-  asm("{\n\t"
-      ".reg .b32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
-      ".reg .b64 p0, p1, p2, p3, q0, q1, q2, q3;\n\t"
-      "shl.b32 l0, %1, 16;\n\t"
-      "and.b32 h0, %1, 0xffff0000;\n\t"
-      "shl.b32 l1, %2, 16;\n\t"
-      "and.b32 h1, %2, 0xffff0000;\n\t"
-      "shl.b32 l2, %3, 16;\n\t"
-      "and.b32 h2, %3, 0xffff0000;\n\t"
-      "shl.b32 l3, %4, 16;\n\t"
-      "and.b32 h3, %4, 0xffff0000;\n\t"
-      "mov.b64 p0, {l0, h0};\n\t"
-      "mov.b64 p1, {l1, h1};\n\t"
-      "mov.b64 p2, {l2, h2};\n\t"
-      "mov.b64 p3, {l3, h3};\n\t"
-      "mov.b64 q0, {%5, %6};\n\t"
-      "mov.b64 q1, {%7, %8};\n\t"
-      "mov.b64 q2, {%9, %10};\n\t"
-      "mov.b64 q3, {%11, %12};\n\t"
-      "fma.rn.f32x2 %0, p0, q0, %0;\n\t"
-      "fma.rn.f32x2 %0, p1, q1, %0;\n\t"
-      "fma.rn.f32x2 %0, p2, q2, %0;\n\t"
-      "fma.rn.f32x2 %0, p3, q3, %0;\n\t"
-      "}"
-      : "+l"(acc)
-      : "r"(w.x), "r"(w.y), "r"(w.z), "r"(w.w), "f"(x0.x), "f"(x0.y), "f"(x0.z), "f"(x0.w),
-        "f"(x1.x), "f"(x1.y), "f"(x1.z), "f"(x1.w));
-}
-
-__device__ __forceinline__ float sum_f32x2(unsigned long long acc) {
-  return __uint_as_float(static_cast<uint32_t>(acc)) +
-         __uint_as_float(static_cast<uint32_t>(acc >> 32));
-}
-
 // Two E4M3 codes (low byte first) as floats, by the hardware conversion.
 __device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two) {
   const __half2_raw r =
@@ -233,43 +196,14 @@ __device__ __forceinline__ float dot16_e4m3_bf16(const uint4 &w, const uint4 &x0
   return s0 + s1;
 }
 
-// sum over q = 0..15 of e4m3(w[q]) * a[q] for 16 codes and 16 fp32 values,
-// two interleaved partial sums
-__device__ __forceinline__ float dot16_e4m3_f32(const uint4 &w, const float4 &a0,
-                                                const float4 &a1, const float4 &a2,
-                                                const float4 &a3) {
-  float s0 = 0.f, s1 = 0.f;
-  float2 p = e4m3x2_to_float2(w.x);
-  s0 = fmaf(p.x, a0.x, s0);
-  s1 = fmaf(p.y, a0.y, s1);
-  p = e4m3x2_to_float2(w.x >> 16);
-  s0 = fmaf(p.x, a0.z, s0);
-  s1 = fmaf(p.y, a0.w, s1);
-  p = e4m3x2_to_float2(w.y);
-  s0 = fmaf(p.x, a1.x, s0);
-  s1 = fmaf(p.y, a1.y, s1);
-  p = e4m3x2_to_float2(w.y >> 16);
-  s0 = fmaf(p.x, a1.z, s0);
-  s1 = fmaf(p.y, a1.w, s1);
-  p = e4m3x2_to_float2(w.z);
-  s0 = fmaf(p.x, a2.x, s0);
-  s1 = fmaf(p.y, a2.y, s1);
-  p = e4m3x2_to_float2(w.z >> 16);
-  s0 = fmaf(p.x, a2.z, s0);
-  s1 = fmaf(p.y, a2.w, s1);
-  p = e4m3x2_to_float2(w.w);
-  s0 = fmaf(p.x, a3.x, s0);
-  s1 = fmaf(p.y, a3.y, s1);
-  p = e4m3x2_to_float2(w.w >> 16);
-  s0 = fmaf(p.x, a3.z, s0);
-  s1 = fmaf(p.y, a3.w, s1);
-  return s0 + s1;
-}
-
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
+}
+
+__device__ __forceinline__ uint16_t bf16_bits(float v) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 
 __device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long *p) {
@@ -290,7 +224,7 @@ __device__ __forceinline__ void phase1_group(const uint4 *__restrict__ g,
                                              const int *plist,
                                              int nq, int k, int H8, int I, int i, float bg,
                                              float bu, bool bias, int act_kind,
-                                             float *__restrict__ act, const float *sg,
+                                             uint16_t *__restrict__ act, const float *sg,
                                              const float *su, int cpb) {
   const int lane = threadIdx.x & 31;
   const int HC = kFp8 ? H8 / 2 : H8;  // 16-byte weight chunks per row
@@ -349,33 +283,33 @@ __device__ __forceinline__ void phase1_group(const uint4 *__restrict__ g,
       const float us = warp_sum(au[q]);
       if (lane == 0)
         act[static_cast<size_t>(plist[q]) * I + i] =
-            bias ? gated_rt(act_kind, gs + bg, us + bu) : gated_rt(act_kind, gs, us);
+            bf16_bits(bias ? gated_rt(act_kind, gs + bg, us + bu) : gated_rt(act_kind, gs, us));
     }
   }
 }
 
 // Phase 2 item: the kR2 dot products of w2 rows r0.. r0+kR2-1 of this CTA
-// (ws: in shared memory, else wg: through L2) with act of one pair; the act
-// chunks are loaded once for the kR2 independent sums.  Lane 0 writes
+// (ws: in shared memory, else wg: through L2) with act of one pair (bf16,
+// a8: 8 values per 16-byte chunk, on chip when cache_act); the act chunks
+// are loaded once for the kR2 independent sums.  Lane 0 writes
 // sdots[r][pair].
 // FP8 weights: 16 codes per chunk, each chunk's partial sum times the scale
 // of its row and block (s2r: the scales of row r0, ipb per row).
 template <bool kFp8>
 __device__ __forceinline__ void phase2_item(const uint4 *ws, const uint4 *__restrict__ wg,
-                                            const float4 *a4, int cache_act, int pair, int r0,
+                                            const uint4 *a8, int cache_act, int pair, int r0,
                                             int nrows, int I, int TK, float *sdots,
                                             const float *s2r, int ipb, int cpb) {
   const int lane = threadIdx.x & 31;
-  const int I8 = I / 8;
-  const float4 *a = a4 + static_cast<size_t>(pair) * (I / 4);
-  if constexpr (kFp8) {
-    const int IC = I / 16;
-    float v[kR2];
+  const uint4 *a = a8 + static_cast<size_t>(pair) * (I / 8);
+  const int IC = kFp8 ? I / 16 : I / 8;  // 16-byte weight chunks per row
+  float v[kR2];
 #pragma unroll
-    for (int rr = 0; rr < kR2; ++rr) v[rr] = 0.f;
-    for (int base = 0; base < IC; base += 32 * kU2) {
-      // the scales of this lane's chunks, loaded ahead of the dot products
-      float sc[kU2][kR2];
+  for (int rr = 0; rr < kR2; ++rr) v[rr] = 0.f;
+  for (int base = 0; base < IC; base += 32 * kU2) {
+    // FP8: the scales of this lane's chunks, loaded ahead of the dot products
+    float sc[kU2][kR2];
+    if (kFp8) {
 #pragma unroll
       for (int j = 0; j < kU2; ++j) {
         const int c = base + lane + 32 * j;
@@ -384,57 +318,33 @@ __device__ __forceinline__ void phase2_item(const uint4 *ws, const uint4 *__rest
           // s2r may point into shared memory: a generic load
           sc[j][rr] = c < IC && r0 + rr < nrows ? s2r[rr * ipb + c / cpb] : 0.f;
       }
+    }
 #pragma unroll
-      for (int j = 0; j < kU2; ++j) {
-        const int c = base + lane + 32 * j;
-        if (c < IC) {
-          const float4 a0 = cache_act ? a[4 * c] : __ldcg(a + 4 * c);
-          const float4 a1 = cache_act ? a[4 * c + 1] : __ldcg(a + 4 * c + 1);
-          const float4 a2 = cache_act ? a[4 * c + 2] : __ldcg(a + 4 * c + 2);
-          const float4 a3 = cache_act ? a[4 * c + 3] : __ldcg(a + 4 * c + 3);
+    for (int j = 0; j < kU2; ++j) {
+      const int c = base + lane + 32 * j;
+      if (c < IC) {
+        // the act values of this chunk: 16 (FP8) or 8 (bf16 weights)
+        const uint4 x0 = cache_act ? a[(kFp8 ? 2 : 1) * c] : __ldcg(a + (kFp8 ? 2 : 1) * c);
+        uint4 x1 = x0;
+        if (kFp8) x1 = cache_act ? a[2 * c + 1] : __ldcg(a + 2 * c + 1);
 #pragma unroll
-          for (int rr = 0; rr < kR2; ++rr) {
-            if (r0 + rr < nrows) {
-              const uint4 wv =
-                  ws != nullptr ? ws[(r0 + rr) * IC + c] : __ldg(wg + (r0 + rr) * IC + c);
-              v[rr] = fmaf(dot16_e4m3_f32(wv, a0, a1, a2, a3), sc[j][rr], v[rr]);
-            }
+        for (int rr = 0; rr < kR2; ++rr) {
+          if (r0 + rr < nrows) {
+            const uint4 wv =
+                ws != nullptr ? ws[(r0 + rr) * IC + c] : __ldg(wg + (r0 + rr) * IC + c);
+            if (kFp8)
+              v[rr] = fmaf(dot16_e4m3_bf16(wv, x0, x1), sc[j][rr], v[rr]);
+            else
+              v[rr] = fma8_bf16(wv, x0, v[rr]);
           }
         }
       }
     }
+  }
 #pragma unroll
-    for (int rr = 0; rr < kR2; ++rr) {
-      const float sv = warp_sum(v[rr]);
-      if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
-    }
-  } else {
-    unsigned long long v[kR2];  // two fp32 partial sums each
-#pragma unroll
-    for (int rr = 0; rr < kR2; ++rr) v[rr] = 0ull;
-    for (int base = 0; base < I8; base += 32 * kU2) {
-#pragma unroll
-      for (int j = 0; j < kU2; ++j) {
-        const int c = base + lane + 32 * j;
-        if (c < I8) {
-          const float4 a0 = cache_act ? a[2 * c] : __ldcg(a + 2 * c);
-          const float4 a1 = cache_act ? a[2 * c + 1] : __ldcg(a + 2 * c + 1);
-#pragma unroll
-          for (int rr = 0; rr < kR2; ++rr) {
-            if (r0 + rr < nrows) {
-              const uint4 wv =
-                  ws != nullptr ? ws[(r0 + rr) * I8 + c] : __ldg(wg + (r0 + rr) * I8 + c);
-              fma8_f32x2(wv, a0, a1, v[rr]);
-            }
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int rr = 0; rr < kR2; ++rr) {
-      const float sv = warp_sum(sum_f32x2(v[rr]));
-      if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
-    }
+  for (int rr = 0; rr < kR2; ++rr) {
+    const float sv = warp_sum(v[rr]);
+    if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
   }
 }
 
@@ -450,85 +360,62 @@ __device__ __forceinline__ void phase2_item(const uint4 *ws, const uint4 *__rest
 constexpr int kU2c = 3;  // bf16: chunks per lane per block (I = 768: one block)
 constexpr int kU2f = 1;  // FP8: chunks of 16 codes per lane per block
 template <bool kFp8>
-__device__ __forceinline__ void phase2_item_onchip(const uint4 *ws, const float4 *sa,
+__device__ __forceinline__ void phase2_item_onchip(const uint4 *ws, const uint4 *sa,
                                                    const float *sc0, int pair, int r0,
                                                    int nrows, int I, int TK, float *sdots,
                                                    int ipb, int cpb) {
   const int lane = threadIdx.x & 31;
+  constexpr int kU = kFp8 ? kU2f : kU2c;
+  const int IC = kFp8 ? I / 16 : I / 8;
   int rows[kR2];
 #pragma unroll
   for (int rr = 0; rr < kR2; ++rr) rows[rr] = min(r0 + rr, nrows - 1);
-  if constexpr (kFp8) {
-    const int IC = I / 16;
-    float v[kR2];
+  float v[kR2];
 #pragma unroll
-    for (int rr = 0; rr < kR2; ++rr) v[rr] = 0.f;
-    for (int base = 0; base < IC; base += 32 * kU2f) {
-      float4 a[kU2f][4];
-      uint4 wv[kU2f][kR2];
-      float sc[kU2f][kR2];
+  for (int rr = 0; rr < kR2; ++rr) v[rr] = 0.f;
+  for (int base = 0; base < IC; base += 32 * kU) {
+    uint4 x0[kU], x1[kU];
+    uint4 wv[kU][kR2];
+    float sc[kU][kR2];
 #pragma unroll
-      for (int j = 0; j < kU2f; ++j) {
-        const int c = min(base + lane + 32 * j, IC - 1);
+    for (int j = 0; j < kU; ++j) {
+      const int c = min(base + lane + 32 * j, IC - 1);
+      if (kFp8) {
+        x0[j] = sa[2 * c];
+        x1[j] = sa[2 * c + 1];
+      } else {
+        x0[j] = sa[c];
+      }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) a[j][q] = sa[4 * c + q];
+      for (int rr = 0; rr < kR2; ++rr) {
+        wv[j][rr] = ws[rows[rr] * IC + c];
+        if (kFp8) sc[j][rr] = sc0[rows[rr] * ipb + c / cpb];  // generic: shared or global
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kU; ++j) {
+      if (base + lane + 32 * j < IC) {
 #pragma unroll
         for (int rr = 0; rr < kR2; ++rr) {
-          wv[j][rr] = ws[rows[rr] * IC + c];
-          sc[j][rr] = sc0[rows[rr] * ipb + c / cpb];  // generic: shared or global
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < kU2f; ++j) {
-        if (base + lane + 32 * j < IC) {
-#pragma unroll
-          for (int rr = 0; rr < kR2; ++rr)
-            v[rr] = fmaf(dot16_e4m3_f32(wv[j][rr], a[j][0], a[j][1], a[j][2], a[j][3]),
-                         sc[j][rr], v[rr]);
+          if (kFp8)
+            v[rr] = fmaf(dot16_e4m3_bf16(wv[j][rr], x0[j], x1[j]), sc[j][rr], v[rr]);
+          else
+            v[rr] = fma8_bf16(wv[j][rr], x0[j], v[rr]);
         }
       }
     }
+  }
 #pragma unroll
-    for (int rr = 0; rr < kR2; ++rr) {
-      const float sv = warp_sum(v[rr]);
-      if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
-    }
-  } else {
-    const int I8 = I / 8;
-    unsigned long long v[kR2];  // two fp32 partial sums each
-#pragma unroll
-    for (int rr = 0; rr < kR2; ++rr) v[rr] = 0ull;
-    for (int base = 0; base < I8; base += 32 * kU2c) {
-      float4 lo[kU2c], hi[kU2c];
-      uint4 wv[kU2c][kR2];
-#pragma unroll
-      for (int j = 0; j < kU2c; ++j) {
-        const int c = min(base + lane + 32 * j, I8 - 1);
-        lo[j] = sa[2 * c];
-        hi[j] = sa[2 * c + 1];
-#pragma unroll
-        for (int rr = 0; rr < kR2; ++rr) wv[j][rr] = ws[rows[rr] * I8 + c];
-      }
-#pragma unroll
-      for (int j = 0; j < kU2c; ++j) {
-        if (base + lane + 32 * j < I8) {
-#pragma unroll
-          for (int rr = 0; rr < kR2; ++rr) fma8_f32x2(wv[j][rr], lo[j], hi[j], v[rr]);
-        }
-      }
-    }
-#pragma unroll
-    for (int rr = 0; rr < kR2; ++rr) {
-      const float sv = warp_sum(sum_f32x2(v[rr]));
-      if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
-    }
+  for (int rr = 0; rr < kR2; ++rr) {
+    const float sv = warp_sum(v[rr]);
+    if (lane == 0 && r0 + rr < nrows) sdots[(r0 + rr) * TK + pair] = sv;
   }
 }
 
 // Dynamic shared memory of a CTA: the token vectors in bf16 [T][H]; a ring of `slots` buffers, each holding this
 // CTA's w2 rows of one chosen expert in bf16 [rows_per_cta][I] (no ring when
 // one expert's rows do not fit: phase 2 then reads w2 through L2); act in
-// fp32 [T*k][I] when it fits; the dot products [rows_per_cta][T*k].
+// bf16 [T*k][I] when it fits; the dot products [rows_per_cta][T*k].
 struct SmemLayout {
   size_t w2_off, act_off, dots_off, scl_off, total;
 };
@@ -546,7 +433,7 @@ __host__ __device__ inline SmemLayout smem_layout(int T, int TK, int H, int I,
   SmemLayout s;
   s.w2_off = static_cast<size_t>(T) * H * 2;
   s.act_off = s.w2_off + static_cast<size_t>(slots) * w2_slot_bytes(rows_per_cta, I, elem);
-  s.dots_off = s.act_off + (cache_act ? static_cast<size_t>(TK) * I * sizeof(float) : 0);
+  s.dots_off = s.act_off + (cache_act ? static_cast<size_t>(TK) * I * 2 : 0);  // bf16
   s.scl_off = s.dots_off + static_cast<size_t>(rows_per_cta) * TK * sizeof(float);
   s.total = s.scl_off + static_cast<size_t>(slots) * rows_per_cta * scl * sizeof(float);
   return s;
@@ -587,8 +474,10 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       smem_layout(T, TK, H, I, rows_per_cta, slots, cache_act, kElem, stage_scl ? ipb : 0);
   const size_t slot_stride = w2_slot_bytes(rows_per_cta, I, kElem);
   uint8_t *sx = smem;  // the token's vector (one-token kernel)
+  // act scratch (T*k*I values): bf16 bits in the caller's fp32-sized buffer
+  uint16_t *act_h = reinterpret_cast<uint16_t *>(act);
   uint8_t *sw2 = smem + lay.w2_off;
-  float *sact = reinterpret_cast<float *>(smem + lay.act_off);
+  uint4 *sact = reinterpret_cast<uint4 *>(smem + lay.act_off);  // act in bf16 [T*k][I]
   float *sdots = reinterpret_cast<float *>(smem + lay.dots_off);
   float *sscl = reinterpret_cast<float *>(smem + lay.scl_off);  // [slots][rows_per_cta][ipb]
   const int h0 = blockIdx.x * rows_per_cta;
@@ -701,7 +590,8 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       if (lane == 0) {
         const float a = b1 != nullptr ? gated_rt(act_kind, ag + bg, au + bu)
                                       : gated_rt(act_kind, ag, au);
-        for (int q = 0; q < np; ++q) act[static_cast<size_t>(L.plist[p0 + q]) * I + i] = a;
+        const uint16_t ab = bf16_bits(a);
+        for (int q = 0; q < np; ++q) act_h[static_cast<size_t>(L.plist[p0 + q]) * I + i] = ab;
       }
     } else {
       // the tokens routed to e, in groups of at most 4 (the row pair is
@@ -712,9 +602,9 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
         const bool bias = b1 != nullptr;
         if (nq == 1)
           phase1_group<1, kFp8 ? 4 : 8, kFp8>(g, u, sx4, pl, nq, k, H8, I, i, bg, bu, bias,
-                                              act_kind, act, sg, su, cpb);
+                                              act_kind, act_h, sg, su, cpb);
         else
-          phase1_group<4, 4, kFp8>(g, u, sx4, pl, nq, k, H8, I, i, bg, bu, bias, act_kind, act,
+          phase1_group<4, 4, kFp8>(g, u, sx4, pl, nq, k, H8, I, i, bg, bu, bias, act_kind, act_h,
                                    sg, su, cpb);
       }
     }
@@ -759,17 +649,16 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
   }
 
   // ------------------------------------------------------------ phase 2
-  const float4 *act4 = reinterpret_cast<const float4 *>(act);
+  const uint4 *act8 = reinterpret_cast<const uint4 *>(act_h);
   // every operand on chip (w2 rows in the ring, act staged below):
   // phase2_item_onchip
   const bool onchip = ring && cache_act;
   if (cache_act) {
     // act was written by other CTAs in this launch: read it from L2
-    const int n4 = TK * I / 4;
-    float4 *d4 = reinterpret_cast<float4 *>(sact);
-    for (int x = threadIdx.x; x < n4; x += kThreads) d4[x] = __ldcg(act4 + x);
+    const int n8 = TK * I / 8;
+    for (int x = threadIdx.x; x < n8; x += kThreads) sact[x] = __ldcg(act8 + x);
     __syncthreads();
-    act4 = d4;
+    act8 = sact;
   }
   const uint64_t tl_act = tl_buf ? global_timer_ns() : 0;
   if (threadIdx.x == 0)
@@ -822,13 +711,13 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
       if (onchip)
         phase2_item_onchip<kFp8>(
             reinterpret_cast<const uint4 *>(sw2 + d * slot_stride),
-            act4 + static_cast<size_t>(pair) * (I / 4),
+            act8 + static_cast<size_t>(pair) * (I / 8),
             !kFp8 ? nullptr
                   : stage_scl ? sscl + static_cast<size_t>(d) * rows_per_cta * ipb : s2 + row0 * ipb,
             pair, rg * kR2, nrows, I, TK, sdots, ipb, cpb);
       else
         phase2_item<kFp8>(ring ? reinterpret_cast<const uint4 *>(sw2 + d * slot_stride) : nullptr,
-                          w2 + row0 * IC, act4, cache_act, pair, rg * kR2, nrows, I, TK, sdots,
+                          w2 + row0 * IC, act8, cache_act, pair, rg * kR2, nrows, I, TK, sdots,
                           s2r, ipb, cpb);
     }
   } else if (rgroups > 0) {
@@ -853,14 +742,14 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm)
         if (onchip)
           phase2_item_onchip<kFp8>(
               reinterpret_cast<const uint4 *>(sw2 + q * slot_stride),
-              act4 + static_cast<size_t>(L.plist[pq]) * (I / 4),
+              act8 + static_cast<size_t>(L.plist[pq]) * (I / 8),
               !kFp8                     ? nullptr
               : stage_scl && d < slots ? sscl + static_cast<size_t>(d) * rows_per_cta * ipb
                                        : s2 + row0 * ipb,
               L.plist[pq], rg * kR2, nrows, I, TK, sdots, ipb, cpb);
         else
           phase2_item<kFp8>(reinterpret_cast<const uint4 *>(sw2 + q * slot_stride), nullptr,
-                            act4, cache_act, L.plist[pq], rg * kR2, nrows, I, TK, sdots,
+                            act8, cache_act, L.plist[pq], rg * kR2, nrows, I, TK, sdots,
                             kFp8 ? s2 + (row0 + rg * kR2) * ipb : nullptr, ipb, cpb);
       }
       before += n_items;
@@ -925,7 +814,7 @@ SmallTConfig small_t_config(int T, int TK, int H, int I, int E, int grid, size_t
     while (n > 0 && size(n, cache) > budget) --n;
     return n;
   };
-  c.cache_act = static_cast<size_t>(TK) * I * sizeof(float) <= kActCacheMax ? 1 : 0;
+  c.cache_act = static_cast<size_t>(TK) * I * 2 <= kActCacheMax ? 1 : 0;
   c.slots = fit(c.cache_act);
   if (c.cache_act && c.slots < std::min(want, 2) && fit(0) > c.slots) {
     c.cache_act = 0;
