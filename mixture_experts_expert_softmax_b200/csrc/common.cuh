@@ -128,12 +128,6 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
 }
 
 // Bring `bytes` of global memory into L2 without waiting.
-// Ask L2 to fetch the 128-byte line holding p (no data comes back; the
-// thread does not wait).
-__device__ __forceinline__ void prefetch_l2_line(const void *p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }

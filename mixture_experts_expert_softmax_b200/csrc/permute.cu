@@ -180,17 +180,6 @@ __global__ void __launch_bounds__(kGroupThreads)
   uint16_t *s_hist = reinterpret_cast<uint16_t *>(s_tot + E);         // [warps][E]
   __shared__ int32_t s_warp_tot[kGroupWarps];
   __shared__ int32_t s_nvalid;
-  if (xs != nullptr) {
-    // The hidden rows do not come from the previous kernel: have L2 fetch
-    // them now, so that the row copy after the sort reads them from L2
-    // rather than waiting on DRAM (a prefetch only warms L2, so it is
-    // correct whatever the previous kernel still writes).
-    const int64_t lines = static_cast<int64_t>(n / k) * (H8 / 8);  // 128-byte lines
-    const char *hb = reinterpret_cast<const char *>(hidden);
-    for (int64_t l = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; l < lines;
-         l += static_cast<int64_t>(gridDim.x) * blockDim.x)
-      prefetch_l2_line(hb + l * 128);
-  }
   grid_dep_wait();
   grid_dep_launch();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
