@@ -201,9 +201,9 @@ int moe_forward_fp8(const uint16_t *hidden, const uint8_t *w1, const float *w1_s
  *     token vectors and per-CTA buffers do not fit the kernel's shared
  *     memory on this device.
  *   - The first call on each device, with that device current, looks up
- *     the array's device address (cudaGetSymbolAddress) and caches it; make
- *     that first call before any stream capture.  cudaDeviceReset between
- *     calls is not supported (the cached address would be stale).
+ *     the array's device address (cudaGetSymbolAddress, a host-side runtime
+ *     query) and caches it for later calls.  cudaDeviceReset between calls
+ *     is not supported (the cached address would be stale).
  *   - All calls share the one array, which keeps the last call's contents.
  *     Nothing in it has to be cleared between calls: every act value is
  *     written before it is read in the same call, and the grid-barrier
