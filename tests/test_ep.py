@@ -165,7 +165,7 @@ def _ep_worker(rank, world, port, shape, q):
 
 
 @pytest.mark.parametrize("world,shape", [(2, (13, 128, 128, 8, 2)), (4, (9, 256, 128, 16, 4)),
-                                         (4, (5, 128, 256, 8, 8))])
+                                         (4, (5, 128, 256, 8, 8)), (8, (6, 128, 128, 16, 3))])
 def test_ep_gloo_ranks_match_single_rank_oracle(world, shape):
     port = _free_port()
     ctx = mp.get_context("spawn")
