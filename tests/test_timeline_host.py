@@ -44,3 +44,20 @@ def test_summary_mma_bins_busy_and_gaps():
 
 def test_summary_of_nothing_is_empty():
     assert moe.timeline_summary([]) == {}
+
+
+def test_decoder_names_match_the_device_codes():
+    """The kind and role codes the kernels write (an enum in the device
+    header) decode to the names timeline_stop reports."""
+    import re
+    src = open(os.path.join(ROOT, "mixture_experts_expert_softmax_b200", "csrc",
+                            "common.cuh")).read()
+    codes = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(kTl\w+)\s*=\s*(\d+)", src)}
+    kinds = {"kTlGemm1": "gemm1", "kTlGemm2": "gemm2", "kTlFused": "gemm_fused",
+             "kTlSmallT": "small_t"}
+    roles = {"kTlProducer": "producer", "kTlMma": "mma", "kTlEpilogue": "epilogue",
+             "kTlPhase1": "phase1", "kTlBarrier": "barrier", "kTlActLoad": "act_load",
+             "kTlW2Wait": "w2_wait", "kTlPhase2": "phase2", "kTlItems": "phase2_dots"}
+    assert set(kinds) | set(roles) <= set(codes)
+    assert {codes[c]: n for c, n in kinds.items()} == moe.TIMELINE_KINDS
+    assert {codes[c]: n for c, n in roles.items()} == moe.TIMELINE_ROLES
